@@ -1,0 +1,275 @@
+/*
+ * convrot_oracle.c -- plain, slow, single-threaded CPU oracle for the ConvRot
+ * W4A4 quantized Linear.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only the tests, the smoke check and the CPU
+ * baseline leg of the benchmark may load this file's library.  The CUDA
+ * library never links, includes or calls it, and it shares no code, header,
+ * table or constant generator with the CUDA path.
+ *
+ * What it computes (sources, by page title and section):
+ *  - "Qwen-Image-Edit-2511 -- INT4 tensorwise W4A4 (+ConvRot, mixed int8
+ *    fallback)" (HF card, intro paragraph): weights are packed signed INT4,
+ *    two codes per byte, rotated with a group-256 regular-Hadamard ConvRot
+ *    rotation; activations are rotated online and quantized dynamically to
+ *    INT4; calibration-free.  Speed table: a "rank-one" s4 MMA kernel, i.e.
+ *    the integer product is rescaled by s_a[m] * s_w[n].
+ *  - "rockerBOO/qwen3-4b-nvfp4-convrot" (file table): group-wise Hadamard
+ *    rotation, group size 256.
+ *  - "Nicolaslas/Rebels_w4a8s" ("What I do differently"): the ConvRot group is
+ *    exactly 256, so K must be a multiple of 256.
+ *  - "JoaoZaokk/Z-Image-Turbo-W4A4-ConvRot" ("Where Z-Image sits"): group
+ *    sizes 256, 64 and 16 exist (the rotation of order 4^s for s = 4, 3, 2).
+ *
+ * Readings the pages leave open, fixed here (each is listed in the design
+ * notes):
+ *  - The regular Hadamard of order 4 is H4 = [[1,1,1,-1],[1,1,-1,1],
+ *    [1,-1,1,1],[-1,1,1,1]]; order 256 is H4 (x) H4 (x) H4 (x) H4, scaled by
+ *    1/16 so that it is orthonormal.
+ *  - It is evaluated as 4 radix-4 butterfly stages, stride 1 first, then 4,
+ *    16, 64.  One butterfly on (a, b, c, d) forms p=a+b, q=a-b, r=c+d,
+ *    t=c-d and writes (p+t, p-t, q+r, r-q).  Every add is one IEEE fp32
+ *    round-to-nearest add with no contraction (compile with
+ *    -ffp-contract=off).  The 1/16 is applied last, as one fp32 multiply.
+ *  - Per-token scale: s_a[m] = amax_k |x'[m,k]| / 7 (one IEEE fp32 divide),
+ *    over the whole row (all groups).  amax == 0 gives s_a = 0 and all codes 0.
+ *  - Code: q = clamp(rint(x' / s_a), -8, 7), rint = round half to even, the
+ *    quotient is a true IEEE fp32 division.
+ *  - Packing: byte i of a row = (q[2i] & 0xF) | ((q[2i+1] & 0xF) << 4).
+ *  - GEMM: acc[m,n] = sum_k q_a[m,k] * q_w[n,k] in int64.
+ *  - Epilogue: y32 = ((float)acc * s_a[m]) * s_w[n] + (float)bias[n], each op
+ *    one fp32 RN op; y = bf16 round-to-nearest-even of y32.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define ORACLE_OK 0
+#define ORACLE_ERR_SHAPE 1
+#define ORACLE_ERR_OVERFLOW 2
+#define ORACLE_ERR_NOMEM 3
+
+/* ---- bf16 <-> fp32 (plain definitions) -------------------------------- */
+
+/* bf16 is the top 16 bits of an IEEE binary32, so widening is a shift. */
+static float bf16_bits_to_f32(uint16_t h) {
+  uint32_t u = ((uint32_t)h) << 16;
+  float f;
+  memcpy(&f, &u, sizeof f);
+  return f;
+}
+
+/* Round-to-nearest-even of binary32 to its top 16 bits; NaN stays NaN. */
+static uint16_t f32_to_bf16_bits_rne(float f) {
+  uint32_t u;
+  memcpy(&u, &f, sizeof u);
+  if ((u & 0x7fffffffu) > 0x7f800000u) return (uint16_t)((u >> 16) | 0x0040u);
+  uint32_t lsb = (u >> 16) & 1u;
+  u += 0x7fffu + lsb;
+  return (uint16_t)(u >> 16);
+}
+
+uint16_t oracle_f32_to_bf16(float f) { return f32_to_bf16_bits_rne(f); }
+float oracle_bf16_to_f32(uint16_t h) { return bf16_bits_to_f32(h); }
+
+/* ---- rotation ----------------------------------------------------------- */
+
+/* log4 of a supported group size (16, 64, 256), or -1. */
+static int group_log4(int group) {
+  switch (group) {
+    case 16: return 2;
+    case 64: return 3;
+    case 256: return 4;
+    default: return -1;
+  }
+}
+
+/* One group of G = 4^S values, in place: S radix-4 stages (stride 1, 4, 16,
+ * ...), then one multiply by 1/sqrt(G) = 2^-S. */
+static void rotate_group(float *v, int S) {
+  int G = 1 << (2 * S);
+  for (int s = 0; s < S; ++s) {
+    int st = 1 << (2 * s);
+    for (int i = 0; i < G; ++i) {
+      if (((i / st) & 3) != 0) continue; /* digit s of i must be 0 */
+      float a = v[i], b = v[i + st], c = v[i + 2 * st], d = v[i + 3 * st];
+      float p = a + b;
+      float q = a - b;
+      float r = c + d;
+      float t = c - d;
+      v[i] = p + t;
+      v[i + st] = p - t;
+      v[i + 2 * st] = q + r;
+      v[i + 3 * st] = r - q;
+    }
+  }
+  float scale = ldexpf(1.0f, -S);
+  for (int i = 0; i < G; ++i) v[i] = v[i] * scale;
+}
+
+/* In-place block-diagonal rotation of an fp32 [M, K] matrix, group by group
+ * along K.  Returns ORACLE_ERR_SHAPE when K is not a multiple of the group. */
+int oracle_rotate_rows_f32(float *data, int M, int K, int group) {
+  int S = group_log4(group);
+  if (S < 0 || M < 0 || K < 0 || K % group != 0) return ORACLE_ERR_SHAPE;
+  for (int m = 0; m < M; ++m)
+    for (int g = 0; g < K / group; ++g) rotate_group(data + (size_t)m * K + (size_t)g * group, S);
+  return ORACLE_OK;
+}
+
+/* ---- packing -------------------------------------------------------------- */
+
+/* Two signed 4-bit codes per byte, the even index in the low nibble. */
+void oracle_pack_codes(const int8_t *q, int64_t n, uint8_t *out) {
+  for (int64_t i = 0; i < n / 2; ++i)
+    out[i] = (uint8_t)(((uint8_t)q[2 * i] & 0x0Fu) | (((uint8_t)q[2 * i + 1] & 0x0Fu) << 4));
+}
+
+/* Inverse of oracle_pack_codes: two's-complement sign extension of nibbles. */
+void oracle_unpack_codes(const uint8_t *in, int64_t n, int8_t *q) {
+  for (int64_t i = 0; i < n / 2; ++i) {
+    int lo = in[i] & 0x0F, hi = (in[i] >> 4) & 0x0F;
+    q[2 * i] = (int8_t)(lo >= 8 ? lo - 16 : lo);
+    q[2 * i + 1] = (int8_t)(hi >= 8 ? hi - 16 : hi);
+  }
+}
+
+/* ---- rotate + per-row quantize ------------------------------------------- */
+
+/* x: bf16 bits [M, K]; outputs: codes [M, K] (optional), packed [M, K/2]
+ * (optional), scales [M], rotated fp32 [M, K] (optional). */
+int oracle_rotate_quant_ex(const uint16_t *x, int M, int K, int group, int8_t *codes,
+                           uint8_t *packed, float *scale, float *rotated) {
+  int S = group_log4(group);
+  if (S < 0 || M < 0 || K <= 0 || K % group != 0) return ORACLE_ERR_SHAPE;
+  float *row = (float *)malloc(sizeof(float) * (size_t)K);
+  int8_t *q = (int8_t *)malloc((size_t)K);
+  if (!row || !q) {
+    free(row);
+    free(q);
+    return ORACLE_ERR_NOMEM;
+  }
+  for (int m = 0; m < M; ++m) {
+    const uint16_t *xr = x + (size_t)m * K;
+    for (int k = 0; k < K; ++k) row[k] = bf16_bits_to_f32(xr[k]); /* S1 widen */
+    for (int g = 0; g < K / group; ++g) rotate_group(row + (size_t)g * group, S); /* S2 */
+    float amax = 0.0f; /* S3 per-token amax over the whole row */
+    for (int k = 0; k < K; ++k) {
+      float a = fabsf(row[k]);
+      if (a > amax) amax = a;
+    }
+    float s = amax / 7.0f;
+    for (int k = 0; k < K; ++k) { /* S4 quantize */
+      int c = 0;
+      if (s != 0.0f) {
+        float r = rintf(row[k] / s);
+        if (r < -8.0f) r = -8.0f;
+        if (r > 7.0f) r = 7.0f;
+        c = (int)r;
+      }
+      q[k] = (int8_t)c;
+    }
+    scale[m] = s;
+    if (codes) memcpy(codes + (size_t)m * K, q, (size_t)K);
+    if (packed) oracle_pack_codes(q, K, packed + (size_t)m * (K / 2));
+    if (rotated) memcpy(rotated + (size_t)m * K, row, sizeof(float) * (size_t)K);
+  }
+  free(row);
+  free(q);
+  return ORACLE_OK;
+}
+
+/* The activation prologue: bf16 x[M, K] -> packed codes [M, K/2] + s_a[M]. */
+int oracle_rotate_quant(const uint16_t *x, int M, int K, uint8_t *xq, float *s_a) {
+  return oracle_rotate_quant_ex(x, M, K, 256, NULL, xq, s_a, NULL);
+}
+
+/* Offline weight preparation: the same math on each output channel (row of
+ * W[N, K]), which gives per-output-channel scales. */
+int oracle_pack_weight(const uint16_t *W, int N, int K, uint8_t *Wq, float *s_w) {
+  return oracle_rotate_quant_ex(W, N, K, 256, NULL, Wq, s_w, NULL);
+}
+
+/* ---- integer GEMM --------------------------------------------------------- */
+
+/* acc[m, n] = sum_k q_a[m, k] * q_w[n, k] over packed operands, in int64.
+ * Rows [m0, m1) only, so a caller can time or check a subset of rows. */
+int oracle_gemm_s64_rows(const uint8_t *xq, const uint8_t *Wq, int M, int N, int K, int m0,
+                         int m1, int64_t *acc) {
+  if (M < 0 || N < 0 || K <= 0 || K % 2 != 0 || m0 < 0 || m1 > M || m0 > m1)
+    return ORACLE_ERR_SHAPE;
+  int8_t *a = (int8_t *)malloc((size_t)K);
+  int8_t *w = (int8_t *)malloc((size_t)K * (size_t)(N > 0 ? N : 1));
+  if (!a || !w) {
+    free(a);
+    free(w);
+    return ORACLE_ERR_NOMEM;
+  }
+  for (int n = 0; n < N; ++n) oracle_unpack_codes(Wq + (size_t)n * (K / 2), K, w + (size_t)n * K);
+  for (int m = m0; m < m1; ++m) {
+    oracle_unpack_codes(xq + (size_t)m * (K / 2), K, a);
+    for (int n = 0; n < N; ++n) {
+      const int8_t *wr = w + (size_t)n * K;
+      int64_t s = 0;
+      for (int k = 0; k < K; ++k) s += (int64_t)a[k] * (int64_t)wr[k];
+      acc[(size_t)(m - m0) * N + n] = s;
+    }
+  }
+  free(a);
+  free(w);
+  return ORACLE_OK;
+}
+
+int oracle_gemm_s64(const uint8_t *xq, const uint8_t *Wq, int M, int N, int K, int64_t *acc) {
+  return oracle_gemm_s64_rows(xq, Wq, M, N, K, 0, M, acc);
+}
+
+/* ---- rank-one epilogue ---------------------------------------------------- */
+
+/* y32 = ((float)acc * s_a[m]) * s_w[n] (+ bias[n]); y16 = bf16 RNE of y32.
+ * acc must fit int32 (|acc| <= 64 K), otherwise ORACLE_ERR_OVERFLOW.  Any of
+ * y32 / y16 / bias may be NULL. */
+int oracle_epilogue(const int64_t *acc, const float *s_a, const float *s_w, const uint16_t *bias,
+                    int M, int N, float *y32, uint16_t *y16) {
+  for (int m = 0; m < M; ++m)
+    for (int n = 0; n < N; ++n) {
+      int64_t a = acc[(size_t)m * N + n];
+      if (a > INT32_MAX || a < INT32_MIN) return ORACLE_ERR_OVERFLOW;
+      float v = (float)a * s_a[m];
+      v = v * s_w[n];
+      if (bias) v = v + bf16_bits_to_f32(bias[n]);
+      if (y32) y32[(size_t)m * N + n] = v;
+      if (y16) y16[(size_t)m * N + n] = f32_to_bf16_bits_rne(v);
+    }
+  return ORACLE_OK;
+}
+
+/* ---- the whole Linear ----------------------------------------------------- */
+
+/* y = epilogue(gemm(rotate_quant(x), Wq)); rows [m0, m1) of y only (the rest
+ * of the prologue still runs on every row it needs: only rows m0..m1-1). */
+int oracle_linear_rows(const uint16_t *x, const uint8_t *Wq, const float *s_w, const uint16_t *bias,
+                       int M, int N, int K, int m0, int m1, float *y32, uint16_t *y16) {
+  if (M < 0 || N <= 0 || K <= 0 || K % 256 != 0 || m0 < 0 || m1 > M || m0 > m1)
+    return ORACLE_ERR_SHAPE;
+  int rows = m1 - m0;
+  uint8_t *xq = (uint8_t *)malloc((size_t)(rows > 0 ? rows : 1) * (size_t)(K / 2));
+  float *s_a = (float *)malloc(sizeof(float) * (size_t)(rows > 0 ? rows : 1));
+  int64_t *acc = (int64_t *)malloc(sizeof(int64_t) * (size_t)(rows > 0 ? rows : 1) * (size_t)N);
+  int rc = ORACLE_ERR_NOMEM;
+  if (xq && s_a && acc) {
+    rc = oracle_rotate_quant(x + (size_t)m0 * K, rows, K, xq, s_a);
+    if (rc == ORACLE_OK) rc = oracle_gemm_s64(xq, Wq, rows, N, K, acc);
+    if (rc == ORACLE_OK) rc = oracle_epilogue(acc, s_a, s_w, bias, rows, N, y32, y16);
+  }
+  free(xq);
+  free(s_a);
+  free(acc);
+  return rc;
+}
+
+int oracle_linear(const uint16_t *x, const uint8_t *Wq, const float *s_w, const uint16_t *bias,
+                  int M, int N, int K, float *y32, uint16_t *y16) {
+  return oracle_linear_rows(x, Wq, s_w, bias, M, N, K, 0, M, y32, y16);
+}
