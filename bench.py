@@ -1,0 +1,463 @@
+#!/usr/bin/env python3
+"""Benchmark of the ConvRot W4A4 quantized Linear on B200.
+
+One *step* is one pass of the whole hot path over one batch of synthetic
+input: for every linear of the workload, the fused ConvRot W4A4 Linear
+(online rotation + per-token INT4 quantization, then the tensor-core W4A4
+GEMM with the rank-one scale + bias epilogue, bf16 out).
+
+Default workload (``qwen3_4b``): the seven linears of one Qwen3-4B
+text-encoder decoder layer (q/k/v/o, gate/up/down; hidden 2560) at two prompt
+lengths, M = 76 and M = 1220 tokens -> 14 linear calls per step.  Other
+workloads: ``dit6b`` (M = 4224, hidden 3840), ``edit20b`` (M = 8704, hidden
+3072), ``small_m`` (M in 1..128), ``small``.
+
+Metric: effective TOPS = sum over the step's linears of 2*M*N*K / step time.
+
+Usage:  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+        [--workload NAME] [--no-e2e]
+Multi-GPU: launched by torchrun; every rank runs the same workload (replicas,
+weak scaling, no data-path collective); the time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import synthetic  # noqa: E402
+
+METRIC = "ConvRot W4A4 linear effective TOPS & % INT8-TC peak; HBM GB/s at M<=16"
+UNIT = "TOPS"
+WORKLOAD_DESC = {
+    "qwen3_4b": "Qwen3-4B text-encoder layer linears (q,k,v,o,gate,up,down; hidden 2560) at M=76 and M=1220",
+    "dit6b": "6B DiT block linears at 1024x1024 (qkv, out, ffn up, ffn down; hidden 3840), M=4224",
+    "edit20b": "20B image-edit DiT linears (to_q/k/v/out, mlp up/down; hidden 3072), M=8704",
+    "small_m": "small-M sweep, M in {1,8,16,64,128} x (K,N) in {(2560,9728),(9728,2560),(3072,12288),(12288,3072)}",
+    "small": "single linear M=32, K=512, N=256",
+}
+L2_FLUSH_BYTES = 256 << 20
+INT8_PER_BF16 = 2.0  # nominal dense int8 : bf16 tensor throughput (4.5 : 2.25 PFLOP/s)
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="qwen3_4b", choices=sorted(WORKLOAD_DESC))
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def step_ops(shapes):
+    return sum(2.0 * s.M * s.N * s.K for s in shapes)
+
+
+def alg_bytes(s):
+    """Algorithmic HBM bytes of one fused linear: x, packed W, s_w, bias, y."""
+    return 2 * s.M * s.K + s.N * s.K // 2 + 4 * s.N + 2 * s.N + 2 * s.M * s.N
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": float(p["hbm_gbs"]), "bf16_tflops": float(p["bf16_tflops"]),
+                "bf16_tflops_sustained": float(p.get("bf16_tflops_sustained", p["bf16_tflops"])),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled every 200 ms while running."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            import tempfile
+            fd, self.path = tempfile.mkstemp(prefix="clocks_", suffix=".csv")
+            os.close(fd)
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200",
+                 "-i", str(self.gpu)], stdout=self.fh, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.fh.close()
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    smax = float(parts[2])
+                except ValueError:
+                    continue
+                for n, v in zip(names, parts[5:9]):
+                    if v.lower().startswith("active"):
+                        reasons.add(n)
+        os.unlink(self.path)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": smax, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ the oracle leg
+
+def cpu_baseline(shapes, workload, budget_s=15.0):
+    """Time the CPU oracle (single thread, as it stands) on a bounded sample:
+    the first ``r`` rows of each linear of the step, r grown until the run
+    takes about ``budget_s``; throughput in the metric's unit (TOPS)."""
+    import oracle
+    inputs = []
+    for s in shapes:
+        x = synthetic.activations(workload, s.M, s.K)
+        w, b = synthetic.weights(workload, s.N, s.K)
+        wq, s_w = oracle.pack_weight(w)
+        inputs.append((s, x, wq, s_w, b))
+    rows = 1
+    while True:
+        t0 = time.perf_counter()
+        ops = 0.0
+        for s, x, wq, s_w, b in inputs:
+            r = min(rows, s.M)
+            oracle.linear(x[:r], wq, s_w, b, s.K)
+            ops += 2.0 * r * s.N * s.K
+        dt = time.perf_counter() - t0
+        if dt >= budget_s / 3 or rows >= max(s.M for s in shapes):
+            break
+        rows = min(max(s.M for s in shapes), rows * max(2, int(budget_s / 3 / max(dt, 1e-3))))
+    return {"value": ops / dt / 1e12, "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": f"first {rows} rows (capped at M) of each of the {len(shapes)} linears of one step "
+                      f"({ops / 1e9:.2f} GOP) in {dt:.1f} s; weight packing untimed",
+            "seconds": dt}
+
+
+# ------------------------------------------------------------------ main
+
+def main():
+    args = parse()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    shapes = synthetic.workload_shapes(args.workload)
+    config = {"workload": args.workload, "description": WORKLOAD_DESC[args.workload],
+              "linears": [f"{s.name}:M{s.M}xK{s.K}xN{s.N}" for s in shapes],
+              "l2": "flushed between timed steps (256 MiB write, outside the events)",
+              "parallelism": f"replicas x{max(world, args.gpus)}" if max(world, args.gpus) > 1 else "single GPU",
+              "codes": "s4 packed weights, s4 activations widened to s8 for tcgen05 kind::i8, int32 accumulate, "
+                       "fp32 epilogue, bf16 out"}
+
+    if args.impl == "reference":
+        return reference_arm(args, shapes, config, world, rank)
+
+    import torch
+    import torch.distributed as dist
+    import rotation_quantized_bit_b200 as rq
+
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    else:
+        torch.cuda.set_device(0)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    rq.load_library()
+
+    # ---- inputs (untimed): activations per (M, K), packed weights per linear
+    xs = {}
+    for s in shapes:
+        if (s.M, s.K) not in xs:
+            xb = synthetic.activations(args.workload, s.M, s.K)
+            xs[(s.M, s.K)] = torch.from_numpy(xb.view(np.int16)).view(torch.bfloat16).to(dev)
+    layers = []
+    for s in shapes:
+        w, b = synthetic.weights(args.workload, s.N, s.K)
+        wd = torch.from_numpy(w.view(np.int16)).view(torch.bfloat16).to(dev)
+        wq, s_w = rq.convrot_pack_weight(wd)
+        bias = torch.from_numpy(b.view(np.int16)).view(torch.bfloat16).to(dev)
+        y = torch.empty((s.M, s.N), dtype=torch.bfloat16, device=dev)
+        layers.append((s, wq, s_w, bias, y))
+        del wd
+    ws_bytes = max(rq.convrot_w4a4_workspace_size(s.M, s.N, s.K) for s in shapes)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    torch.cuda.synchronize()
+
+    nlin = len(layers)
+
+    def run_step(evs=None):
+        for i, (s, wq, s_w, bias, y) in enumerate(layers):
+            if evs is not None:
+                evs[i][0].record(stream)
+            rq.convrot_w4a4_quantize(xs[(s.M, s.K)], ws)
+            if evs is not None:
+                evs[i][1].record(stream)
+            rq.convrot_w4a4_gemm_quantized(ws, s.M, wq, s_w, bias, out=y)
+            if evs is not None:
+                evs[i][2].record(stream)
+
+    for _ in range(max(args.warmup, 3)):
+        flush.zero_()
+        run_step()
+    torch.cuda.synchronize()
+
+    counts0 = rq.convrot_dispatch_counts()
+    step_events = [[[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(nlin)]
+                   for _ in range(args.steps)]
+    sampler = ClockSampler(torch.cuda.current_device()) if rank == 0 or world == 1 else None
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    if sampler:
+        sampler.start()
+    for k in range(args.steps):
+        flush.zero_()  # L2 flush, outside the step's events
+        run_step(step_events[k])
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop() if sampler else None
+    counts1 = rq.convrot_dispatch_counts()
+    err = rq.convrot_device_error()
+    if err:
+        raise RuntimeError(f"device error word {err:#x}: a bounded wait expired")
+
+    # per-linear, per-kernel times (ms), summed over the K steps
+    t_quant = np.zeros(nlin)
+    t_gemm = np.zeros(nlin)
+    for k in range(args.steps):
+        for i in range(nlin):
+            e0, e1, e2 = step_events[k][i]
+            t_quant[i] += e0.elapsed_time(e1)
+            t_gemm[i] += e1.elapsed_time(e2)
+    total_ms = float(t_quant.sum() + t_gemm.sum())
+    if world > 1:
+        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms_per_step = total_ms / args.steps
+    ops = step_ops(shapes)
+    n_rep = world if world > 1 else 1
+    value = n_rep * ops * args.steps / (total_ms * 1e-3) / 1e12
+
+    peaks = load_peaks()
+    int8_peak = peaks["bf16_tflops"] * INT8_PER_BF16
+    detail = []
+    for i, (s, *_rest) in enumerate(layers):
+        tq, tg = t_quant[i] / args.steps, t_gemm[i] / args.steps
+        op = 2.0 * s.M * s.N * s.K
+        gemm_bytes = s.N * s.K // 2 + s.M * s.K + 4 * s.M + 6 * s.N + 2 * s.M * s.N
+        detail.append({
+            "linear": s.name, "M": s.M, "K": s.K, "N": s.N,
+            "us_total": round((tq + tg) * 1e3, 2), "us_prologue": round(tq * 1e3, 2), "us_gemm": round(tg * 1e3, 2),
+            "tops_fused": round(op / ((tq + tg) * 1e-3) / 1e12, 1),
+            "gemm_tops": round(op / (tg * 1e-3) / 1e12, 1),
+            "gemm_frac_int8_peak": round(op / (tg * 1e-3) / 1e12 / int8_peak, 3),
+            "gemm_hbm_gbs": round(gemm_bytes / (tg * 1e-3) / 1e9, 1),
+            "prologue_hbm_gbs": round((2.5 * s.M * s.K + 4 * s.M) / (tq * 1e-3) / 1e9, 1),
+        })
+    # dominant kernel = the single launch class with the largest share of the step
+    cand = []
+    for i, (s, *_r) in enumerate(layers):
+        cand.append(("gemm", i, t_gemm[i]))
+        cand.append(("prologue", i, t_quant[i]))
+    kind, idx, tsum = max(cand, key=lambda c: c[2])
+    s = layers[idx][0]
+    t_launch = tsum / args.steps * 1e-3  # seconds per launch
+    if kind == "gemm":
+        ridge = int8_peak * 1e12 / (peaks["hbm_gbs"] * 1e9)
+        gemm_bytes = s.N * s.K // 2 + s.M * s.K + 4 * s.M + 6 * s.N + 2 * s.M * s.N
+        intensity = 2.0 * s.M * s.N * s.K / gemm_bytes
+        if intensity >= ridge:
+            roof = {"bound": "tensor", "achieved": 2.0 * s.M * s.N * s.K / t_launch / 1e12,
+                    "peak": int8_peak, "unit": "TFLOP/s"}
+        else:
+            roof = {"bound": "hbm", "achieved": gemm_bytes / t_launch / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s"}
+        kname = "w4a4_tc_gemm_kernel"
+    else:
+        roof = {"bound": "hbm", "achieved": (2.5 * s.M * s.K + 4 * s.M) / t_launch / 1e9,
+                "peak": peaks["hbm_gbs"], "unit": "GB/s"}
+        kname = "rotate_quant_kernel"
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["kernel"] = kname
+    roof["launch"] = f"{s.name} M{s.M} K{s.K} N{s.N}"
+    roof["peak_source"] = (f"{peaks['source']} bf16 dense burst {peaks['bf16_tflops']} TFLOP/s x {INT8_PER_BF16} "
+                           "(nominal int8:bf16)" if roof["bound"] == "tensor" else f"{peaks['source']} HBM copy")
+    roof["share_of_step"] = tsum / total_ms if world == 1 else None
+    roof["traffic"] = committed_traffic(kname, s)
+
+    launches = (counts1["rotate_quant"] - counts0["rotate_quant"]) + (counts1["tc_gemm"] - counts0["tc_gemm"]) + \
+               (counts1["tc_gemm_splitk"] - counts0["tc_gemm_splitk"])
+
+    e2e = None
+    if not args.no_e2e:
+        e2e = end_to_end(args, rq, torch, dev, stream, shapes, xs, layers, ws, flush, world, dist)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(shapes, args.workload)
+
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": max(world, 1), "steps": args.steps,
+        "warmup": max(args.warmup, 3), "ms_per_step": round(ms_per_step, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "s8", "data": "synthetic",
+        "config": config, "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches,
+        "clocks": clocks, "detail": detail,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def committed_traffic(kernel, s):
+    """DRAM bytes per launch from the committed ncu summary (profiles/traffic.json),
+    if it was taken on this launch shape and on the current kernel source."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    try:
+        with open(path) as f:
+            rec = json.load(f)
+        ent = rec.get(kernel)
+        if not ent or ent.get("source_sha256") != source_sha(kernel):
+            return None
+        scale = 1.0
+        if ent.get("shape") != [s.M, s.K, s.N]:
+            return None
+        return ent["dram_bytes_per_launch"] * scale
+    except (OSError, ValueError, KeyError):
+        return None
+
+
+def source_sha(kernel):
+    fname = {"w4a4_tc_gemm_kernel": "gemm.cu", "rotate_quant_kernel": "rotate_quant.cu"}[kernel]
+    with open(os.path.join(ROOT, "rotation_quantized_bit_b200", "csrc", fname), "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()
+
+
+def end_to_end(args, rq, torch, dev, stream, shapes, xs, layers, ws, flush, world, dist):
+    """Same step through the public fused call, with the step's inputs copied
+    from pinned host memory and every output read back, inside the timing."""
+    host_x = {k: v.cpu().pin_memory() for k, v in xs.items()}
+    host_y = [torch.empty(y.shape, dtype=y.dtype).pin_memory() for (_, _, _, _, y) in layers]
+    h2d = sum(v.numel() * 2 for v in host_x.values())
+    d2h = sum(y.numel() * 2 for y in host_y)
+
+    def step():
+        for k, v in host_x.items():
+            xs[k].copy_(v, non_blocking=True)
+        for (s, wq, s_w, bias, y) in layers:
+            rq.convrot_w4a4_linear(xs[(s.M, s.K)], wq, s_w, bias, out=y, workspace=ws)
+        for (s, wq, s_w, bias, y), hy in zip(layers, host_y):
+            hy.copy_(y, non_blocking=True)
+
+    for _ in range(max(args.warmup, 3)):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    total = 0.0
+    for _ in range(args.steps):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        step()
+        e1.record(stream)
+        e1.synchronize()
+        total += e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([total], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total = float(t.item())
+    n_rep = world if world > 1 else 1
+    return {"value": round(n_rep * step_ops(shapes) * args.steps / (total * 1e-3) / 1e12, 2), "unit": UNIT,
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "ms_per_step": round(total / args.steps, 4),
+            "api": "convrot_w4a4_linear (C ABI) per linear, pinned host->device x, device->host y"}
+
+
+def reference_arm(args, shapes, config, world, rank):
+    """The CPU oracle as the reference arm: rank 0 only, bounded sample per step."""
+    if rank != 0:
+        return
+    import oracle
+    inputs = []
+    for s in shapes:
+        x = synthetic.activations(args.workload, s.M, s.K)
+        w, b = synthetic.weights(args.workload, s.N, s.K)
+        wq, s_w = oracle.pack_weight(w)
+        inputs.append((s, x, wq, s_w, b))
+    rows = 2  # rows per linear per step: keeps a step near a few seconds
+
+    def step():
+        ops = 0.0
+        for s, x, wq, s_w, b in inputs:
+            r = min(rows, s.M)
+            oracle.linear(x[:r], wq, s_w, b, s.K)
+            ops += 2.0 * r * s.N * s.K
+        return ops
+
+    for _ in range(max(args.warmup, 3) if args.warmup else 0):
+        step()
+    t0 = time.perf_counter()
+    ops = 0.0
+    for _ in range(args.steps):
+        ops += step()
+    dt = time.perf_counter() - t0
+    value = ops / dt / 1e12
+    sample = f"first {rows} rows of each of the {len(shapes)} linears per step ({ops / args.steps / 1e9:.2f} GOP/step)"
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": max(world, 1), "steps": args.steps,
+            "warmup": max(args.warmup, 3), "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32/int64", "data": "synthetic", "config": config,
+            "impl": "reference",
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,174 @@
+/*
+ * convrot.h -- C ABI of the B200 (sm_100a) ConvRot W4A4 quantized Linear.
+ *
+ * The method (sources by page title and section):
+ *   "Qwen-Image-Edit-2511 -- INT4 tensorwise W4A4 (+ConvRot, mixed int8
+ *   fallback)", intro paragraph: weights are packed signed INT4, two codes per
+ *   byte, after a group-256 regular-Hadamard ConvRot rotation; activations are
+ *   rotated online and quantized dynamically to INT4 inside the kernel;
+ *   calibration-free.  Same card, speed table: a fused ConvRot + rank-one s4
+ *   MMA kernel (integer product rescaled by s_a[m] * s_w[n]).
+ *   "rockerBOO/qwen3-4b-nvfp4-convrot", file table: group-wise Hadamard
+ *   rotation, group size 256.
+ *   "Nicolaslas/Rebels_w4a8s", "What I do differently": the ConvRot group is
+ *   exactly 256, so K must be divisible by 256.
+ *
+ * Definitions used by every entry point:
+ *   R        block-diagonal rotation along K: each group of 256 channels is
+ *            multiplied by H/16, H = H4 (x) H4 (x) H4 (x) H4 with
+ *            H4 = [[1,1,1,-1],[1,1,-1,1],[1,-1,1,1],[-1,1,1,1]], evaluated
+ *            in fp32 as 4 radix-4 butterfly stages (stride 1, 4, 16, 64; each
+ *            butterfly (a,b,c,d) -> (p+t, p-t, q+r, r-q) with p=a+b, q=a-b,
+ *            r=c+d, t=c-d, no FMA contraction), then one multiply by 1/16.
+ *   scale    s[r] = amax_k |R(v)[r,k]| / 7 (one fp32 IEEE division), per row.
+ *   code     q = clamp(rint(R(v)/s), -8, 7), a true IEEE fp32 division and
+ *            round half to even; s == 0 gives q == 0.
+ *   packing  byte i of a row = (q[2i] & 0xF) | ((q[2i+1] & 0xF) << 4).
+ *   linear   acc[m,n] = sum_k q_a[m,k] q_w[n,k] (exact int32), then
+ *            y[m,n] = acc * s_a[m] * s_w[n] + bias[n], rounded to bf16 (RNE).
+ *
+ * Conventions for every call:
+ *   - All pointers are DEVICE pointers, owned by the caller; the library never
+ *     allocates per call.  Pointers must be 16-byte aligned.
+ *   - Matrices are row-major and dense (row stride == number of columns).
+ *   - bf16 tensors are passed as uint16_t bit patterns.
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream); every
+ *     call only enqueues work on it and returns.  Argument errors are reported
+ *     synchronously, before anything is enqueued.  Launch failures return
+ *     CONVROT_ERR_CUDA.  A device-side wait that gave up (see
+ *     convrot_device_error) is reported asynchronously.
+ *   - Shapes: M >= 1, N >= 1 (N % 8 == 0 for the linear/GEMM outputs),
+ *     K >= 256 with K % 256 == 0, K <= 32768.
+ *   - The GPU must be sm_100 (B200); anything else gives CONVROT_ERR_DEVICE.
+ */
+#ifndef CONVROT_H_
+#define CONVROT_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  CONVROT_OK = 0,
+  CONVROT_ERR_NULL = 1,      /* a required pointer is NULL */
+  CONVROT_ERR_SHAPE = 2,     /* M < 1, N < 1, N % 8, K % 256, K > 32768 */
+  CONVROT_ERR_ALIGN = 3,     /* a pointer is not 16-byte aligned */
+  CONVROT_ERR_DEVICE = 4,    /* no CUDA device, or the current device is not sm_100 */
+  CONVROT_ERR_WORKSPACE = 5, /* workspace NULL or smaller than the *_workspace_size */
+  CONVROT_ERR_CUDA = 6,      /* a CUDA runtime/driver call failed */
+  CONVROT_ERR_TIMEOUT = 7    /* a bounded device-side wait expired (async) */
+} convrot_status_t;
+
+/* Human-readable name of a status code (static storage, never NULL). */
+const char *convrot_status_string(convrot_status_t status);
+
+/* Offline weight preparation ("weights ... with ConvRot rotation", packed
+ * signed INT4, per-output-channel scales; Qwen-Image-Edit-2511 W4A4 card,
+ * intro).  Rotates each row n of W along K, quantizes it with its own scale
+ * s_w[n] and packs it.
+ *   W    [N, K] bf16 bits      (input)
+ *   Wq   [N, K/2] uint8        (output, packed codes)
+ *   s_w  [N] float             (output)
+ * Bit-identical to convrot_rotate_quant applied to W. */
+convrot_status_t convrot_pack_weight(const uint16_t *W, int N, int K, uint8_t *Wq, float *s_w,
+                                     void *stream);
+
+/* Online activation prologue (rotation + dynamic per-token INT4, same card,
+ * intro).
+ *   x    [M, K] bf16 bits      (input)
+ *   xq   [M, K/2] uint8        (output, packed codes)
+ *   s_a  [M] float             (output, per-token scale) */
+convrot_status_t convrot_rotate_quant(const uint16_t *x, int M, int K, uint8_t *xq, float *s_a,
+                                      void *stream);
+
+/* Bytes of workspace w4a4_gemm* needs for (M, N, K). */
+size_t convrot_gemm_workspace_size(int M, int N, int K);
+
+/* Integer GEMM with the rank-one epilogue (the "rank-one s4 MMA", same card,
+ * speed table) on codes that are already quantized.
+ *   xq   [M, K/2] uint8, s_a [M] float     (from convrot_rotate_quant)
+ *   Wq   [N, K/2] uint8, s_w [N] float     (from convrot_pack_weight)
+ *   bias [N] bf16 bits, or NULL for none
+ *   y    [M, N] bf16 bits                  (output)
+ *   workspace: device memory of at least convrot_gemm_workspace_size bytes
+ *   (scratch, contents undefined afterwards).
+ * Every code nibble is accepted, including -8. */
+convrot_status_t w4a4_gemm(const uint8_t *xq, const float *s_a, const uint8_t *Wq,
+                           const float *s_w, const uint16_t *bias, int M, int N, int K,
+                           uint16_t *y, void *workspace, size_t workspace_bytes, void *stream);
+
+/* Same kernels, different sink: the exact int32 accumulator acc[M, N]
+ * (scales and bias are not applied; s_a / s_w / bias are ignored and may be
+ * NULL).  For parity checks. */
+convrot_status_t w4a4_gemm_s32(const uint8_t *xq, const uint8_t *Wq, int M, int N, int K,
+                               int32_t *acc, void *workspace, size_t workspace_bytes,
+                               void *stream);
+
+/* Same kernels, fp32 sink y32[M, N] = acc * s_a[m] * s_w[n] + bias[n] before
+ * the bf16 rounding.  For parity checks. */
+convrot_status_t w4a4_gemm_f32(const uint8_t *xq, const float *s_a, const uint8_t *Wq,
+                               const float *s_w, const uint16_t *bias, int M, int N, int K,
+                               float *y32, void *workspace, size_t workspace_bytes,
+                               void *stream);
+
+/* Bytes of workspace convrot_w4a4_linear* needs for (M, N, K). */
+size_t convrot_w4a4_workspace_size(int M, int N, int K);
+
+/* The fused ConvRot W4A4 Linear: y = W4A4(x) with x rotated and quantized
+ * online (same card, intro and speed table).
+ *   x    [M, K] bf16 bits  (input activations)
+ *   Wq   [N, K/2] uint8, s_w [N] float (from convrot_pack_weight)
+ *   bias [N] bf16 bits or NULL
+ *   y    [M, N] bf16 bits  (output)
+ *   workspace: >= convrot_w4a4_workspace_size bytes of device scratch (holds
+ *   the activation codes and scales between the two kernels). */
+convrot_status_t convrot_w4a4_linear(const uint16_t *x, const uint8_t *Wq, const float *s_w,
+                                     const uint16_t *bias, int M, int N, int K, uint16_t *y,
+                                     void *workspace, size_t workspace_bytes, void *stream);
+
+/* The fused Linear with an fp32 sink (before the bf16 rounding).  For parity
+ * checks. */
+convrot_status_t convrot_w4a4_linear_f32(const uint16_t *x, const uint8_t *Wq, const float *s_w,
+                                         const uint16_t *bias, int M, int N, int K, float *y32,
+                                         void *workspace, size_t workspace_bytes, void *stream);
+
+/* The two launches that make up convrot_w4a4_linear, for callers that want
+ * to time or schedule them separately; convrot_w4a4_linear is exactly
+ * convrot_w4a4_quantize followed by convrot_w4a4_gemm_quantized on the same
+ * workspace and stream.
+ *   convrot_w4a4_quantize: x [M, K] bf16 -> the workspace (activation codes
+ *     in the GEMM's operand layout + per-token scales).  workspace_bytes >=
+ *     convrot_w4a4_workspace_size(M, N, K) for every N it will be used with.
+ *   convrot_w4a4_gemm_quantized: workspace (from convrot_w4a4_quantize with
+ *     the same M, K) x Wq -> y [M, N] bf16. */
+convrot_status_t convrot_w4a4_quantize(const uint16_t *x, int M, int K, void *workspace,
+                                       size_t workspace_bytes, void *stream);
+convrot_status_t convrot_w4a4_gemm_quantized(const uint8_t *Wq, const float *s_w,
+                                             const uint16_t *bias, int M, int N, int K,
+                                             uint16_t *y, const void *workspace,
+                                             size_t workspace_bytes, void *stream);
+
+/* Device-side error word of the current device: bit 0 = a bounded wait
+ * inside a kernel expired (the kernel skipped its remaining work and
+ * returned; its outputs are invalid).  Synchronizes `stream`, copies the word
+ * to *code and clears it.  Returns CONVROT_ERR_TIMEOUT when the word was
+ * non-zero, CONVROT_OK otherwise. */
+convrot_status_t convrot_device_error(void *stream, uint32_t *code);
+
+/* Host-side count of how many times each kernel path was enqueued by this
+ * process: counts[0] = rotate/quant prologue, [1] = packed-code unpack pass,
+ * [2] = tensor-core GEMM without split-K, [3] = tensor-core GEMM with split-K
+ * (cluster reduction).  `n` is the array length; at most 4 are written. */
+void convrot_dispatch_counts(uint64_t *counts, int n);
+
+/* Library build identifier (static string). */
+const char *convrot_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* CONVROT_H_ */

@@ -1,0 +1,266 @@
+"""Python binding of the B200 ConvRot W4A4 quantized Linear (``libconvrot_b200.so``).
+
+Argument marshalling only: every step of the computation runs in the CUDA
+kernels behind the C ABI declared in ``include/convrot.h``.  PyTorch supplies
+device memory and streams.  There is no fallback: if the shared library is
+missing or the device is not an sm_100 GPU, the calls raise.
+
+The functions carry the C names:
+
+    convrot_pack_weight(W)                  -> (Wq, s_w)
+    convrot_rotate_quant(x)                 -> (xq, s_a)
+    w4a4_gemm(xq, s_a, Wq, s_w, bias)       -> y   (bf16)
+    w4a4_gemm_s32(xq, Wq, K)                -> acc (int32)
+    w4a4_gemm_f32(xq, s_a, Wq, s_w, bias)   -> y32 (fp32)
+    convrot_w4a4_linear(x, Wq, s_w, bias)   -> y   (bf16)
+    convrot_w4a4_linear_f32(x, Wq, s_w, bias) -> y32 (fp32)
+
+Tensors are torch CUDA tensors: bf16 as ``torch.bfloat16``, packed codes as
+``torch.uint8`` [rows, K/2], scales ``torch.float32``.  Outputs may be passed
+in (``out=``) or are allocated with torch; the workspace likewise.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libconvrot_b200.so")
+
+STATUS = {
+    0: "CONVROT_OK", 1: "CONVROT_ERR_NULL", 2: "CONVROT_ERR_SHAPE", 3: "CONVROT_ERR_ALIGN",
+    4: "CONVROT_ERR_DEVICE", 5: "CONVROT_ERR_WORKSPACE", 6: "CONVROT_ERR_CUDA", 7: "CONVROT_ERR_TIMEOUT",
+}
+
+# Every symbol include/convrot.h declares (the tests check the export list).
+EXPORTS = [
+    "convrot_status_string", "convrot_pack_weight", "convrot_rotate_quant", "convrot_gemm_workspace_size",
+    "w4a4_gemm", "w4a4_gemm_s32", "w4a4_gemm_f32", "convrot_w4a4_workspace_size", "convrot_w4a4_linear",
+    "convrot_w4a4_linear_f32", "convrot_w4a4_quantize", "convrot_w4a4_gemm_quantized", "convrot_device_error",
+    "convrot_dispatch_counts", "convrot_version",
+]
+
+
+class ConvRotError(RuntimeError):
+    def __init__(self, fn: str, code: int, msg: str):
+        super().__init__(f"{fn} failed: {msg}")
+        self.code = code
+        self.status = STATUS.get(code, str(code))
+
+
+_lib = None
+
+
+def load_library():
+    """Load libconvrot_b200.so (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"{LIB_PATH} is missing: build it with `python -m rotation_quantized_bit_b200.build` "
+            "(nvcc, sm_100a). There is no CPU or fallback path.")
+    lib = ctypes.CDLL(LIB_PATH)
+    P, I, Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+    lib.convrot_status_string.argtypes = [I]
+    lib.convrot_status_string.restype = ctypes.c_char_p
+    lib.convrot_version.restype = ctypes.c_char_p
+    lib.convrot_pack_weight.argtypes = [P, I, I, P, P, P]
+    lib.convrot_rotate_quant.argtypes = [P, I, I, P, P, P]
+    lib.convrot_gemm_workspace_size.argtypes = [I, I, I]
+    lib.convrot_gemm_workspace_size.restype = Z
+    lib.convrot_w4a4_workspace_size.argtypes = [I, I, I]
+    lib.convrot_w4a4_workspace_size.restype = Z
+    lib.w4a4_gemm.argtypes = [P, P, P, P, P, I, I, I, P, P, Z, P]
+    lib.w4a4_gemm_s32.argtypes = [P, P, I, I, I, P, P, Z, P]
+    lib.w4a4_gemm_f32.argtypes = [P, P, P, P, P, I, I, I, P, P, Z, P]
+    lib.convrot_w4a4_linear.argtypes = [P, P, P, P, I, I, I, P, P, Z, P]
+    lib.convrot_w4a4_linear_f32.argtypes = [P, P, P, P, I, I, I, P, P, Z, P]
+    lib.convrot_w4a4_quantize.argtypes = [P, I, I, P, Z, P]
+    lib.convrot_w4a4_gemm_quantized.argtypes = [P, P, P, I, I, I, P, P, Z, P]
+    lib.convrot_device_error.argtypes = [P, ctypes.POINTER(ctypes.c_uint32)]
+    lib.convrot_dispatch_counts.argtypes = [ctypes.POINTER(ctypes.c_uint64), I]
+    lib.convrot_dispatch_counts.restype = None
+    for name in lib_status_fns():
+        getattr(lib, name).restype = I
+    _lib = lib
+    return lib
+
+
+def lib_status_fns():
+    return ["convrot_pack_weight", "convrot_rotate_quant", "w4a4_gemm", "w4a4_gemm_s32", "w4a4_gemm_f32",
+            "convrot_w4a4_linear", "convrot_w4a4_linear_f32", "convrot_w4a4_quantize",
+            "convrot_w4a4_gemm_quantized", "convrot_device_error"]
+
+
+def _check(fn: str, rc: int):
+    if rc != 0:
+        raise ConvRotError(fn, rc, load_library().convrot_status_string(rc).decode())
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _need(t, name, dtype, shape=None):
+    if t is None:
+        return
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+
+
+def convrot_gemm_workspace_size(M: int, N: int, K: int) -> int:
+    return int(load_library().convrot_gemm_workspace_size(M, N, K))
+
+
+def convrot_w4a4_workspace_size(M: int, N: int, K: int) -> int:
+    return int(load_library().convrot_w4a4_workspace_size(M, N, K))
+
+
+def _workspace(ws, nbytes, device):
+    if ws is None:
+        ws = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=device)
+    _need(ws, "workspace", torch.uint8)
+    return ws
+
+
+def convrot_rotate_quant(x, xq=None, s_a=None, stream=None):
+    lib = load_library()
+    M, K = x.shape
+    _need(x, "x", torch.bfloat16)
+    xq = torch.empty((M, K // 2), dtype=torch.uint8, device=x.device) if xq is None else xq
+    s_a = torch.empty((M,), dtype=torch.float32, device=x.device) if s_a is None else s_a
+    _need(xq, "xq", torch.uint8, (M, K // 2))
+    _need(s_a, "s_a", torch.float32, (M,))
+    _check("convrot_rotate_quant", lib.convrot_rotate_quant(_ptr(x), M, K, _ptr(xq), _ptr(s_a), _stream(stream)))
+    return xq, s_a
+
+
+def convrot_pack_weight(W, Wq=None, s_w=None, stream=None):
+    lib = load_library()
+    N, K = W.shape
+    _need(W, "W", torch.bfloat16)
+    Wq = torch.empty((N, K // 2), dtype=torch.uint8, device=W.device) if Wq is None else Wq
+    s_w = torch.empty((N,), dtype=torch.float32, device=W.device) if s_w is None else s_w
+    _need(Wq, "Wq", torch.uint8, (N, K // 2))
+    _need(s_w, "s_w", torch.float32, (N,))
+    _check("convrot_pack_weight", lib.convrot_pack_weight(_ptr(W), N, K, _ptr(Wq), _ptr(s_w), _stream(stream)))
+    return Wq, s_w
+
+
+def _gemm(fn_name, out_dtype, xq, s_a, Wq, s_w, bias, out, workspace, stream):
+    lib = load_library()
+    M, K = xq.shape[0], xq.shape[1] * 2
+    N = Wq.shape[0]
+    _need(xq, "xq", torch.uint8)
+    _need(Wq, "Wq", torch.uint8, (N, K // 2))
+    _need(s_a, "s_a", torch.float32, (M,))
+    _need(s_w, "s_w", torch.float32, (N,))
+    _need(bias, "bias", torch.bfloat16, (N,))
+    out = torch.empty((M, N), dtype=out_dtype, device=xq.device) if out is None else out
+    _need(out, "out", out_dtype, (M, N))
+    ws = _workspace(workspace, convrot_gemm_workspace_size(M, N, K), xq.device)
+    fn = getattr(lib, fn_name)
+    if fn_name == "w4a4_gemm_s32":
+        rc = fn(_ptr(xq), _ptr(Wq), M, N, K, _ptr(out), _ptr(ws), ws.numel(), _stream(stream))
+    else:
+        rc = fn(_ptr(xq), _ptr(s_a), _ptr(Wq), _ptr(s_w), _ptr(bias), M, N, K, _ptr(out), _ptr(ws), ws.numel(),
+                _stream(stream))
+    _check(fn_name, rc)
+    return out
+
+
+def w4a4_gemm(xq, s_a, Wq, s_w, bias=None, out=None, workspace=None, stream=None):
+    return _gemm("w4a4_gemm", torch.bfloat16, xq, s_a, Wq, s_w, bias, out, workspace, stream)
+
+
+def w4a4_gemm_f32(xq, s_a, Wq, s_w, bias=None, out=None, workspace=None, stream=None):
+    return _gemm("w4a4_gemm_f32", torch.float32, xq, s_a, Wq, s_w, bias, out, workspace, stream)
+
+
+def w4a4_gemm_s32(xq, Wq, out=None, workspace=None, stream=None):
+    return _gemm("w4a4_gemm_s32", torch.int32, xq, None, Wq, None, None, out, workspace, stream)
+
+
+def _linear(fn_name, out_dtype, x, Wq, s_w, bias, out, workspace, stream):
+    lib = load_library()
+    M, K = x.shape
+    N = Wq.shape[0]
+    _need(x, "x", torch.bfloat16)
+    _need(Wq, "Wq", torch.uint8, (N, K // 2))
+    _need(s_w, "s_w", torch.float32, (N,))
+    _need(bias, "bias", torch.bfloat16, (N,))
+    out = torch.empty((M, N), dtype=out_dtype, device=x.device) if out is None else out
+    _need(out, "out", out_dtype, (M, N))
+    ws = _workspace(workspace, convrot_w4a4_workspace_size(M, N, K), x.device)
+    rc = getattr(lib, fn_name)(_ptr(x), _ptr(Wq), _ptr(s_w), _ptr(bias), M, N, K, _ptr(out), _ptr(ws), ws.numel(),
+                               _stream(stream))
+    _check(fn_name, rc)
+    return out
+
+
+def convrot_w4a4_linear(x, Wq, s_w, bias=None, out=None, workspace=None, stream=None):
+    return _linear("convrot_w4a4_linear", torch.bfloat16, x, Wq, s_w, bias, out, workspace, stream)
+
+
+def convrot_w4a4_linear_f32(x, Wq, s_w, bias=None, out=None, workspace=None, stream=None):
+    return _linear("convrot_w4a4_linear_f32", torch.float32, x, Wq, s_w, bias, out, workspace, stream)
+
+
+def convrot_w4a4_quantize(x, workspace, stream=None):
+    """First launch of the fused Linear: x -> activation codes + scales in ``workspace``."""
+    M, K = x.shape
+    _need(x, "x", torch.bfloat16)
+    _need(workspace, "workspace", torch.uint8)
+    _check("convrot_w4a4_quantize", load_library().convrot_w4a4_quantize(
+        _ptr(x), M, K, _ptr(workspace), workspace.numel(), _stream(stream)))
+    return workspace
+
+
+def convrot_w4a4_gemm_quantized(workspace, M, Wq, s_w, bias=None, out=None, stream=None):
+    """Second launch of the fused Linear: ``workspace`` (from convrot_w4a4_quantize) x Wq -> y."""
+    N, K = Wq.shape[0], Wq.shape[1] * 2
+    _need(Wq, "Wq", torch.uint8)
+    _need(s_w, "s_w", torch.float32, (N,))
+    _need(bias, "bias", torch.bfloat16, (N,))
+    _need(workspace, "workspace", torch.uint8)
+    out = torch.empty((M, N), dtype=torch.bfloat16, device=Wq.device) if out is None else out
+    _need(out, "out", torch.bfloat16, (M, N))
+    _check("convrot_w4a4_gemm_quantized", load_library().convrot_w4a4_gemm_quantized(
+        _ptr(Wq), _ptr(s_w), _ptr(bias), M, N, K, _ptr(out), _ptr(workspace), workspace.numel(), _stream(stream)))
+    return out
+
+
+def convrot_device_error(stream=None) -> int:
+    """Synchronize, read and clear the device error word; raise on a timeout."""
+    lib = load_library()
+    code = ctypes.c_uint32(0)
+    rc = lib.convrot_device_error(_stream(stream), ctypes.byref(code))
+    if rc not in (0, 7):
+        _check("convrot_device_error", rc)
+    return int(code.value)
+
+
+def convrot_dispatch_counts():
+    lib = load_library()
+    arr = (ctypes.c_uint64 * 4)()
+    lib.convrot_dispatch_counts(arr, 4)
+    return {"rotate_quant": arr[0], "unpack_codes": arr[1], "tc_gemm": arr[2], "tc_gemm_splitk": arr[3]}
+
+
+def convrot_version() -> str:
+    return load_library().convrot_version().decode()

@@ -1,0 +1,255 @@
+// api.cu -- the extern "C" boundary of libconvrot_b200.so (declared in
+// include/convrot.h).  Validates arguments on the host, carves the caller's
+// workspace and enqueues the kernels on the caller's stream.  No allocation,
+// no host synchronisation (except convrot_device_error, which is a query).
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cstdint>
+#include <cstring>
+
+#include "../../include/convrot.h"
+#include "kernels.cuh"
+#include "ptx.cuh"
+
+namespace convrot {
+
+__device__ uint32_t g_device_error = 0;
+
+namespace {
+
+std::atomic<uint64_t> g_counts[4];
+
+constexpr int kMaxK = 32768;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Cached per device: is it sm_100?  and its SM count.
+struct DeviceInfo {
+  int ok = -1;  // -1 unknown, 0 no, 1 yes
+  int sms = 0;
+};
+DeviceInfo g_dev[64];
+
+convrot_status_t check_device(int* sms_out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return CONVROT_ERR_DEVICE;
+  if (dev >= 64) return CONVROT_ERR_DEVICE;
+  DeviceInfo& d = g_dev[dev];
+  if (d.ok < 0) {
+    int major = 0, minor = 0, sms = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return CONVROT_ERR_DEVICE;
+    d.ok = (major == 10 && minor == 0) ? 1 : 0;
+    d.sms = sms;
+  }
+  if (d.ok != 1) return CONVROT_ERR_DEVICE;
+  if (sms_out) *sms_out = d.sms;
+  return CONVROT_OK;
+}
+
+convrot_status_t check_mk(int M, int K) {
+  if (M < 1 || K < 256 || K % 256 != 0 || K > kMaxK) return CONVROT_ERR_SHAPE;
+  return CONVROT_OK;
+}
+
+convrot_status_t check_mnk(int M, int N, int K) {
+  if (check_mk(M, K) != CONVROT_OK || N < 1 || N % 8 != 0) return CONVROT_ERR_SHAPE;
+  return CONVROT_OK;
+}
+
+convrot_status_t from_cuda(cudaError_t e) { return e == cudaSuccess ? CONVROT_OK : CONVROT_ERR_CUDA; }
+
+size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+// Workspace layout shared by the GEMM and the fused Linear:
+//   [0, M*K)            activation codes as signed bytes (operand layout)
+//   [M*K, M*K + 4M)     per-token scales (fused Linear only)
+size_t codes_bytes(int M, int K) { return round_up(static_cast<size_t>(M) * static_cast<size_t>(K), 256); }
+
+convrot_status_t gemm_common(const uint8_t* xq, const float* s_a, const uint8_t* Wq, const float* s_w,
+                             const uint16_t* bias, int M, int N, int K, void* out, GemmSink sink, void* ws,
+                             size_t ws_bytes, void* stream) {
+  if (!xq || !Wq || !out) return CONVROT_ERR_NULL;
+  if (sink != GemmSink::kS32 && (!s_a || !s_w)) return CONVROT_ERR_NULL;
+  convrot_status_t st = check_mnk(M, N, K);
+  if (st != CONVROT_OK) return st;
+  if (!aligned16(xq) || !aligned16(Wq) || !aligned16(out) || (s_a && !aligned16(s_a)) ||
+      (s_w && !aligned16(s_w)) || (bias && !aligned16(bias)))
+    return CONVROT_ERR_ALIGN;
+  if (!ws || ws_bytes < convrot_gemm_workspace_size(M, N, K)) return CONVROT_ERR_WORKSPACE;
+  if (!aligned16(ws)) return CONVROT_ERR_ALIGN;
+  int sms = 0;
+  st = check_device(&sms);
+  if (st != CONVROT_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int8_t* xs8 = static_cast<int8_t*>(ws);
+  if (cudaError_t e = launch_unpack_codes(xq, M, K, xs8, s); e != cudaSuccess) return CONVROT_ERR_CUDA;
+  GemmArgs a{xs8, s_a, Wq, s_w, bias, out, M, N, K};
+  return from_cuda(launch_w4a4_gemm(a, sink, choose_tiling(M, N, K, sms), s));
+}
+
+convrot_status_t quantize_common(const uint16_t* x, int M, int K, void* ws, size_t ws_bytes, void* stream) {
+  if (!x) return CONVROT_ERR_NULL;
+  convrot_status_t st = check_mk(M, K);
+  if (st != CONVROT_OK) return st;
+  if (!aligned16(x)) return CONVROT_ERR_ALIGN;
+  if (!ws || ws_bytes < convrot_w4a4_workspace_size(M, 8, K)) return CONVROT_ERR_WORKSPACE;
+  if (!aligned16(ws)) return CONVROT_ERR_ALIGN;
+  st = check_device(nullptr);
+  if (st != CONVROT_OK) return st;
+  int8_t* xs8 = static_cast<int8_t*>(ws);
+  float* s_a = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + codes_bytes(M, K));
+  RotateQuantOut o{nullptr, xs8, s_a};
+  return from_cuda(launch_rotate_quant(x, M, K, o, static_cast<cudaStream_t>(stream)));
+}
+
+convrot_status_t gemm_quantized_common(const uint8_t* Wq, const float* s_w, const uint16_t* bias, int M, int N,
+                                       int K, void* out, GemmSink sink, const void* ws, size_t ws_bytes,
+                                       void* stream) {
+  if (!Wq || !s_w || !out) return CONVROT_ERR_NULL;
+  convrot_status_t st = check_mnk(M, N, K);
+  if (st != CONVROT_OK) return st;
+  if (!aligned16(Wq) || !aligned16(s_w) || !aligned16(out) || (bias && !aligned16(bias))) return CONVROT_ERR_ALIGN;
+  if (!ws || ws_bytes < convrot_w4a4_workspace_size(M, N, K)) return CONVROT_ERR_WORKSPACE;
+  if (!aligned16(ws)) return CONVROT_ERR_ALIGN;
+  int sms = 0;
+  st = check_device(&sms);
+  if (st != CONVROT_OK) return st;
+  const int8_t* xs8 = static_cast<const int8_t*>(ws);
+  const float* s_a = reinterpret_cast<const float*>(static_cast<const uint8_t*>(ws) + codes_bytes(M, K));
+  GemmArgs a{xs8, s_a, Wq, s_w, bias, out, M, N, K};
+  return from_cuda(launch_w4a4_gemm(a, sink, choose_tiling(M, N, K, sms), static_cast<cudaStream_t>(stream)));
+}
+
+convrot_status_t linear_common(const uint16_t* x, const uint8_t* Wq, const float* s_w, const uint16_t* bias, int M,
+                               int N, int K, void* out, GemmSink sink, void* ws, size_t ws_bytes, void* stream) {
+  if (!x || !Wq || !s_w || !out) return CONVROT_ERR_NULL;
+  convrot_status_t st = check_mnk(M, N, K);
+  if (st != CONVROT_OK) return st;
+  if (!aligned16(x) || !aligned16(Wq) || !aligned16(s_w) || !aligned16(out) || (bias && !aligned16(bias)))
+    return CONVROT_ERR_ALIGN;
+  if (!ws || ws_bytes < convrot_w4a4_workspace_size(M, N, K)) return CONVROT_ERR_WORKSPACE;
+  if (!aligned16(ws)) return CONVROT_ERR_ALIGN;
+  st = quantize_common(x, M, K, ws, ws_bytes, stream);
+  if (st != CONVROT_OK) return st;
+  return gemm_quantized_common(Wq, s_w, bias, M, N, K, out, sink, ws, ws_bytes, stream);
+}
+
+}  // namespace
+
+void count_dispatch(int which) {
+  if (which >= 0 && which < 4) g_counts[which].fetch_add(1, std::memory_order_relaxed);
+}
+
+}  // namespace convrot
+
+using namespace convrot;
+
+extern "C" {
+
+const char* convrot_status_string(convrot_status_t status) {
+  switch (status) {
+    case CONVROT_OK: return "CONVROT_OK";
+    case CONVROT_ERR_NULL: return "CONVROT_ERR_NULL: a required pointer is NULL";
+    case CONVROT_ERR_SHAPE: return "CONVROT_ERR_SHAPE: need M>=1, N>=1, N%8==0, K%256==0, 256<=K<=32768";
+    case CONVROT_ERR_ALIGN: return "CONVROT_ERR_ALIGN: pointers must be 16-byte aligned";
+    case CONVROT_ERR_DEVICE: return "CONVROT_ERR_DEVICE: needs an sm_100 (B200) device";
+    case CONVROT_ERR_WORKSPACE: return "CONVROT_ERR_WORKSPACE: workspace missing or too small";
+    case CONVROT_ERR_CUDA: return "CONVROT_ERR_CUDA: a CUDA call failed";
+    case CONVROT_ERR_TIMEOUT: return "CONVROT_ERR_TIMEOUT: a bounded device-side wait expired";
+  }
+  return "CONVROT_ERR_UNKNOWN";
+}
+
+const char* convrot_version(void) { return "convrot-b200 sm_100a"; }
+
+convrot_status_t convrot_rotate_quant(const uint16_t* x, int M, int K, uint8_t* xq, float* s_a, void* stream) {
+  if (!x || !xq || !s_a) return CONVROT_ERR_NULL;
+  convrot_status_t st = check_mk(M, K);
+  if (st != CONVROT_OK) return st;
+  if (!aligned16(x) || !aligned16(xq) || !aligned16(s_a)) return CONVROT_ERR_ALIGN;
+  st = check_device(nullptr);
+  if (st != CONVROT_OK) return st;
+  RotateQuantOut o{xq, nullptr, s_a};
+  return from_cuda(launch_rotate_quant(x, M, K, o, static_cast<cudaStream_t>(stream)));
+}
+
+convrot_status_t convrot_pack_weight(const uint16_t* W, int N, int K, uint8_t* Wq, float* s_w, void* stream) {
+  return convrot_rotate_quant(W, N, K, Wq, s_w, stream);
+}
+
+size_t convrot_gemm_workspace_size(int M, int N, int K) {
+  (void)N;
+  if (check_mk(M, K) != CONVROT_OK) return 0;
+  return codes_bytes(M, K);
+}
+
+size_t convrot_w4a4_workspace_size(int M, int N, int K) {
+  (void)N;
+  if (check_mk(M, K) != CONVROT_OK) return 0;
+  return codes_bytes(M, K) + round_up(static_cast<size_t>(M) * sizeof(float), 256);
+}
+
+convrot_status_t w4a4_gemm(const uint8_t* xq, const float* s_a, const uint8_t* Wq, const float* s_w,
+                           const uint16_t* bias, int M, int N, int K, uint16_t* y, void* workspace,
+                           size_t workspace_bytes, void* stream) {
+  return gemm_common(xq, s_a, Wq, s_w, bias, M, N, K, y, GemmSink::kBF16, workspace, workspace_bytes, stream);
+}
+
+convrot_status_t w4a4_gemm_s32(const uint8_t* xq, const uint8_t* Wq, int M, int N, int K, int32_t* acc,
+                               void* workspace, size_t workspace_bytes, void* stream) {
+  return gemm_common(xq, nullptr, Wq, nullptr, nullptr, M, N, K, acc, GemmSink::kS32, workspace, workspace_bytes,
+                     stream);
+}
+
+convrot_status_t w4a4_gemm_f32(const uint8_t* xq, const float* s_a, const uint8_t* Wq, const float* s_w,
+                               const uint16_t* bias, int M, int N, int K, float* y32, void* workspace,
+                               size_t workspace_bytes, void* stream) {
+  return gemm_common(xq, s_a, Wq, s_w, bias, M, N, K, y32, GemmSink::kF32, workspace, workspace_bytes, stream);
+}
+
+convrot_status_t convrot_w4a4_linear(const uint16_t* x, const uint8_t* Wq, const float* s_w, const uint16_t* bias,
+                                     int M, int N, int K, uint16_t* y, void* workspace, size_t workspace_bytes,
+                                     void* stream) {
+  return linear_common(x, Wq, s_w, bias, M, N, K, y, GemmSink::kBF16, workspace, workspace_bytes, stream);
+}
+
+convrot_status_t convrot_w4a4_linear_f32(const uint16_t* x, const uint8_t* Wq, const float* s_w,
+                                         const uint16_t* bias, int M, int N, int K, float* y32, void* workspace,
+                                         size_t workspace_bytes, void* stream) {
+  return linear_common(x, Wq, s_w, bias, M, N, K, y32, GemmSink::kF32, workspace, workspace_bytes, stream);
+}
+
+convrot_status_t convrot_w4a4_quantize(const uint16_t* x, int M, int K, void* workspace, size_t workspace_bytes,
+                                       void* stream) {
+  return quantize_common(x, M, K, workspace, workspace_bytes, stream);
+}
+
+convrot_status_t convrot_w4a4_gemm_quantized(const uint8_t* Wq, const float* s_w, const uint16_t* bias, int M, int N,
+                                             int K, uint16_t* y, const void* workspace, size_t workspace_bytes,
+                                             void* stream) {
+  return gemm_quantized_common(Wq, s_w, bias, M, N, K, y, GemmSink::kBF16, workspace, workspace_bytes, stream);
+}
+
+convrot_status_t convrot_device_error(void* stream, uint32_t* code) {
+  if (!code) return CONVROT_ERR_NULL;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) return CONVROT_ERR_CUDA;
+  uint32_t v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_device_error, sizeof(v)) != cudaSuccess) return CONVROT_ERR_CUDA;
+  const uint32_t zero = 0;
+  if (cudaMemcpyToSymbol(g_device_error, &zero, sizeof(zero)) != cudaSuccess) return CONVROT_ERR_CUDA;
+  *code = v;
+  return v ? CONVROT_ERR_TIMEOUT : CONVROT_OK;
+}
+
+void convrot_dispatch_counts(uint64_t* counts, int n) {
+  if (!counts) return;
+  for (int i = 0; i < n && i < 4; ++i) counts[i] = g_counts[i].load(std::memory_order_relaxed);
+}
+
+}  // extern "C"

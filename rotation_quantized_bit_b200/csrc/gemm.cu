@@ -1,0 +1,415 @@
+// gemm.cu -- W4A4 integer GEMM with the rank-one epilogue on sm_100a
+// tensor cores (tcgen05.mma kind::i8, accumulators in tensor memory).
+//
+// What it computes ("Qwen-Image-Edit-2511 -- INT4 tensorwise W4A4
+// (+ConvRot...)", speed table: a rank-one s4 MMA kernel):
+//   acc[m, n] = sum_k q_a[m, k] * q_w[n, k]            (exact int32)
+//   y[m, n]   = acc * s_a[m] * s_w[n] + bias[n]        (fp32, then bf16 RNE)
+//
+// Mapping to the B200 tensor core.  sm_100a has no 4-bit integer MMA kind,
+// so the 4-bit codes are widened to bytes for kind::i8.  The weight tile
+// is the MMA "A" operand and lives in tensor memory (swap-AB: MMA M = 128
+// output channels, MMA N = BT tokens):
+//   * a TMA producer warp streams packed weight tiles (128 rows x 64 bytes =
+//     128 K values) and activation byte tiles (BT rows x 128 bytes, 128-byte
+//     swizzle) into a ring of shared-memory stages;
+//   * four unpack warps turn each packed weight row into 32 tensor-memory
+//     columns with three integer ops per 8 codes: the low nibbles of a
+//     32-bit word are codes (0,2,4,6), the high nibbles (1,3,5,7); moving a
+//     two's-complement nibble into the high half of a byte gives the signed
+//     byte 16 * q_w, so (w << 4) & 0xF0F0F0F0 and w & 0xF0F0F0F0 are the
+//     two halves, already sign-correct;
+//   * one thread issues tcgen05.mma kind::i8 (A = s8 weights from tensor
+//     memory, B = s8 activations from shared memory, K = 32 per
+//     instruction).  The activation bytes are stored in the matching per-8
+//     chunk order, so the contraction pairs the right codes;
+//   * the accumulator is exactly 16 * acc (|16 acc| <= 1024 K < 2^31), and
+//     the epilogue shifts it right by 4.
+// Split-K (for small M) runs the K-slices of one output tile as a thread
+// block cluster and adds the int32 partial tiles through distributed shared
+// memory; the sum is exact and independent of order.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "kernels.cuh"
+#include "ptx.cuh"
+
+namespace convrot {
+
+namespace {
+
+constexpr int kThreads = 192;    // warp 0 TMA, warp 1 MMA, warps 2..5 unpack + epilogue
+constexpr int kRows = 128;       // output channels per tile (MMA M)
+constexpr int kKB = 128;         // K values per pipeline step
+constexpr int kWTileBytes = kRows * kKB / 2;  // 8 KB packed weights per step
+constexpr int kASlots = 2;       // tensor-memory A buffers (32 columns each)
+
+struct Params {
+  const float* s_a;
+  const float* s_w;
+  const uint16_t* bias;
+  void* out;
+  int M, N, K;
+  int BT, splits, kb_total, kb_per_split, nstages, tmem_cols;
+};
+
+struct SharedHeader {
+  uint64_t full[16];
+  uint64_t empty[16];
+  uint64_t a_full[kASlots];
+  uint64_t a_empty[kASlots];
+  uint64_t acc_full;
+  uint32_t tmem_base;
+};
+
+__device__ __forceinline__ void unpack_row_to_tmem(const uint8_t* wstage, int row, uint32_t taddr) {
+  // The weight tile landed with the 64-byte TMA swizzle: 16-byte chunk c of
+  // row r sits at chunk c ^ ((r >> 1) & 3).
+  uint32_t cols[32];
+  const int sw = (row >> 1) & 3;
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    const uint4 v = *reinterpret_cast<const uint4*>(wstage + row * 64 + ((c ^ sw) << 4));
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      cols[8 * c + 2 * j] = (w[j] << 4) & 0xF0F0F0F0u;
+      cols[8 * c + 2 * j + 1] = w[j] & 0xF0F0F0F0u;
+    }
+  }
+  tmem_st_32x32b_x32(taddr, cols);
+}
+
+template <int SINK>
+__device__ __forceinline__ void store_output(const Params& p, int m, int n, int32_t dsum) {
+  const int32_t acc = dsum >> 4;  // the weights entered the MMA as 16 * q_w
+  const size_t idx = static_cast<size_t>(m) * p.N + n;
+  if (SINK == static_cast<int>(GemmSink::kS32)) {
+    static_cast<int32_t*>(p.out)[idx] = acc;
+    return;
+  }
+  float y = __fmul_rn(__fmul_rn(__int2float_rn(acc), __ldg(p.s_a + m)), __ldg(p.s_w + n));
+  if (p.bias) y = __fadd_rn(y, __uint_as_float(static_cast<uint32_t>(__ldg(p.bias + n)) << 16));
+  if (SINK == static_cast<int>(GemmSink::kF32)) {
+    static_cast<float*>(p.out)[idx] = y;
+  } else {
+    static_cast<uint16_t*>(p.out)[idx] = __bfloat16_as_ushort(__float2bfloat16_rn(y));
+  }
+}
+
+template <int SINK>
+__global__ void __launch_bounds__(kThreads, 1)
+    w4a4_tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_x,
+                        const __grid_constant__ Params p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  // 1024-byte alignment for the swizzled stage tiles.
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int BT = p.BT;
+  const int stage_bytes = kWTileBytes + BT * kKB;
+  SharedHeader* hdr = reinterpret_cast<SharedHeader*>(smem + p.nstages * stage_bytes);
+  int32_t* red = reinterpret_cast<int32_t*>(reinterpret_cast<uint8_t*>(hdr) + 1024);  // split-K partials
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n0 = blockIdx.x * kRows;
+  const int m0 = blockIdx.y * BT;
+  // K blocks of this split: an even share [j*KB/S, (j+1)*KB/S), never empty
+  // because S <= KB.
+  const int split = blockIdx.z;
+  const int kb0 = (split * p.kb_total) / p.splits;
+  const int nkb = ((split + 1) * p.kb_total) / p.splits - kb0;
+  const int ns = p.nstages;
+  const uint32_t a_col0 = static_cast<uint32_t>(p.tmem_cols - 32 * kASlots);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < ns; ++s) {
+      mbar_init(&hdr->full[s], 1);
+      mbar_init(&hdr->empty[s], 1 + 4);  // MMA commit + one arrive per unpack warp
+    }
+    for (int a = 0; a < kASlots; ++a) {
+      mbar_init(&hdr->a_full[a], 4);
+      mbar_init(&hdr->a_empty[a], 1);
+    }
+    mbar_init(&hdr->acc_full, 1);
+    fence_mbarrier_init();
+    prefetch_tmap(&tm_w);
+    prefetch_tmap(&tm_x);
+  }
+  if (warp == 1) {
+    tmem_alloc(&hdr->tmem_base, static_cast<uint32_t>(p.tmem_cols));
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = hdr->tmem_base;
+
+  if (warp == 0) {
+    // ------------------------------------------------ TMA producer
+    if (lane == 0) {
+      const uint32_t bytes = static_cast<uint32_t>(stage_bytes);
+      int issued = 0;
+      for (int i = 0; i < nkb; ++i) {
+        const int s = i % ns;
+        if (i >= ns && !mbar_wait(&hdr->empty[s], ((i / ns) - 1) & 1)) break;
+        uint8_t* st = smem + s * stage_bytes;
+        mbar_arrive_expect_tx(&hdr->full[s], bytes);
+        tma_load_2d(st, &tm_w, &hdr->full[s], (kb0 + i) * (kKB / 2), n0);
+        tma_load_2d(st + kWTileBytes, &tm_x, &hdr->full[s], (kb0 + i) * kKB, m0);
+        ++issued;
+      }
+      // Drain: every issued load has landed before the block may exit.
+      for (int i = (issued > ns ? issued - ns : 0); i < issued; ++i)
+        mbar_wait(&hdr->full[i % ns], (i / ns) & 1);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc = umma_idesc_i8(kRows, BT, /*a_signed=*/true, /*b_signed=*/true);
+      bool ok = true;
+      for (int i = 0; i < nkb && ok; ++i) {
+        const int s = i % ns, a = i % kASlots;
+        ok = mbar_wait(&hdr->full[s], (i / ns) & 1) && mbar_wait(&hdr->a_full[a], (i / kASlots) & 1);
+        if (!ok) break;
+        tc_fence_after();
+        const uint64_t bdesc = umma_desc_k_sw128(smem_u32(smem + s * stage_bytes + kWTileBytes));
+#pragma unroll
+        for (int kk = 0; kk < kKB / 32; ++kk) {
+          umma_i8_ts(tmem, tmem + a_col0 + 32 * a + 8 * kk, bdesc + 2 * kk, idesc, (i > 0 || kk > 0) ? 1u : 0u);
+        }
+        umma_commit(&hdr->empty[s]);
+        umma_commit(&hdr->a_empty[a]);
+      }
+      umma_commit(&hdr->acc_full);
+      mbar_wait(&hdr->acc_full, 0);  // all MMAs retired before teardown
+    }
+  } else {
+    // ------------------------------------------------ unpack, then epilogue
+    const int quad = warp & 3;  // tensor-memory lane quadrant of this warp
+    const int row = quad * 32 + lane;
+    const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
+    bool ok = true;
+    for (int i = 0; i < nkb; ++i) {
+      const int s = i % ns, a = i % kASlots;
+      ok = mbar_wait(&hdr->full[s], (i / ns) & 1);
+      if (ok && i >= kASlots) ok = mbar_wait(&hdr->a_empty[a], ((i / kASlots) - 1) & 1);
+      ok = __all_sync(0xffffffffu, ok);  // tcgen05.st below is warp-collective
+      if (!ok) break;
+      unpack_row_to_tmem(smem + s * stage_bytes, row, tmem + lane_base + a_col0 + 32 * a);
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&hdr->empty[s]);
+        mbar_arrive(&hdr->a_full[a]);
+      }
+    }
+    if (ok) ok = mbar_wait(&hdr->acc_full, 0);
+    ok = __all_sync(0xffffffffu, ok);  // tcgen05.ld below is warp-collective
+    tc_fence_after();
+
+    const int n = n0 + row;
+    if (p.splits == 1) {
+      if (ok && nkb > 0) {
+        for (int c = 0; c < BT; c += 16) {
+          uint32_t v[16];
+          tmem_ld_32x32b_x16(tmem + lane_base + static_cast<uint32_t>(c), v);
+          tmem_wait_ld();
+          if (n < p.N) {
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+              const int m = m0 + c + j;
+              if (m < p.M) store_output<SINK>(p, m, n, static_cast<int32_t>(v[j]));
+            }
+          }
+        }
+      }
+    } else {
+      // Partial tile -> own shared memory, column-major [BT][128].
+      for (int c = 0; c < BT; c += 16) {
+        uint32_t v[16];
+        tmem_ld_32x32b_x16(tmem + lane_base + static_cast<uint32_t>(c), v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int j = 0; j < 16; ++j) red[(c + j) * kRows + row] = (ok && nkb > 0) ? static_cast<int32_t>(v[j]) : 0;
+      }
+    }
+  }
+
+  if (p.splits > 1) {
+    __syncwarp();    // the cluster barrier below is .aligned: reconverge first
+    cluster_sync();  // every CTA of the cluster has its partial tile in shared memory
+    if (warp >= 2) {
+      const int quad = warp & 3;
+      const int row = quad * 32 + lane;
+      const int n = n0 + row;
+      const uint32_t rank = cluster_ctarank();
+      for (int c = static_cast<int>(rank); c < BT; c += p.splits) {
+        const int m = m0 + c;
+        if (m >= p.M || n >= p.N) continue;
+        const uint32_t local = smem_u32(red + c * kRows + row);
+        int32_t sum = 0;
+        for (int j = 0; j < p.splits; ++j) sum += ld_shared_cluster_s32(map_shared_rank(local, static_cast<uint32_t>(j)));
+        store_output<SINK>(p, m, n, sum);
+      }
+    }
+    __syncwarp();
+    cluster_sync();  // nobody leaves while a peer still reads its shared memory
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, static_cast<uint32_t>(p.tmem_cols));
+  }
+}
+
+// ---------------------------------------------------------------- host side
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  }
+  return fn;
+}
+
+// 2-D uint8 tensor [rows, cols] (row stride = cols bytes), box [box_rows, box_cols].
+bool make_map_u8(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows,
+                 uint32_t box_cols, CUtensorMapSwizzle swz) {
+  EncodeTiledFn fn = get_encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols};
+  cuuint32_t box[2] = {box_cols, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+int shared_bytes_for(int BT, int nstages, int splits) {
+  int bytes = 1024 /*alignment slack*/ + nstages * (kWTileBytes + BT * kKB) + 1024 /*header*/;
+  if (splits > 1) bytes += BT * kRows * 4;
+  return bytes;
+}
+
+template <int SINK>
+cudaError_t launch_sink(const CUtensorMap& tw, const CUtensorMap& tx, const Params& prm, const GemmTiling& t,
+                        cudaStream_t stream) {
+  static int attr_done_dev = -1;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (attr_done_dev != dev) {
+    cudaError_t e = cudaFuncSetAttribute(w4a4_tc_gemm_kernel<SINK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         227 * 1024);
+    if (e != cudaSuccess) return e;
+    attr_done_dev = dev;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(t.n_tiles, t.m_tiles, t.splits);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = static_cast<size_t>(t.smem_bytes);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  int nattr = 0;
+  if (t.splits > 1) {
+    attr[nattr].id = cudaLaunchAttributeClusterDimension;
+    attr[nattr].val.clusterDim.x = 1;
+    attr[nattr].val.clusterDim.y = 1;
+    attr[nattr].val.clusterDim.z = static_cast<unsigned>(t.splits);
+    ++nattr;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = nattr;
+  return cudaLaunchKernelEx(&cfg, w4a4_tc_gemm_kernel<SINK>, tw, tx, prm);
+}
+
+}  // namespace
+
+GemmTiling choose_tiling(int M, int N, int K, int num_sms) {
+  GemmTiling t{};
+  const int kb_total = K / kKB;
+  // Tokens per tile: one tile when M fits, else the fewest tiles of <= 192.
+  const int max_bt = 192;
+  int m_tiles = (M + max_bt - 1) / max_bt;
+  int bt = (M + m_tiles - 1) / m_tiles;
+  bt = ((bt + 15) / 16) * 16;
+  if (bt < 16) bt = 16;
+  t.BT = bt;
+  t.m_tiles = (M + bt - 1) / bt;
+  t.n_tiles = (N + kRows - 1) / kRows;
+  // Split K across a cluster until the grid covers two CTAs per SM.
+  const int tiles = t.m_tiles * t.n_tiles;
+  int splits = 1;
+  while (splits < 8 && tiles * splits * 2 <= 2 * num_sms && splits * 2 <= kb_total) splits *= 2;
+  const int kbps = (kb_total + splits - 1) / splits;  // the largest share
+  t.splits = splits;
+  t.kb_per_split = kbps;
+  // Pipeline depth: as many stages as fit two CTAs per SM (~110 KB each).
+  const int stage = kWTileBytes + bt * kKB;
+  int ns = (110 * 1024 - 2048 - (splits > 1 ? bt * kRows * 4 : 0)) / stage;
+  if (ns > 8) ns = 8;
+  if (ns > kbps) ns = kbps < 2 ? 2 : kbps;
+  if (ns < 2) ns = 2;
+  t.nstages = ns;
+  int cols = 32;
+  while (cols < bt + 32 * kASlots) cols *= 2;
+  t.tmem_cols = cols;
+  t.smem_bytes = shared_bytes_for(bt, ns, splits);
+  // Never let more CTAs share an SM than its 512 tensor-memory columns can
+  // hold: a CTA blocked in tcgen05.alloc while its cluster peers wait for it
+  // could deadlock.  Shared memory per CTA is padded so that at most
+  // 512 / cols CTAs fit in the SM's 228 KB.
+  const int max_ctas = 512 / cols;
+  const int min_smem = (228 * 1024) / (max_ctas + 1) + 1;
+  if (t.smem_bytes < min_smem) t.smem_bytes = min_smem;
+  return t;
+}
+
+cudaError_t launch_w4a4_gemm(const GemmArgs& a, GemmSink sink, const GemmTiling& t, cudaStream_t stream) {
+  CUtensorMap tw, tx;
+  if (!make_map_u8(&tw, a.Wq, static_cast<uint64_t>(a.N), static_cast<uint64_t>(a.K / 2), kRows, kKB / 2,
+                   CU_TENSOR_MAP_SWIZZLE_64B))
+    return cudaErrorInvalidValue;
+  if (!make_map_u8(&tx, a.xs8, static_cast<uint64_t>(a.M), static_cast<uint64_t>(a.K), static_cast<uint32_t>(t.BT),
+                   kKB, CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorInvalidValue;
+  Params prm{};
+  prm.s_a = a.s_a;
+  prm.s_w = a.s_w;
+  prm.bias = a.bias;
+  prm.out = a.out;
+  prm.M = a.M;
+  prm.N = a.N;
+  prm.K = a.K;
+  prm.BT = t.BT;
+  prm.splits = t.splits;
+  prm.kb_total = a.K / kKB;
+  prm.kb_per_split = t.kb_per_split;
+  prm.nstages = t.nstages;
+  prm.tmem_cols = t.tmem_cols;
+  cudaError_t e;
+  switch (sink) {
+    case GemmSink::kBF16: e = launch_sink<0>(tw, tx, prm, t, stream); break;
+    case GemmSink::kF32: e = launch_sink<1>(tw, tx, prm, t, stream); break;
+    default: e = launch_sink<2>(tw, tx, prm, t, stream); break;
+  }
+  count_dispatch(t.splits > 1 ? 3 : 2);
+  return e;
+}
+
+}  // namespace convrot

@@ -1,0 +1,59 @@
+// kernels.cuh -- internal launch interface between the C ABI (api.cu) and the
+// CUDA kernels (rotate_quant.cu, gemm.cu).  Not installed, not part of the ABI.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cstdint>
+
+namespace convrot {
+
+// Rows are processed by the prologue in 8-element chunks; the activation
+// operand of the tensor-core GEMM stores each chunk's codes in the order
+// (0, 2, 4, 6, 1, 3, 5, 7), the order in which a packed 32-bit word of weight
+// nibbles splits into its low and high nibbles.
+
+// Output sinks of the rotate/quant prologue (packed or s8 may be null).
+struct RotateQuantOut {
+  uint8_t* packed;  // [M, K/2] two codes per byte, or null
+  int8_t* s8;       // [M, K] codes as signed bytes in chunk order (0,2,4,6,1,3,5,7), or null
+  float* scale;     // [M]
+};
+
+cudaError_t launch_rotate_quant(const uint16_t* x, int M, int K, RotateQuantOut out, cudaStream_t stream);
+
+// Packed codes [M, K/2] -> signed-byte operand layout [M, K].
+cudaError_t launch_unpack_codes(const uint8_t* packed, int M, int K, int8_t* s8, cudaStream_t stream);
+
+enum class GemmSink : int { kBF16 = 0, kF32 = 1, kS32 = 2 };
+
+struct GemmTiling {
+  int BT;           // tokens per CTA tile (MMA N), multiple of 16 in [16, 192]
+  int m_tiles;      // ceil(M / BT)
+  int n_tiles;      // ceil(N / 128)
+  int splits;       // split-K factor = cluster size (1 .. 8)
+  int kb_per_split; // 128-wide K blocks per split
+  int nstages;      // depth of the shared-memory TMA ring
+  int tmem_cols;    // tensor-memory columns allocated per CTA (power of two)
+  int smem_bytes;   // dynamic shared memory per CTA
+};
+
+GemmTiling choose_tiling(int M, int N, int K, int num_sms);
+
+struct GemmArgs {
+  const int8_t* xs8;      // [M, K] activation codes (operand layout)
+  const float* s_a;       // [M]   (ignored by the s32 sink)
+  const uint8_t* Wq;      // [N, K/2] packed weight codes
+  const float* s_w;       // [N]
+  const uint16_t* bias;   // [N] or null
+  void* out;              // [M, N] bf16 / f32 / s32
+  int M, N, K;
+};
+
+// Builds the tensor maps and launches the tensor-core GEMM.
+cudaError_t launch_w4a4_gemm(const GemmArgs& a, GemmSink sink, const GemmTiling& t, cudaStream_t stream);
+
+// Host-side dispatch counters (see convrot_dispatch_counts).
+void count_dispatch(int which);
+
+}  // namespace convrot

@@ -1,0 +1,88 @@
+"""Host-side checks of the C ABI (no GPU needed): the library loads, exports
+every symbol include/convrot.h declares, and rejects bad arguments before it
+touches a device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from rotation_quantized_bit_b200 import build
+    build.build()
+    import rotation_quantized_bit_b200 as rq
+    return rq.load_library()
+
+
+def declared_functions():
+    with open(os.path.join(ROOT, "include", "convrot.h")) as f:
+        text = f.read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b([a-z_0-9]+)\s*\(", text)) - {"if", "sizeof"})
+
+
+def test_header_declares_the_public_names():
+    names = declared_functions()
+    for need in ["convrot_pack_weight", "convrot_rotate_quant", "w4a4_gemm", "convrot_w4a4_linear"]:
+        assert need in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    import rotation_quantized_bit_b200 as rq
+    names = declared_functions()
+    for n in names:
+        assert hasattr(lib, n), f"{n} declared in include/convrot.h but not exported"
+    assert sorted(rq.EXPORTS) == names
+
+
+def test_status_strings(lib):
+    for code in range(8):
+        s = lib.convrot_status_string(code).decode()
+        assert s.startswith("CONVROT_")
+    assert b"UNKNOWN" in lib.convrot_status_string(99)
+
+
+def test_workspace_sizes(lib):
+    assert lib.convrot_w4a4_workspace_size(32, 256, 512) >= 32 * 512 + 32 * 4
+    assert lib.convrot_gemm_workspace_size(1220, 9728, 2560) >= 1220 * 2560
+    assert lib.convrot_w4a4_workspace_size(32, 256, 300) == 0  # bad K
+    assert lib.convrot_w4a4_workspace_size(0, 256, 512) == 0
+
+
+FAKE = ctypes.c_void_p(0x10000)      # never dereferenced: validation fails first
+FAKE_ODD = ctypes.c_void_p(0x10001)  # misaligned
+
+
+@pytest.mark.parametrize("M,N,K,code", [
+    (0, 256, 512, 2), (32, 0, 512, 2), (32, 12, 512, 2), (32, 256, 500, 2), (32, 256, 128, 2),
+    (32, 256, 65536, 2),
+])
+def test_shape_errors_are_synchronous(lib, M, N, K, code):
+    rc = lib.convrot_w4a4_linear(FAKE, FAKE, FAKE, None, M, N, K, FAKE, FAKE, 1 << 30, None)
+    assert rc == code
+
+
+def test_null_alignment_and_workspace_errors(lib):
+    assert lib.convrot_w4a4_linear(None, FAKE, FAKE, None, 32, 256, 512, FAKE, FAKE, 1 << 30, None) == 1
+    assert lib.convrot_w4a4_linear(FAKE_ODD, FAKE, FAKE, None, 32, 256, 512, FAKE, FAKE, 1 << 30, None) == 3
+    assert lib.convrot_w4a4_linear(FAKE, FAKE, FAKE, None, 32, 256, 512, FAKE, FAKE, 16, None) == 5
+    assert lib.convrot_w4a4_linear(FAKE, FAKE, FAKE, None, 32, 256, 512, FAKE, None, 1 << 30, None) == 5
+    assert lib.convrot_rotate_quant(FAKE, 4, 512, None, FAKE, None) == 1
+    assert lib.w4a4_gemm_s32(FAKE, FAKE, 4, 256, 512, FAKE_ODD, FAKE, 1 << 30, None) == 3
+    assert lib.w4a4_gemm(FAKE, None, FAKE, FAKE, None, 4, 256, 512, FAKE, FAKE, 1 << 30, None) == 1
+
+
+def test_dispatch_counters_without_a_gpu(lib):
+    import torch
+    arr = (ctypes.c_uint64 * 4)()
+    lib.convrot_dispatch_counts(arr, 4)
+    if not torch.cuda.is_available():
+        assert list(arr) == [0, 0, 0, 0]  # argument errors never reach a launch
+
+
+def test_version(lib):
+    assert b"sm_100a" in lib.convrot_version()

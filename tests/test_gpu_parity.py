@@ -1,0 +1,235 @@
+"""GPU parity: the CUDA path through the C ABI against the CPU oracle, element
+by element, on the same seeded inputs.
+
+Bar (stated by the method's contract):
+  * codes (packed bytes), scales (raw fp32 bits) and the int32 accumulators:
+    bit-exact;
+  * fp32 output: |y - y_oracle| <= 1e-5 * max|y_oracle|;
+  * bf16 output: within one bf16 ulp of the oracle's bf16.
+Small cases span several tiles and ragged tails; the full workload shapes
+(the ones the benchmark times, through the same entry point and launch
+configuration) are checked on sampled rows that include the first tile, a
+middle tile and the M tail.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synthetic
+from tests.gpu_util import dev, dev_bf16, f32_bits, host, host_bits
+
+pytestmark = pytest.mark.gpu
+
+F32_TOL = 1e-5
+
+
+@pytest.fixture(scope="module")
+def rq():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    import rotation_quantized_bit_b200 as rq
+    rq.load_library()
+    return rq
+
+
+def bf16_ulp_diff(a_bits, b_bits):
+    """|a - b| in units of bf16 ulps, via the monotone integer mapping."""
+    def key(u):
+        u = u.astype(np.int32)
+        return np.where(u & 0x8000, 0x8000 - (u & 0x7FFF), 0x8000 + u)
+    return np.abs(key(a_bits) - key(b_bits))
+
+
+def check_f32(y, ref):
+    scale = max(float(np.max(np.abs(ref))), 1e-30)
+    err = float(np.max(np.abs(y.astype(np.float64) - ref.astype(np.float64))))
+    assert err <= F32_TOL * scale, f"max err {err} > {F32_TOL} * {scale}"
+
+
+# ------------------------------------------------------------- rotate / quant
+
+RQ_CASES = [("small", 32, 512), ("qwen3_4b", 77, 2560), ("qwen3_4b", 1, 256), ("dit6b", 300, 3840),
+            ("edit20b", 5, 12288), ("qwen3_4b", 129, 9728), ("dit6b", 64, 10240)]
+
+
+@pytest.mark.parametrize("workload,M,K", RQ_CASES)
+def test_rotate_quant_bit_exact(rq, workload, M, K):
+    x = synthetic.activations(workload, M, K)
+    xq_ref, s_ref = oracle.rotate_quant(x)
+    xq, s = rq.convrot_rotate_quant(dev_bf16(x))
+    assert np.array_equal(f32_bits(host(s)), f32_bits(s_ref))
+    assert np.array_equal(host(xq), xq_ref)
+
+
+def special_rows(K=512):
+    rows = []
+    z = np.zeros(K)
+    rows.append(z.copy())                                    # all zero -> s = 0, codes 0
+    for v1 in (8, 24, 40, 56, 72, 88, 104):                  # exact half-integer ties
+        r = z.copy(); r[0] = 112.0; r[256] = v1; rows.append(r)
+    for A, B in ((1.421875, 1.3203125), (1.53125, 1.421875), (2.0625, 1.03125),
+                 (2.546875, 1.2734375), (2.609375, 1.3046875)):  # division vs reciprocal ties
+        r = z.copy(); r[0] = A; r[256] = B; rows.append(r)
+    r = z.copy(); r[:] = 3.0; rows.append(r)                 # constant vector
+    r = z.copy(); r[5] = -1e-38; r[300] = 3e-39; rows.append(r)  # subnormal scale
+    r = z.copy(); r[7] = 3.0e38; r[8] = -2.5e38; rows.append(r)  # huge values
+    r = z.copy(); r[::3] = 1e-30; rows.append(r)             # tiny values
+    return synthetic.to_bf16_bits(np.stack(rows))
+
+
+def test_rotate_quant_special_rows(rq):
+    x = special_rows()
+    xq_ref, s_ref = oracle.rotate_quant(x)
+    xq, s = rq.convrot_rotate_quant(dev_bf16(x))
+    assert np.array_equal(f32_bits(host(s)), f32_bits(s_ref))
+    assert np.array_equal(host(xq), xq_ref)
+
+
+@pytest.mark.parametrize("workload,N,K", [("small", 256, 512), ("qwen3_4b", 1024, 2560), ("dit6b", 136, 3840)])
+def test_pack_weight_bit_exact(rq, workload, N, K):
+    w, _ = synthetic.weights(workload, N, K)
+    wq_ref, s_ref = oracle.pack_weight(w)
+    wq, s = rq.convrot_pack_weight(dev_bf16(w))
+    assert np.array_equal(host(wq), wq_ref)
+    assert np.array_equal(f32_bits(host(s)), f32_bits(s_ref))
+
+
+# ------------------------------------------------------------- GEMM sinks
+
+GEMM_CASES = [(8, 256, 256), (32, 256, 512), (77, 264, 768), (1, 128, 2560), (16, 2560, 2560),
+              (200, 384, 1024), (300, 1000, 512), (193, 136, 256), (600, 4096, 512)]
+
+
+def random_codes(seed, rows, K):
+    rng = np.random.default_rng(seed)
+    return rng.integers(0, 256, size=(rows, K // 2), dtype=np.uint8)  # every nibble, -8 included
+
+
+@pytest.mark.parametrize("M,N,K", GEMM_CASES)
+def test_gemm_s32_bit_exact(rq, M, N, K):
+    xq = random_codes(M * 7 + K, M, K)
+    wq = random_codes(N * 13 + K, N, K)
+    ref = oracle.gemm_s64(xq, wq, K)
+    acc = rq.w4a4_gemm_s32(dev(xq), dev(wq))
+    assert np.array_equal(host(acc).astype(np.int64), ref)
+
+
+def test_gemm_s32_extremes(rq):
+    K = 3840
+    for a, b, want in ((0x77, 0x77, 49 * K), (0x88, 0x88, 64 * K), (0x88, 0x77, -56 * K)):
+        xq = np.full((24, K // 2), a, np.uint8)
+        wq = np.full((136, K // 2), b, np.uint8)
+        assert np.all(host(rq.w4a4_gemm_s32(dev(xq), dev(wq))) == want)
+
+
+@pytest.mark.parametrize("M,N,K", [(32, 256, 512), (77, 264, 768), (193, 136, 256), (600, 4096, 512)])
+def test_gemm_f32_and_bf16(rq, M, N, K):
+    x = synthetic.activations("qwen3_4b", M, K)
+    w, b = synthetic.weights("qwen3_4b", N, K)
+    xq, s_a = oracle.rotate_quant(x)
+    wq, s_w = oracle.pack_weight(w)
+    acc = oracle.gemm_s64(xq, wq, K)
+    y32_ref, y16_ref = oracle.epilogue(acc, s_a, s_w, b)
+    args = (dev(xq), dev(s_a), dev(wq), dev(s_w), dev_bf16(b))
+    y32 = host(rq.w4a4_gemm_f32(*args))
+    check_f32(y32, y32_ref)
+    assert np.array_equal(f32_bits(y32), f32_bits(y32_ref))  # same op order as the oracle -> identical bits
+    y16 = host_bits(rq.w4a4_gemm(*args))
+    assert bf16_ulp_diff(y16, y16_ref).max() <= 1
+    # no bias
+    y32n = host(rq.w4a4_gemm_f32(dev(xq), dev(s_a), dev(wq), dev(s_w), None))
+    check_f32(y32n, oracle.epilogue(acc, s_a, s_w, None)[0])
+
+
+# ------------------------------------------------------------- fused Linear
+
+LINEAR_CASES = [("small", 32, 512, 256), ("qwen3_4b", 77, 2560, 264), ("qwen3_4b", 1, 2560, 1024),
+                ("dit6b", 250, 3840, 384), ("edit20b", 16, 3072, 12288), ("qwen3_4b", 8, 9728, 2560)]
+
+
+@pytest.mark.parametrize("workload,M,K,N", LINEAR_CASES)
+def test_linear_matches_oracle(rq, workload, M, K, N):
+    x = synthetic.activations(workload, M, K)
+    w, b = synthetic.weights(workload, N, K)
+    wq, s_w = oracle.pack_weight(w)
+    y32_ref, y16_ref = oracle.linear(x, wq, s_w, b, K)
+    dx, dwq, dsw, db = dev_bf16(x), dev(wq), dev(s_w), dev_bf16(b)
+    y32 = host(rq.convrot_w4a4_linear_f32(dx, dwq, dsw, db))
+    check_f32(y32, y32_ref)
+    assert np.array_equal(f32_bits(y32), f32_bits(y32_ref))
+    y16 = host_bits(rq.convrot_w4a4_linear(dx, dwq, dsw, db))
+    assert bf16_ulp_diff(y16, y16_ref).max() <= 1
+
+
+def sample_rows(M, BT_guess=192):
+    rows = set(range(min(M, 8)))
+    rows |= set(range(max(0, M - 8), M))
+    mid = M // 2
+    rows |= set(range(max(0, mid - 4), min(M, mid + 4)))
+    return sorted(rows)
+
+
+FULL = [s for wl in ("qwen3_4b", "dit6b", "edit20b", "small_m") for s in synthetic.workload_shapes(wl)]
+
+
+@pytest.mark.parametrize("shape", FULL, ids=lambda s: f"{s.name}-M{s.M}-K{s.K}-N{s.N}")
+def test_full_size_linear_sampled_rows(rq, shape):
+    wl = next(w for w in ("qwen3_4b", "dit6b", "edit20b", "small_m")
+              if shape in synthetic.workload_shapes(w))
+    M, K, N = shape.M, shape.K, shape.N
+    x = synthetic.activations(wl, M, K)
+    w, b = synthetic.weights(wl, N, K)
+    dwq, dsw = rq.convrot_pack_weight(dev_bf16(w))
+    wq = host(dwq)
+    y32 = host(rq.convrot_w4a4_linear_f32(dev_bf16(x), dwq, dsw, dev_bf16(b)))
+    y16 = host_bits(rq.convrot_w4a4_linear(dev_bf16(x), dwq, dsw, dev_bf16(b)))
+    rows = sample_rows(M)
+    # the weights prepared on the GPU are the oracle's, checked on sampled rows
+    wrows = sorted(set(range(min(N, 4))) | set(range(max(0, N - 4), N)))
+    wq_ref, sw_ref = oracle.pack_weight(w[wrows])
+    assert np.array_equal(wq[wrows], wq_ref) and np.array_equal(f32_bits(host(dsw)[wrows]), f32_bits(sw_ref))
+    for r0, r1 in _runs(rows):
+        ref32, ref16 = oracle.linear(x, wq, host(dsw), b, K, rows=(r0, r1))
+        check_f32(y32[r0:r1], ref32)
+        assert np.array_equal(f32_bits(y32[r0:r1]), f32_bits(ref32))
+        assert bf16_ulp_diff(y16[r0:r1], ref16).max() <= 1
+
+
+def _runs(rows):
+    out, start, prev = [], rows[0], rows[0]
+    for r in rows[1:]:
+        if r != prev + 1:
+            out.append((start, prev + 1))
+            start = r
+        prev = r
+    out.append((start, prev + 1))
+    return out
+
+
+# ------------------------------------------------------------- boundary behaviour
+
+
+def test_errors_raise_before_launch(rq):
+    x = torch.zeros((4, 300), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(rq.ConvRotError) as e:
+        rq.convrot_rotate_quant(x)
+    assert e.value.status == "CONVROT_ERR_SHAPE"
+    buf = torch.zeros(4 * 512 * 2 + 16, dtype=torch.uint8, device="cuda")
+    lib = rq.load_library()
+    import ctypes
+    rc = lib.convrot_rotate_quant(ctypes.c_void_p(buf.data_ptr() + 2), 4, 512, ctypes.c_void_p(buf.data_ptr()),
+                                  ctypes.c_void_p(buf.data_ptr()), None)
+    assert rq.STATUS[rc] == "CONVROT_ERR_ALIGN"
+
+
+def test_dispatch_counts_and_no_device_error(rq):
+    before = rq.convrot_dispatch_counts()
+    x = dev_bf16(synthetic.activations("small", 32, 512))
+    w, b = synthetic.weights("small", 256, 512)
+    wq, s_w = rq.convrot_pack_weight(dev_bf16(w))
+    rq.convrot_w4a4_linear(x, wq, s_w, dev_bf16(b))
+    after = rq.convrot_dispatch_counts()
+    assert after["rotate_quant"] == before["rotate_quant"] + 2
+    assert after["tc_gemm"] + after["tc_gemm_splitk"] == before["tc_gemm"] + before["tc_gemm_splitk"] + 1
+    assert rq.convrot_device_error() == 0
