@@ -164,6 +164,11 @@ convrot_status_t convrot_device_error(void *stream, uint32_t *code);
  * (cluster reduction).  `n` is the array length; at most 4 are written. */
 void convrot_dispatch_counts(uint64_t *counts, int n);
 
+/* Description of the last CUDA call of this library that failed on the
+ * calling thread (which call, error name and text); "" if none.  Valid until
+ * the next failing call on the same thread. */
+const char *convrot_last_error(void);
+
 /* Library build identifier (static string). */
 const char *convrot_version(void);
 

@@ -39,7 +39,7 @@ EXPORTS = [
     "convrot_status_string", "convrot_pack_weight", "convrot_rotate_quant", "convrot_gemm_workspace_size",
     "w4a4_gemm", "w4a4_gemm_s32", "w4a4_gemm_f32", "convrot_w4a4_workspace_size", "convrot_w4a4_linear",
     "convrot_w4a4_linear_f32", "convrot_w4a4_quantize", "convrot_w4a4_gemm_quantized", "convrot_device_error",
-    "convrot_dispatch_counts", "convrot_version",
+    "convrot_dispatch_counts", "convrot_last_error", "convrot_version",
 ]
 
 
@@ -67,6 +67,7 @@ def load_library():
     lib.convrot_status_string.argtypes = [I]
     lib.convrot_status_string.restype = ctypes.c_char_p
     lib.convrot_version.restype = ctypes.c_char_p
+    lib.convrot_last_error.restype = ctypes.c_char_p
     lib.convrot_pack_weight.argtypes = [P, I, I, P, P, P]
     lib.convrot_rotate_quant.argtypes = [P, I, I, P, P, P]
     lib.convrot_gemm_workspace_size.argtypes = [I, I, I]
@@ -97,7 +98,10 @@ def lib_status_fns():
 
 def _check(fn: str, rc: int):
     if rc != 0:
-        raise ConvRotError(fn, rc, load_library().convrot_status_string(rc).decode())
+        lib = load_library()
+        msg = lib.convrot_status_string(rc).decode()
+        last = lib.convrot_last_error().decode()
+        raise ConvRotError(fn, rc, msg + (f" [{last}]" if last and rc == 6 else ""))
 
 
 def _ptr(t):

@@ -7,6 +7,7 @@
 
 #include <atomic>
 #include <cstdint>
+#include <cstdio>
 #include <cstring>
 
 #include "../../include/convrot.h"
@@ -62,6 +63,8 @@ convrot_status_t check_mnk(int M, int N, int K) {
 }
 
 convrot_status_t from_cuda(cudaError_t e) { return e == cudaSuccess ? CONVROT_OK : CONVROT_ERR_CUDA; }
+
+convrot_status_t check_device(int* sms_out);
 
 size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
@@ -145,6 +148,34 @@ void count_dispatch(int which) {
   if (which >= 0 && which < 4) g_counts[which].fetch_add(1, std::memory_order_relaxed);
 }
 
+namespace {
+thread_local char g_last_error[256] = "";
+}
+
+cudaError_t note_cuda(cudaError_t e, const char* where) {
+  if (e != cudaSuccess) snprintf(g_last_error, sizeof(g_last_error), "%s: %s (%s)", where, cudaGetErrorName(e),
+                                 cudaGetErrorString(e));
+  return e;
+}
+
+cudaError_t ensure_dynamic_smem(const void* kernel, int bytes, int* cache) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (bytes <= cache[dev]) return cudaSuccess;
+  int optin = 0;
+  e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+  if (e != cudaSuccess) return e;
+  cudaFuncAttributes fa;
+  e = cudaFuncGetAttributes(&fa, kernel);
+  if (e != cudaSuccess) return e;
+  if (bytes + static_cast<int>(fa.sharedSizeBytes) > optin) return cudaErrorInvalidValue;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess) cache[dev] = bytes;
+  return e;
+}
+
 }  // namespace convrot
 
 using namespace convrot;
@@ -166,6 +197,8 @@ const char* convrot_status_string(convrot_status_t status) {
 }
 
 const char* convrot_version(void) { return "convrot-b200 sm_100a"; }
+
+const char* convrot_last_error(void) { return g_last_error; }
 
 convrot_status_t convrot_rotate_quant(const uint16_t* x, int M, int K, uint8_t* xq, float* s_a, void* stream) {
   if (!x || !xq || !s_a) return CONVROT_ERR_NULL;

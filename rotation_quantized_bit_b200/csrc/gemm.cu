@@ -310,15 +310,9 @@ int shared_bytes_for(int BT, int nstages, int splits) {
 template <int SINK>
 cudaError_t launch_sink(const CUtensorMap& tw, const CUtensorMap& tx, const Params& prm, const GemmTiling& t,
                         cudaStream_t stream) {
-  static int attr_done_dev = -1;
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (attr_done_dev != dev) {
-    cudaError_t e = cudaFuncSetAttribute(w4a4_tc_gemm_kernel<SINK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         227 * 1024);
-    if (e != cudaSuccess) return e;
-    attr_done_dev = dev;
-  }
+  static int cache[64] = {0};
+  cudaError_t e = ensure_dynamic_smem(reinterpret_cast<const void*>(w4a4_tc_gemm_kernel<SINK>), t.smem_bytes, cache);
+  if (e != cudaSuccess) return note_cuda(e, "w4a4_gemm: dynamic shared memory attribute");
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(t.n_tiles, t.m_tiles, t.splits);
   cfg.blockDim = dim3(kThreads, 1, 1);
@@ -335,7 +329,7 @@ cudaError_t launch_sink(const CUtensorMap& tw, const CUtensorMap& tx, const Para
   }
   cfg.attrs = attr;
   cfg.numAttrs = nattr;
-  return cudaLaunchKernelEx(&cfg, w4a4_tc_gemm_kernel<SINK>, tw, tx, prm);
+  return note_cuda(cudaLaunchKernelEx(&cfg, w4a4_tc_gemm_kernel<SINK>, tw, tx, prm), "w4a4_gemm: launch");
 }
 
 }  // namespace
@@ -384,10 +378,10 @@ cudaError_t launch_w4a4_gemm(const GemmArgs& a, GemmSink sink, const GemmTiling&
   CUtensorMap tw, tx;
   if (!make_map_u8(&tw, a.Wq, static_cast<uint64_t>(a.N), static_cast<uint64_t>(a.K / 2), kRows, kKB / 2,
                    CU_TENSOR_MAP_SWIZZLE_64B))
-    return cudaErrorInvalidValue;
+    return note_cuda(cudaErrorInvalidValue, "w4a4_gemm: weight tensor map");
   if (!make_map_u8(&tx, a.xs8, static_cast<uint64_t>(a.M), static_cast<uint64_t>(a.K), static_cast<uint32_t>(t.BT),
                    kKB, CU_TENSOR_MAP_SWIZZLE_128B))
-    return cudaErrorInvalidValue;
+    return note_cuda(cudaErrorInvalidValue, "w4a4_gemm: activation tensor map");
   Params prm{};
   prm.s_a = a.s_a;
   prm.s_w = a.s_w;

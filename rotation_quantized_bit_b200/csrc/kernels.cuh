@@ -56,4 +56,11 @@ cudaError_t launch_w4a4_gemm(const GemmArgs& a, GemmSink sink, const GemmTiling&
 // Host-side dispatch counters (see convrot_dispatch_counts).
 void count_dispatch(int which);
 
+// Remember the last failing CUDA call (see convrot_last_error).
+cudaError_t note_cuda(cudaError_t e, const char* where);
+
+// Raise a kernel's dynamic shared-memory limit to `bytes` on the current
+// device if needed (checked against the opt-in maximum minus static usage).
+cudaError_t ensure_dynamic_smem(const void* kernel, int bytes, int* cache);
+
 }  // namespace convrot

@@ -155,21 +155,15 @@ int num_sms_cached() {
 }  // namespace
 
 cudaError_t launch_rotate_quant(const uint16_t* x, int M, int K, RotateQuantOut out, cudaStream_t stream) {
-  const size_t smem = static_cast<size_t>(K) * sizeof(float);
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(rotate_quant_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         65536 * static_cast<int>(sizeof(float)) > 227 * 1024
-                                             ? 227 * 1024
-                                             : 65536 * static_cast<int>(sizeof(float)));
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  const int smem = K * static_cast<int>(sizeof(float));
+  static int cache[64] = {0};
+  cudaError_t e = ensure_dynamic_smem(reinterpret_cast<const void*>(rotate_quant_kernel), smem, cache);
+  if (e != cudaSuccess) return note_cuda(e, "rotate_quant: dynamic shared memory attribute");
   int grid = num_sms_cached() * 4;
   if (grid > M) grid = M;
   rotate_quant_kernel<<<grid, kThreads, smem, stream>>>(x, M, K, out);
   count_dispatch(0);
-  return cudaGetLastError();
+  return note_cuda(cudaGetLastError(), "rotate_quant: launch");
 }
 
 cudaError_t launch_unpack_codes(const uint8_t* packed, int M, int K, int8_t* s8, cudaStream_t stream) {
@@ -178,7 +172,7 @@ cudaError_t launch_unpack_codes(const uint8_t* packed, int M, int K, int8_t* s8,
   if (grid > num_sms_cached() * 8) grid = num_sms_cached() * 8;
   unpack_codes_kernel<<<grid, kThreads, 0, stream>>>(packed, M, K, s8);
   count_dispatch(1);
-  return cudaGetLastError();
+  return note_cuda(cudaGetLastError(), "unpack_codes: launch");
 }
 
 }  // namespace convrot
