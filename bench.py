@@ -60,6 +60,8 @@ def parse():
     ap.add_argument("--workload", default="qwen3_4b", choices=sorted(WORKLOAD_DESC))
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--only", default=None, help="restrict the workload to the linear with this name")
+    ap.add_argument("--no-graph", action="store_true", help="launch the step eagerly instead of replaying a CUDA graph")
     return ap.parse_args()
 
 
@@ -180,9 +182,15 @@ def main():
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     shapes = synthetic.workload_shapes(args.workload)
+    if args.only:
+        shapes = [s for s in shapes if s.name == args.only]
+        if not shapes:
+            raise SystemExit(f"no linear named {args.only!r} in workload {args.workload}")
     config = {"workload": args.workload, "description": WORKLOAD_DESC[args.workload],
               "linears": [f"{s.name}:M{s.M}xK{s.K}xN{s.N}" for s in shapes],
               "l2": "flushed between timed steps (256 MiB write, outside the events)",
+              "launch": "each step replayed from a CUDA graph (2 kernels per linear)" if not args.no_graph
+                        else "eager launches",
               "parallelism": f"replicas x{max(world, args.gpus)}" if max(world, args.gpus) > 1 else "single GPU",
               "codes": "s4 packed weights, s4 activations widened to s8 for tcgen05 kind::i8, int32 accumulate, "
                        "fp32 epilogue, bf16 out"}
@@ -243,9 +251,27 @@ def main():
         run_step()
     torch.cuda.synchronize()
 
-    counts0 = rq.convrot_dispatch_counts()
-    step_events = [[[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(nlin)]
+    # One CUDA graph per timed step (each with its own events): a replay runs
+    # the step's launches back to back, with no host gaps between them.
+    # external=True: recorded inside a graph capture these become event-record
+    # nodes that are timestamped on every replay (internal events would only
+    # mark cross-stream dependencies).
+    step_events = [[[torch.cuda.Event(enable_timing=True, external=True) for _ in range(3)] for _ in range(nlin)]
                    for _ in range(args.steps)]
+    graphs = []
+    if not args.no_graph:
+        for k in range(args.steps):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                run_step(step_events[k])
+            graphs.append(g)
+        for g in graphs[:1]:  # one untimed replay of the captured work
+            flush.zero_()
+            g.replay()
+        torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+
+    counts0 = rq.convrot_dispatch_counts()
     sampler = ClockSampler(torch.cuda.current_device()) if rank == 0 or world == 1 else None
     if world > 1:
         dist.barrier()
@@ -254,7 +280,10 @@ def main():
         sampler.start()
     for k in range(args.steps):
         flush.zero_()  # L2 flush, outside the step's events
-        run_step(step_events[k])
+        if graphs:
+            graphs[k].replay()
+        else:
+            run_step(step_events[k])
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
@@ -263,6 +292,11 @@ def main():
     err = rq.convrot_device_error()
     if err:
         raise RuntimeError(f"device error word {err:#x}: a bounded wait expired")
+    if graphs:  # launches of a replayed graph are not seen by the host counters
+        launches = 2 * nlin * args.steps
+    else:
+        launches = (counts1["rotate_quant"] - counts0["rotate_quant"]) + (counts1["tc_gemm"] - counts0["tc_gemm"]) + \
+                   (counts1["tc_gemm_splitk"] - counts0["tc_gemm_splitk"])
 
     # per-linear, per-kernel times (ms), summed over the K steps
     t_quant = np.zeros(nlin)
@@ -328,9 +362,6 @@ def main():
     roof["share_of_step"] = tsum / total_ms if world == 1 else None
     roof["traffic"] = committed_traffic(kname, s)
 
-    launches = (counts1["rotate_quant"] - counts0["rotate_quant"]) + (counts1["tc_gemm"] - counts0["tc_gemm"]) + \
-               (counts1["tc_gemm_splitk"] - counts0["tc_gemm_splitk"])
-
     e2e = None
     if not args.no_e2e:
         e2e = end_to_end(args, rq, torch, dev, stream, shapes, xs, layers, ws, flush, world, dist)
@@ -348,6 +379,7 @@ def main():
     }
     if rank == 0:
         print(json.dumps(line), flush=True)
+    del graphs
     if world > 1:
         dist.destroy_process_group()
 

@@ -83,16 +83,19 @@ __device__ __forceinline__ void unpack_row_to_tmem(const uint8_t* wstage, int ro
   tmem_st_32x32b_x32(taddr, cols);
 }
 
+// One output element from the MMA sum (16 * acc): scales and bias already
+// loaded by the caller.
 template <int SINK>
-__device__ __forceinline__ void store_output(const Params& p, int m, int n, int32_t dsum) {
+__device__ __forceinline__ void store_output(const Params& p, int m, int n, int32_t dsum, float sa, float sw,
+                                             float bv) {
   const int32_t acc = dsum >> 4;  // the weights entered the MMA as 16 * q_w
   const size_t idx = static_cast<size_t>(m) * p.N + n;
   if (SINK == static_cast<int>(GemmSink::kS32)) {
     static_cast<int32_t*>(p.out)[idx] = acc;
     return;
   }
-  float y = __fmul_rn(__fmul_rn(__int2float_rn(acc), __ldg(p.s_a + m)), __ldg(p.s_w + n));
-  if (p.bias) y = __fadd_rn(y, __uint_as_float(static_cast<uint32_t>(__ldg(p.bias + n)) << 16));
+  float y = __fmul_rn(__fmul_rn(__int2float_rn(acc), sa), sw);
+  if (p.bias) y = __fadd_rn(y, bv);
   if (SINK == static_cast<int>(GemmSink::kF32)) {
     static_cast<float*>(p.out)[idx] = y;
   } else {
@@ -110,7 +113,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int BT = p.BT;
   const int stage_bytes = kWTileBytes + BT * kKB;
   SharedHeader* hdr = reinterpret_cast<SharedHeader*>(smem + p.nstages * stage_bytes);
-  int32_t* red = reinterpret_cast<int32_t*>(reinterpret_cast<uint8_t*>(hdr) + 1024);  // split-K partials
+  float* sa_tile = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(hdr) + 1024);   // s_a of the BT tokens
+  int32_t* red = reinterpret_cast<int32_t*>(reinterpret_cast<uint8_t*>(hdr) + 2048);  // split-K partials
+  const int red_pitch = BT + 4;  // int32 per partial-tile row (16-byte rows, bank-conflict free)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n0 = blockIdx.x * kRows;
@@ -190,6 +195,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int quad = warp & 3;  // tensor-memory lane quadrant of this warp
     const int row = quad * 32 + lane;
     const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
+    const int et = threadIdx.x - 64;  // 0..127 over the four unpack/epilogue warps
+    if (SINK != static_cast<int>(GemmSink::kS32)) {
+      for (int c = et; c < BT; c += 128) sa_tile[c] = (m0 + c < p.M) ? __ldg(p.s_a + m0 + c) : 0.0f;
+    }
     bool ok = true;
     for (int i = 0; i < nkb; ++i) {
       const int s = i % ns, a = i % kASlots;
@@ -209,10 +218,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (ok) ok = mbar_wait(&hdr->acc_full, 0);
     ok = __all_sync(0xffffffffu, ok);  // tcgen05.ld below is warp-collective
     tc_fence_after();
+    named_barrier(1, 128);  // sa_tile written by all four epilogue warps
 
     const int n = n0 + row;
     if (p.splits == 1) {
       if (ok && nkb > 0) {
+        const float sw = (SINK != static_cast<int>(GemmSink::kS32) && n < p.N) ? __ldg(p.s_w + n) : 0.0f;
+        const float bv = (p.bias && n < p.N) ? __uint_as_float(static_cast<uint32_t>(__ldg(p.bias + n)) << 16) : 0.0f;
         for (int c = 0; c < BT; c += 16) {
           uint32_t v[16];
           tmem_ld_32x32b_x16(tmem + lane_base + static_cast<uint32_t>(c), v);
@@ -221,19 +233,25 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
               const int m = m0 + c + j;
-              if (m < p.M) store_output<SINK>(p, m, n, static_cast<int32_t>(v[j]));
+              if (m < p.M) store_output<SINK>(p, m, n, static_cast<int32_t>(v[j]), sa_tile[c + j], sw, bv);
             }
           }
         }
       }
     } else {
-      // Partial tile -> own shared memory, column-major [BT][128].
+      // Partial tile -> own shared memory, row-major [128][BT + 4].
       for (int c = 0; c < BT; c += 16) {
         uint32_t v[16];
         tmem_ld_32x32b_x16(tmem + lane_base + static_cast<uint32_t>(c), v);
         tmem_wait_ld();
+        const bool keep = ok && nkb > 0;
 #pragma unroll
-        for (int j = 0; j < 16; ++j) red[(c + j) * kRows + row] = (ok && nkb > 0) ? static_cast<int32_t>(v[j]) : 0;
+        for (int q = 0; q < 4; ++q) {
+          int4 w = keep ? make_int4(static_cast<int32_t>(v[4 * q]), static_cast<int32_t>(v[4 * q + 1]),
+                                    static_cast<int32_t>(v[4 * q + 2]), static_cast<int32_t>(v[4 * q + 3]))
+                        : make_int4(0, 0, 0, 0);
+          *reinterpret_cast<int4*>(red + row * red_pitch + c + 4 * q) = w;
+        }
       }
     }
   }
@@ -242,17 +260,34 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();    // the cluster barrier below is .aligned: reconverge first
     cluster_sync();  // every CTA of the cluster has its partial tile in shared memory
     if (warp >= 2) {
+      // CTA `rank` finishes the 4-token groups g = rank, rank + S, ... of the
+      // tile: all S partials of a group are loaded (16 bytes each) before
+      // they are summed, so the remote loads overlap.
       const int quad = warp & 3;
       const int row = quad * 32 + lane;
       const int n = n0 + row;
       const uint32_t rank = cluster_ctarank();
-      for (int c = static_cast<int>(rank); c < BT; c += p.splits) {
-        const int m = m0 + c;
-        if (m >= p.M || n >= p.N) continue;
-        const uint32_t local = smem_u32(red + c * kRows + row);
-        int32_t sum = 0;
-        for (int j = 0; j < p.splits; ++j) sum += ld_shared_cluster_s32(map_shared_rank(local, static_cast<uint32_t>(j)));
-        store_output<SINK>(p, m, n, sum);
+      const float sw = (SINK != static_cast<int>(GemmSink::kS32) && n < p.N) ? __ldg(p.s_w + n) : 0.0f;
+      const float bv = (p.bias && n < p.N) ? __uint_as_float(static_cast<uint32_t>(__ldg(p.bias + n)) << 16) : 0.0f;
+      const uint32_t row_addr = smem_u32(red + row * red_pitch);
+      for (int g = static_cast<int>(rank); g < BT / 4; g += p.splits) {
+        if (m0 + 4 * g >= p.M || n >= p.N) continue;
+        int4 part[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          if (j < p.splits) part[j] = ld_shared_cluster_v4(map_shared_rank(row_addr + 16u * g, static_cast<uint32_t>(j)));
+        int4 sum = make_int4(0, 0, 0, 0);
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          if (j < p.splits) {
+            sum.x += part[j].x; sum.y += part[j].y; sum.z += part[j].z; sum.w += part[j].w;
+          }
+        const int32_t sv[4] = {sum.x, sum.y, sum.z, sum.w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int m = m0 + 4 * g + q;
+          if (m < p.M) store_output<SINK>(p, m, n, sv[q], sa_tile[4 * g + q], sw, bv);
+        }
       }
     }
     __syncwarp();
@@ -302,8 +337,8 @@ bool make_map_u8(CUtensorMap* map, const void* base, uint64_t rows, uint64_t col
 }
 
 int shared_bytes_for(int BT, int nstages, int splits) {
-  int bytes = 1024 /*alignment slack*/ + nstages * (kWTileBytes + BT * kKB) + 1024 /*header*/;
-  if (splits > 1) bytes += BT * kRows * 4;
+  int bytes = 1024 /*alignment slack*/ + nstages * (kWTileBytes + BT * kKB) + 2048 /*header + s_a tile*/;
+  if (splits > 1) bytes += (BT + 4) * kRows * 4;
   return bytes;
 }
 
@@ -355,7 +390,7 @@ GemmTiling choose_tiling(int M, int N, int K, int num_sms) {
   t.kb_per_split = kbps;
   // Pipeline depth: as many stages as fit two CTAs per SM (~110 KB each).
   const int stage = kWTileBytes + bt * kKB;
-  int ns = (110 * 1024 - 2048 - (splits > 1 ? bt * kRows * 4 : 0)) / stage;
+  int ns = (110 * 1024 - 3072 - (splits > 1 ? (bt + 4) * kRows * 4 : 0)) / stage;
   if (ns > 8) ns = 8;
   if (ns > kbps) ns = kbps < 2 ? 2 : kbps;
   if (ns < 2) ns = 2;

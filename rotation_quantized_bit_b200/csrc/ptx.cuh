@@ -209,10 +209,19 @@ __device__ __forceinline__ uint32_t map_shared_rank(uint32_t local_addr, uint32_
   return r;
 }
 
-__device__ __forceinline__ int32_t ld_shared_cluster_s32(uint32_t addr) {
-  int32_t v;
-  asm volatile("ld.shared::cluster.s32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+// 16-byte load from (possibly another CTA's) shared memory in the cluster.
+// Ordered only by the cluster barriers around it, so several can be in flight.
+__device__ __forceinline__ int4 ld_shared_cluster_v4(uint32_t addr) {
+  int4 v;
+  asm volatile("ld.shared::cluster.v4.s32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(addr));
   return v;
+}
+
+// Named barrier over `count` threads (a multiple of 32).
+__device__ __forceinline__ void named_barrier(uint32_t id, uint32_t count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
 // ---------------------------------------------------------------- PDL

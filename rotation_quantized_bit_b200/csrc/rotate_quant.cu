@@ -8,12 +8,32 @@
 //      group-256 regular-Hadamard rotation, activations rotated online),
 //   3. s = amax / 7 over the row (dynamic per-token INT4, same paragraph),
 //   4. q = clamp(rint(x' / s), -8, 7) and write the codes.
-// Bit-exact contract: the butterflies use the fixed stage order (stride 1, 4,
-// 16, 64) and association (p=a+b, q=a-b, r=c+d, t=c-d -> p+t, p-t, q+r, r-q)
-// with explicitly rounded adds (no contraction), the 1/16 is one multiply,
-// the quotient is a correctly rounded IEEE division and rint is round half to
-// even -- the same operations in the same order as any plain fp32 evaluation
-// of the definition, so the codes and scales are identical bit for bit.
+//
+// Bit-exact contract.  The butterflies use the fixed stage order (stride 1,
+// 4, 16, 64) and association (p=a+b, q=a-b, r=c+d, t=c-d -> p+t, p-t, q+r,
+// r-q), every add is a correctly rounded fp32 add (packed f32x2 or scalar, no
+// contraction), the 1/16 is one multiply, the scale is an IEEE division, and
+// each code equals rint(fl(x' / s)) with ties to even, so codes and scales are
+// identical bit for bit to any plain fp32 evaluation of that definition.
+//
+// Layout.  A lane owns one half (128 channels) of a 256-channel group and
+// keeps it in registers as 64 fp32 pairs; pair i holds channels i and i + 64
+// of the half, so the radix-4 stages on channel bits (0,1), (2,3), (4,5) are
+// packed f32x2 butterflies, and the stage on bits (6,7) combines the two
+// members of a pair and the two halves held by the lane pair (lane ^ 1), one
+// shuffle per two channels.  Input is staged through shared memory: a warp
+// copies its 8 KB tile (16 groups) with coalesced 16-byte cp.async into
+// XOR-swizzled slots, so both the copy and each lane's 16 reads of its own
+// 256 bytes are free of bank conflicts.  The next row block is prefetched
+// while the current one is computed.  Codes leave through the same buffer
+// and coalesced 16-byte stores.
+//
+// Quantization.  y = x' * rcp(s) (rcp correctly rounded), then rint via the
+// addition of 1.5 * 2^23, whose low byte is the two's-complement code.  For
+// |y| < 8, y and the correctly rounded quotient differ by less than 2^-19.8,
+// so the codes agree unless some |y - rint(y)| lies within 2^-19 of one half;
+// a lane that sees such a value (or a row whose scale is subnormal or zero)
+// recomputes its codes with the correctly rounded division.
 #include <cuda_runtime.h>
 
 #include <cstdint>
@@ -24,99 +44,290 @@ namespace convrot {
 
 namespace {
 
-constexpr int kThreads = 256;
+typedef unsigned long long u64;
 
-__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
-__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+constexpr int kTileBytes = 8192;          // 16 groups x 256 bf16 per warp
+constexpr int kMaxWarps = 8;              // at most 128 groups per row block
+constexpr float kMagic = 12582912.0f;     // 1.5 * 2^23: x + kMagic rounds x to an integer, ties to even
+constexpr float kTieGuard = 0.5f - 1.0f / 524288.0f;  // 0.5 - 2^-19
+constexpr float kMinNormal = 1.17549435e-38f;         // 2^-126
 
-// One block rotates and quantizes one row at a time, holding the row in
-// shared memory as fp32.
-__global__ void __launch_bounds__(kThreads) rotate_quant_kernel(const uint16_t* __restrict__ x, int M, int K,
-                                                                RotateQuantOut out) {
-  extern __shared__ float row[];  // K floats
-  __shared__ float red_f[kThreads / 32];
-  const int tid = threadIdx.x;
-  const int lane = tid & 31, warp = tid >> 5;
-  const int nchunk = K >> 3;  // 8-element chunks
-  const int nbfly = K >> 2;   // radix-4 butterflies per stage
+// ---------------------------------------------------------------- helpers
 
-  for (int m = blockIdx.x; m < M; m += gridDim.x) {
-    const uint4* src = reinterpret_cast<const uint4*>(x + static_cast<size_t>(m) * K);
-    for (int c = tid; c < nchunk; c += kThreads) {
-      uint4 v = __ldg(src + c);
-      float* d = row + 8 * c;
-      d[0] = bf16_lo(v.x); d[1] = bf16_hi(v.x);
-      d[2] = bf16_lo(v.y); d[3] = bf16_hi(v.y);
-      d[4] = bf16_lo(v.z); d[5] = bf16_hi(v.z);
-      d[6] = bf16_lo(v.w); d[7] = bf16_hi(v.w);
-    }
-    // Four radix-4 stages; stage s pairs indices that differ only in base-4
-    // digit s (stride 4^s).
+__device__ __forceinline__ u64 f2(float lo, float hi) {
+  u64 d;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(d) : "f"(lo), "f"(hi));
+  return d;
+}
+__device__ __forceinline__ void f2_split(u64 v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ u64 f2_add(u64 a, u64 b) {
+  u64 d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ u64 f2_sub(u64 a, u64 b) {
+  u64 d;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ u64 f2_mul(u64 a, u64 b) {
+  u64 d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// One radix-4 butterfly on packed pairs: (a,b,c,d) -> (p+t, p-t, q+r, r-q).
+__device__ __forceinline__ void bfly4(u64& a, u64& b, u64& c, u64& d) {
+  const u64 p = f2_add(a, b), q = f2_sub(a, b), r = f2_add(c, d), t = f2_sub(c, d);
+  a = f2_add(p, t);
+  b = f2_sub(p, t);
+  c = f2_add(q, r);
+  d = f2_sub(r, q);
+}
+
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, bool valid) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(valid ? 16 : 0) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+// Byte 0 of four words -> one word (the code bytes of four rounded floats).
+__device__ __forceinline__ uint32_t gather_b0(uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  const uint32_t ab = __byte_perm(a, b, 0x0040);  // [a0, b0, .., ..]
+  const uint32_t cd = __byte_perm(c, d, 0x0040);  // [c0, d0, .., ..]
+  return __byte_perm(ab, cd, 0x5410);             // [a0, b0, c0, d0]
+}
+
+// Eight codes as bytes (natural order, two words) -> packed nibbles, even index low.
+__device__ __forceinline__ uint32_t pack_nibbles(uint32_t lo4, uint32_t hi4) {
+  const uint32_t a = lo4 & 0x0F0F0F0Fu, b = hi4 & 0x0F0F0F0Fu;
+  const uint32_t a2 = a | (a >> 4), b2 = b | (b >> 4);  // bytes 0 and 2 hold two codes each
+  return __byte_perm(a2, b2, 0x6420);
+}
+
+// Sixteen codes of two chunks (8 + 8, natural order) -> staging.  s8 layout:
+// per chunk the operand order (0,2,4,6,1,3,5,7), 16 bytes per chunk pair in
+// slot (pair ^ (region & 7)) of the lane's 128-byte region.  Packed layout: 4
+// bytes per chunk, 8 bytes per chunk pair, at region * 64 + 8 * pair.
+template <bool PACKED>
+__device__ __forceinline__ void stage_chunk_pair(uint8_t* stage, int region, int pair, const uint32_t (&c)[16]) {
+  if (PACKED) {
+    const uint32_t w0 = pack_nibbles(gather_b0(c[0], c[1], c[2], c[3]), gather_b0(c[4], c[5], c[6], c[7]));
+    const uint32_t w1 = pack_nibbles(gather_b0(c[8], c[9], c[10], c[11]), gather_b0(c[12], c[13], c[14], c[15]));
+    *reinterpret_cast<uint2*>(stage + 64 * region + 8 * pair) = make_uint2(w0, w1);
+  } else {
+    uint4 o;
+    o.x = gather_b0(c[0], c[2], c[4], c[6]);
+    o.y = gather_b0(c[1], c[3], c[5], c[7]);
+    o.z = gather_b0(c[8], c[10], c[12], c[14]);
+    o.w = gather_b0(c[9], c[11], c[13], c[15]);
+    *reinterpret_cast<uint4*>(stage + 128 * region + 16 * (pair ^ (region & 7))) = o;
+  }
+}
+
+struct RQParams {
+  const uint16_t* x;
+  int M, K;
+  int G;        // groups of 256 per row
+  int R;        // rows per block
+  int nblocks;  // ceil(M / R)
+  RotateQuantOut out;
+};
+
+// Shared-memory slot of logical 16-byte chunk c = 16 * region + k of the input
+// tile: k XOR the region's low three bits.
+__device__ __forceinline__ int in_slot(int c) { return (c & ~15) | ((c & 15) ^ ((c >> 4) & 7)); }
+
+template <bool PACKED>
+__global__ void __launch_bounds__(kMaxWarps * 32, 1) rotate_quant_kernel(const __grid_constant__ RQParams p) {
+  extern __shared__ __align__(16) uint8_t smem[];
+  __shared__ uint32_t row_amax[2][128];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  uint8_t* const wbuf0 = smem + (2 * warp) * kTileBytes;
+  uint8_t* const wbuf1 = smem + (2 * warp + 1) * kTileBytes;
+  const int groups_per_block = p.R * p.G;
+  const size_t row_bytes = static_cast<size_t>(p.K) * 2;
+  const size_t total_bytes = static_cast<size_t>(p.M) * row_bytes;
+  const uint8_t* xb = reinterpret_cast<const uint8_t*>(p.x);
+
+  // Coalesced copy of this warp's tile of row block b into buffer `buf`.
+  auto prefetch = [&](int b, int buf) {
+    const size_t base = static_cast<size_t>(b) * p.R * row_bytes + static_cast<size_t>(warp) * kTileBytes;
+    const size_t block_end = min(static_cast<size_t>(b + 1) * p.R * row_bytes, total_bytes);
+    const uint32_t s0 = smem_addr(buf ? wbuf1 : wbuf0);
 #pragma unroll
-    for (int s = 0; s < 4; ++s) {
-      __syncthreads();
+    for (int i = 0; i < kTileBytes / 512; ++i) {
+      const int c = 32 * i + lane;
+      const size_t g = base + 16 * static_cast<size_t>(c);
+      const bool valid = g < block_end;
+      cp_async16(s0 + 16 * in_slot(c), valid ? xb + g : xb, valid);
+    }
+    cp_async_commit();
+  };
+
+  for (int i = threadIdx.x; i < 2 * 128; i += blockDim.x) (&row_amax[0][0])[i] = 0u;
+  __syncthreads();
+
+  int it = 0;
+  if (static_cast<int>(blockIdx.x) < p.nblocks) prefetch(blockIdx.x, 0);
+  for (int b = blockIdx.x; b < p.nblocks; b += gridDim.x, ++it) {
+    const int buf = it & 1;
+    uint8_t* const tile = buf ? wbuf1 : wbuf0;
+    uint32_t* const amax_slot = row_amax[it & 1];
+    const int nb = b + gridDim.x;
+    if (nb < p.nblocks) {
+      prefetch(nb, buf ^ 1);
+      cp_async_wait<1>();
+    } else {
+      cp_async_wait<0>();
+    }
+    __syncwarp();
+
+    // This lane's half-group.
+    const int f = 16 * warp + (lane >> 1);  // group index within the block
+    const int h = lane & 1;                 // which half of the group
+    const bool active = f < groups_per_block;
+    const int rloc = active ? f / p.G : 0;
+    const int row = b * p.R + rloc;
+    const bool live = active && row < p.M;
+
+    // ---- 128 bf16 -> 64 fp32 pairs: pair i = (channel i, channel i + 64)
+    u64 P[64];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const uint4 lo = *reinterpret_cast<const uint4*>(tile + 16 * ((lane << 4) | (k ^ (lane & 7))));
+      const uint4 hi = *reinterpret_cast<const uint4*>(tile + 16 * ((lane << 4) | ((k + 8) ^ (lane & 7))));
+      const uint32_t w0[4] = {lo.x, lo.y, lo.z, lo.w};
+      const uint32_t w1[4] = {hi.x, hi.y, hi.z, hi.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        P[8 * k + 2 * e] = f2(__uint_as_float(w0[e] << 16), __uint_as_float(w1[e] << 16));
+        P[8 * k + 2 * e + 1] = f2(__uint_as_float(w0[e] & 0xFFFF0000u), __uint_as_float(w1[e] & 0xFFFF0000u));
+      }
+    }
+    __syncwarp();  // the tile buffer becomes the output staging area below
+
+    // ---- rotation: stages on channel bits (0,1), (2,3), (4,5), packed
+#pragma unroll
+    for (int s = 0; s < 3; ++s) {
       const int st = 1 << (2 * s);
-      for (int b = tid; b < nbfly; b += kThreads) {
-        const int g = b >> 6, li = b & 63;
-        const int low = li & (st - 1);
-        const int high = li >> (2 * s);
-        const int i = g * 256 + ((high << (2 * s + 2)) | low);
-        const float a = row[i], bb = row[i + st], c = row[i + 2 * st], d = row[i + 3 * st];
-        const float p = __fadd_rn(a, bb), q = __fsub_rn(a, bb), r = __fadd_rn(c, d), t = __fsub_rn(c, d);
-        row[i] = __fadd_rn(p, t);
-        row[i + st] = __fsub_rn(p, t);
-        row[i + 2 * st] = __fadd_rn(q, r);
-        row[i + 3 * st] = __fsub_rn(r, q);
-      }
-    }
-    __syncthreads();
-    float amax = 0.0f;
-    for (int k = tid; k < K; k += kThreads) {
-      const float v = __fmul_rn(row[k], 0.0625f);
-      row[k] = v;
-      amax = fmaxf(amax, fabsf(v));
-    }
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-    if (lane == 0) red_f[warp] = amax;
-    __syncthreads();
-    if (tid < 32) {
-      float v = tid < kThreads / 32 ? red_f[tid] : 0.0f;
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-      if (tid == 0) red_f[0] = v;
+      for (int i = 0; i < 64; ++i)
+        if (((i >> (2 * s)) & 3) == 0) bfly4(P[i], P[i + st], P[i + 2 * st], P[i + 3 * st]);
     }
+    // stage on bits (6,7): bit 6 within the pair, bit 7 across the lane pair.
+    // Lane h=0 holds (a, b), lane h=1 holds (c, d); u = own sum, w = own
+    // difference; the partner's w completes (p+t, p-t) resp. (q+r, r-q).
+#pragma unroll
+    for (int i = 0; i < 64; ++i) {
+      float a, c;
+      f2_split(P[i], a, c);
+      const float u = __fadd_rn(a, c), w = __fsub_rn(a, c);
+      const float r = __shfl_xor_sync(0xffffffffu, w, 1);
+      P[i] = f2(__fadd_rn(u, r), __fsub_rn(u, r));
+    }
+    // x' = v * 1/16, and the lane's amax
+    const u64 sixteenth = f2(0.0625f, 0.0625f);
+    float m = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 64; ++i) {
+      P[i] = f2_mul(P[i], sixteenth);
+      float a, c;
+      f2_split(P[i], a, c);
+      m = max3(m, fabsf(a), fabsf(c));
+    }
+    if (live) atomicMax(&amax_slot[rloc], __float_as_uint(m));
     __syncthreads();
-    const float scale = __fdiv_rn(red_f[0], 7.0f);
-    if (tid == 0) out.scale[m] = scale;
+    const float scale = __fdiv_rn(__uint_as_float(amax_slot[rloc]), 7.0f);
+    // The other slot is free now (its last readers finished before this
+    // barrier): clear it for the next block.
+    if (static_cast<int>(threadIdx.x) < 128) row_amax[(it + 1) & 1][threadIdx.x] = 0u;
 
-    for (int c = tid; c < nchunk; c += kThreads) {
-      int q[8];
+    // ---- quantize into the staging area (region `lane` of `tile`)
+    const bool fast = scale >= kMinNormal;
+    float emax = 0.0f;
+    if (fast) {
+      const float rcp = __frcp_rn(scale);
+      const u64 rr = f2(rcp, rcp), mg = f2(kMagic, kMagic);
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        int v = 0;
-        if (scale != 0.0f) {
-          v = __float2int_rn(__fdiv_rn(row[8 * c + j], scale));
-          v = min(7, max(-8, v));
+      for (int k = 0; k < 8; k += 2) {
+        // pairs 8k .. 8k+15 hold chunks k, k+1 (.x) and k+8, k+9 (.y)
+        uint32_t cx[16], cy[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const u64 y = f2_mul(P[8 * k + e], rr);
+          const u64 t = f2_add(y, mg);
+          const u64 d = f2_sub(y, f2_sub(t, mg));  // y - rint(y), exact
+          float tx, ty, dx, dy;
+          f2_split(t, tx, ty);
+          f2_split(d, dx, dy);
+          emax = max3(emax, fabsf(dx), fabsf(dy));
+          cx[e] = __float_as_uint(tx);
+          cy[e] = __float_as_uint(ty);
         }
-        q[j] = v;
-      }
-      if (out.packed) {
-        uint32_t w = 0;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) w |= (static_cast<uint32_t>(q[j]) & 0xFu) << (4 * j);
-        reinterpret_cast<uint32_t*>(out.packed + static_cast<size_t>(m) * (K >> 1))[c] = w;
-      }
-      if (out.s8) {
-        uint2 w;
-        w.x = (static_cast<uint32_t>(q[0]) & 0xFFu) | ((static_cast<uint32_t>(q[2]) & 0xFFu) << 8) |
-              ((static_cast<uint32_t>(q[4]) & 0xFFu) << 16) | ((static_cast<uint32_t>(q[6]) & 0xFFu) << 24);
-        w.y = (static_cast<uint32_t>(q[1]) & 0xFFu) | ((static_cast<uint32_t>(q[3]) & 0xFFu) << 8) |
-              ((static_cast<uint32_t>(q[5]) & 0xFFu) << 16) | ((static_cast<uint32_t>(q[7]) & 0xFFu) << 24);
-        reinterpret_cast<uint2*>(out.s8 + static_cast<size_t>(m) * K)[c] = w;
+        stage_chunk_pair<PACKED>(tile, lane, k >> 1, cx);
+        stage_chunk_pair<PACKED>(tile, lane, (k + 8) >> 1, cy);
       }
     }
-    __syncthreads();
+    if (!fast || emax >= kTieGuard) {
+      // Exact path: a zero or subnormal scale, or a value next to a tie.
+#pragma unroll
+      for (int k = 0; k < 8; k += 2) {
+        uint32_t cx[16], cy[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          float a, c;
+          f2_split(P[8 * k + e], a, c);
+          int qa = 0, qc = 0;
+          if (scale != 0.0f) {
+            qa = min(7, max(-8, __float2int_rn(__fdiv_rn(a, scale))));
+            qc = min(7, max(-8, __float2int_rn(__fdiv_rn(c, scale))));
+          }
+          cx[e] = static_cast<uint32_t>(qa);
+          cy[e] = static_cast<uint32_t>(qc);
+        }
+        stage_chunk_pair<PACKED>(tile, lane, k >> 1, cx);
+        stage_chunk_pair<PACKED>(tile, lane, (k + 8) >> 1, cy);
+      }
+    }
+    if (live && h == 0 && f % p.G == 0) p.out.scale[row] = scale;
+    __syncwarp();
+
+    // ---- coalesced copy-out of the warp's codes (16 groups x 256 codes)
+    {
+      constexpr int kOutTile = kTileBytes / (PACKED ? 4 : 2);  // 2 KB packed, 4 KB as bytes
+      const size_t code_row = PACKED ? static_cast<size_t>(p.K) / 2 : static_cast<size_t>(p.K);
+      const size_t block_end = min(static_cast<size_t>(b + 1) * p.R * code_row, static_cast<size_t>(p.M) * code_row);
+      const size_t base = static_cast<size_t>(b) * p.R * code_row + static_cast<size_t>(warp) * kOutTile;
+      uint8_t* dst = PACKED ? p.out.packed : reinterpret_cast<uint8_t*>(p.out.s8);
+#pragma unroll
+      for (int i = 0; i < kOutTile / 512; ++i) {
+        const int c = 32 * i + lane;
+        uint4 v;
+        if (PACKED) {
+          v = *reinterpret_cast<const uint4*>(tile + 16 * c);
+        } else {
+          const int region = c >> 3, k = c & 7;
+          v = *reinterpret_cast<const uint4*>(tile + 128 * region + 16 * (k ^ (region & 7)));
+        }
+        const size_t g = base + 16 * static_cast<size_t>(c);
+        if (g < block_end) *reinterpret_cast<uint4*>(dst + g) = v;
+      }
+    }
+    __syncwarp();
   }
 }
 
@@ -124,10 +335,10 @@ __global__ void __launch_bounds__(kThreads) rotate_quant_kernel(const uint16_t* 
 // index in the low nibble); its low nibbles are codes (0,2,4,6) and its high
 // nibbles (1,3,5,7).  u = nibble ^ 8 = q + 8 in [0, 15]; the signed byte is
 // (u + 0x78) ^ 0x80 = u - 8 (mod 256), with no carry between bytes.
-__global__ void __launch_bounds__(kThreads) unpack_codes_kernel(const uint8_t* __restrict__ packed, int M, int K,
-                                                                int8_t* __restrict__ s8) {
+__global__ void __launch_bounds__(256) unpack_codes_kernel(const uint8_t* __restrict__ packed, int M, int K,
+                                                           int8_t* __restrict__ s8) {
   const int lane = threadIdx.x & 31;
-  const int warps_per_block = kThreads / 32;
+  const int warps_per_block = blockDim.x / 32;
   const int nword = K >> 3;
   for (int m = blockIdx.x * warps_per_block + (threadIdx.x >> 5); m < M; m += gridDim.x * warps_per_block) {
     const uint32_t* src = reinterpret_cast<const uint32_t*>(packed + static_cast<size_t>(m) * (K >> 1));
@@ -142,35 +353,61 @@ __global__ void __launch_bounds__(kThreads) unpack_codes_kernel(const uint8_t* _
 }
 
 int num_sms_cached() {
-  static int n = 0;
-  if (n == 0) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    if (n <= 0) n = 148;
+  static int n[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) dev = 0;
+  if (n[dev] == 0) {
+    cudaDeviceGetAttribute(&n[dev], cudaDevAttrMultiProcessorCount, dev);
+    if (n[dev] <= 0) n[dev] = 148;
   }
-  return n;
+  return n[dev];
 }
 
 }  // namespace
 
 cudaError_t launch_rotate_quant(const uint16_t* x, int M, int K, RotateQuantOut out, cudaStream_t stream) {
-  const int smem = K * static_cast<int>(sizeof(float));
-  static int cache[64] = {0};
-  cudaError_t e = ensure_dynamic_smem(reinterpret_cast<const void*>(rotate_quant_kernel), smem, cache);
+  RQParams p{};
+  p.x = x;
+  p.M = M;
+  p.K = K;
+  p.G = K / 256;
+  // Rows per block: at most 128 groups (8 warps) per block, and few enough
+  // rows that every SM gets about two blocks.
+  const int sms = num_sms_cached();
+  int R = 128 / p.G;
+  const int spread = M / (2 * sms);
+  if (spread < R) R = spread < 1 ? 1 : spread;
+  p.R = R;
+  p.nblocks = (M + R - 1) / R;
+  p.out = out;
+  const int warps = (R * p.G + 15) / 16;
+  const int smem = warps * 2 * kTileBytes;
+  const bool packed = out.packed != nullptr;
+  const void* kfn = packed ? reinterpret_cast<const void*>(rotate_quant_kernel<true>)
+                           : reinterpret_cast<const void*>(rotate_quant_kernel<false>);
+  static int cache_packed[64] = {0}, cache_s8[64] = {0};
+  cudaError_t e = ensure_dynamic_smem(kfn, smem, packed ? cache_packed : cache_s8);
   if (e != cudaSuccess) return note_cuda(e, "rotate_quant: dynamic shared memory attribute");
-  int grid = num_sms_cached() * 4;
-  if (grid > M) grid = M;
-  rotate_quant_kernel<<<grid, kThreads, smem, stream>>>(x, M, K, out);
+  int per_sm = 0;
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kfn, warps * 32, smem);
+  if (e != cudaSuccess) return note_cuda(e, "rotate_quant: occupancy query");
+  if (per_sm < 1) per_sm = 1;
+  int grid = sms * per_sm;
+  if (grid > p.nblocks) grid = p.nblocks;
+  if (packed)
+    rotate_quant_kernel<true><<<grid, warps * 32, smem, stream>>>(p);
+  else
+    rotate_quant_kernel<false><<<grid, warps * 32, smem, stream>>>(p);
   count_dispatch(0);
   return note_cuda(cudaGetLastError(), "rotate_quant: launch");
 }
 
 cudaError_t launch_unpack_codes(const uint8_t* packed, int M, int K, int8_t* s8, cudaStream_t stream) {
-  const int per_block = kThreads / 32;
+  const int per_block = 8;
   int grid = (M + per_block - 1) / per_block;
   if (grid > num_sms_cached() * 8) grid = num_sms_cached() * 8;
-  unpack_codes_kernel<<<grid, kThreads, 0, stream>>>(packed, M, K, s8);
+  unpack_codes_kernel<<<grid, 256, 0, stream>>>(packed, M, K, s8);
   count_dispatch(1);
   return note_cuda(cudaGetLastError(), "unpack_codes: launch");
 }

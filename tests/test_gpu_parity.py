@@ -73,9 +73,21 @@ def special_rows(K=512):
         r = z.copy(); r[0] = A; r[256] = B; rows.append(r)
     r = z.copy(); r[:] = 3.0; rows.append(r)                 # constant vector
     r = z.copy(); r[5] = -1e-38; r[300] = 3e-39; rows.append(r)  # subnormal scale
-    r = z.copy(); r[7] = 3.0e38; r[8] = -2.5e38; rows.append(r)  # huge values
+    r = z.copy(); r[7] = 1.0e37; r[8] = -8.0e36; rows.append(r)  # huge values, partial sums stay finite
     r = z.copy(); r[::3] = 1e-30; rows.append(r)             # tiny values
     return synthetic.to_bf16_bits(np.stack(rows))
+
+
+@pytest.mark.parametrize("M", [1, 7, 77, 300, 1220])
+@pytest.mark.parametrize("K", [256, 512, 2560, 3072, 3840, 9728, 12288, 32768])
+def test_rotate_quant_shape_grid(rq, M, K):
+    if M * K > 1220 * 12288:
+        pytest.skip("keeps the CPU oracle within seconds")
+    x = synthetic.activations("qwen3_4b", M, K, seed_extra=K)
+    xq_ref, s_ref = oracle.rotate_quant(x)
+    xq, s = rq.convrot_rotate_quant(dev_bf16(x))
+    assert np.array_equal(f32_bits(host(s)), f32_bits(s_ref))
+    assert np.array_equal(host(xq), xq_ref)
 
 
 def test_rotate_quant_special_rows(rq):
@@ -160,6 +172,18 @@ def test_linear_matches_oracle(rq, workload, M, K, N):
     assert np.array_equal(f32_bits(y32), f32_bits(y32_ref))
     y16 = host_bits(rq.convrot_w4a4_linear(dx, dwq, dsw, db))
     assert bf16_ulp_diff(y16, y16_ref).max() <= 1
+
+
+def test_linear_special_rows(rq):
+    # Ties, division-vs-reciprocal cases, zero / subnormal / huge rows through
+    # the fused path (its prologue writes byte codes for the GEMM operand).
+    x = special_rows()
+    M, K, N = x.shape[0], x.shape[1], 264
+    w, b = synthetic.weights("qwen3_4b", N, K)
+    wq, s_w = oracle.pack_weight(w)
+    y32_ref, _ = oracle.linear(x, wq, s_w, b, K)
+    y32 = host(rq.convrot_w4a4_linear_f32(dev_bf16(x), dev(wq), dev(s_w), dev_bf16(b)))
+    assert np.array_equal(f32_bits(y32), f32_bits(y32_ref))
 
 
 def sample_rows(M, BT_guess=192):
