@@ -135,6 +135,27 @@ convrot_status_t convrot_w4a4_linear_f32(const uint16_t *x, const uint8_t *Wq, c
                                          const uint16_t *bias, int M, int N, int K, float *y32,
                                          void *workspace, size_t workspace_bytes, void *stream);
 
+/* The fused Linear without a caller-supplied workspace, for callers that
+ * cannot allocate device memory: code running inside a host framework that
+ * owns all device allocations and forbids side allocations, fixed-budget
+ * deployments that must not grow their footprint after start-up, and plugin
+ * or foreign-language callers with no binding to a CUDA allocator.  The pages
+ * have no counterpart of this call; it is a deployment convenience.
+ *   Same arguments and results as convrot_w4a4_linear, minus the workspace.
+ *   Scratch: a static 32 MiB device array inside the library (held by every
+ *   GPU that loads the library until the process exits).  Shapes whose
+ *   convrot_w4a4_workspace_size exceeds 32 MiB return CONVROT_ERR_WORKSPACE
+ *   (convrot_last_error says by how much).  Allocates nothing: no cudaMalloc,
+ *   no cudaFree.
+ *   The first call on each device looks up the array's device address
+ *   (cudaGetSymbolAddress) with that device current; make that first call
+ *   before any stream capture.
+ *   Every call shares the one array and it keeps the last call's contents, so
+ *   calls that overlap on the GPU (e.g. on two streams at once) race. */
+convrot_status_t convrot_w4a4_linear_noalloc(const uint16_t *x, const uint8_t *Wq,
+                                             const float *s_w, const uint16_t *bias, int M,
+                                             int N, int K, uint16_t *y, void *stream);
+
 /* The two launches that make up convrot_w4a4_linear, for callers that want
  * to time or schedule them separately; convrot_w4a4_linear is exactly
  * convrot_w4a4_quantize followed by convrot_w4a4_gemm_quantized on the same

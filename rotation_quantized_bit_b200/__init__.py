@@ -38,7 +38,7 @@ STATUS = {
 EXPORTS = [
     "convrot_status_string", "convrot_pack_weight", "convrot_rotate_quant", "convrot_gemm_workspace_size",
     "w4a4_gemm", "w4a4_gemm_s32", "w4a4_gemm_f32", "convrot_w4a4_workspace_size", "convrot_w4a4_linear",
-    "convrot_w4a4_linear_f32", "convrot_w4a4_quantize", "convrot_w4a4_gemm_quantized", "convrot_device_error",
+    "convrot_w4a4_linear_f32", "convrot_w4a4_linear_noalloc", "convrot_w4a4_quantize", "convrot_w4a4_gemm_quantized", "convrot_device_error",
     "convrot_dispatch_counts", "convrot_last_error", "convrot_version",
 ]
 
@@ -79,6 +79,7 @@ def load_library():
     lib.w4a4_gemm_f32.argtypes = [P, P, P, P, P, I, I, I, P, P, Z, P]
     lib.convrot_w4a4_linear.argtypes = [P, P, P, P, I, I, I, P, P, Z, P]
     lib.convrot_w4a4_linear_f32.argtypes = [P, P, P, P, I, I, I, P, P, Z, P]
+    lib.convrot_w4a4_linear_noalloc.argtypes = [P, P, P, P, I, I, I, P, P]
     lib.convrot_w4a4_quantize.argtypes = [P, I, I, P, Z, P]
     lib.convrot_w4a4_gemm_quantized.argtypes = [P, P, P, I, I, I, P, P, Z, P]
     lib.convrot_device_error.argtypes = [P, ctypes.POINTER(ctypes.c_uint32)]
@@ -92,7 +93,7 @@ def load_library():
 
 def lib_status_fns():
     return ["convrot_pack_weight", "convrot_rotate_quant", "w4a4_gemm", "w4a4_gemm_s32", "w4a4_gemm_f32",
-            "convrot_w4a4_linear", "convrot_w4a4_linear_f32", "convrot_w4a4_quantize",
+            "convrot_w4a4_linear", "convrot_w4a4_linear_f32", "convrot_w4a4_linear_noalloc", "convrot_w4a4_quantize",
             "convrot_w4a4_gemm_quantized", "convrot_device_error"]
 
 
@@ -223,6 +224,28 @@ def convrot_w4a4_linear(x, Wq, s_w, bias=None, out=None, workspace=None, stream=
 
 def convrot_w4a4_linear_f32(x, Wq, s_w, bias=None, out=None, workspace=None, stream=None):
     return _linear("convrot_w4a4_linear_f32", torch.float32, x, Wq, s_w, bias, out, workspace, stream)
+
+
+def convrot_w4a4_linear_noalloc(x, Wq, s_w, bias=None, out=None, stream=None):
+    """The fused Linear using the library's own static scratch instead of a
+    workspace (for callers that cannot allocate device memory; see
+    include/convrot.h).  ``out`` is the caller's; nothing else is allocated by
+    the library.  Shapes needing more than 32 MiB of scratch raise."""
+    M, K = x.shape
+    N = Wq.shape[0]
+    _need(x, "x", torch.bfloat16)
+    _need(Wq, "Wq", torch.uint8, (N, K // 2))
+    _need(s_w, "s_w", torch.float32, (N,))
+    _need(bias, "bias", torch.bfloat16, (N,))
+    out = torch.empty((M, N), dtype=torch.bfloat16, device=x.device) if out is None else out
+    _need(out, "out", torch.bfloat16, (M, N))
+    rc = load_library().convrot_w4a4_linear_noalloc(_ptr(x), _ptr(Wq), _ptr(s_w), _ptr(bias), M, N, K, _ptr(out),
+                                                    _stream(stream))
+    if rc != 0:
+        lib = load_library()
+        raise ConvRotError("convrot_w4a4_linear_noalloc", rc,
+                           lib.convrot_status_string(rc).decode() + f" [{lib.convrot_last_error().decode()}]")
+    return out
 
 
 def convrot_w4a4_quantize(x, workspace, stream=None):
