@@ -235,37 +235,47 @@ def main():
 
     nlin = len(layers)
 
-    def run_step(evs=None):
+    def run_step(evs=None, per_kernel=False):
+        """One step.  With per_kernel, an event sits between the two launches of
+        each linear (which serialises them); otherwise events only bracket each
+        linear, so the GEMM's programmatic launch overlaps the prologue."""
+        cur = torch.cuda.current_stream()  # the capture stream while a graph is being captured
         for i, (s, wq, s_w, bias, y) in enumerate(layers):
             if evs is not None:
-                evs[i][0].record(stream)
+                evs[i][0].record(cur)
             rq.convrot_w4a4_quantize(xs[(s.M, s.K)], ws)
-            if evs is not None:
-                evs[i][1].record(stream)
+            if evs is not None and per_kernel:
+                evs[i][1].record(cur)
             rq.convrot_w4a4_gemm_quantized(ws, s.M, wq, s_w, bias, out=y)
             if evs is not None:
-                evs[i][2].record(stream)
+                evs[i][2].record(cur)
 
     for _ in range(max(args.warmup, 3)):
         flush.zero_()
         run_step()
     torch.cuda.synchronize()
 
-    # One CUDA graph per timed step (each with its own events): a replay runs
-    # the step's launches back to back, with no host gaps between them.
-    # external=True: recorded inside a graph capture these become event-record
-    # nodes that are timestamped on every replay (internal events would only
-    # mark cross-stream dependencies).
-    step_events = [[[torch.cuda.Event(enable_timing=True, external=True) for _ in range(3)] for _ in range(nlin)]
-                   for _ in range(args.steps)]
-    graphs = []
+    # One CUDA graph per timed step (each with its own events); a replay runs
+    # the step's launches back to back, with no host gaps.  External events:
+    # recorded inside a capture they become event-record nodes timestamped on
+    # every replay.
+    def make_events():
+        return [[[torch.cuda.Event(enable_timing=True, external=True) for _ in range(3)] for _ in range(nlin)]
+                for _ in range(args.steps)]
+
+    step_events, kern_events = make_events(), make_events()
+    graphs, kgraphs = [], []
     if not args.no_graph:
         for k in range(args.steps):
             g = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g):
                 run_step(step_events[k])
             graphs.append(g)
-        for g in graphs[:1]:  # one untimed replay of the captured work
+            g2 = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g2):
+                run_step(kern_events[k], per_kernel=True)
+            kgraphs.append(g2)
+        for g in (graphs[0], kgraphs[0]):  # one untimed replay of each
             flush.zero_()
             g.replay()
         torch.cuda.synchronize()
@@ -289,6 +299,15 @@ def main():
         dist.barrier()
     clocks = sampler.stop() if sampler else None
     counts1 = rq.convrot_dispatch_counts()
+    # Per-kernel breakdown (for the roofline of the dominant kernel): the same
+    # step with the two launches of each linear separated by an event.
+    for k in range(args.steps):
+        flush.zero_()
+        if kgraphs:
+            kgraphs[k].replay()
+        else:
+            run_step(kern_events[k], per_kernel=True)
+    torch.cuda.synchronize()
     err = rq.convrot_device_error()
     if err:
         raise RuntimeError(f"device error word {err:#x}: a bounded wait expired")
@@ -298,15 +317,18 @@ def main():
         launches = (counts1["rotate_quant"] - counts0["rotate_quant"]) + (counts1["tc_gemm"] - counts0["tc_gemm"]) + \
                    (counts1["tc_gemm_splitk"] - counts0["tc_gemm_splitk"])
 
-    # per-linear, per-kernel times (ms), summed over the K steps
+    # per-linear times of the timed steps, and per-kernel times of the breakdown
+    # steps (ms), summed over the K steps
+    t_lin = np.zeros(nlin)
     t_quant = np.zeros(nlin)
     t_gemm = np.zeros(nlin)
     for k in range(args.steps):
         for i in range(nlin):
-            e0, e1, e2 = step_events[k][i]
+            t_lin[i] += step_events[k][i][0].elapsed_time(step_events[k][i][2])
+            e0, e1, e2 = kern_events[k][i]
             t_quant[i] += e0.elapsed_time(e1)
             t_gemm[i] += e1.elapsed_time(e2)
-    total_ms = float(t_quant.sum() + t_gemm.sum())
+    total_ms = float(t_lin.sum())
     if world > 1:
         t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
@@ -323,10 +345,11 @@ def main():
         tq, tg = t_quant[i] / args.steps, t_gemm[i] / args.steps
         op = 2.0 * s.M * s.N * s.K
         gemm_bytes = s.N * s.K // 2 + s.M * s.K + 4 * s.M + 6 * s.N + 2 * s.M * s.N
+        tl = t_lin[i] / args.steps
         detail.append({
             "linear": s.name, "M": s.M, "K": s.K, "N": s.N,
-            "us_total": round((tq + tg) * 1e3, 2), "us_prologue": round(tq * 1e3, 2), "us_gemm": round(tg * 1e3, 2),
-            "tops_fused": round(op / ((tq + tg) * 1e-3) / 1e12, 1),
+            "us_linear": round(tl * 1e3, 2), "us_prologue": round(tq * 1e3, 2), "us_gemm": round(tg * 1e3, 2),
+            "tops_fused": round(op / (tl * 1e-3) / 1e12, 1),
             "gemm_tops": round(op / (tg * 1e-3) / 1e12, 1),
             "gemm_frac_int8_peak": round(op / (tg * 1e-3) / 1e12 / int8_peak, 3),
             "gemm_hbm_gbs": round(gemm_bytes / (tg * 1e-3) / 1e9, 1),
@@ -359,7 +382,7 @@ def main():
     roof["launch"] = f"{s.name} M{s.M} K{s.K} N{s.N}"
     roof["peak_source"] = (f"{peaks['source']} bf16 dense burst {peaks['bf16_tflops']} TFLOP/s x {INT8_PER_BF16} "
                            "(nominal int8:bf16)" if roof["bound"] == "tensor" else f"{peaks['source']} HBM copy")
-    roof["share_of_step"] = tsum / total_ms if world == 1 else None
+    roof["share_of_breakdown"] = float(tsum / (t_quant.sum() + t_gemm.sum()))
     roof["traffic"] = committed_traffic(kname, s)
 
     e2e = None
@@ -379,7 +402,7 @@ def main():
     }
     if rank == 0:
         print(json.dumps(line), flush=True)
-    del graphs
+    del graphs, kgraphs
     if world > 1:
         dist.destroy_process_group()
 

@@ -179,6 +179,15 @@ convrot_status_t convrot_w4a4_gemm_quantized(const uint8_t *Wq, const float *s_w
  * non-zero, CONVROT_OK otherwise. */
 convrot_status_t convrot_device_error(void *stream, uint32_t *code);
 
+/* Exercises the failure path of the bounded device-side waits (the failure
+ * detection described above): launches a one-thread kernel that waits on a
+ * barrier nothing ever arrives at, for at most limit_us microseconds
+ * (1..1000000).  Afterwards convrot_device_error reports CONVROT_ERR_TIMEOUT
+ * (and clears the word).  While the word is set, every later bounded wait
+ * gives up at once, so call convrot_device_error before further work.  Touches
+ * no caller memory; the context stays usable. */
+convrot_status_t convrot_selftest_timeout(unsigned int limit_us, void *stream);
+
 /* Host-side count of how many times each kernel path was enqueued by this
  * process: counts[0] = rotate/quant prologue, [1] = packed-code unpack pass,
  * [2] = tensor-core GEMM without split-K, [3] = tensor-core GEMM with split-K

@@ -39,7 +39,7 @@ EXPORTS = [
     "convrot_status_string", "convrot_pack_weight", "convrot_rotate_quant", "convrot_gemm_workspace_size",
     "w4a4_gemm", "w4a4_gemm_s32", "w4a4_gemm_f32", "convrot_w4a4_workspace_size", "convrot_w4a4_linear",
     "convrot_w4a4_linear_f32", "convrot_w4a4_linear_noalloc", "convrot_w4a4_quantize", "convrot_w4a4_gemm_quantized", "convrot_device_error",
-    "convrot_dispatch_counts", "convrot_last_error", "convrot_version",
+    "convrot_dispatch_counts", "convrot_last_error", "convrot_selftest_timeout", "convrot_version",
 ]
 
 
@@ -83,6 +83,7 @@ def load_library():
     lib.convrot_w4a4_quantize.argtypes = [P, I, I, P, Z, P]
     lib.convrot_w4a4_gemm_quantized.argtypes = [P, P, P, I, I, I, P, P, Z, P]
     lib.convrot_device_error.argtypes = [P, ctypes.POINTER(ctypes.c_uint32)]
+    lib.convrot_selftest_timeout.argtypes = [ctypes.c_uint, P]
     lib.convrot_dispatch_counts.argtypes = [ctypes.POINTER(ctypes.c_uint64), I]
     lib.convrot_dispatch_counts.restype = None
     for name in lib_status_fns():
@@ -94,7 +95,7 @@ def load_library():
 def lib_status_fns():
     return ["convrot_pack_weight", "convrot_rotate_quant", "w4a4_gemm", "w4a4_gemm_s32", "w4a4_gemm_f32",
             "convrot_w4a4_linear", "convrot_w4a4_linear_f32", "convrot_w4a4_linear_noalloc", "convrot_w4a4_quantize",
-            "convrot_w4a4_gemm_quantized", "convrot_device_error"]
+            "convrot_w4a4_gemm_quantized", "convrot_device_error", "convrot_selftest_timeout"]
 
 
 def _check(fn: str, rc: int):
@@ -280,6 +281,11 @@ def convrot_device_error(stream=None) -> int:
     if rc not in (0, 7):
         _check("convrot_device_error", rc)
     return int(code.value)
+
+
+def convrot_selftest_timeout(limit_us: int = 20000, stream=None):
+    """Run the bounded-wait failure path once (see include/convrot.h)."""
+    _check("convrot_selftest_timeout", load_library().convrot_selftest_timeout(int(limit_us), _stream(stream)))
 
 
 def convrot_dispatch_counts():

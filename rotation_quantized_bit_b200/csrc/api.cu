@@ -150,6 +150,23 @@ void count_dispatch(int which) {
 
 namespace {
 thread_local char g_last_error[256] = "";
+
+// One thread waits on an mbarrier that nothing ever arrives at; the bounded
+// wait gives up after limit_ns and records the timeout bit.
+__global__ void selftest_timeout_kernel(unsigned long long limit_ns) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_mbarrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) (void)mbar_wait_for(&bar, 0, limit_ns);
+}
+}  // namespace
+
+cudaError_t launch_selftest_timeout(unsigned int limit_us, cudaStream_t stream) {
+  selftest_timeout_kernel<<<1, 32, 0, stream>>>(static_cast<unsigned long long>(limit_us) * 1000ull);
+  return note_cuda(cudaGetLastError(), "selftest_timeout: launch");
 }
 
 cudaError_t note_cuda(cudaError_t e, const char* where) {
@@ -266,6 +283,13 @@ convrot_status_t convrot_w4a4_gemm_quantized(const uint8_t* Wq, const float* s_w
                                              int K, uint16_t* y, const void* workspace, size_t workspace_bytes,
                                              void* stream) {
   return gemm_quantized_common(Wq, s_w, bias, M, N, K, y, GemmSink::kBF16, workspace, workspace_bytes, stream);
+}
+
+convrot_status_t convrot_selftest_timeout(unsigned int limit_us, void* stream) {
+  if (limit_us == 0 || limit_us > 1000000u) return CONVROT_ERR_SHAPE;
+  convrot_status_t st = check_device(nullptr);
+  if (st != CONVROT_OK) return st;
+  return from_cuda(launch_selftest_timeout(limit_us, static_cast<cudaStream_t>(stream)));
 }
 
 convrot_status_t convrot_device_error(void* stream, uint32_t* code) {

@@ -85,8 +85,8 @@ __device__ __forceinline__ void unpack_row_to_tmem(const uint8_t* wstage, int ro
 
 // One output element from the MMA sum (16 * acc): scales and bias already
 // loaded by the caller.
-template <int SINK>
-__device__ __forceinline__ void store_output(const Params& p, int m, int n, int32_t dsum, float sa, float sw,
+template <int SINK, class P>
+__device__ __forceinline__ void store_output(const P& p, int m, int n, int32_t dsum, float sa, float sw,
                                              float bv) {
   const int32_t acc = dsum >> 4;  // the weights entered the MMA as 16 * q_w
   const size_t idx = static_cast<size_t>(m) * p.N + n;
@@ -115,7 +115,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   SharedHeader* hdr = reinterpret_cast<SharedHeader*>(smem + p.nstages * stage_bytes);
   float* sa_tile = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(hdr) + 1024);   // s_a of the BT tokens
   int32_t* red = reinterpret_cast<int32_t*>(reinterpret_cast<uint8_t*>(hdr) + 2048);  // split-K partials
-  const int red_pitch = BT + 4;  // int32 per partial-tile row (16-byte rows, bank-conflict free)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n0 = blockIdx.x * kRows;
@@ -155,8 +154,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------ TMA producer
     if (lane == 0) {
       const uint32_t bytes = static_cast<uint32_t>(stage_bytes);
-      int issued = 0;
-      for (int i = 0; i < nkb; ++i) {
+      // The weights do not depend on the preceding prologue kernel: the first
+      // stages' weight tiles are requested before waiting for it.
+      const int prime = nkb < ns ? nkb : ns;
+      for (int i = 0; i < prime; ++i) {
+        mbar_arrive_expect_tx(&hdr->full[i], bytes);
+        tma_load_2d(smem + i * stage_bytes, &tm_w, &hdr->full[i], (kb0 + i) * (kKB / 2), n0);
+      }
+      pdl_wait();
+      for (int i = 0; i < prime; ++i)
+        tma_load_2d(smem + i * stage_bytes + kWTileBytes, &tm_x, &hdr->full[i], (kb0 + i) * kKB, m0);
+      int issued = prime;
+      for (int i = prime; i < nkb; ++i) {
         const int s = i % ns;
         if (i >= ns && !mbar_wait(&hdr->empty[s], ((i / ns) - 1) & 1)) break;
         uint8_t* st = smem + s * stage_bytes;
@@ -196,9 +205,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int row = quad * 32 + lane;
     const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
     const int et = threadIdx.x - 64;  // 0..127 over the four unpack/epilogue warps
-    if (SINK != static_cast<int>(GemmSink::kS32)) {
-      for (int c = et; c < BT; c += 128) sa_tile[c] = (m0 + c < p.M) ? __ldg(p.s_a + m0 + c) : 0.0f;
-    }
     bool ok = true;
     for (int i = 0; i < nkb; ++i) {
       const int s = i % ns, a = i % kASlots;
@@ -214,6 +220,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive(&hdr->empty[s]);
         mbar_arrive(&hdr->a_full[a]);
       }
+    }
+    pdl_wait();  // s_a comes from the preceding prologue kernel
+    if (SINK != static_cast<int>(GemmSink::kS32)) {
+      for (int c = et; c < BT; c += 128) sa_tile[c] = (m0 + c < p.M) ? __ldg(p.s_a + m0 + c) : 0.0f;
     }
     if (ok) ok = mbar_wait(&hdr->acc_full, 0);
     ok = __all_sync(0xffffffffu, ok);  // tcgen05.ld below is warp-collective
@@ -239,7 +249,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     } else {
-      // Partial tile -> own shared memory, row-major [128][BT + 4].
+      // Push the partial tile to its owners.  4-token group g belongs to CTA
+      // g % S of the cluster, which keeps the partials of its groups in slots
+      // [source rank][g / S][row] (16 bytes each); the stores are
+      // fire-and-forget and become visible at the cluster barrier.
+      const int S = p.splits;
+      const int ngl = (BT / 4 + S - 1) / S;
+      const uint32_t me = cluster_ctarank();
+      const uint32_t red_base = smem_u32(red);
       for (int c = 0; c < BT; c += 16) {
         uint32_t v[16];
         tmem_ld_32x32b_x16(tmem + lane_base + static_cast<uint32_t>(c), v);
@@ -247,10 +264,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         const bool keep = ok && nkb > 0;
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-          int4 w = keep ? make_int4(static_cast<int32_t>(v[4 * q]), static_cast<int32_t>(v[4 * q + 1]),
-                                    static_cast<int32_t>(v[4 * q + 2]), static_cast<int32_t>(v[4 * q + 3]))
-                        : make_int4(0, 0, 0, 0);
-          *reinterpret_cast<int4*>(red + row * red_pitch + c + 4 * q) = w;
+          const int g = c / 4 + q;
+          const int4 w = keep ? make_int4(static_cast<int32_t>(v[4 * q]), static_cast<int32_t>(v[4 * q + 1]),
+                                          static_cast<int32_t>(v[4 * q + 2]), static_cast<int32_t>(v[4 * q + 3]))
+                              : make_int4(0, 0, 0, 0);
+          const uint32_t slot = ((static_cast<uint32_t>(me) * ngl + static_cast<uint32_t>(g / S)) * kRows + row) * 16u;
+          st_shared_cluster_v4(map_shared_rank(red_base + slot, static_cast<uint32_t>(g % S)), w);
         }
       }
     }
@@ -258,30 +277,28 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (p.splits > 1) {
     __syncwarp();    // the cluster barrier below is .aligned: reconverge first
-    cluster_sync();  // every CTA of the cluster has its partial tile in shared memory
+    cluster_sync();  // every partial has reached its owner's shared memory
     if (warp >= 2) {
-      // CTA `rank` finishes the 4-token groups g = rank, rank + S, ... of the
-      // tile: all S partials of a group are loaded (16 bytes each) before
-      // they are summed, so the remote loads overlap.
+      // This CTA sums, from its own shared memory, the S partials of the
+      // groups it owns and writes their outputs.  No CTA touches another's
+      // shared memory after the barrier, so none has to wait before exiting.
+      const int S = p.splits;
+      const int ngl = (BT / 4 + S - 1) / S;
       const int quad = warp & 3;
       const int row = quad * 32 + lane;
       const int n = n0 + row;
-      const uint32_t rank = cluster_ctarank();
+      const int rank = static_cast<int>(cluster_ctarank());
       const float sw = (SINK != static_cast<int>(GemmSink::kS32) && n < p.N) ? __ldg(p.s_w + n) : 0.0f;
       const float bv = (p.bias && n < p.N) ? __uint_as_float(static_cast<uint32_t>(__ldg(p.bias + n)) << 16) : 0.0f;
-      const uint32_t row_addr = smem_u32(red + row * red_pitch);
-      for (int g = static_cast<int>(rank); g < BT / 4; g += p.splits) {
-        if (m0 + 4 * g >= p.M || n >= p.N) continue;
-        int4 part[8];
-#pragma unroll
-        for (int j = 0; j < 8; ++j)
-          if (j < p.splits) part[j] = ld_shared_cluster_v4(map_shared_rank(row_addr + 16u * g, static_cast<uint32_t>(j)));
+      const int4* red4 = reinterpret_cast<const int4*>(red);
+      for (int gl = 0; gl < ngl; ++gl) {
+        const int g = gl * S + rank;
+        if (g >= BT / 4 || m0 + 4 * g >= p.M || n >= p.N) continue;
         int4 sum = make_int4(0, 0, 0, 0);
-#pragma unroll
-        for (int j = 0; j < 8; ++j)
-          if (j < p.splits) {
-            sum.x += part[j].x; sum.y += part[j].y; sum.z += part[j].z; sum.w += part[j].w;
-          }
+        for (int j = 0; j < S; ++j) {
+          const int4 v = red4[(j * ngl + gl) * kRows + row];
+          sum.x += v.x; sum.y += v.y; sum.z += v.z; sum.w += v.w;
+        }
         const int32_t sv[4] = {sum.x, sum.y, sum.z, sum.w};
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
@@ -290,8 +307,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
-    __syncwarp();
-    cluster_sync();  // nobody leaves while a peer still reads its shared memory
   }
 
   tc_fence_before();
@@ -300,6 +315,228 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem, static_cast<uint32_t>(p.tmem_cols));
+  }
+}
+
+
+// ---------------------------------------------------------------- persistent kernel (large M)
+//
+// One CTA per SM walks the output tiles (tile t -> m tile t % m_tiles, n tile
+// t / m_tiles) with a k-block stream that does not drain between tiles:
+//   warp 0      TMA producer (ring of `nstages` shared-memory stages)
+//   warp 1      TMEM allocation (all 512 columns) and the MMA-issuing thread
+//   warps 2..5  weight unpack into four 32-column A slots of tensor memory
+//   warps 6..9  epilogue, draining one of two 192-column accumulators while
+//               the MMA fills the other
+constexpr int kPThreads = 320;
+constexpr int kPASlots = 4;
+constexpr uint32_t kPAccStride = 192;  // column offset of accumulator 1
+constexpr uint32_t kPAColBase = 384;   // first A-slot column
+
+struct PParams {
+  const float* s_a;
+  const float* s_w;
+  const uint16_t* bias;
+  void* out;
+  int M, N, K;
+  int BT, m_tiles, num_tiles, nstages;
+};
+
+struct PHeader {
+  uint64_t full[8];
+  uint64_t empty[8];
+  uint64_t a_full[kPASlots];
+  uint64_t a_empty[kPASlots];
+  uint64_t acc_full[2];
+  uint64_t acc_empty[2];
+  uint32_t tmem_base;
+};
+
+template <int SINK>
+__global__ void __launch_bounds__(kPThreads, 1)
+    w4a4_tc_gemm_persistent_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_x,
+                                   const __grid_constant__ PParams p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int BT = p.BT;
+  const int ns = p.nstages;
+  const int stage_bytes = kWTileBytes + BT * kKB;
+  PHeader* hdr = reinterpret_cast<PHeader*>(smem + ns * stage_bytes);
+  float* sa_buf = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(hdr) + 1024);  // [2][192]
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int kbn = p.K / kKB;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < ns; ++s) {
+      mbar_init(&hdr->full[s], 1);
+      mbar_init(&hdr->empty[s], 1 + 4);  // MMA commit + one arrive per unpack warp
+    }
+    for (int a = 0; a < kPASlots; ++a) {
+      mbar_init(&hdr->a_full[a], 4);
+      mbar_init(&hdr->a_empty[a], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&hdr->acc_full[b], 1);
+      mbar_init(&hdr->acc_empty[b], 4);  // one arrive per epilogue warp
+    }
+    fence_mbarrier_init();
+    prefetch_tmap(&tm_w);
+    prefetch_tmap(&tm_x);
+  }
+  if (warp == 1) {
+    tmem_alloc(&hdr->tmem_base, 512u);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = hdr->tmem_base;
+
+  if (warp == 0) {
+    // ------------------------------------------------ TMA producer
+    if (lane == 0) {
+      const uint32_t bytes = static_cast<uint32_t>(stage_bytes);
+      const int my_tiles = (p.num_tiles - static_cast<int>(blockIdx.x) + static_cast<int>(gridDim.x) - 1) /
+                           static_cast<int>(gridDim.x);
+      const int total = my_tiles * kbn;
+      auto coords = [&](int i, int& m0, int& n0, int& kb) {
+        const int tile = static_cast<int>(blockIdx.x) + (i / kbn) * static_cast<int>(gridDim.x);
+        m0 = (tile % p.m_tiles) * BT;
+        n0 = (tile / p.m_tiles) * kRows;
+        kb = i % kbn;
+      };
+      // Weight tiles of the first stages do not depend on the preceding
+      // prologue kernel: request them before waiting for it.
+      const int prime = total < ns ? total : ns;
+      for (int i = 0; i < prime; ++i) {
+        int m0, n0, kb;
+        coords(i, m0, n0, kb);
+        mbar_arrive_expect_tx(&hdr->full[i], bytes);
+        tma_load_2d(smem + i * stage_bytes, &tm_w, &hdr->full[i], kb * (kKB / 2), n0);
+      }
+      pdl_wait();
+      for (int i = 0; i < prime; ++i) {
+        int m0, n0, kb;
+        coords(i, m0, n0, kb);
+        tma_load_2d(smem + i * stage_bytes + kWTileBytes, &tm_x, &hdr->full[i], kb * kKB, m0);
+      }
+      int it = prime;
+      for (; it < total; ++it) {
+        const int s = it % ns;
+        if (!mbar_wait(&hdr->empty[s], ((it / ns) - 1) & 1)) break;
+        int m0, n0, kb;
+        coords(it, m0, n0, kb);
+        uint8_t* st = smem + s * stage_bytes;
+        mbar_arrive_expect_tx(&hdr->full[s], bytes);
+        tma_load_2d(st, &tm_w, &hdr->full[s], kb * (kKB / 2), n0);
+        tma_load_2d(st + kWTileBytes, &tm_x, &hdr->full[s], kb * kKB, m0);
+      }
+      // Drain: every issued load has landed before the block may exit.
+      for (int i = (it > ns ? it - ns : 0); i < it; ++i) mbar_wait(&hdr->full[i % ns], (i / ns) & 1);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc = umma_idesc_i8(kRows, BT, /*a_signed=*/true, /*b_signed=*/true);
+      int it = 0, tc = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < p.num_tiles && ok; tile += gridDim.x, ++tc) {
+        const int b = tc & 1;
+        if (tc >= 2 && !mbar_wait(&hdr->acc_empty[b], ((tc / 2) - 1) & 1)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem + static_cast<uint32_t>(b) * kPAccStride;
+        for (int kb = 0; kb < kbn; ++kb, ++it) {
+          const int s = it % ns, a = it % kPASlots;
+          if (!mbar_wait(&hdr->full[s], (it / ns) & 1) || !mbar_wait(&hdr->a_full[a], (it / kPASlots) & 1)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint64_t bdesc = umma_desc_k_sw128(smem_u32(smem + s * stage_bytes + kWTileBytes));
+#pragma unroll
+          for (int kk = 0; kk < kKB / 32; ++kk)
+            umma_i8_ts(d_tmem, tmem + kPAColBase + 32 * a + 8 * kk, bdesc + 2 * kk, idesc,
+                       (kb > 0 || kk > 0) ? 1u : 0u);
+          umma_commit(&hdr->empty[s]);
+          umma_commit(&hdr->a_empty[a]);
+        }
+        umma_commit(&hdr->acc_full[b]);
+      }
+    }
+  } else if (warp < 6) {
+    // ------------------------------------------------ weight unpack
+    const int quad = warp & 3;
+    const int row = quad * 32 + lane;
+    const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
+    int it = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < p.num_tiles && ok; tile += gridDim.x) {
+      for (int kb = 0; kb < kbn; ++kb, ++it) {
+        const int s = it % ns, a = it % kPASlots;
+        bool w = mbar_wait(&hdr->full[s], (it / ns) & 1);
+        if (w && it >= kPASlots) w = mbar_wait(&hdr->a_empty[a], ((it / kPASlots) - 1) & 1);
+        ok = __all_sync(0xffffffffu, w);  // tcgen05.st below is warp-collective
+        if (!ok) break;
+        unpack_row_to_tmem(smem + s * stage_bytes, row, tmem + lane_base + kPAColBase + 32 * a);
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(&hdr->empty[s]);
+          mbar_arrive(&hdr->a_full[a]);
+        }
+      }
+    }
+  } else {
+    // ------------------------------------------------ epilogue
+    const int quad = warp & 3;
+    const int row = quad * 32 + lane;
+    const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
+    const int et = threadIdx.x - 192;  // 0..127
+    pdl_wait();  // s_a comes from the preceding prologue kernel
+    int tc = 0;
+    for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++tc) {
+      const int b = tc & 1;
+      const int m0 = (tile % p.m_tiles) * BT, n0 = (tile / p.m_tiles) * kRows;
+      float* sa = sa_buf + 192 * b;
+      if (SINK != static_cast<int>(GemmSink::kS32))
+        for (int c = et; c < BT; c += 128) sa[c] = (m0 + c < p.M) ? __ldg(p.s_a + m0 + c) : 0.0f;
+      named_barrier(1, 128);  // s_a of this tile staged; all warps are done with tile tc - 2
+      const int n = n0 + row;
+      const float sw = (SINK != static_cast<int>(GemmSink::kS32) && n < p.N) ? __ldg(p.s_w + n) : 0.0f;
+      const float bv = (p.bias && n < p.N) ? __uint_as_float(static_cast<uint32_t>(__ldg(p.bias + n)) << 16) : 0.0f;
+      // On a failed wait the warp skips the tile's work but keeps taking part
+      // in the named barrier above, so no peer waits on it forever.
+      const bool ok = __all_sync(0xffffffffu, mbar_wait(&hdr->acc_full[b], (tc / 2) & 1));
+      tc_fence_after();
+      const uint32_t acc = tmem + lane_base + static_cast<uint32_t>(b) * kPAccStride;
+      for (int c = 0; ok && c < BT; c += 16) {
+        uint32_t v[16];
+        tmem_ld_32x32b_x16(acc + static_cast<uint32_t>(c), v);
+        tmem_wait_ld();
+        if (n < p.N) {
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const int m = m0 + c + j;
+            if (m < p.M) store_output<SINK>(p, m, n, static_cast<int32_t>(v[j]), sa[c + j], sw, bv);
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&hdr->acc_empty[b]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, 512u);
   }
 }
 
@@ -338,7 +575,7 @@ bool make_map_u8(CUtensorMap* map, const void* base, uint64_t rows, uint64_t col
 
 int shared_bytes_for(int BT, int nstages, int splits) {
   int bytes = 1024 /*alignment slack*/ + nstages * (kWTileBytes + BT * kKB) + 2048 /*header + s_a tile*/;
-  if (splits > 1) bytes += (BT + 4) * kRows * 4;
+  if (splits > 1) bytes += splits * ((BT / 4 + splits - 1) / splits) * kRows * 16;
   return bytes;
 }
 
@@ -353,8 +590,11 @@ cudaError_t launch_sink(const CUtensorMap& tw, const CUtensorMap& tx, const Para
   cfg.blockDim = dim3(kThreads, 1, 1);
   cfg.dynamicSmemBytes = static_cast<size_t>(t.smem_bytes);
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   int nattr = 0;
+  attr[nattr].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[nattr].val.programmaticStreamSerializationAllowed = 1;
+  ++nattr;
   if (t.splits > 1) {
     attr[nattr].id = cudaLaunchAttributeClusterDimension;
     attr[nattr].val.clusterDim.x = 1;
@@ -367,10 +607,78 @@ cudaError_t launch_sink(const CUtensorMap& tw, const CUtensorMap& tx, const Para
   return note_cuda(cudaLaunchKernelEx(&cfg, w4a4_tc_gemm_kernel<SINK>, tw, tx, prm), "w4a4_gemm: launch");
 }
 
+template <int SINK>
+cudaError_t launch_persistent(const CUtensorMap& tw, const CUtensorMap& tx, const PParams& prm, const GemmTiling& t,
+                              cudaStream_t stream) {
+  static int cache[64] = {0};
+  const void* kfn = reinterpret_cast<const void*>(w4a4_tc_gemm_persistent_kernel<SINK>);
+  cudaError_t e = ensure_dynamic_smem(kfn, t.smem_bytes, cache);
+  if (e != cudaSuccess) return note_cuda(e, "w4a4_gemm: dynamic shared memory attribute");
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(t.grid, 1, 1);
+  cfg.blockDim = dim3(kPThreads, 1, 1);
+  cfg.dynamicSmemBytes = static_cast<size_t>(t.smem_bytes);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return note_cuda(cudaLaunchKernelEx(&cfg, w4a4_tc_gemm_persistent_kernel<SINK>, tw, tx, prm),
+                   "w4a4_gemm: persistent launch");
+}
+
+// Estimated cycles of the persistent kernel for a token tile of BT: rounds
+// of tiles per SM x k blocks x the slower of the MMA (2 * BT cycles per k
+// block at 8192 int8 MACs/clk) and a per-k-block floor of 256 cycles for the
+// fixed work every k block carries whatever BT is (the 8 KB weight tile
+// fetched from L2 and unpacked into tensor memory).
+long persistent_cost(int M, int N, int K, int BT, int num_sms) {
+  const long tiles = static_cast<long>((M + BT - 1) / BT) * ((N + kRows - 1) / kRows);
+  const long rounds = (tiles + num_sms - 1) / num_sms;
+  const long per_kb = 2L * BT > 256 ? 2L * BT : 256;
+  return rounds * (K / kKB) * per_kb;
+}
+
 }  // namespace
 
 GemmTiling choose_tiling(int M, int N, int K, int num_sms) {
   GemmTiling t{};
+  // Large M: the persistent kernel, with the token tile BT (multiple of 16,
+  // <= 192) of the lowest estimated cost, when it yields at least half as
+  // many tiles as SMs.
+  {
+    int best_bt = 0;
+    long best = -1;
+    for (int bt = 192; bt >= 64; bt -= 16) {
+      const long tiles = static_cast<long>((M + bt - 1) / bt) * ((N + kRows - 1) / kRows);
+      if (2 * tiles < num_sms) continue;
+      const long c = persistent_cost(M, N, K, bt, num_sms);
+      if (best < 0 || c < best) {
+        best = c;
+        best_bt = bt;
+      }
+    }
+    if (best_bt > 0 && M > 128) {
+      t.persistent = true;
+      t.BT = best_bt;
+      t.m_tiles = (M + best_bt - 1) / best_bt;
+      t.n_tiles = (N + kRows - 1) / kRows;
+      t.splits = 1;
+      t.kb_per_split = K / kKB;
+      const int stage = kWTileBytes + best_bt * kKB;
+      int ns = (220 * 1024 - 4096) / stage;
+      if (ns > 8) ns = 8;
+      t.nstages = ns;
+      t.tmem_cols = 512;
+      t.smem_bytes = 1024 + ns * stage + 1024 + 2 * 192 * 4;
+      if (t.smem_bytes < 120 * 1024) t.smem_bytes = 120 * 1024;  // one CTA per SM (it owns all of TMEM)
+      const long tiles = static_cast<long>(t.m_tiles) * t.n_tiles;
+      t.grid = static_cast<int>(tiles < num_sms ? tiles : num_sms);
+      return t;
+    }
+  }
+  // Small M: one CTA per (tile, K slice), slices of a tile form a cluster.
   const int kb_total = K / kKB;
   // Tokens per tile: one tile when M fits, else the fewest tiles of <= 192.
   const int max_bt = 192;
@@ -390,7 +698,7 @@ GemmTiling choose_tiling(int M, int N, int K, int num_sms) {
   t.kb_per_split = kbps;
   // Pipeline depth: as many stages as fit two CTAs per SM (~110 KB each).
   const int stage = kWTileBytes + bt * kKB;
-  int ns = (110 * 1024 - 3072 - (splits > 1 ? (bt + 4) * kRows * 4 : 0)) / stage;
+  int ns = (110 * 1024 - 3072 - (splits > 1 ? splits * ((bt / 4 + splits - 1) / splits) * kRows * 16 : 0)) / stage;
   if (ns > 8) ns = 8;
   if (ns > kbps) ns = kbps < 2 ? 2 : kbps;
   if (ns < 2) ns = 2;
@@ -406,6 +714,8 @@ GemmTiling choose_tiling(int M, int N, int K, int num_sms) {
   const int max_ctas = 512 / cols;
   const int min_smem = (228 * 1024) / (max_ctas + 1) + 1;
   if (t.smem_bytes < min_smem) t.smem_bytes = min_smem;
+  t.persistent = false;
+  t.grid = t.n_tiles * t.m_tiles * t.splits;
   return t;
 }
 
@@ -417,6 +727,28 @@ cudaError_t launch_w4a4_gemm(const GemmArgs& a, GemmSink sink, const GemmTiling&
   if (!make_map_u8(&tx, a.xs8, static_cast<uint64_t>(a.M), static_cast<uint64_t>(a.K), static_cast<uint32_t>(t.BT),
                    kKB, CU_TENSOR_MAP_SWIZZLE_128B))
     return note_cuda(cudaErrorInvalidValue, "w4a4_gemm: activation tensor map");
+  if (t.persistent) {
+    PParams pp{};
+    pp.s_a = a.s_a;
+    pp.s_w = a.s_w;
+    pp.bias = a.bias;
+    pp.out = a.out;
+    pp.M = a.M;
+    pp.N = a.N;
+    pp.K = a.K;
+    pp.BT = t.BT;
+    pp.m_tiles = t.m_tiles;
+    pp.num_tiles = t.m_tiles * t.n_tiles;
+    pp.nstages = t.nstages;
+    cudaError_t e;
+    switch (sink) {
+      case GemmSink::kBF16: e = launch_persistent<0>(tw, tx, pp, t, stream); break;
+      case GemmSink::kF32: e = launch_persistent<1>(tw, tx, pp, t, stream); break;
+      default: e = launch_persistent<2>(tw, tx, pp, t, stream); break;
+    }
+    count_dispatch(2);
+    return e;
+  }
   Params prm{};
   prm.s_a = a.s_a;
   prm.s_w = a.s_w;

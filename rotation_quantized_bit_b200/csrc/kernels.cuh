@@ -28,6 +28,8 @@ cudaError_t launch_unpack_codes(const uint8_t* packed, int M, int K, int8_t* s8,
 enum class GemmSink : int { kBF16 = 0, kF32 = 1, kS32 = 2 };
 
 struct GemmTiling {
+  bool persistent;  // one CTA per SM over all tiles (large M) vs one CTA per tile/split (small M)
+  int grid;         // CTAs launched
   int BT;           // tokens per CTA tile (MMA N), multiple of 16 in [16, 192]
   int m_tiles;      // ceil(M / BT)
   int n_tiles;      // ceil(N / 128)

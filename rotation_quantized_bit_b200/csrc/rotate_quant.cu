@@ -155,6 +155,9 @@ template <bool PACKED>
 __global__ void __launch_bounds__(kMaxWarps * 32, 1) rotate_quant_kernel(const __grid_constant__ RQParams p) {
   extern __shared__ __align__(16) uint8_t smem[];
   __shared__ uint32_t row_amax[2][128];
+  // Let the dependent GEMM launch now: it streams its weights meanwhile and
+  // waits (griddepcontrol.wait) for this grid before reading codes or scales.
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   uint8_t* const wbuf0 = smem + (2 * warp) * kTileBytes;
   uint8_t* const wbuf1 = smem + (2 * warp + 1) * kTileBytes;
@@ -283,24 +286,40 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) rotate_quant_kernel(const _
       }
     }
     if (!fast || emax >= kTieGuard) {
-      // Exact path: a zero or subnormal scale, or a value next to a tie.
+      // Exact path (rare): a zero or subnormal scale (every code by the
+      // division), or a lane with a value next to a tie (only those values
+      // are divided; the others keep the reciprocal result, which is exact
+      // for them).  A rolled loop over a local copy keeps this path small.
+      float v[128];
 #pragma unroll
-      for (int k = 0; k < 8; k += 2) {
-        uint32_t cx[16], cy[16];
+      for (int i = 0; i < 64; ++i) f2_split(P[i], v[i], v[i + 64]);
+      const float rcp = fast ? __frcp_rn(scale) : 0.0f;
+#pragma unroll 1
+      for (int k = 0; k < 16; ++k) {  // chunk k: channels 8k .. 8k+7 of the half
+        uint32_t q[8];
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          float a, c;
-          f2_split(P[8 * k + e], a, c);
-          int qa = 0, qc = 0;
-          if (scale != 0.0f) {
-            qa = min(7, max(-8, __float2int_rn(__fdiv_rn(a, scale))));
-            qc = min(7, max(-8, __float2int_rn(__fdiv_rn(c, scale))));
+        for (int e = 0; e < 8; ++e) {
+          const float x = v[8 * k + e];
+          int qq = 0;
+          if (fast) {
+            const float y = __fmul_rn(x, rcp);
+            const float r = __fsub_rn(__fadd_rn(y, kMagic), kMagic);
+            qq = static_cast<int>(r);
+            if (fabsf(__fsub_rn(y, r)) >= kTieGuard) qq = __float2int_rn(__fdiv_rn(x, scale));
+          } else if (scale != 0.0f) {
+            qq = min(7, max(-8, __float2int_rn(__fdiv_rn(x, scale))));
           }
-          cx[e] = static_cast<uint32_t>(qa);
-          cy[e] = static_cast<uint32_t>(qc);
+          q[e] = static_cast<uint32_t>(qq);
         }
-        stage_chunk_pair<PACKED>(tile, lane, k >> 1, cx);
-        stage_chunk_pair<PACKED>(tile, lane, (k + 8) >> 1, cy);
+        if (PACKED) {
+          uint32_t w = 0;
+#pragma unroll
+          for (int e = 0; e < 8; ++e) w |= (q[e] & 0xFu) << (4 * e);
+          *reinterpret_cast<uint32_t*>(tile + 64 * lane + 4 * k) = w;
+        } else {
+          const uint2 o = make_uint2(gather_b0(q[0], q[2], q[4], q[6]), gather_b0(q[1], q[3], q[5], q[7]));
+          *reinterpret_cast<uint2*>(tile + 128 * lane + 16 * ((k >> 1) ^ (lane & 7)) + 8 * (k & 1)) = o;
+        }
       }
     }
     if (live && h == 0 && f % p.G == 0) p.out.scale[row] = scale;
@@ -372,12 +391,43 @@ cudaError_t launch_rotate_quant(const uint16_t* x, int M, int K, RotateQuantOut 
   p.M = M;
   p.K = K;
   p.G = K / 256;
-  // Rows per block: at most 128 groups (8 warps) per block, and few enough
-  // rows that every SM gets about two blocks.
+  // Rows per block R: a block holds R*G half-group pairs (at most 128 groups,
+  // 8 warps).  Pick the R with the fewest waves of blocks over the SMs and,
+  // among those, the fewest warps on the busiest SM.
   const int sms = num_sms_cached();
-  int R = 128 / p.G;
-  const int spread = M / (2 * sms);
-  if (spread < R) R = spread < 1 ? 1 : spread;
+  const bool packed_out = out.packed != nullptr;
+  const void* kfn_sel = packed_out ? reinterpret_cast<const void*>(rotate_quant_kernel<true>)
+                                   : reinterpret_cast<const void*>(rotate_quant_kernel<false>);
+  static int regs_cache[2][64] = {{0}};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) dev = 0;
+  int& regs = regs_cache[packed_out ? 1 : 0][dev];
+  if (regs == 0) {
+    cudaFuncAttributes fa;
+    regs = (cudaFuncGetAttributes(&fa, kfn_sel) == cudaSuccess && fa.numRegs > 0) ? fa.numRegs : 255;
+  }
+  const int warp_regs = ((regs * 32 + 255) / 256) * 256;
+  int best_R = 1;
+  long best_key = -1;
+  for (int R = 1; R <= 128 / p.G; ++R) {
+    const int nb = (M + R - 1) / R;
+    const int w = (R * p.G + 15) / 16;
+    int per_sm = 65536 / (warp_regs * w);
+    per_sm = min(per_sm, (228 * 1024) / (w * 2 * kTileBytes + 2048));
+    per_sm = min(per_sm, 64 / w);
+    if (per_sm < 1) continue;
+    const long slots = static_cast<long>(sms) * per_sm;
+    const long waves = (nb + slots - 1) / slots;
+    const long busiest = static_cast<long>((nb + sms - 1) / sms) * w;  // warps on the busiest SM per wave
+    const long key = waves * 100000 + (waves > 1 ? 0 : busiest);
+    if (best_key < 0 || key < best_key || (key == best_key && R > best_R)) {
+      best_key = key;
+      best_R = R;
+    }
+    if (R > M) break;
+  }
+  const int R = best_R;
   p.R = R;
   p.nblocks = (M + R - 1) / R;
   p.out = out;

@@ -110,7 +110,9 @@ def test_pack_weight_bit_exact(rq, workload, N, K):
 # ------------------------------------------------------------- GEMM sinks
 
 GEMM_CASES = [(8, 256, 256), (32, 256, 512), (77, 264, 768), (1, 128, 2560), (16, 2560, 2560),
-              (200, 384, 1024), (300, 1000, 512), (193, 136, 256), (600, 4096, 512)]
+              (200, 384, 1024), (300, 1000, 512), (193, 136, 256), (600, 4096, 512),
+              # persistent large-M path: several tiles per SM, ragged M and N tails
+              (1000, 1280, 1024), (777, 2056, 768), (2100, 1024, 256)]
 
 
 def random_codes(seed, rows, K):
@@ -157,7 +159,8 @@ def test_gemm_f32_and_bf16(rq, M, N, K):
 # ------------------------------------------------------------- fused Linear
 
 LINEAR_CASES = [("small", 32, 512, 256), ("qwen3_4b", 77, 2560, 264), ("qwen3_4b", 1, 2560, 1024),
-                ("dit6b", 250, 3840, 384), ("edit20b", 16, 3072, 12288), ("qwen3_4b", 8, 9728, 2560)]
+                ("dit6b", 250, 3840, 384), ("edit20b", 16, 3072, 12288), ("qwen3_4b", 8, 9728, 2560),
+                ("dit6b", 600, 3840, 1024), ("qwen3_4b", 1220, 2560, 1024)]
 
 
 @pytest.mark.parametrize("workload,M,K,N", LINEAR_CASES)
