@@ -25,13 +25,14 @@
 //     chunk order, so the contraction pairs the right codes;
 //   * the accumulator is exactly 16 * acc (|16 acc| <= 1024 K < 2^31), and
 //     the epilogue shifts it right by 4.
-// Split-K (for small M) runs the K-slices of one output tile as a thread
-// block cluster and adds the int32 partial tiles through distributed shared
-// memory; the sum is exact and independent of order.
+// Work is cut into units of one 128-wide K block of one output tile; see
+// the kernel below for the two schedules (whole tiles for large M, stream-K
+// for small M) and the exact cross-CTA reduction of split tiles.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cstdint>
 
 #include "kernels.cuh"
@@ -41,46 +42,34 @@ namespace convrot {
 
 namespace {
 
-constexpr int kThreads = 192;    // warp 0 TMA, warp 1 MMA, warps 2..5 unpack + epilogue
 constexpr int kRows = 128;       // output channels per tile (MMA M)
-constexpr int kKB = 128;         // K values per pipeline step
-constexpr int kWTileBytes = kRows * kKB / 2;  // 8 KB packed weights per step
-constexpr int kASlots = 2;       // tensor-memory A buffers (32 columns each)
+constexpr int kKB = 256;         // K values per unit (pipeline step)
+constexpr int kWTileBytes = kRows * kKB / 2;  // 16 KB packed weights per unit
+constexpr int kXBox = 128;       // K bytes per activation TMA box (the 128-byte swizzle span)
+constexpr int kMaxStages = 16;   // depth limit of the shared-memory TMA ring
+constexpr int kDoneRing = 32;    // MMA completion barriers, one per unit mod 32 (>= stages, >= A slots)
+constexpr int kMaxASlots = 8;    // tensor-memory A slots (64 columns each)
 
-struct Params {
-  const float* s_a;
-  const float* s_w;
-  const uint16_t* bias;
-  void* out;
-  int M, N, K;
-  int BT, splits, kb_total, kb_per_split, nstages, tmem_cols;
-};
-
-struct SharedHeader {
-  uint64_t full[16];
-  uint64_t empty[16];
-  uint64_t a_full[kASlots];
-  uint64_t a_empty[kASlots];
-  uint64_t acc_full;
-  uint32_t tmem_base;
-};
-
+// One packed weight row of a unit (128 bytes = 256 codes) -> 64 tensor-memory
+// columns of signed bytes.  The tile landed with the 128-byte TMA swizzle:
+// 16-byte chunk c of row r sits at chunk c ^ (r & 7).
 __device__ __forceinline__ void unpack_row_to_tmem(const uint8_t* wstage, int row, uint32_t taddr) {
-  // The weight tile landed with the 64-byte TMA swizzle: 16-byte chunk c of
-  // row r sits at chunk c ^ ((r >> 1) & 3).
-  uint32_t cols[32];
-  const int sw = (row >> 1) & 3;
+  const int sw = row & 7;
 #pragma unroll
-  for (int c = 0; c < 4; ++c) {
-    const uint4 v = *reinterpret_cast<const uint4*>(wstage + row * 64 + ((c ^ sw) << 4));
-    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  for (int h = 0; h < 2; ++h) {
+    uint32_t cols[32];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      cols[8 * c + 2 * j] = (w[j] << 4) & 0xF0F0F0F0u;
-      cols[8 * c + 2 * j + 1] = w[j] & 0xF0F0F0F0u;
+    for (int c = 0; c < 4; ++c) {
+      const uint4 v = *reinterpret_cast<const uint4*>(wstage + row * 128 + (((4 * h + c) ^ sw) << 4));
+      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        cols[8 * c + 2 * j] = (w[j] << 4) & 0xF0F0F0F0u;
+        cols[8 * c + 2 * j + 1] = w[j] & 0xF0F0F0F0u;
+      }
     }
+    tmem_st_32x32b_x32(taddr + 32u * h, cols);
   }
-  tmem_st_32x32b_x32(taddr, cols);
 }
 
 // One output element from the MMA sum (16 * acc): scales and bias already
@@ -103,235 +92,33 @@ __device__ __forceinline__ void store_output(const P& p, int m, int n, int32_t d
   }
 }
 
-template <int SINK>
-__global__ void __launch_bounds__(kThreads, 1)
-    w4a4_tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_x,
-                        const __grid_constant__ Params p) {
-  extern __shared__ __align__(1024) uint8_t smem_raw[];
-  // 1024-byte alignment for the swizzled stage tiles.
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  const int BT = p.BT;
-  const int stage_bytes = kWTileBytes + BT * kKB;
-  SharedHeader* hdr = reinterpret_cast<SharedHeader*>(smem + p.nstages * stage_bytes);
-  float* sa_tile = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(hdr) + 1024);   // s_a of the BT tokens
-  int32_t* red = reinterpret_cast<int32_t*>(reinterpret_cast<uint8_t*>(hdr) + 2048);  // split-K partials
-
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int n0 = blockIdx.x * kRows;
-  const int m0 = blockIdx.y * BT;
-  // K blocks of this split: an even share [j*KB/S, (j+1)*KB/S), never empty
-  // because S <= KB.
-  const int split = blockIdx.z;
-  const int kb0 = (split * p.kb_total) / p.splits;
-  const int nkb = ((split + 1) * p.kb_total) / p.splits - kb0;
-  const int ns = p.nstages;
-  const uint32_t a_col0 = static_cast<uint32_t>(p.tmem_cols - 32 * kASlots);
-
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < ns; ++s) {
-      mbar_init(&hdr->full[s], 1);
-      mbar_init(&hdr->empty[s], 1 + 4);  // MMA commit + one arrive per unpack warp
-    }
-    for (int a = 0; a < kASlots; ++a) {
-      mbar_init(&hdr->a_full[a], 4);
-      mbar_init(&hdr->a_empty[a], 1);
-    }
-    mbar_init(&hdr->acc_full, 1);
-    fence_mbarrier_init();
-    prefetch_tmap(&tm_w);
-    prefetch_tmap(&tm_x);
-  }
-  if (warp == 1) {
-    tmem_alloc(&hdr->tmem_base, static_cast<uint32_t>(p.tmem_cols));
-    tmem_relinquish();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = hdr->tmem_base;
-
-  if (warp == 0) {
-    // ------------------------------------------------ TMA producer
-    if (lane == 0) {
-      const uint32_t bytes = static_cast<uint32_t>(stage_bytes);
-      // The weights do not depend on the preceding prologue kernel: the first
-      // stages' weight tiles are requested before waiting for it.
-      const int prime = nkb < ns ? nkb : ns;
-      for (int i = 0; i < prime; ++i) {
-        mbar_arrive_expect_tx(&hdr->full[i], bytes);
-        tma_load_2d(smem + i * stage_bytes, &tm_w, &hdr->full[i], (kb0 + i) * (kKB / 2), n0);
-      }
-      pdl_wait();
-      for (int i = 0; i < prime; ++i)
-        tma_load_2d(smem + i * stage_bytes + kWTileBytes, &tm_x, &hdr->full[i], (kb0 + i) * kKB, m0);
-      int issued = prime;
-      for (int i = prime; i < nkb; ++i) {
-        const int s = i % ns;
-        if (i >= ns && !mbar_wait(&hdr->empty[s], ((i / ns) - 1) & 1)) break;
-        uint8_t* st = smem + s * stage_bytes;
-        mbar_arrive_expect_tx(&hdr->full[s], bytes);
-        tma_load_2d(st, &tm_w, &hdr->full[s], (kb0 + i) * (kKB / 2), n0);
-        tma_load_2d(st + kWTileBytes, &tm_x, &hdr->full[s], (kb0 + i) * kKB, m0);
-        ++issued;
-      }
-      // Drain: every issued load has landed before the block may exit.
-      for (int i = (issued > ns ? issued - ns : 0); i < issued; ++i)
-        mbar_wait(&hdr->full[i % ns], (i / ns) & 1);
-    }
-  } else if (warp == 1) {
-    // ------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      const uint32_t idesc = umma_idesc_i8(kRows, BT, /*a_signed=*/true, /*b_signed=*/true);
-      bool ok = true;
-      for (int i = 0; i < nkb && ok; ++i) {
-        const int s = i % ns, a = i % kASlots;
-        ok = mbar_wait(&hdr->full[s], (i / ns) & 1) && mbar_wait(&hdr->a_full[a], (i / kASlots) & 1);
-        if (!ok) break;
-        tc_fence_after();
-        const uint64_t bdesc = umma_desc_k_sw128(smem_u32(smem + s * stage_bytes + kWTileBytes));
-#pragma unroll
-        for (int kk = 0; kk < kKB / 32; ++kk) {
-          umma_i8_ts(tmem, tmem + a_col0 + 32 * a + 8 * kk, bdesc + 2 * kk, idesc, (i > 0 || kk > 0) ? 1u : 0u);
-        }
-        umma_commit(&hdr->empty[s]);
-        umma_commit(&hdr->a_empty[a]);
-      }
-      umma_commit(&hdr->acc_full);
-      mbar_wait(&hdr->acc_full, 0);  // all MMAs retired before teardown
-    }
-  } else {
-    // ------------------------------------------------ unpack, then epilogue
-    const int quad = warp & 3;  // tensor-memory lane quadrant of this warp
-    const int row = quad * 32 + lane;
-    const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
-    const int et = threadIdx.x - 64;  // 0..127 over the four unpack/epilogue warps
-    bool ok = true;
-    for (int i = 0; i < nkb; ++i) {
-      const int s = i % ns, a = i % kASlots;
-      ok = mbar_wait(&hdr->full[s], (i / ns) & 1);
-      if (ok && i >= kASlots) ok = mbar_wait(&hdr->a_empty[a], ((i / kASlots) - 1) & 1);
-      ok = __all_sync(0xffffffffu, ok);  // tcgen05.st below is warp-collective
-      if (!ok) break;
-      unpack_row_to_tmem(smem + s * stage_bytes, row, tmem + lane_base + a_col0 + 32 * a);
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(&hdr->empty[s]);
-        mbar_arrive(&hdr->a_full[a]);
-      }
-    }
-    pdl_wait();  // s_a comes from the preceding prologue kernel
-    if (SINK != static_cast<int>(GemmSink::kS32)) {
-      for (int c = et; c < BT; c += 128) sa_tile[c] = (m0 + c < p.M) ? __ldg(p.s_a + m0 + c) : 0.0f;
-    }
-    if (ok) ok = mbar_wait(&hdr->acc_full, 0);
-    ok = __all_sync(0xffffffffu, ok);  // tcgen05.ld below is warp-collective
-    tc_fence_after();
-    named_barrier(1, 128);  // sa_tile written by all four epilogue warps
-
-    const int n = n0 + row;
-    if (p.splits == 1) {
-      if (ok && nkb > 0) {
-        const float sw = (SINK != static_cast<int>(GemmSink::kS32) && n < p.N) ? __ldg(p.s_w + n) : 0.0f;
-        const float bv = (p.bias && n < p.N) ? __uint_as_float(static_cast<uint32_t>(__ldg(p.bias + n)) << 16) : 0.0f;
-        for (int c = 0; c < BT; c += 16) {
-          uint32_t v[16];
-          tmem_ld_32x32b_x16(tmem + lane_base + static_cast<uint32_t>(c), v);
-          tmem_wait_ld();
-          if (n < p.N) {
-#pragma unroll
-            for (int j = 0; j < 16; ++j) {
-              const int m = m0 + c + j;
-              if (m < p.M) store_output<SINK>(p, m, n, static_cast<int32_t>(v[j]), sa_tile[c + j], sw, bv);
-            }
-          }
-        }
-      }
-    } else {
-      // Push the partial tile to its owners.  4-token group g belongs to CTA
-      // g % S of the cluster, which keeps the partials of its groups in slots
-      // [source rank][g / S][row] (16 bytes each); the stores are
-      // fire-and-forget and become visible at the cluster barrier.
-      const int S = p.splits;
-      const int ngl = (BT / 4 + S - 1) / S;
-      const uint32_t me = cluster_ctarank();
-      const uint32_t red_base = smem_u32(red);
-      for (int c = 0; c < BT; c += 16) {
-        uint32_t v[16];
-        tmem_ld_32x32b_x16(tmem + lane_base + static_cast<uint32_t>(c), v);
-        tmem_wait_ld();
-        const bool keep = ok && nkb > 0;
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const int g = c / 4 + q;
-          const int4 w = keep ? make_int4(static_cast<int32_t>(v[4 * q]), static_cast<int32_t>(v[4 * q + 1]),
-                                          static_cast<int32_t>(v[4 * q + 2]), static_cast<int32_t>(v[4 * q + 3]))
-                              : make_int4(0, 0, 0, 0);
-          const uint32_t slot = ((static_cast<uint32_t>(me) * ngl + static_cast<uint32_t>(g / S)) * kRows + row) * 16u;
-          st_shared_cluster_v4(map_shared_rank(red_base + slot, static_cast<uint32_t>(g % S)), w);
-        }
-      }
-    }
-  }
-
-  if (p.splits > 1) {
-    __syncwarp();    // the cluster barrier below is .aligned: reconverge first
-    cluster_sync();  // every partial has reached its owner's shared memory
-    if (warp >= 2) {
-      // This CTA sums, from its own shared memory, the S partials of the
-      // groups it owns and writes their outputs.  No CTA touches another's
-      // shared memory after the barrier, so none has to wait before exiting.
-      const int S = p.splits;
-      const int ngl = (BT / 4 + S - 1) / S;
-      const int quad = warp & 3;
-      const int row = quad * 32 + lane;
-      const int n = n0 + row;
-      const int rank = static_cast<int>(cluster_ctarank());
-      const float sw = (SINK != static_cast<int>(GemmSink::kS32) && n < p.N) ? __ldg(p.s_w + n) : 0.0f;
-      const float bv = (p.bias && n < p.N) ? __uint_as_float(static_cast<uint32_t>(__ldg(p.bias + n)) << 16) : 0.0f;
-      const int4* red4 = reinterpret_cast<const int4*>(red);
-      for (int gl = 0; gl < ngl; ++gl) {
-        const int g = gl * S + rank;
-        if (g >= BT / 4 || m0 + 4 * g >= p.M || n >= p.N) continue;
-        int4 sum = make_int4(0, 0, 0, 0);
-        for (int j = 0; j < S; ++j) {
-          const int4 v = red4[(j * ngl + gl) * kRows + row];
-          sum.x += v.x; sum.y += v.y; sum.z += v.z; sum.w += v.w;
-        }
-        const int32_t sv[4] = {sum.x, sum.y, sum.z, sum.w};
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const int m = m0 + 4 * g + q;
-          if (m < p.M) store_output<SINK>(p, m, n, sv[q], sa_tile[4 * g + q], sw, bv);
-        }
-      }
-    }
-  }
-
-  tc_fence_before();
-  __syncthreads();
-  if (warp == 1) {
-    __syncwarp();
-    tc_fence_after();
-    tmem_dealloc(tmem, static_cast<uint32_t>(p.tmem_cols));
-  }
-}
-
-
-// ---------------------------------------------------------------- persistent kernel (large M)
+// ---------------------------------------------------------------- the kernel
 //
-// One CTA per SM walks the output tiles (tile t -> m tile t % m_tiles, n tile
-// t / m_tiles) with a k-block stream that does not drain between tiles:
+// One CTA per SM walks its list of units; a unit is one 128-wide K block of
+// one output tile (BT tokens x 128 output channels).  Two schedules:
+//   * tiles (large M): CTA c takes the whole tiles c, c + grid, c + 2 grid ...
+//     (neighbouring CTAs share activation and weight tiles in L2);
+//   * stream-K (small M, fewer tiles than SMs): the units of all tiles, in
+//     tile-major order, are cut into `grid` contiguous ranges of equal size,
+//     so every SM streams the same share of the weights.
+// Consecutive units of one tile form a segment, summed in one tensor-memory
+// accumulator.  A segment that covers all K blocks of its tile is stored
+// directly.  Otherwise (stream-K only; at most the first and the last
+// segment of a CTA) its int32 partial tile goes to the CTA's slot in global
+// memory and the CTA bumps the tile's arrival counter; the CTA that arrives
+// last adds the other contributors' slots to its own accumulator, stores the
+// tile and resets the counter to zero for the next launch.  Integer addition
+// is exact, so no output bit depends on the order of arrival.
 //   warp 0      TMA producer (ring of `nstages` shared-memory stages)
 //   warp 1      TMEM allocation (all 512 columns) and the MMA-issuing thread
-//   warps 2..5  weight unpack into four 32-column A slots of tensor memory
-//   warps 6..9  epilogue, draining one of two 192-column accumulators while
-//               the MMA fills the other
+//   warps 2..5  weight unpack into 64-column A slots of tensor memory
+//   warps 6..9  epilogue, draining one of two accumulators while the MMA
+//               fills the other
+// The MMA thread commits once per unit, to done[unit % 32]; that one
+// completion frees both the unit's shared-memory stage (for the TMA producer)
+// and its A slot (for the unpack warps).  A unit of 256 K values is 8 MMAs,
+// so the waits and the commit of the issuing thread are spread over 8.
 constexpr int kPThreads = 320;
-constexpr int kPASlots = 4;
-constexpr uint32_t kPAccStride = 192;  // column offset of accumulator 1
-constexpr uint32_t kPAColBase = 384;   // first A-slot column
 
 struct PParams {
   const float* s_a;
@@ -339,42 +126,93 @@ struct PParams {
   const uint16_t* bias;
   void* out;
   int M, N, K;
-  int BT, m_tiles, num_tiles, nstages;
+  int BT, m_tiles, num_tiles, nstages, kbn;
+  int acc_stride;   // tensor-memory columns per accumulator (BT rounded up to 32)
+  int a_slots;      // A slots of 64 columns after the two accumulators
+  int stream_k;     // 0: whole tiles round-robin, 1: stream-K ranges
+  int units;        // num_tiles * kbn
+  uint32_t* ctr;    // [num_tiles] arrival counters (stream-K), zero between launches
+  int32_t* slots;   // [2 * grid][BT][128] partial tiles (stream-K)
 };
 
 struct PHeader {
-  uint64_t full[8];
-  uint64_t empty[8];
-  uint64_t a_full[kPASlots];
-  uint64_t a_empty[kPASlots];
+  uint64_t full[kMaxStages];
+  uint64_t done[kDoneRing];     // unit i's MMAs have completed (its stage and A slot are free)
+  uint64_t a_full[kMaxASlots];
   uint64_t acc_full[2];
   uint64_t acc_empty[2];
   uint32_t tmem_base;
+  uint32_t last_flag;
 };
+
+// First unit of CTA c under stream-K (c in [0, grid]; strictly increasing
+// because grid <= units).
+__device__ __forceinline__ int sk_begin(const PParams& p, int c) {
+  return static_cast<int>((static_cast<long long>(c) * p.units) / static_cast<int>(gridDim.x));
+}
+
+// The CTA whose stream-K range holds unit u.
+__device__ __forceinline__ int sk_owner(const PParams& p, int u) {
+  const int G = static_cast<int>(gridDim.x);
+  int c = static_cast<int>((static_cast<long long>(u) * G) / p.units);
+  while (c + 1 < G && sk_begin(p, c + 1) <= u) ++c;
+  while (c > 0 && sk_begin(p, c) > u) --c;
+  return c;
+}
+
+// Number of units of this CTA.
+__device__ __forceinline__ int unit_count(const PParams& p) {
+  if (p.stream_k) return sk_begin(p, blockIdx.x + 1) - sk_begin(p, blockIdx.x);
+  const int my_tiles =
+      (p.num_tiles - static_cast<int>(blockIdx.x) + static_cast<int>(gridDim.x) - 1) / static_cast<int>(gridDim.x);
+  return my_tiles * p.kbn;
+}
+
+// Tile and K block of this CTA's first unit, and the step to the next unit.
+__device__ __forceinline__ void unit_first(const PParams& p, int u0, int& tile, int& kb) {
+  if (p.stream_k) {
+    tile = u0 / p.kbn;
+    kb = u0 - tile * p.kbn;
+  } else {
+    tile = static_cast<int>(blockIdx.x);
+    kb = 0;
+  }
+}
+__device__ __forceinline__ void unit_next(const PParams& p, int& tile, int& kb) {
+  if (++kb == p.kbn) {
+    kb = 0;
+    tile += p.stream_k ? 1 : static_cast<int>(gridDim.x);
+  }
+}
+
+// Partial-tile slot layout: 16-token chunks, each [128 rows][16 tokens], so
+// a thread (one row) moves 64 contiguous bytes per chunk.
+__device__ __forceinline__ int32_t* slot_chunk(int32_t* slot, int c, int row) {
+  return slot + (c >> 4) * (kRows * 16) + row * 16;
+}
 
 template <int SINK>
 __global__ void __launch_bounds__(kPThreads, 1)
-    w4a4_tc_gemm_persistent_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_x,
-                                   const __grid_constant__ PParams p) {
+    w4a4_tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_x,
+                        const __grid_constant__ PParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int BT = p.BT;
   const int ns = p.nstages;
   const int stage_bytes = kWTileBytes + BT * kKB;
+  const int nas = p.a_slots;
+  const uint32_t a_col0 = 2u * static_cast<uint32_t>(p.acc_stride);
   PHeader* hdr = reinterpret_cast<PHeader*>(smem + ns * stage_bytes);
   float* sa_buf = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(hdr) + 1024);  // [2][192]
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int kbn = p.K / kKB;
+  const int kbn = p.kbn;
+  const int u0 = p.stream_k ? sk_begin(p, blockIdx.x) : 0;
+  const int total = unit_count(p);
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < ns; ++s) {
-      mbar_init(&hdr->full[s], 1);
-      mbar_init(&hdr->empty[s], 1 + 4);  // MMA commit + one arrive per unpack warp
-    }
-    for (int a = 0; a < kPASlots; ++a) {
-      mbar_init(&hdr->a_full[a], 4);
-      mbar_init(&hdr->a_empty[a], 1);
-    }
+    for (int s = 0; s < ns; ++s) mbar_init(&hdr->full[s], 1);
+    for (int r = 0; r < kDoneRing; ++r) mbar_init(&hdr->done[r], 1);  // one MMA commit
+    for (int a = 0; a < nas; ++a) mbar_init(&hdr->a_full[a], 4);      // one arrive per unpack warp
     for (int b = 0; b < 2; ++b) {
       mbar_init(&hdr->acc_full[b], 1);
       mbar_init(&hdr->acc_empty[b], 4);  // one arrive per epilogue warp
@@ -396,40 +234,32 @@ __global__ void __launch_bounds__(kPThreads, 1)
     // ------------------------------------------------ TMA producer
     if (lane == 0) {
       const uint32_t bytes = static_cast<uint32_t>(stage_bytes);
-      const int my_tiles = (p.num_tiles - static_cast<int>(blockIdx.x) + static_cast<int>(gridDim.x) - 1) /
-                           static_cast<int>(gridDim.x);
-      const int total = my_tiles * kbn;
-      auto coords = [&](int i, int& m0, int& n0, int& kb) {
-        const int tile = static_cast<int>(blockIdx.x) + (i / kbn) * static_cast<int>(gridDim.x);
-        m0 = (tile % p.m_tiles) * BT;
-        n0 = (tile / p.m_tiles) * kRows;
-        kb = i % kbn;
-      };
       // Weight tiles of the first stages do not depend on the preceding
       // prologue kernel: request them before waiting for it.
       const int prime = total < ns ? total : ns;
-      for (int i = 0; i < prime; ++i) {
-        int m0, n0, kb;
-        coords(i, m0, n0, kb);
+      int tile, kb;
+      unit_first(p, u0, tile, kb);
+      for (int i = 0; i < prime; ++i, unit_next(p, tile, kb)) {
         mbar_arrive_expect_tx(&hdr->full[i], bytes);
-        tma_load_2d(smem + i * stage_bytes, &tm_w, &hdr->full[i], kb * (kKB / 2), n0);
+        tma_load_2d(smem + i * stage_bytes, &tm_w, &hdr->full[i], kb * (kKB / 2), (tile / p.m_tiles) * kRows);
       }
       pdl_wait();
-      for (int i = 0; i < prime; ++i) {
-        int m0, n0, kb;
-        coords(i, m0, n0, kb);
-        tma_load_2d(smem + i * stage_bytes + kWTileBytes, &tm_x, &hdr->full[i], kb * kKB, m0);
+      unit_first(p, u0, tile, kb);
+      for (int i = 0; i < prime; ++i, unit_next(p, tile, kb)) {
+        uint8_t* xs = smem + i * stage_bytes + kWTileBytes;
+        tma_load_2d(xs, &tm_x, &hdr->full[i], kb * kKB, (tile % p.m_tiles) * BT);
+        tma_load_2d(xs + BT * kXBox, &tm_x, &hdr->full[i], kb * kKB + kXBox, (tile % p.m_tiles) * BT);
       }
-      int it = prime;
-      for (; it < total; ++it) {
-        const int s = it % ns;
-        if (!mbar_wait(&hdr->empty[s], ((it / ns) - 1) & 1)) break;
-        int m0, n0, kb;
-        coords(it, m0, n0, kb);
+      int it = prime, s = prime % ns;  // stage of unit `it`
+      for (; it < total; ++it, unit_next(p, tile, kb)) {
+        const int w = it - ns;  // the unit that last used stage s
+        if (!mbar_wait(&hdr->done[w % kDoneRing], (w / kDoneRing) & 1)) break;
         uint8_t* st = smem + s * stage_bytes;
         mbar_arrive_expect_tx(&hdr->full[s], bytes);
-        tma_load_2d(st, &tm_w, &hdr->full[s], kb * (kKB / 2), n0);
-        tma_load_2d(st + kWTileBytes, &tm_x, &hdr->full[s], kb * kKB, m0);
+        tma_load_2d(st, &tm_w, &hdr->full[s], kb * (kKB / 2), (tile / p.m_tiles) * kRows);
+        tma_load_2d(st + kWTileBytes, &tm_x, &hdr->full[s], kb * kKB, (tile % p.m_tiles) * BT);
+        tma_load_2d(st + kWTileBytes + BT * kXBox, &tm_x, &hdr->full[s], kb * kKB + kXBox, (tile % p.m_tiles) * BT);
+        if (++s == ns) s = 0;
       }
       // Drain: every issued load has landed before the block may exit.
       for (int i = (it > ns ? it - ns : 0); i < it; ++i) mbar_wait(&hdr->full[i % ns], (i / ns) & 1);
@@ -438,32 +268,41 @@ __global__ void __launch_bounds__(kPThreads, 1)
     // ------------------------------------------------ MMA issuer
     if (lane == 0) {
       const uint32_t idesc = umma_idesc_i8(kRows, BT, /*a_signed=*/true, /*b_signed=*/true);
-      int it = 0, tc = 0;
-      bool ok = true;
-      for (int tile = blockIdx.x; tile < p.num_tiles && ok; tile += gridDim.x, ++tc) {
-        const int b = tc & 1;
-        if (tc >= 2 && !mbar_wait(&hdr->acc_empty[b], ((tc / 2) - 1) & 1)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        const uint32_t d_tmem = tmem + static_cast<uint32_t>(b) * kPAccStride;
-        for (int kb = 0; kb < kbn; ++kb, ++it) {
-          const int s = it % ns, a = it % kPASlots;
-          if (!mbar_wait(&hdr->full[s], (it / ns) & 1) || !mbar_wait(&hdr->a_full[a], (it / kPASlots) & 1)) {
-            ok = false;
-            break;
-          }
+      int seg = 0, tile, kb, s = 0, ph = 0, a = 0, aph = 0;
+      bool first = true;
+      uint32_t d_tmem = tmem;
+      unit_first(p, u0, tile, kb);
+      for (int i = 0; i < total; ++i, unit_next(p, tile, kb)) {
+        if (i == 0 || kb == 0) {  // a segment starts: take accumulator seg & 1
+          const int b = seg & 1;
+          if (seg >= 2 && !mbar_wait(&hdr->acc_empty[b], ((seg / 2) - 1) & 1)) break;
           tc_fence_after();
-          const uint64_t bdesc = umma_desc_k_sw128(smem_u32(smem + s * stage_bytes + kWTileBytes));
-#pragma unroll
-          for (int kk = 0; kk < kKB / 32; ++kk)
-            umma_i8_ts(d_tmem, tmem + kPAColBase + 32 * a + 8 * kk, bdesc + 2 * kk, idesc,
-                       (kb > 0 || kk > 0) ? 1u : 0u);
-          umma_commit(&hdr->empty[s]);
-          umma_commit(&hdr->a_empty[a]);
+          d_tmem = tmem + static_cast<uint32_t>(b * p.acc_stride);
+          first = true;
         }
-        umma_commit(&hdr->acc_full[b]);
+        if (!mbar_wait(&hdr->full[s], ph & 1) || !mbar_wait(&hdr->a_full[a], aph & 1)) break;
+        tc_fence_after();
+        const uint64_t bdesc0 = umma_desc_k_sw128(smem_u32(smem + s * stage_bytes + kWTileBytes));
+        const uint64_t bdesc1 = umma_desc_k_sw128(smem_u32(smem + s * stage_bytes + kWTileBytes + BT * kXBox));
+        const uint32_t a_tmem = tmem + a_col0 + 64u * static_cast<uint32_t>(a);
+#pragma unroll
+        for (int kk = 0; kk < kKB / 32; ++kk)
+          umma_i8_ts(d_tmem, a_tmem + 8 * kk, (kk < 4 ? bdesc0 : bdesc1) + 2 * (kk & 3), idesc,
+                     (first && kk == 0) ? 0u : 1u);
+        first = false;
+        umma_commit(&hdr->done[i % kDoneRing]);
+        if (++a == nas) {
+          a = 0;
+          ++aph;
+        }
+        if (i == total - 1 || kb == kbn - 1) {  // the segment ends
+          umma_commit(&hdr->acc_full[seg & 1]);
+          ++seg;
+        }
+        if (++s == ns) {
+          s = 0;
+          ++ph;
+        }
       }
     }
   } else if (warp < 6) {
@@ -471,24 +310,24 @@ __global__ void __launch_bounds__(kPThreads, 1)
     const int quad = warp & 3;
     const int row = quad * 32 + lane;
     const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
-    int it = 0;
-    bool ok = true;
-    for (int tile = blockIdx.x; tile < p.num_tiles && ok; tile += gridDim.x) {
-      for (int kb = 0; kb < kbn; ++kb, ++it) {
-        const int s = it % ns, a = it % kPASlots;
-        bool w = mbar_wait(&hdr->full[s], (it / ns) & 1);
-        if (w && it >= kPASlots) w = mbar_wait(&hdr->a_empty[a], ((it / kPASlots) - 1) & 1);
-        ok = __all_sync(0xffffffffu, w);  // tcgen05.st below is warp-collective
-        if (!ok) break;
-        unpack_row_to_tmem(smem + s * stage_bytes, row, tmem + lane_base + kPAColBase + 32 * a);
-        tmem_wait_st();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) {
-          mbar_arrive(&hdr->empty[s]);
-          mbar_arrive(&hdr->a_full[a]);
-        }
+    for (int it = 0, s = 0, ph = 0, a = 0; it < total; ++it) {
+      bool w = mbar_wait(&hdr->full[s], ph & 1);
+      if (w && it >= nas) {
+        const int u = it - nas;  // the unit that last used A slot a
+        w = mbar_wait(&hdr->done[u % kDoneRing], (u / kDoneRing) & 1);
       }
+      if (!__all_sync(0xffffffffu, w)) break;  // tcgen05.st below is warp-collective
+      tc_fence_after();
+      unpack_row_to_tmem(smem + s * stage_bytes, row, tmem + lane_base + a_col0 + 64u * static_cast<uint32_t>(a));
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&hdr->a_full[a]);
+      if (++s == ns) {
+        s = 0;
+        ++ph;
+      }
+      if (++a == nas) a = 0;
     }
   } else {
     // ------------------------------------------------ epilogue
@@ -496,38 +335,134 @@ __global__ void __launch_bounds__(kPThreads, 1)
     const int row = quad * 32 + lane;
     const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
     const int et = threadIdx.x - 192;  // 0..127
-    pdl_wait();  // s_a comes from the preceding prologue kernel
-    int tc = 0;
-    for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++tc) {
-      const int b = tc & 1;
+    pdl_wait();  // s_a and the zeroed counters come from the preceding kernel
+    int seg = 0, seg_kb0 = 0, tile, kb;
+    unit_first(p, u0, tile, kb);
+    for (int i = 0; i < total; ++i, unit_next(p, tile, kb)) {
+      if (i == 0 || kb == 0) seg_kb0 = kb;
+      if (!(i == total - 1 || kb == kbn - 1)) continue;
+      // Segment `seg` (K blocks seg_kb0 .. kb of `tile`) ends at unit i.
+      const int b = seg & 1;
+      const bool whole = seg_kb0 == 0 && kb == kbn - 1;
       const int m0 = (tile % p.m_tiles) * BT, n0 = (tile / p.m_tiles) * kRows;
       float* sa = sa_buf + 192 * b;
       if (SINK != static_cast<int>(GemmSink::kS32))
         for (int c = et; c < BT; c += 128) sa[c] = (m0 + c < p.M) ? __ldg(p.s_a + m0 + c) : 0.0f;
-      named_barrier(1, 128);  // s_a of this tile staged; all warps are done with tile tc - 2
+      named_barrier(1, 128);  // s_a staged; all warps are done with segment seg - 2
       const int n = n0 + row;
       const float sw = (SINK != static_cast<int>(GemmSink::kS32) && n < p.N) ? __ldg(p.s_w + n) : 0.0f;
       const float bv = (p.bias && n < p.N) ? __uint_as_float(static_cast<uint32_t>(__ldg(p.bias + n)) << 16) : 0.0f;
-      // On a failed wait the warp skips the tile's work but keeps taking part
-      // in the named barrier above, so no peer waits on it forever.
-      const bool ok = __all_sync(0xffffffffu, mbar_wait(&hdr->acc_full[b], (tc / 2) & 1));
+      // On a failed wait the warp skips the segment's data but keeps taking
+      // part in the named barriers and the counter protocol, so no peer (in
+      // this CTA or another) is left waiting and the counters stay balanced.
+      const bool ok = __all_sync(0xffffffffu, mbar_wait(&hdr->acc_full[b], (seg / 2) & 1));
       tc_fence_after();
-      const uint32_t acc = tmem + lane_base + static_cast<uint32_t>(b) * kPAccStride;
-      for (int c = 0; ok && c < BT; c += 16) {
-        uint32_t v[16];
-        tmem_ld_32x32b_x16(acc + static_cast<uint32_t>(c), v);
-        tmem_wait_ld();
-        if (n < p.N) {
+      const uint32_t acc = tmem + lane_base + static_cast<uint32_t>(b * p.acc_stride);
+      if (whole) {
+        for (int c = 0; ok && c < BT; c += 16) {
+          uint32_t v[16];
+          tmem_ld_32x32b_x16(acc + static_cast<uint32_t>(c), v);
+          tmem_wait_ld();
+          if (n < p.N) {
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const int m = m0 + c + j;
-            if (m < p.M) store_output<SINK>(p, m, n, static_cast<int32_t>(v[j]), sa[c + j], sw, bv);
+            for (int j = 0; j < 16; ++j) {
+              const int m = m0 + c + j;
+              if (m < p.M) store_output<SINK>(p, m, n, static_cast<int32_t>(v[j]), sa[c + j], sw, bv);
+            }
           }
+        }
+      } else {
+        // Partial tile: publish it, then count the arrival.
+        int32_t* mine = p.slots + static_cast<size_t>(2 * blockIdx.x + (seg == 0 ? 0 : 1)) * BT * kRows;
+        for (int c = 0; ok && c < BT; c += 16) {
+          uint32_t v[16];
+          tmem_ld_32x32b_x16(acc + static_cast<uint32_t>(c), v);
+          tmem_wait_ld();
+          int4* dst = reinterpret_cast<int4*>(slot_chunk(mine, c, row));
+#pragma unroll
+          for (int r = 0; r < 4; ++r)
+            dst[r] = make_int4(static_cast<int32_t>(v[4 * r]), static_cast<int32_t>(v[4 * r + 1]),
+                               static_cast<int32_t>(v[4 * r + 2]), static_cast<int32_t>(v[4 * r + 3]));
+        }
+        __threadfence();        // this thread's slot stores precede the arrival below
+        named_barrier(1, 128);  // ... for all 128 threads
+        const int c_first = sk_owner(p, tile * kbn), c_last = sk_owner(p, tile * kbn + kbn - 1);
+        if (et == 0)
+          hdr->last_flag = atomicAdd(p.ctr + tile, 1u) == static_cast<uint32_t>(c_last - c_first) ? 1u : 0u;
+        named_barrier(1, 128);
+        if (hdr->last_flag) {
+          __threadfence();  // every other contributor's slot is visible now
+          // 32 tokens at a time: the own accumulator from tensor memory plus
+          // the other contributors' slots.
+          for (int h = 0; ok && h < BT; h += 32) {
+            int32_t sum[32];
+#pragma unroll
+            for (int q = 0; q < 2; ++q) {
+              if (h + 16 * q < BT) {  // uniform across the warp (tcgen05.ld is collective)
+                uint32_t v[16];
+                tmem_ld_32x32b_x16(acc + static_cast<uint32_t>(h + 16 * q), v);
+                tmem_wait_ld();
+#pragma unroll
+                for (int j = 0; j < 16; ++j) sum[16 * q + j] = static_cast<int32_t>(v[j]);
+              }
+            }
+            // Two contributors per round: 16 independent 16-byte loads in flight.
+            for (int cc = c_first;;) {
+              int sl[2] = {-1, -1};
+#pragma unroll
+              for (int e = 0; e < 2; ++e) {
+                if (cc == static_cast<int>(blockIdx.x)) ++cc;
+                // Tile `tile` is CTA cc's first segment when cc's range
+                // starts inside it, else its last.
+                if (cc <= c_last) sl[e] = 2 * cc + (sk_begin(p, cc) >= tile * kbn ? 0 : 1), ++cc;
+              }
+              if (sl[0] < 0) break;
+              int4 v[2][8];
+#pragma unroll
+              for (int e = 0; e < 2; ++e) {
+                if (sl[e] < 0) continue;
+                int32_t* other = p.slots + static_cast<size_t>(sl[e]) * BT * kRows;
+#pragma unroll
+                for (int q = 0; q < 2; ++q) {
+                  if (h + 16 * q < BT) {
+                    const int4* src = reinterpret_cast<const int4*>(slot_chunk(other, h + 16 * q, row));
+#pragma unroll
+                    for (int r = 0; r < 4; ++r) v[e][4 * q + r] = __ldcg(src + r);
+                  }
+                }
+              }
+#pragma unroll
+              for (int e = 0; e < 2; ++e) {
+                if (sl[e] < 0) continue;
+#pragma unroll
+                for (int q = 0; q < 2; ++q) {
+                  if (h + 16 * q < BT) {
+#pragma unroll
+                    for (int r = 0; r < 4; ++r) {
+                      sum[16 * q + 4 * r] += v[e][4 * q + r].x;
+                      sum[16 * q + 4 * r + 1] += v[e][4 * q + r].y;
+                      sum[16 * q + 4 * r + 2] += v[e][4 * q + r].z;
+                      sum[16 * q + 4 * r + 3] += v[e][4 * q + r].w;
+                    }
+                  }
+                }
+              }
+            }
+            if (n < p.N) {
+#pragma unroll
+              for (int j = 0; j < 32; ++j) {
+                const int m = m0 + h + j;
+                if (h + j < BT && m < p.M) store_output<SINK>(p, m, n, sum[j], sa[h + j], sw, bv);
+              }
+            }
+          }
+          if (et == 0) p.ctr[tile] = 0u;  // ready for the next launch
         }
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&hdr->acc_empty[b]);
+      ++seg;
     }
   }
 
@@ -573,45 +508,11 @@ bool make_map_u8(CUtensorMap* map, const void* base, uint64_t rows, uint64_t col
   return r == CUDA_SUCCESS;
 }
 
-int shared_bytes_for(int BT, int nstages, int splits) {
-  int bytes = 1024 /*alignment slack*/ + nstages * (kWTileBytes + BT * kKB) + 2048 /*header + s_a tile*/;
-  if (splits > 1) bytes += splits * ((BT / 4 + splits - 1) / splits) * kRows * 16;
-  return bytes;
-}
-
 template <int SINK>
-cudaError_t launch_sink(const CUtensorMap& tw, const CUtensorMap& tx, const Params& prm, const GemmTiling& t,
+cudaError_t launch_sink(const CUtensorMap& tw, const CUtensorMap& tx, const PParams& prm, const GemmTiling& t,
                         cudaStream_t stream) {
   static int cache[64] = {0};
-  cudaError_t e = ensure_dynamic_smem(reinterpret_cast<const void*>(w4a4_tc_gemm_kernel<SINK>), t.smem_bytes, cache);
-  if (e != cudaSuccess) return note_cuda(e, "w4a4_gemm: dynamic shared memory attribute");
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(t.n_tiles, t.m_tiles, t.splits);
-  cfg.blockDim = dim3(kThreads, 1, 1);
-  cfg.dynamicSmemBytes = static_cast<size_t>(t.smem_bytes);
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[2];
-  int nattr = 0;
-  attr[nattr].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[nattr].val.programmaticStreamSerializationAllowed = 1;
-  ++nattr;
-  if (t.splits > 1) {
-    attr[nattr].id = cudaLaunchAttributeClusterDimension;
-    attr[nattr].val.clusterDim.x = 1;
-    attr[nattr].val.clusterDim.y = 1;
-    attr[nattr].val.clusterDim.z = static_cast<unsigned>(t.splits);
-    ++nattr;
-  }
-  cfg.attrs = attr;
-  cfg.numAttrs = nattr;
-  return note_cuda(cudaLaunchKernelEx(&cfg, w4a4_tc_gemm_kernel<SINK>, tw, tx, prm), "w4a4_gemm: launch");
-}
-
-template <int SINK>
-cudaError_t launch_persistent(const CUtensorMap& tw, const CUtensorMap& tx, const PParams& prm, const GemmTiling& t,
-                              cudaStream_t stream) {
-  static int cache[64] = {0};
-  const void* kfn = reinterpret_cast<const void*>(w4a4_tc_gemm_persistent_kernel<SINK>);
+  const void* kfn = reinterpret_cast<const void*>(w4a4_tc_gemm_kernel<SINK>);
   cudaError_t e = ensure_dynamic_smem(kfn, t.smem_bytes, cache);
   if (e != cudaSuccess) return note_cuda(e, "w4a4_gemm: dynamic shared memory attribute");
   cudaLaunchConfig_t cfg = {};
@@ -624,152 +525,165 @@ cudaError_t launch_persistent(const CUtensorMap& tw, const CUtensorMap& tx, cons
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return note_cuda(cudaLaunchKernelEx(&cfg, w4a4_tc_gemm_persistent_kernel<SINK>, tw, tx, prm),
-                   "w4a4_gemm: persistent launch");
+  return note_cuda(cudaLaunchKernelEx(&cfg, w4a4_tc_gemm_kernel<SINK>, tw, tx, prm), "w4a4_gemm: launch");
 }
 
-// Estimated cycles of the persistent kernel for a token tile of BT: rounds
-// of tiles per SM x k blocks x the slower of the MMA (2 * BT cycles per k
-// block at 8192 int8 MACs/clk) and a per-k-block floor of 256 cycles for the
-// fixed work every k block carries whatever BT is (the 8 KB weight tile
-// fetched from L2 and unpacked into tensor memory).
+// Estimated cycles of the whole-tile schedule for a token tile of BT: rounds
+// of tiles per SM x units x the slower of the MMA (4 * BT cycles per 256-K
+// unit at 8192 int8 MACs/clk) and a per-unit floor of 640 cycles that every
+// unit costs whatever BT is (issuing its 8 MMAs and commit, and the 16 KB
+// weight tile fetched and unpacked into tensor memory).
 long persistent_cost(int M, int N, int K, int BT, int num_sms) {
   const long tiles = static_cast<long>((M + BT - 1) / BT) * ((N + kRows - 1) / kRows);
   const long rounds = (tiles + num_sms - 1) / num_sms;
-  const long per_kb = 2L * BT > 256 ? 2L * BT : 256;
-  return rounds * (K / kKB) * per_kb;
+  const long per_unit = 4L * BT > 640 ? 4L * BT : 640;
+  return rounds * (K / kKB) * per_unit;
 }
 
 }  // namespace
 
+namespace {
+
+// Stages of BT-token units that fit the shared memory of one CTA, and the
+// dynamic shared memory for them (padded so that one CTA, which owns all of
+// tensor memory, occupies an SM).
+void set_stages(GemmTiling& t) {
+  const int stage = kWTileBytes + t.BT * kKB;
+  int ns = (220 * 1024 - 4096) / stage;
+  if (ns > kMaxStages) ns = kMaxStages;
+  t.nstages = ns;
+  t.smem_bytes = 1024 + ns * stage + 1024 + 2 * 192 * 4;
+  if (t.smem_bytes < 120 * 1024) t.smem_bytes = 120 * 1024;
+  // Tensor memory: two accumulators of BT (rounded up to 32) columns, then
+  // 64-column A slots in the rest of the 512.
+  t.acc_stride = (t.BT + 31) / 32 * 32;
+  t.a_slots = (512 - 2 * t.acc_stride) / 64;
+  if (t.a_slots > kMaxASlots) t.a_slots = kMaxASlots;
+}
+
+}  // namespace
+
+// Stream-K grid: the number of CTAs g (at most one per SM) with the lowest
+// modelled time.  The weights stream at the lower of the HBM rate and what g
+// SMs pull (kSmBps each); a split tile then costs its last CTA one round of
+// L2 loads (kRoundSec) per 32 tokens for every two other contributors.
+int streamk_grid(int units, int kbn, int BT, int max_grid) {
+  constexpr double kHbmBps = 6.0e12, kSmBps = 150e9, kRoundSec = 0.4e-6;
+  const double unit_w = kWTileBytes, unit_all = kWTileBytes + static_cast<double>(BT) * kKB;
+  double best = 0;
+  int best_g = 1;
+  const int gmax = units < max_grid ? units : max_grid;
+  for (int g = 1; g <= gmax; ++g) {
+    const int most = (units + g - 1) / g, least = units / g;
+    int parts = 1;  // contributors of the most split tile
+    if (!(units % g == 0 && least % kbn == 0)) {
+      parts = (kbn + least - 1) / least + 1;
+      if (units % g == 0 && kbn % least == 0) parts = kbn / least;
+    }
+    const double t_stream = std::max(units * unit_w / kHbmBps, most * unit_all / kSmBps);
+    const double t_red = ((parts - 1 + 1) / 2) * ((BT + 31) / 32) * kRoundSec;
+    const double t = t_stream + t_red;
+    if (g == 1 || t < best * 0.999) {
+      best = t;
+      best_g = g;
+    }
+  }
+  return best_g;
+}
+
+size_t streamk_scratch_bytes(const GemmTiling& t) {
+  if (!t.stream_k) return 0;
+  return static_cast<size_t>(2 * kMaxGemmGrid) * static_cast<size_t>(t.BT) * kRows * sizeof(int32_t);
+}
+
 GemmTiling choose_tiling(int M, int N, int K, int num_sms) {
   GemmTiling t{};
-  // Large M: the persistent kernel, with the token tile BT (multiple of 16,
-  // <= 192) of the lowest estimated cost, when it yields at least half as
-  // many tiles as SMs.
-  {
+  const int kbn = K / kKB;
+  const int G = num_sms < kMaxGemmGrid ? num_sms : kMaxGemmGrid;
+  t.n_tiles = (N + kRows - 1) / kRows;
+  // Large M: whole tiles, with the token tile BT (multiple of 16, <= 192) of
+  // the lowest estimated cost, when it yields at least half as many tiles as
+  // SMs.
+  if (M > 128) {
     int best_bt = 0;
     long best = -1;
     for (int bt = 192; bt >= 64; bt -= 16) {
-      const long tiles = static_cast<long>((M + bt - 1) / bt) * ((N + kRows - 1) / kRows);
-      if (2 * tiles < num_sms) continue;
-      const long c = persistent_cost(M, N, K, bt, num_sms);
+      const long tiles = static_cast<long>((M + bt - 1) / bt) * t.n_tiles;
+      if (2 * tiles < G) continue;
+      const long c = persistent_cost(M, N, K, bt, G);
       if (best < 0 || c < best) {
         best = c;
         best_bt = bt;
       }
     }
-    if (best_bt > 0 && M > 128) {
-      t.persistent = true;
+    if (best_bt > 0) {
+      t.stream_k = false;
       t.BT = best_bt;
       t.m_tiles = (M + best_bt - 1) / best_bt;
-      t.n_tiles = (N + kRows - 1) / kRows;
-      t.splits = 1;
-      t.kb_per_split = K / kKB;
-      const int stage = kWTileBytes + best_bt * kKB;
-      int ns = (220 * 1024 - 4096) / stage;
-      if (ns > 8) ns = 8;
-      t.nstages = ns;
-      t.tmem_cols = 512;
-      t.smem_bytes = 1024 + ns * stage + 1024 + 2 * 192 * 4;
-      if (t.smem_bytes < 120 * 1024) t.smem_bytes = 120 * 1024;  // one CTA per SM (it owns all of TMEM)
-      const long tiles = static_cast<long>(t.m_tiles) * t.n_tiles;
-      t.grid = static_cast<int>(tiles < num_sms ? tiles : num_sms);
+      t.units = t.m_tiles * t.n_tiles * kbn;
+      const int tiles = t.m_tiles * t.n_tiles;
+      t.grid = tiles < G ? tiles : G;
+      set_stages(t);
       return t;
     }
   }
-  // Small M: one CTA per (tile, K slice), slices of a tile form a cluster.
-  const int kb_total = K / kKB;
-  // Tokens per tile: one tile when M fits, else the fewest tiles of <= 192.
-  const int max_bt = 192;
-  int m_tiles = (M + max_bt - 1) / max_bt;
-  int bt = (M + m_tiles - 1) / m_tiles;
-  bt = ((bt + 15) / 16) * 16;
+  // Small M (or few tiles): stream-K over tiles of BT = M rounded up to 16
+  // (at most 128) tokens.
+  int bt = M <= 128 ? ((M + 15) / 16) * 16 : 128;
   if (bt < 16) bt = 16;
   t.BT = bt;
   t.m_tiles = (M + bt - 1) / bt;
-  t.n_tiles = (N + kRows - 1) / kRows;
-  // Split K across a cluster until the grid covers two CTAs per SM.
   const int tiles = t.m_tiles * t.n_tiles;
-  int splits = 1;
-  while (splits < 8 && tiles * splits * 2 <= 2 * num_sms && splits * 2 <= kb_total) splits *= 2;
-  const int kbps = (kb_total + splits - 1) / splits;  // the largest share
-  t.splits = splits;
-  t.kb_per_split = kbps;
-  // Pipeline depth: as many stages as fit two CTAs per SM (~110 KB each).
-  const int stage = kWTileBytes + bt * kKB;
-  int ns = (110 * 1024 - 3072 - (splits > 1 ? splits * ((bt / 4 + splits - 1) / splits) * kRows * 16 : 0)) / stage;
-  if (ns > 8) ns = 8;
-  if (ns > kbps) ns = kbps < 2 ? 2 : kbps;
-  if (ns < 2) ns = 2;
-  t.nstages = ns;
-  int cols = 32;
-  while (cols < bt + 32 * kASlots) cols *= 2;
-  t.tmem_cols = cols;
-  t.smem_bytes = shared_bytes_for(bt, ns, splits);
-  // Never let more CTAs share an SM than its 512 tensor-memory columns can
-  // hold: a CTA blocked in tcgen05.alloc while its cluster peers wait for it
-  // could deadlock.  Shared memory per CTA is padded so that at most
-  // 512 / cols CTAs fit in the SM's 228 KB.
-  const int max_ctas = 512 / cols;
-  const int min_smem = (228 * 1024) / (max_ctas + 1) + 1;
-  if (t.smem_bytes < min_smem) t.smem_bytes = min_smem;
-  t.persistent = false;
-  t.grid = t.n_tiles * t.m_tiles * t.splits;
+  t.units = tiles * kbn;
+  if (tiles > kMaxSplitTiles) {
+    // More tiles than counters (N > 128 * 1024): whole tiles balance anyway.
+    t.stream_k = false;
+    t.grid = tiles < G ? tiles : G;
+  } else {
+    t.stream_k = true;
+    t.grid = streamk_grid(t.units, kbn, bt, G);
+  }
+  set_stages(t);
   return t;
 }
 
 cudaError_t launch_w4a4_gemm(const GemmArgs& a, GemmSink sink, const GemmTiling& t, cudaStream_t stream) {
   CUtensorMap tw, tx;
   if (!make_map_u8(&tw, a.Wq, static_cast<uint64_t>(a.N), static_cast<uint64_t>(a.K / 2), kRows, kKB / 2,
-                   CU_TENSOR_MAP_SWIZZLE_64B))
+                   CU_TENSOR_MAP_SWIZZLE_128B))
     return note_cuda(cudaErrorInvalidValue, "w4a4_gemm: weight tensor map");
   if (!make_map_u8(&tx, a.xs8, static_cast<uint64_t>(a.M), static_cast<uint64_t>(a.K), static_cast<uint32_t>(t.BT),
-                   kKB, CU_TENSOR_MAP_SWIZZLE_128B))
+                   kXBox, CU_TENSOR_MAP_SWIZZLE_128B))
     return note_cuda(cudaErrorInvalidValue, "w4a4_gemm: activation tensor map");
-  if (t.persistent) {
-    PParams pp{};
-    pp.s_a = a.s_a;
-    pp.s_w = a.s_w;
-    pp.bias = a.bias;
-    pp.out = a.out;
-    pp.M = a.M;
-    pp.N = a.N;
-    pp.K = a.K;
-    pp.BT = t.BT;
-    pp.m_tiles = t.m_tiles;
-    pp.num_tiles = t.m_tiles * t.n_tiles;
-    pp.nstages = t.nstages;
-    cudaError_t e;
-    switch (sink) {
-      case GemmSink::kBF16: e = launch_persistent<0>(tw, tx, pp, t, stream); break;
-      case GemmSink::kF32: e = launch_persistent<1>(tw, tx, pp, t, stream); break;
-      default: e = launch_persistent<2>(tw, tx, pp, t, stream); break;
-    }
-    count_dispatch(2);
-    return e;
-  }
-  Params prm{};
-  prm.s_a = a.s_a;
-  prm.s_w = a.s_w;
-  prm.bias = a.bias;
-  prm.out = a.out;
-  prm.M = a.M;
-  prm.N = a.N;
-  prm.K = a.K;
-  prm.BT = t.BT;
-  prm.splits = t.splits;
-  prm.kb_total = a.K / kKB;
-  prm.kb_per_split = t.kb_per_split;
-  prm.nstages = t.nstages;
-  prm.tmem_cols = t.tmem_cols;
+  if (t.grid < 1 || t.grid > kMaxGemmGrid || (t.stream_k && (!a.ctr || !a.slots)) || t.a_slots < 2 ||
+      t.nstages < 1 || t.nstages > kMaxStages)
+    return note_cuda(cudaErrorInvalidValue, "w4a4_gemm: tiling");
+  PParams pp{};
+  pp.s_a = a.s_a;
+  pp.s_w = a.s_w;
+  pp.bias = a.bias;
+  pp.out = a.out;
+  pp.M = a.M;
+  pp.N = a.N;
+  pp.K = a.K;
+  pp.BT = t.BT;
+  pp.m_tiles = t.m_tiles;
+  pp.num_tiles = t.m_tiles * t.n_tiles;
+  pp.nstages = t.nstages;
+  pp.kbn = a.K / kKB;
+  pp.acc_stride = t.acc_stride;
+  pp.a_slots = t.a_slots;
+  pp.stream_k = t.stream_k ? 1 : 0;
+  pp.units = t.units;
+  pp.ctr = a.ctr;
+  pp.slots = a.slots;
   cudaError_t e;
   switch (sink) {
-    case GemmSink::kBF16: e = launch_sink<0>(tw, tx, prm, t, stream); break;
-    case GemmSink::kF32: e = launch_sink<1>(tw, tx, prm, t, stream); break;
-    default: e = launch_sink<2>(tw, tx, prm, t, stream); break;
+    case GemmSink::kBF16: e = launch_sink<0>(tw, tx, pp, t, stream); break;
+    case GemmSink::kF32: e = launch_sink<1>(tw, tx, pp, t, stream); break;
+    default: e = launch_sink<2>(tw, tx, pp, t, stream); break;
   }
-  count_dispatch(t.splits > 1 ? 3 : 2);
+  count_dispatch(t.stream_k ? 3 : 2);
   return e;
 }
 

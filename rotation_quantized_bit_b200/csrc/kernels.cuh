@@ -18,29 +18,40 @@ struct RotateQuantOut {
   uint8_t* packed;  // [M, K/2] two codes per byte, or null
   int8_t* s8;       // [M, K] codes as signed bytes in chunk order (0,2,4,6,1,3,5,7), or null
   float* scale;     // [M]
+  uint32_t* zero;   // [nzero] words set to zero (the GEMM's tile counters), or null
+  int nzero;
 };
 
 cudaError_t launch_rotate_quant(const uint16_t* x, int M, int K, RotateQuantOut out, cudaStream_t stream);
 
 // Packed codes [M, K/2] -> signed-byte operand layout [M, K].
-cudaError_t launch_unpack_codes(const uint8_t* packed, int M, int K, int8_t* s8, cudaStream_t stream);
+// Also sets zero[0 .. nzero) to zero (the GEMM's tile counters) when non-null.
+cudaError_t launch_unpack_codes(const uint8_t* packed, int M, int K, int8_t* s8, uint32_t* zero, int nzero,
+                                cudaStream_t stream);
 
 enum class GemmSink : int { kBF16 = 0, kF32 = 1, kS32 = 2 };
 
+// Limits of the stream-K scratch reserved in the workspace.
+constexpr int kMaxGemmGrid = 160;     // CTAs (one per SM); two partial-tile slots each
+constexpr int kMaxSplitTiles = 1024;  // per-tile arrival counters
+
 struct GemmTiling {
-  bool persistent;  // one CTA per SM over all tiles (large M) vs one CTA per tile/split (small M)
-  int grid;         // CTAs launched
-  int BT;           // tokens per CTA tile (MMA N), multiple of 16 in [16, 192]
+  bool stream_k;    // stream-K ranges of K-block units (small M) vs whole tiles round-robin (large M)
+  int grid;         // CTAs launched, at most one per SM
+  int BT;           // tokens per tile (MMA N), multiple of 16 in [16, 192]
   int m_tiles;      // ceil(M / BT)
   int n_tiles;      // ceil(N / 128)
-  int splits;       // split-K factor = cluster size (1 .. 8)
-  int kb_per_split; // 128-wide K blocks per split
+  int units;        // m_tiles * n_tiles * K / 128
   int nstages;      // depth of the shared-memory TMA ring
-  int tmem_cols;    // tensor-memory columns allocated per CTA (power of two)
   int smem_bytes;   // dynamic shared memory per CTA
+  int acc_stride;   // tensor-memory columns per accumulator
+  int a_slots;      // 64-column tensor-memory slots for unpacked weights
 };
 
 GemmTiling choose_tiling(int M, int N, int K, int num_sms);
+
+// Bytes of partial-tile slots a tiling needs (0 for whole tiles).
+size_t streamk_scratch_bytes(const GemmTiling& t);
 
 struct GemmArgs {
   const int8_t* xs8;      // [M, K] activation codes (operand layout)
@@ -50,6 +61,8 @@ struct GemmArgs {
   const uint16_t* bias;   // [N] or null
   void* out;              // [M, N] bf16 / f32 / s32
   int M, N, K;
+  uint32_t* ctr;          // [kMaxSplitTiles] tile counters, zero on entry (stream-K)
+  int32_t* slots;         // streamk_scratch_bytes of partial tiles (stream-K)
 };
 
 // Builds the tensor maps and launches the tensor-core GEMM.

@@ -48,7 +48,7 @@ extern "C" convrot_status_t convrot_w4a4_linear_noalloc(const uint16_t* x, const
   if (need == 0 || N < 1 || N % 8 != 0) return CONVROT_ERR_SHAPE;
   if (need > kNoAllocScratchBytes) {
     char msg[160];
-    snprintf(msg, sizeof(msg), "convrot_w4a4_linear_noalloc: M*K needs %zu bytes of scratch, above the %zu-byte limit",
+    snprintf(msg, sizeof(msg), "convrot_w4a4_linear_noalloc: the shape needs %zu bytes of scratch, above the %zu-byte limit",
              need, kNoAllocScratchBytes);
     note_cuda(cudaErrorInvalidValue, msg);
     return CONVROT_ERR_WORKSPACE;
@@ -66,6 +66,7 @@ extern "C" convrot_status_t convrot_w4a4_linear_noalloc(const uint16_t* x, const
     g_scratch_ptr[dev] = p;
   }
   // Nothing in the scratch needs to start at zero: the first kernel writes
-  // every code and scale that the second one reads.
+  // every code and scale that the second one reads and zeroes the GEMM's
+  // tile counters.
   return convrot_w4a4_linear(x, Wq, s_w, bias, M, N, K, y, g_scratch_ptr[dev], kNoAllocScratchBytes, stream);
 }

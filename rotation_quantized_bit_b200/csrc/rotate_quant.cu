@@ -28,12 +28,19 @@
 // while the current one is computed.  Codes leave through the same buffer
 // and coalesced 16-byte stores.
 //
-// Quantization.  y = x' * rcp(s) (rcp correctly rounded), then rint via the
-// addition of 1.5 * 2^23, whose low byte is the two's-complement code.  For
-// |y| < 8, y and the correctly rounded quotient differ by less than 2^-19.8,
-// so the codes agree unless some |y - rint(y)| lies within 2^-19 of one half;
-// a lane that sees such a value (or a row whose scale is subnormal or zero)
-// recomputes its codes with the correctly rounded division.
+// Quantization.  The code is rint(q) with q the correctly rounded quotient
+// x' / s.  q is formed without a division by Markstein's correction (P.
+// Markstein, "Computation of elementary functions on the IBM RISC System/6000
+// processor", IBM J. Res. Develop. 34(1), 1990; restated as Markstein's
+// theorem in Muller et al., "Handbook of Floating-Point Arithmetic", ch. on
+// division with an FMA): with y = RN(1/s), q0 = RN(x' y) is within two ulps of
+// x'/s; one step q1 = RN(q0 + RN(x' - s q0) y) makes it faithful, and a second
+// step from a faithful q1, whose remainder x' - s q1 is exact, returns
+// RN(x'/s) itself.  Both remainders are fused multiply-adds.  The theorem needs
+// the remainders and products clear of underflow, which holds for every scale
+// s >= 2^-100 wherever the code can be nonzero; rows with a smaller scale (zero
+// included) take the IEEE division.  rint is the addition of 1.5 * 2^23, whose
+// low byte is then the two's-complement code.
 #include <cuda_runtime.h>
 
 #include <cstdint>
@@ -49,8 +56,7 @@ typedef unsigned long long u64;
 constexpr int kTileBytes = 8192;          // 16 groups x 256 bf16 per warp
 constexpr int kMaxWarps = 8;              // at most 128 groups per row block
 constexpr float kMagic = 12582912.0f;     // 1.5 * 2^23: x + kMagic rounds x to an integer, ties to even
-constexpr float kTieGuard = 0.5f - 1.0f / 524288.0f;  // 0.5 - 2^-19
-constexpr float kMinNormal = 1.17549435e-38f;         // 2^-126
+constexpr float kMinScale = 7.88860905e-31f;           // 2^-100: below it, codes by division
 
 // ---------------------------------------------------------------- helpers
 
@@ -75,6 +81,11 @@ __device__ __forceinline__ u64 f2_sub(u64 a, u64 b) {
 __device__ __forceinline__ u64 f2_mul(u64 a, u64 b) {
   u64 d;
   asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ u64 f2_fma(u64 a, u64 b, u64 c) {
+  u64 d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
   return d;
 }
 __device__ __forceinline__ float max3(float a, float b, float c) {
@@ -182,6 +193,8 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) rotate_quant_kernel(const _
   };
 
   for (int i = threadIdx.x; i < 2 * 128; i += blockDim.x) (&row_amax[0][0])[i] = 0u;
+  if (blockIdx.x == 0 && p.out.zero)
+    for (int i = threadIdx.x; i < p.out.nzero; i += blockDim.x) p.out.zero[i] = 0u;
   __syncthreads();
 
   int it = 0;
@@ -260,56 +273,40 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) rotate_quant_kernel(const _
     if (static_cast<int>(threadIdx.x) < 128) row_amax[(it + 1) & 1][threadIdx.x] = 0u;
 
     // ---- quantize into the staging area (region `lane` of `tile`)
-    const bool fast = scale >= kMinNormal;
-    float emax = 0.0f;
-    if (fast) {
+    if (scale >= kMinScale) {
       const float rcp = __frcp_rn(scale);
-      const u64 rr = f2(rcp, rcp), mg = f2(kMagic, kMagic);
+      const u64 rr = f2(rcp, rcp), ns = f2(-scale, -scale), mg = f2(kMagic, kMagic);
 #pragma unroll
       for (int k = 0; k < 8; k += 2) {
         // pairs 8k .. 8k+15 hold chunks k, k+1 (.x) and k+8, k+9 (.y)
         uint32_t cx[16], cy[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
-          const u64 y = f2_mul(P[8 * k + e], rr);
-          const u64 t = f2_add(y, mg);
-          const u64 d = f2_sub(y, f2_sub(t, mg));  // y - rint(y), exact
-          float tx, ty, dx, dy;
-          f2_split(t, tx, ty);
-          f2_split(d, dx, dy);
-          emax = max3(emax, fabsf(dx), fabsf(dy));
+          const u64 x = P[8 * k + e];
+          u64 q = f2_mul(x, rr);
+          q = f2_fma(f2_fma(ns, q, x), rr, q);  // faithful
+          q = f2_fma(f2_fma(ns, q, x), rr, q);  // RN(x / s)
+          float tx, ty;
+          f2_split(f2_add(q, mg), tx, ty);
           cx[e] = __float_as_uint(tx);
           cy[e] = __float_as_uint(ty);
         }
         stage_chunk_pair<PACKED>(tile, lane, k >> 1, cx);
         stage_chunk_pair<PACKED>(tile, lane, (k + 8) >> 1, cy);
       }
-    }
-    if (!fast || emax >= kTieGuard) {
-      // Exact path (rare): a zero or subnormal scale (every code by the
-      // division), or a lane with a value next to a tie (only those values
-      // are divided; the others keep the reciprocal result, which is exact
-      // for them).  A rolled loop over a local copy keeps this path small.
+    } else {
+      // Zero or tiny scale (a whole row takes this branch): IEEE division,
+      // in a rolled loop over a local copy to keep the code small.
       float v[128];
 #pragma unroll
       for (int i = 0; i < 64; ++i) f2_split(P[i], v[i], v[i + 64]);
-      const float rcp = fast ? __frcp_rn(scale) : 0.0f;
 #pragma unroll 1
       for (int k = 0; k < 16; ++k) {  // chunk k: channels 8k .. 8k+7 of the half
         uint32_t q[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
-          const float x = v[8 * k + e];
-          int qq = 0;
-          if (fast) {
-            const float y = __fmul_rn(x, rcp);
-            const float r = __fsub_rn(__fadd_rn(y, kMagic), kMagic);
-            qq = static_cast<int>(r);
-            if (fabsf(__fsub_rn(y, r)) >= kTieGuard) qq = __float2int_rn(__fdiv_rn(x, scale));
-          } else if (scale != 0.0f) {
-            qq = min(7, max(-8, __float2int_rn(__fdiv_rn(x, scale))));
-          }
-          q[e] = static_cast<uint32_t>(qq);
+          const int qq = scale != 0.0f ? __float2int_rn(__fdiv_rn(v[8 * k + e], scale)) : 0;
+          q[e] = static_cast<uint32_t>(min(7, max(-8, qq)));
         }
         if (PACKED) {
           uint32_t w = 0;
@@ -355,7 +352,9 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) rotate_quant_kernel(const _
 // nibbles (1,3,5,7).  u = nibble ^ 8 = q + 8 in [0, 15]; the signed byte is
 // (u + 0x78) ^ 0x80 = u - 8 (mod 256), with no carry between bytes.
 __global__ void __launch_bounds__(256) unpack_codes_kernel(const uint8_t* __restrict__ packed, int M, int K,
-                                                           int8_t* __restrict__ s8) {
+                                                           int8_t* __restrict__ s8, uint32_t* zero, int nzero) {
+  if (blockIdx.x == 0 && zero)
+    for (int i = threadIdx.x; i < nzero; i += blockDim.x) zero[i] = 0u;
   const int lane = threadIdx.x & 31;
   const int warps_per_block = blockDim.x / 32;
   const int nword = K >> 3;
@@ -453,11 +452,12 @@ cudaError_t launch_rotate_quant(const uint16_t* x, int M, int K, RotateQuantOut 
   return note_cuda(cudaGetLastError(), "rotate_quant: launch");
 }
 
-cudaError_t launch_unpack_codes(const uint8_t* packed, int M, int K, int8_t* s8, cudaStream_t stream) {
+cudaError_t launch_unpack_codes(const uint8_t* packed, int M, int K, int8_t* s8, uint32_t* zero, int nzero,
+                                cudaStream_t stream) {
   const int per_block = 8;
   int grid = (M + per_block - 1) / per_block;
   if (grid > num_sms_cached() * 8) grid = num_sms_cached() * 8;
-  unpack_codes_kernel<<<grid, 256, 0, stream>>>(packed, M, K, s8);
+  unpack_codes_kernel<<<grid, 256, 0, stream>>>(packed, M, K, s8, zero, nzero);
   count_dispatch(1);
   return note_cuda(cudaGetLastError(), "unpack_codes: launch");
 }

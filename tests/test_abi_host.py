@@ -51,6 +51,24 @@ def test_workspace_sizes(lib):
     assert lib.convrot_gemm_workspace_size(1220, 9728, 2560) >= 1220 * 2560
     assert lib.convrot_w4a4_workspace_size(32, 256, 300) == 0  # bad K
     assert lib.convrot_w4a4_workspace_size(0, 256, 512) == 0
+    assert lib.convrot_w4a4_workspace_size(32, 250, 512) == 0  # N % 8 != 0
+
+
+def _r256(v):
+    return (v + 255) // 256 * 256
+
+
+def test_workspace_layout(lib):
+    # Large M (whole tiles): codes, scales and 4 KB of tile counters.
+    M, N, K = 4224, 3840, 3840
+    assert lib.convrot_w4a4_workspace_size(M, N, K) == _r256(M * K) + _r256(4 * M) + 4096
+    assert lib.convrot_gemm_workspace_size(M, N, K) == lib.convrot_w4a4_workspace_size(M, N, K)
+    # Small M (stream-K): plus two partial tiles of BT x 128 int32 per CTA
+    # slot (160 slots), BT = M rounded up to 16.
+    for M, bt in ((1, 16), (16, 16), (76, 80), (128, 128)):
+        N, K = 9728, 2560
+        want = _r256(M * K) + _r256(4 * M) + 4096 + 2 * 160 * bt * 128 * 4
+        assert lib.convrot_w4a4_workspace_size(M, N, K) == want, (M, bt)
 
 
 FAKE = ctypes.c_void_p(0x10000)      # never dereferenced: validation fails first

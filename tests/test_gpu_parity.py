@@ -78,6 +78,57 @@ def special_rows(K=512):
     return synthetic.to_bf16_bits(np.stack(rows))
 
 
+def near_tie_rows(n_rows=384, K=512, seed=11):
+    """Rows whose quotients x'/s_a sit at or next to a half-integer, kept only
+    where a quotient formed as x' * fl(1/s_a) would round to another code than
+    the division: the cases a reciprocal-based quantizer gets wrong.
+
+    Each row holds A at channel 0 (group 0 rotates to +-A/16, the row amax)
+    and B at channel 256 (group 1 rotates to +-B/16).  Two families:
+      * exact ties: A = 7 m 2^e, B = (k + 1/2) m 2^e, so fl(A/16)/7 is exact
+        and B/16 divided by it is exactly k + 1/2;
+      * near ties: A = c B with c = 14 / (2k + 1), so the quotient is
+        (k + 1/2)(1 + d) with d the rounding of s_a = fl(fl(A/16) / 7).
+    The filter runs in numpy fp32 (IEEE division and multiplication)."""
+    rng = np.random.default_rng(seed)
+    f = np.float32
+    cand = []
+    for _ in range(40000):
+        if len(cand) >= 2 * n_rows:
+            break
+        k = int(rng.integers(0, 7))
+        e = float(2.0 ** int(rng.integers(-20, 20)))
+        if rng.random() < 0.5:
+            m = int(rng.integers(1, 37))
+            A, B = 7 * m * e, (k + 0.5) * m * e
+        else:
+            B = float(synthetic.bf16_bits_to_f32(synthetic.to_bf16_bits(np.array([rng.uniform(0.5, 1.0) * e])))[0])
+            A = 14.0 / (2 * k + 1) * B
+        bits = synthetic.to_bf16_bits(np.array([A, B]))
+        Af, Bf = synthetic.bf16_bits_to_f32(bits).astype(np.float32)
+        if Af != np.float32(A) or Bf != np.float32(B) or abs(Af) <= abs(Bf):
+            continue
+        s = f(f(Af / f(16)) / f(7))
+        x = f(Bf / f(16))
+        if np.rint(f(x / s)) != np.rint(f(x * f(f(1) / s))):
+            cand.append((float(Af), float(Bf)))
+    cand = sorted(set(cand))[:n_rows]
+    rows = np.zeros((len(cand), K))
+    for i, (A, B) in enumerate(cand):
+        rows[i, 0] = A
+        rows[i, 256] = -B if i % 2 else B
+    return synthetic.to_bf16_bits(rows)
+
+
+def test_rotate_quant_near_ties(rq):
+    x = near_tie_rows()
+    assert x.shape[0] >= 32, "the search found too few rows that separate division from reciprocal"
+    xq_ref, s_ref = oracle.rotate_quant(x)
+    xq, s = rq.convrot_rotate_quant(dev_bf16(x))
+    assert np.array_equal(f32_bits(host(s)), f32_bits(s_ref))
+    assert np.array_equal(host(xq), xq_ref)
+
+
 @pytest.mark.parametrize("M", [1, 7, 77, 300, 1220])
 @pytest.mark.parametrize("K", [256, 512, 2560, 3072, 3840, 9728, 12288, 32768])
 def test_rotate_quant_shape_grid(rq, M, K):
@@ -111,6 +162,9 @@ def test_pack_weight_bit_exact(rq, workload, N, K):
 
 GEMM_CASES = [(8, 256, 256), (32, 256, 512), (77, 264, 768), (1, 128, 2560), (16, 2560, 2560),
               (200, 384, 1024), (300, 1000, 512), (193, 136, 256), (600, 4096, 512),
+              # stream-K: one tile over 96 CTAs; CTAs with two partial tiles;
+              # ragged N with more units than SMs; the largest small-M tile
+              (3, 8, 12288), (16, 1032, 9728), (128, 2056, 768), (64, 136, 32768),
               # persistent large-M path: several tiles per SM, ragged M and N tails
               (1000, 1280, 1024), (777, 2056, 768), (2100, 1024, 256)]
 
@@ -175,6 +229,28 @@ def test_linear_matches_oracle(rq, workload, M, K, N):
     assert np.array_equal(f32_bits(y32), f32_bits(y32_ref))
     y16 = host_bits(rq.convrot_w4a4_linear(dx, dwq, dsw, db))
     assert bf16_ulp_diff(y16, y16_ref).max() <= 1
+
+
+def test_quantize_once_gemm_many(rq):
+    # Projections sharing one input: one quantization, several GEMMs on the
+    # same workspace (the stream-K tile counters must be back at zero after
+    # each), then the counters read back.
+    M, K = 76, 2560
+    x = synthetic.activations("qwen3_4b", M, K)
+    xq_ref, s_a = oracle.rotate_quant(x)
+    shapes = [4096, 1024, 1032, 9728]
+    ws = torch.empty(max(rq.convrot_w4a4_workspace_size(M, N, K) for N in shapes), dtype=torch.uint8,
+                     device="cuda")
+    rq.convrot_w4a4_quantize(dev_bf16(x), ws)
+    for N in shapes:
+        w, b = synthetic.weights("qwen3_4b", N, K)
+        wq, s_w = oracle.pack_weight(w)
+        y16_ref = oracle.epilogue(oracle.gemm_s64(xq_ref, wq, K), s_a, s_w, b)[1]
+        y16 = host_bits(rq.convrot_w4a4_gemm_quantized(ws, M, dev(wq), dev(s_w), dev_bf16(b)))
+        assert bf16_ulp_diff(y16, y16_ref).max() <= 1, N
+    r256 = lambda v: (v + 255) // 256 * 256
+    ctr_off = r256(M * K) + r256(4 * M)
+    assert int(ws[ctr_off:ctr_off + 4096].count_nonzero()) == 0
 
 
 def test_linear_special_rows(rq):
@@ -258,5 +334,5 @@ def test_dispatch_counts_and_no_device_error(rq):
     rq.convrot_w4a4_linear(x, wq, s_w, dev_bf16(b))
     after = rq.convrot_dispatch_counts()
     assert after["rotate_quant"] == before["rotate_quant"] + 2
-    assert after["tc_gemm"] + after["tc_gemm_splitk"] == before["tc_gemm"] + before["tc_gemm_splitk"] + 1
+    assert after["tc_gemm"] + after["tc_gemm_streamk"] == before["tc_gemm"] + before["tc_gemm_streamk"] + 1
     assert rq.convrot_device_error() == 0
