@@ -315,7 +315,7 @@ def main():
         launches = 2 * nlin * args.steps
     else:
         launches = (counts1["rotate_quant"] - counts0["rotate_quant"]) + (counts1["tc_gemm"] - counts0["tc_gemm"]) + \
-                   (counts1["tc_gemm_streamk"] - counts0["tc_gemm_streamk"])
+                   (counts1["tc_gemm_splitk"] - counts0["tc_gemm_splitk"])
 
     # per-linear times of the timed steps, and per-kernel times of the breakdown
     # steps (ms), summed over the K steps

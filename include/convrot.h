@@ -84,10 +84,8 @@ convrot_status_t convrot_pack_weight(const uint16_t *W, int N, int K, uint8_t *W
 convrot_status_t convrot_rotate_quant(const uint16_t *x, int M, int K, uint8_t *xq, float *s_a,
                                       void *stream);
 
-/* Bytes of workspace w4a4_gemm* needs for (M, N, K) on the current device
- * (0 for an invalid shape).  It holds the activation codes widened to bytes,
- * 4 KB of tile counters and, for small M, the partial tiles of the stream-K
- * schedule (2 x 160 x BT x 512 bytes, BT = M rounded up to 16, at most 128). */
+/* Bytes of workspace w4a4_gemm* needs for (M, N, K) (0 for an invalid
+ * shape): the activation codes widened to bytes, M * K rounded up to 256. */
 size_t convrot_gemm_workspace_size(int M, int N, int K);
 
 /* Integer GEMM with the rank-one epilogue (the "rank-one s4 MMA", same card,
@@ -117,9 +115,9 @@ convrot_status_t w4a4_gemm_f32(const uint8_t *xq, const float *s_a, const uint8_
                                float *y32, void *workspace, size_t workspace_bytes,
                                void *stream);
 
-/* Bytes of workspace convrot_w4a4_linear* needs for (M, N, K) on the current
- * device (0 for an invalid shape): the workspace of w4a4_gemm plus the M
- * per-token scales. */
+/* Bytes of workspace convrot_w4a4_linear* needs for (M, N, K) (0 for an
+ * invalid shape): the workspace of w4a4_gemm plus the M per-token scales,
+ * each part rounded up to 256 bytes. */
 size_t convrot_w4a4_workspace_size(int M, int N, int K);
 
 /* The fused ConvRot W4A4 Linear: y = W4A4(x) with x rotated and quantized
@@ -169,12 +167,9 @@ convrot_status_t convrot_w4a4_linear_noalloc(const uint16_t *x, const uint8_t *W
  *     in the GEMM's operand layout + per-token scales).  workspace_bytes >=
  *     convrot_w4a4_workspace_size(M, N, K) for every N it will be used with.
  *   convrot_w4a4_gemm_quantized: workspace (from convrot_w4a4_quantize with
- *     the same M, K) x Wq -> y [M, N] bf16.  It may be called several times
- *     on one quantization (e.g. projections that share their input), one
- *     call at a time per workspace: it only reads the codes and scales, and
- *     the tile counters it uses are back at zero when it completes.  After a
- *     device-side timeout (convrot_device_error) quantize again before the
- *     next convrot_w4a4_gemm_quantized. */
+ *     the same M, K) x Wq -> y [M, N] bf16.  It only reads the workspace, so
+ *     one quantization may serve several GEMMs (e.g. projections that share
+ *     their input). */
 convrot_status_t convrot_w4a4_quantize(const uint16_t *x, int M, int K, void *workspace,
                                        size_t workspace_bytes, void *stream);
 convrot_status_t convrot_w4a4_gemm_quantized(const uint8_t *Wq, const float *s_w,
@@ -200,9 +195,9 @@ convrot_status_t convrot_selftest_timeout(unsigned int limit_us, void *stream);
 
 /* Host-side count of how many times each kernel path was enqueued by this
  * process: counts[0] = rotate/quant prologue, [1] = packed-code unpack pass,
- * [2] = tensor-core GEMM over whole output tiles (large M), [3] = the same
- * GEMM under the stream-K schedule (small M: K blocks spread evenly over the
- * SMs, split tiles summed exactly through the workspace).  `n` is the array
+ * [2] = tensor-core GEMM over whole output tiles, [3] = the same GEMM with
+ * each tile's K split over a thread-block cluster (few tiles, small M; the
+ * partial tiles are summed exactly in shared memory).  `n` is the array
  * length; at most 4 are written. */
 void convrot_dispatch_counts(uint64_t *counts, int n);
 

@@ -292,7 +292,7 @@ def convrot_dispatch_counts():
     lib = load_library()
     arr = (ctypes.c_uint64 * 4)()
     lib.convrot_dispatch_counts(arr, 4)
-    return {"rotate_quant": arr[0], "unpack_codes": arr[1], "tc_gemm": arr[2], "tc_gemm_streamk": arr[3]}
+    return {"rotate_quant": arr[0], "unpack_codes": arr[1], "tc_gemm": arr[2], "tc_gemm_splitk": arr[3]}
 
 
 def convrot_version() -> str:

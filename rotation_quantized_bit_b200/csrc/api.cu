@@ -69,28 +69,13 @@ convrot_status_t check_device(int* sms_out);
 size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 // Workspace layout shared by the GEMM and the fused Linear:
-//   codes   [M*K] bytes        activation codes as signed bytes (operand layout)
-//   s_a     [M] float          per-token scales (fused Linear only)
-//   ctr     [kMaxSplitTiles]   per-tile arrival counters of the stream-K GEMM,
-//                              zeroed by the kernel that writes the codes and
-//                              left at zero by every GEMM that completes
-//   slots   partial int32 tiles of the stream-K GEMM (small M only)
+//   codes   [M*K] bytes   activation codes as signed bytes (operand layout)
+//   s_a     [M] float     per-token scales (fused Linear only)
 // each region starting on a 256-byte boundary.
 size_t codes_bytes(int M, int K) { return round_up(static_cast<size_t>(M) * static_cast<size_t>(K), 256); }
 size_t sa_offset(int M, int K) { return codes_bytes(M, K); }
-size_t ctr_offset(int M, int K) { return sa_offset(M, K) + round_up(static_cast<size_t>(M) * sizeof(float), 256); }
-size_t slots_offset(int M, int K) { return ctr_offset(M, K) + kMaxSplitTiles * sizeof(uint32_t); }
-
-// The tiling the GEMM will use on the current device (148 SMs assumed when
-// no device can be queried, as on a host without a GPU).
-GemmTiling tiling_for(int M, int N, int K) {
-  int sms = 0;
-  if (check_device(&sms) != CONVROT_OK || sms <= 0) sms = 148;
-  return choose_tiling(M, N, K, sms);
-}
-
-size_t workspace_bytes_for(int M, int N, int K) {
-  return slots_offset(M, K) + streamk_scratch_bytes(tiling_for(M, N, K));
+size_t workspace_bytes_for(int M, int K) {
+  return sa_offset(M, K) + round_up(static_cast<size_t>(M) * sizeof(float), 256);
 }
 
 convrot_status_t gemm_common(const uint8_t* xq, const float* s_a, const uint8_t* Wq, const float* s_w,
@@ -103,21 +88,16 @@ convrot_status_t gemm_common(const uint8_t* xq, const float* s_a, const uint8_t*
   if (!aligned16(xq) || !aligned16(Wq) || !aligned16(out) || (s_a && !aligned16(s_a)) ||
       (s_w && !aligned16(s_w)) || (bias && !aligned16(bias)))
     return CONVROT_ERR_ALIGN;
-  if (!ws || ws_bytes < workspace_bytes_for(M, N, K)) return CONVROT_ERR_WORKSPACE;
+  if (!ws || ws_bytes < codes_bytes(M, K)) return CONVROT_ERR_WORKSPACE;
   if (!aligned16(ws)) return CONVROT_ERR_ALIGN;
   int sms = 0;
   st = check_device(&sms);
   if (st != CONVROT_OK) return st;
-  const GemmTiling t = choose_tiling(M, N, K, sms);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  uint8_t* base = static_cast<uint8_t*>(ws);
-  int8_t* xs8 = reinterpret_cast<int8_t*>(base);
-  uint32_t* ctr = reinterpret_cast<uint32_t*>(base + ctr_offset(M, K));
-  int32_t* slots = reinterpret_cast<int32_t*>(base + slots_offset(M, K));
-  if (cudaError_t e = launch_unpack_codes(xq, M, K, xs8, ctr, kMaxSplitTiles, s); e != cudaSuccess)
-    return CONVROT_ERR_CUDA;
-  GemmArgs a{xs8, s_a, Wq, s_w, bias, out, M, N, K, ctr, slots};
-  return from_cuda(launch_w4a4_gemm(a, sink, t, s));
+  int8_t* xs8 = static_cast<int8_t*>(ws);
+  if (cudaError_t e = launch_unpack_codes(xq, M, K, xs8, s); e != cudaSuccess) return CONVROT_ERR_CUDA;
+  GemmArgs a{xs8, s_a, Wq, s_w, bias, out, M, N, K};
+  return from_cuda(launch_w4a4_gemm(a, sink, choose_tiling(M, N, K, sms), s));
 }
 
 convrot_status_t quantize_common(const uint16_t* x, int M, int K, void* ws, size_t ws_bytes, void* stream) {
@@ -125,13 +105,12 @@ convrot_status_t quantize_common(const uint16_t* x, int M, int K, void* ws, size
   convrot_status_t st = check_mk(M, K);
   if (st != CONVROT_OK) return st;
   if (!aligned16(x)) return CONVROT_ERR_ALIGN;
-  if (!ws || ws_bytes < slots_offset(M, K)) return CONVROT_ERR_WORKSPACE;
+  if (!ws || ws_bytes < workspace_bytes_for(M, K)) return CONVROT_ERR_WORKSPACE;
   if (!aligned16(ws)) return CONVROT_ERR_ALIGN;
   st = check_device(nullptr);
   if (st != CONVROT_OK) return st;
   uint8_t* base = static_cast<uint8_t*>(ws);
-  RotateQuantOut o{nullptr, reinterpret_cast<int8_t*>(base), reinterpret_cast<float*>(base + sa_offset(M, K)),
-                   reinterpret_cast<uint32_t*>(base + ctr_offset(M, K)), kMaxSplitTiles};
+  RotateQuantOut o{nullptr, reinterpret_cast<int8_t*>(base), reinterpret_cast<float*>(base + sa_offset(M, K))};
   return from_cuda(launch_rotate_quant(x, M, K, o, static_cast<cudaStream_t>(stream)));
 }
 
@@ -142,19 +121,15 @@ convrot_status_t gemm_quantized_common(const uint8_t* Wq, const float* s_w, cons
   convrot_status_t st = check_mnk(M, N, K);
   if (st != CONVROT_OK) return st;
   if (!aligned16(Wq) || !aligned16(s_w) || !aligned16(out) || (bias && !aligned16(bias))) return CONVROT_ERR_ALIGN;
-  if (!ws || ws_bytes < workspace_bytes_for(M, N, K)) return CONVROT_ERR_WORKSPACE;
+  if (!ws || ws_bytes < workspace_bytes_for(M, K)) return CONVROT_ERR_WORKSPACE;
   if (!aligned16(ws)) return CONVROT_ERR_ALIGN;
   int sms = 0;
   st = check_device(&sms);
   if (st != CONVROT_OK) return st;
-  const GemmTiling t = choose_tiling(M, N, K, sms);
-  // The GEMM only reads the codes and scales; the counters and slots are
-  // its scratch (the counters return to zero when it completes).
-  uint8_t* base = const_cast<uint8_t*>(static_cast<const uint8_t*>(ws));
+  const uint8_t* base = static_cast<const uint8_t*>(ws);
   GemmArgs a{reinterpret_cast<const int8_t*>(base), reinterpret_cast<const float*>(base + sa_offset(M, K)), Wq, s_w,
-             bias, out, M, N, K, reinterpret_cast<uint32_t*>(base + ctr_offset(M, K)),
-             reinterpret_cast<int32_t*>(base + slots_offset(M, K))};
-  return from_cuda(launch_w4a4_gemm(a, sink, t, static_cast<cudaStream_t>(stream)));
+             bias, out, M, N, K};
+  return from_cuda(launch_w4a4_gemm(a, sink, choose_tiling(M, N, K, sms), static_cast<cudaStream_t>(stream)));
 }
 
 convrot_status_t linear_common(const uint16_t* x, const uint8_t* Wq, const float* s_w, const uint16_t* bias, int M,
@@ -164,8 +139,8 @@ convrot_status_t linear_common(const uint16_t* x, const uint8_t* Wq, const float
   if (st != CONVROT_OK) return st;
   if (!aligned16(x) || !aligned16(Wq) || !aligned16(s_w) || !aligned16(out) || (bias && !aligned16(bias)))
     return CONVROT_ERR_ALIGN;
-  // Check the whole workspace before the first launch.
-  if (!ws || ws_bytes < workspace_bytes_for(M, N, K)) return CONVROT_ERR_WORKSPACE;
+  if (!ws || ws_bytes < workspace_bytes_for(M, K)) return CONVROT_ERR_WORKSPACE;
+  if (!aligned16(ws)) return CONVROT_ERR_ALIGN;
   st = quantize_common(x, M, K, ws, ws_bytes, stream);
   if (st != CONVROT_OK) return st;
   return gemm_quantized_common(Wq, s_w, bias, M, N, K, out, sink, ws, ws_bytes, stream);
@@ -253,7 +228,7 @@ convrot_status_t convrot_rotate_quant(const uint16_t* x, int M, int K, uint8_t* 
   if (!aligned16(x) || !aligned16(xq) || !aligned16(s_a)) return CONVROT_ERR_ALIGN;
   st = check_device(nullptr);
   if (st != CONVROT_OK) return st;
-  RotateQuantOut o{xq, nullptr, s_a, nullptr, 0};
+  RotateQuantOut o{xq, nullptr, s_a};
   return from_cuda(launch_rotate_quant(x, M, K, o, static_cast<cudaStream_t>(stream)));
 }
 
@@ -263,12 +238,12 @@ convrot_status_t convrot_pack_weight(const uint16_t* W, int N, int K, uint8_t* W
 
 size_t convrot_gemm_workspace_size(int M, int N, int K) {
   if (check_mnk(M, N, K) != CONVROT_OK) return 0;
-  return workspace_bytes_for(M, N, K);
+  return codes_bytes(M, K);
 }
 
 size_t convrot_w4a4_workspace_size(int M, int N, int K) {
   if (check_mnk(M, N, K) != CONVROT_OK) return 0;
-  return workspace_bytes_for(M, N, K);
+  return workspace_bytes_for(M, K);
 }
 
 convrot_status_t w4a4_gemm(const uint8_t* xq, const float* s_a, const uint8_t* Wq, const float* s_w,

@@ -25,9 +25,10 @@
 //     chunk order, so the contraction pairs the right codes;
 //   * the accumulator is exactly 16 * acc (|16 acc| <= 1024 K < 2^31), and
 //     the epilogue shifts it right by 4.
-// Work is cut into units of one 128-wide K block of one output tile; see
-// the kernel below for the two schedules (whole tiles for large M, stream-K
-// for small M) and the exact cross-CTA reduction of split tiles.
+// Work is cut into units of one 256-wide K block of one output tile; see
+// the kernel below for the two schedules (whole tiles, and K split over a
+// thread-block cluster when there are few tiles) and the exact reduction of
+// split tiles in shared memory.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -94,21 +95,17 @@ __device__ __forceinline__ void store_output(const P& p, int m, int n, int32_t d
 
 // ---------------------------------------------------------------- the kernel
 //
-// One CTA per SM walks its list of units; a unit is one 128-wide K block of
-// one output tile (BT tokens x 128 output channels).  Two schedules:
-//   * tiles (large M): CTA c takes the whole tiles c, c + grid, c + 2 grid ...
-//     (neighbouring CTAs share activation and weight tiles in L2);
-//   * stream-K (small M, fewer tiles than SMs): the units of all tiles, in
-//     tile-major order, are cut into `grid` contiguous ranges of equal size,
-//     so every SM streams the same share of the weights.
-// Consecutive units of one tile form a segment, summed in one tensor-memory
-// accumulator.  A segment that covers all K blocks of its tile is stored
-// directly.  Otherwise (stream-K only; at most the first and the last
-// segment of a CTA) its int32 partial tile goes to the CTA's slot in global
-// memory and the CTA bumps the tile's arrival counter; the CTA that arrives
-// last adds the other contributors' slots to its own accumulator, stores the
-// tile and resets the counter to zero for the next launch.  Integer addition
-// is exact, so no output bit depends on the order of arrival.
+// A unit is one 256-wide K block of one output tile (BT tokens x 128 output
+// channels).  Two schedules:
+//   * whole tiles (splits == 1): one CTA per SM walks the tiles c, c + grid,
+//     c + 2 grid ... (neighbouring CTAs share activation and weight tiles in
+//     L2), each tile's units summed in one tensor-memory accumulator;
+//   * split-K (splits == S > 1, few tiles): the S CTAs of a thread-block
+//     cluster take even shares of one tile's K blocks.  Each pushes its int32
+//     partial tile, in 4-token groups, into the shared memory of the CTA that
+//     owns the group (group g -> CTA g % S); after one cluster barrier every
+//     CTA adds the S partials of its own groups and stores them.  Integer
+//     addition is exact, so the result does not depend on the split.
 //   warp 0      TMA producer (ring of `nstages` shared-memory stages)
 //   warp 1      TMEM allocation (all 512 columns) and the MMA-issuing thread
 //   warps 2..5  weight unpack into 64-column A slots of tensor memory
@@ -129,10 +126,7 @@ struct PParams {
   int BT, m_tiles, num_tiles, nstages, kbn;
   int acc_stride;   // tensor-memory columns per accumulator (BT rounded up to 32)
   int a_slots;      // A slots of 64 columns after the two accumulators
-  int stream_k;     // 0: whole tiles round-robin, 1: stream-K ranges
-  int units;        // num_tiles * kbn
-  uint32_t* ctr;    // [num_tiles] arrival counters (stream-K), zero between launches
-  int32_t* slots;   // [2 * grid][BT][128] partial tiles (stream-K)
+  int splits;       // 1: whole tiles; S > 1: the cluster of S CTAs splits one tile's K
 };
 
 struct PHeader {
@@ -142,53 +136,27 @@ struct PHeader {
   uint64_t acc_full[2];
   uint64_t acc_empty[2];
   uint32_t tmem_base;
-  uint32_t last_flag;
 };
 
-// First unit of CTA c under stream-K (c in [0, grid]; strictly increasing
-// because grid <= units).
-__device__ __forceinline__ int sk_begin(const PParams& p, int c) {
-  return static_cast<int>((static_cast<long long>(c) * p.units) / static_cast<int>(gridDim.x));
-}
-
-// The CTA whose stream-K range holds unit u.
-__device__ __forceinline__ int sk_owner(const PParams& p, int u) {
-  const int G = static_cast<int>(gridDim.x);
-  int c = static_cast<int>((static_cast<long long>(u) * G) / p.units);
-  while (c + 1 < G && sk_begin(p, c + 1) <= u) ++c;
-  while (c > 0 && sk_begin(p, c) > u) --c;
-  return c;
-}
-
-// Number of units of this CTA.
-__device__ __forceinline__ int unit_count(const PParams& p) {
-  if (p.stream_k) return sk_begin(p, blockIdx.x + 1) - sk_begin(p, blockIdx.x);
-  const int my_tiles =
-      (p.num_tiles - static_cast<int>(blockIdx.x) + static_cast<int>(gridDim.x) - 1) / static_cast<int>(gridDim.x);
-  return my_tiles * p.kbn;
-}
-
-// Tile and K block of this CTA's first unit, and the step to the next unit.
-__device__ __forceinline__ void unit_first(const PParams& p, int u0, int& tile, int& kb) {
-  if (p.stream_k) {
-    tile = u0 / p.kbn;
-    kb = u0 - tile * p.kbn;
+// This CTA's first unit (tile, K block) and number of units.
+__device__ __forceinline__ void unit_range(const PParams& p, int& tile, int& kb, int& count) {
+  if (p.splits > 1) {
+    const int j = static_cast<int>(blockIdx.x) % p.splits;  // rank in the cluster
+    tile = static_cast<int>(blockIdx.x) / p.splits;
+    kb = (j * p.kbn) / p.splits;
+    count = ((j + 1) * p.kbn) / p.splits - kb;
   } else {
     tile = static_cast<int>(blockIdx.x);
     kb = 0;
+    count = (p.num_tiles - tile + static_cast<int>(gridDim.x) - 1) / static_cast<int>(gridDim.x) * p.kbn;
   }
 }
+// The unit after (tile, kb) in this CTA's list.
 __device__ __forceinline__ void unit_next(const PParams& p, int& tile, int& kb) {
   if (++kb == p.kbn) {
     kb = 0;
-    tile += p.stream_k ? 1 : static_cast<int>(gridDim.x);
+    tile += static_cast<int>(gridDim.x);
   }
-}
-
-// Partial-tile slot layout: 16-token chunks, each [128 rows][16 tokens], so
-// a thread (one row) moves 64 contiguous bytes per chunk.
-__device__ __forceinline__ int32_t* slot_chunk(int32_t* slot, int c, int row) {
-  return slot + (c >> 4) * (kRows * 16) + row * 16;
 }
 
 template <int SINK>
@@ -204,10 +172,11 @@ __global__ void __launch_bounds__(kPThreads, 1)
   const uint32_t a_col0 = 2u * static_cast<uint32_t>(p.acc_stride);
   PHeader* hdr = reinterpret_cast<PHeader*>(smem + ns * stage_bytes);
   float* sa_buf = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(hdr) + 1024);  // [2][192]
+  int32_t* red = reinterpret_cast<int32_t*>(reinterpret_cast<uint8_t*>(hdr) + 2560);  // split-K partials
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int kbn = p.kbn;
-  const int u0 = p.stream_k ? sk_begin(p, blockIdx.x) : 0;
-  const int total = unit_count(p);
+  int tile0, kb0, total;
+  unit_range(p, tile0, kb0, total);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < ns; ++s) mbar_init(&hdr->full[s], 1);
@@ -237,14 +206,14 @@ __global__ void __launch_bounds__(kPThreads, 1)
       // Weight tiles of the first stages do not depend on the preceding
       // prologue kernel: request them before waiting for it.
       const int prime = total < ns ? total : ns;
-      int tile, kb;
-      unit_first(p, u0, tile, kb);
+      int tile = tile0, kb = kb0;
       for (int i = 0; i < prime; ++i, unit_next(p, tile, kb)) {
         mbar_arrive_expect_tx(&hdr->full[i], bytes);
         tma_load_2d(smem + i * stage_bytes, &tm_w, &hdr->full[i], kb * (kKB / 2), (tile / p.m_tiles) * kRows);
       }
       pdl_wait();
-      unit_first(p, u0, tile, kb);
+      tile = tile0;
+      kb = kb0;
       for (int i = 0; i < prime; ++i, unit_next(p, tile, kb)) {
         uint8_t* xs = smem + i * stage_bytes + kWTileBytes;
         tma_load_2d(xs, &tm_x, &hdr->full[i], kb * kKB, (tile % p.m_tiles) * BT);
@@ -266,43 +235,46 @@ __global__ void __launch_bounds__(kPThreads, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------ MMA issuer
+    // The unpack warps arrive on a_full only after they have seen the unit's
+    // stage complete (weights and activations landed), so a_full alone says
+    // both operands are in place.  The loop over a segment's units is kept
+    // free of branches other than its own back edge: a branch between
+    // tcgen05.mma groups costs about as much as an MMA.
     if (lane == 0) {
       const uint32_t idesc = umma_idesc_i8(kRows, BT, /*a_signed=*/true, /*b_signed=*/true);
-      int seg = 0, tile, kb, s = 0, ph = 0, a = 0, aph = 0;
-      bool first = true;
-      uint32_t d_tmem = tmem;
-      unit_first(p, u0, tile, kb);
-      for (int i = 0; i < total; ++i, unit_next(p, tile, kb)) {
-        if (i == 0 || kb == 0) {  // a segment starts: take accumulator seg & 1
-          const int b = seg & 1;
-          if (seg >= 2 && !mbar_wait(&hdr->acc_empty[b], ((seg / 2) - 1) & 1)) break;
-          tc_fence_after();
-          d_tmem = tmem + static_cast<uint32_t>(b * p.acc_stride);
-          first = true;
-        }
-        if (!mbar_wait(&hdr->full[s], ph & 1) || !mbar_wait(&hdr->a_full[a], aph & 1)) break;
+      const uint32_t x1 = static_cast<uint32_t>(BT * kXBox);  // second activation box of a stage
+      int kb = kb0, seg = 0, s = 0, a = 0;
+      uint32_t aph = 0;
+      bool ok = true;
+      for (int i = 0; i < total && ok;) {
+        const int len = min(total - i, kbn - kb);  // units of this segment
+        const int b = seg & 1;
+        if (seg >= 2 && !mbar_wait(&hdr->acc_empty[b], ((seg / 2) - 1) & 1)) break;
         tc_fence_after();
-        const uint64_t bdesc0 = umma_desc_k_sw128(smem_u32(smem + s * stage_bytes + kWTileBytes));
-        const uint64_t bdesc1 = umma_desc_k_sw128(smem_u32(smem + s * stage_bytes + kWTileBytes + BT * kXBox));
-        const uint32_t a_tmem = tmem + a_col0 + 64u * static_cast<uint32_t>(a);
+        const uint32_t d_tmem = tmem + static_cast<uint32_t>(b * p.acc_stride);
+        for (int j = 0; j < len; ++j, ++i) {
+          if (!mbar_wait(&hdr->a_full[a], aph)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t xs = smem_u32(smem + s * stage_bytes + kWTileBytes);
+          const uint64_t bd0 = umma_desc_k_sw128(xs), bd1 = umma_desc_k_sw128(xs + x1);
+          const uint32_t at = tmem + a_col0 + 64u * static_cast<uint32_t>(a);
+          const uint32_t acc0 = j > 0 ? 1u : 0u;
 #pragma unroll
-        for (int kk = 0; kk < kKB / 32; ++kk)
-          umma_i8_ts(d_tmem, a_tmem + 8 * kk, (kk < 4 ? bdesc0 : bdesc1) + 2 * (kk & 3), idesc,
-                     (first && kk == 0) ? 0u : 1u);
-        first = false;
-        umma_commit(&hdr->done[i % kDoneRing]);
-        if (++a == nas) {
-          a = 0;
-          ++aph;
+          for (int kk = 0; kk < kKB / 32; ++kk)
+            umma_i8_ts(d_tmem, at + 8 * kk, (kk < 4 ? bd0 : bd1) + 2 * (kk & 3), idesc, kk == 0 ? acc0 : 1u);
+          umma_commit(&hdr->done[i & (kDoneRing - 1)]);
+          s = (s + 1 == ns) ? 0 : s + 1;
+          const bool wrap = a + 1 == nas;
+          a = wrap ? 0 : a + 1;
+          aph ^= wrap ? 1u : 0u;
         }
-        if (i == total - 1 || kb == kbn - 1) {  // the segment ends
-          umma_commit(&hdr->acc_full[seg & 1]);
-          ++seg;
-        }
-        if (++s == ns) {
-          s = 0;
-          ++ph;
-        }
+        if (!ok) break;
+        umma_commit(&hdr->acc_full[b]);  // the segment's accumulator is complete
+        ++seg;
+        kb = 0;
       }
     }
   } else if (warp < 6) {
@@ -335,30 +307,26 @@ __global__ void __launch_bounds__(kPThreads, 1)
     const int row = quad * 32 + lane;
     const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
     const int et = threadIdx.x - 192;  // 0..127
-    pdl_wait();  // s_a and the zeroed counters come from the preceding kernel
-    int seg = 0, seg_kb0 = 0, tile, kb;
-    unit_first(p, u0, tile, kb);
+    pdl_wait();  // s_a comes from the preceding kernel
+    int seg = 0, tile = tile0, kb = kb0;
     for (int i = 0; i < total; ++i, unit_next(p, tile, kb)) {
-      if (i == 0 || kb == 0) seg_kb0 = kb;
       if (!(i == total - 1 || kb == kbn - 1)) continue;
-      // Segment `seg` (K blocks seg_kb0 .. kb of `tile`) ends at unit i.
+      // Segment `seg` (this CTA's units of `tile`) ends at unit i.
       const int b = seg & 1;
-      const bool whole = seg_kb0 == 0 && kb == kbn - 1;
       const int m0 = (tile % p.m_tiles) * BT, n0 = (tile / p.m_tiles) * kRows;
-      float* sa = sa_buf + 192 * b;
-      if (SINK != static_cast<int>(GemmSink::kS32))
-        for (int c = et; c < BT; c += 128) sa[c] = (m0 + c < p.M) ? __ldg(p.s_a + m0 + c) : 0.0f;
-      named_barrier(1, 128);  // s_a staged; all warps are done with segment seg - 2
       const int n = n0 + row;
-      const float sw = (SINK != static_cast<int>(GemmSink::kS32) && n < p.N) ? __ldg(p.s_w + n) : 0.0f;
-      const float bv = (p.bias && n < p.N) ? __uint_as_float(static_cast<uint32_t>(__ldg(p.bias + n)) << 16) : 0.0f;
       // On a failed wait the warp skips the segment's data but keeps taking
-      // part in the named barriers and the counter protocol, so no peer (in
-      // this CTA or another) is left waiting and the counters stay balanced.
+      // part in the named and cluster barriers, so no peer is left waiting.
       const bool ok = __all_sync(0xffffffffu, mbar_wait(&hdr->acc_full[b], (seg / 2) & 1));
       tc_fence_after();
       const uint32_t acc = tmem + lane_base + static_cast<uint32_t>(b * p.acc_stride);
-      if (whole) {
+      if (p.splits == 1) {
+        float* sa = sa_buf + 192 * b;
+        if (SINK != static_cast<int>(GemmSink::kS32))
+          for (int c = et; c < BT; c += 128) sa[c] = (m0 + c < p.M) ? __ldg(p.s_a + m0 + c) : 0.0f;
+        named_barrier(1, 128);  // s_a staged; all warps are done with segment seg - 2
+        const float sw = (SINK != static_cast<int>(GemmSink::kS32) && n < p.N) ? __ldg(p.s_w + n) : 0.0f;
+        const float bv = (p.bias && n < p.N) ? __uint_as_float(static_cast<uint32_t>(__ldg(p.bias + n)) << 16) : 0.0f;
         for (int c = 0; ok && c < BT; c += 16) {
           uint32_t v[16];
           tmem_ld_32x32b_x16(acc + static_cast<uint32_t>(c), v);
@@ -372,97 +340,74 @@ __global__ void __launch_bounds__(kPThreads, 1)
           }
         }
       } else {
-        // Partial tile: publish it, then count the arrival.
-        int32_t* mine = p.slots + static_cast<size_t>(2 * blockIdx.x + (seg == 0 ? 0 : 1)) * BT * kRows;
-        for (int c = 0; ok && c < BT; c += 16) {
+        // Push the partial tile to its owners: 4-token group g belongs to CTA
+        // g % S of the cluster, which keeps it in red[source rank][g / S][row]
+        // (16 bytes).  The stores become visible at the cluster barrier.
+        const int S = p.splits;
+        const int ngl = (BT / 4 + S - 1) / S;
+        const uint32_t me = cluster_ctarank();
+        const uint32_t red_base = smem_u32(red);
+        for (int c = 0; c < BT; c += 16) {
           uint32_t v[16];
-          tmem_ld_32x32b_x16(acc + static_cast<uint32_t>(c), v);
-          tmem_wait_ld();
-          int4* dst = reinterpret_cast<int4*>(slot_chunk(mine, c, row));
-#pragma unroll
-          for (int r = 0; r < 4; ++r)
-            dst[r] = make_int4(static_cast<int32_t>(v[4 * r]), static_cast<int32_t>(v[4 * r + 1]),
-                               static_cast<int32_t>(v[4 * r + 2]), static_cast<int32_t>(v[4 * r + 3]));
-        }
-        __threadfence();        // this thread's slot stores precede the arrival below
-        named_barrier(1, 128);  // ... for all 128 threads
-        const int c_first = sk_owner(p, tile * kbn), c_last = sk_owner(p, tile * kbn + kbn - 1);
-        if (et == 0)
-          hdr->last_flag = atomicAdd(p.ctr + tile, 1u) == static_cast<uint32_t>(c_last - c_first) ? 1u : 0u;
-        named_barrier(1, 128);
-        if (hdr->last_flag) {
-          __threadfence();  // every other contributor's slot is visible now
-          // 32 tokens at a time: the own accumulator from tensor memory plus
-          // the other contributors' slots.
-          for (int h = 0; ok && h < BT; h += 32) {
-            int32_t sum[32];
-#pragma unroll
-            for (int q = 0; q < 2; ++q) {
-              if (h + 16 * q < BT) {  // uniform across the warp (tcgen05.ld is collective)
-                uint32_t v[16];
-                tmem_ld_32x32b_x16(acc + static_cast<uint32_t>(h + 16 * q), v);
-                tmem_wait_ld();
-#pragma unroll
-                for (int j = 0; j < 16; ++j) sum[16 * q + j] = static_cast<int32_t>(v[j]);
-              }
-            }
-            // Two contributors per round: 16 independent 16-byte loads in flight.
-            for (int cc = c_first;;) {
-              int sl[2] = {-1, -1};
-#pragma unroll
-              for (int e = 0; e < 2; ++e) {
-                if (cc == static_cast<int>(blockIdx.x)) ++cc;
-                // Tile `tile` is CTA cc's first segment when cc's range
-                // starts inside it, else its last.
-                if (cc <= c_last) sl[e] = 2 * cc + (sk_begin(p, cc) >= tile * kbn ? 0 : 1), ++cc;
-              }
-              if (sl[0] < 0) break;
-              int4 v[2][8];
-#pragma unroll
-              for (int e = 0; e < 2; ++e) {
-                if (sl[e] < 0) continue;
-                int32_t* other = p.slots + static_cast<size_t>(sl[e]) * BT * kRows;
-#pragma unroll
-                for (int q = 0; q < 2; ++q) {
-                  if (h + 16 * q < BT) {
-                    const int4* src = reinterpret_cast<const int4*>(slot_chunk(other, h + 16 * q, row));
-#pragma unroll
-                    for (int r = 0; r < 4; ++r) v[e][4 * q + r] = __ldcg(src + r);
-                  }
-                }
-              }
-#pragma unroll
-              for (int e = 0; e < 2; ++e) {
-                if (sl[e] < 0) continue;
-#pragma unroll
-                for (int q = 0; q < 2; ++q) {
-                  if (h + 16 * q < BT) {
-#pragma unroll
-                    for (int r = 0; r < 4; ++r) {
-                      sum[16 * q + 4 * r] += v[e][4 * q + r].x;
-                      sum[16 * q + 4 * r + 1] += v[e][4 * q + r].y;
-                      sum[16 * q + 4 * r + 2] += v[e][4 * q + r].z;
-                      sum[16 * q + 4 * r + 3] += v[e][4 * q + r].w;
-                    }
-                  }
-                }
-              }
-            }
-            if (n < p.N) {
-#pragma unroll
-              for (int j = 0; j < 32; ++j) {
-                const int m = m0 + h + j;
-                if (h + j < BT && m < p.M) store_output<SINK>(p, m, n, sum[j], sa[h + j], sw, bv);
-              }
-            }
+          if (ok) {
+            tmem_ld_32x32b_x16(acc + static_cast<uint32_t>(c), v);
+            tmem_wait_ld();
           }
-          if (et == 0) p.ctr[tile] = 0u;  // ready for the next launch
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const int g = c / 4 + q;
+            const int4 w = ok ? make_int4(static_cast<int32_t>(v[4 * q]), static_cast<int32_t>(v[4 * q + 1]),
+                                          static_cast<int32_t>(v[4 * q + 2]), static_cast<int32_t>(v[4 * q + 3]))
+                              : make_int4(0, 0, 0, 0);
+            const uint32_t slot = ((me * ngl + static_cast<uint32_t>(g / S)) * kRows + row) * 16u;
+            st_shared_cluster_v4(map_shared_rank(red_base + slot, static_cast<uint32_t>(g % S)), w);
+          }
         }
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&hdr->acc_empty[b]);
       ++seg;
+    }
+  }
+
+  if (p.splits > 1) {
+    __syncwarp();    // the cluster barrier below is .aligned: reconverge first
+    cluster_sync();  // every partial has reached its owner's shared memory
+    if (warp >= 6) {
+      // Sum, from this CTA's own shared memory, the S partials of the groups
+      // it owns and store them.  No CTA touches another's shared memory after
+      // the barrier, so none has to wait before exiting.
+      const int S = p.splits;
+      const int ngl = (BT / 4 + S - 1) / S;
+      const int row = (warp & 3) * 32 + lane;
+      const int n = (tile0 / p.m_tiles) * kRows + row;
+      const int m0 = (tile0 % p.m_tiles) * BT;
+      const int rank = static_cast<int>(cluster_ctarank());
+      const float sw = (SINK != static_cast<int>(GemmSink::kS32) && n < p.N) ? __ldg(p.s_w + n) : 0.0f;
+      const float bv = (p.bias && n < p.N) ? __uint_as_float(static_cast<uint32_t>(__ldg(p.bias + n)) << 16) : 0.0f;
+      const int4* red4 = reinterpret_cast<const int4*>(red);
+      for (int gl = 0; gl < ngl; ++gl) {
+        const int g = gl * S + rank;
+        if (g >= BT / 4 || m0 + 4 * g >= p.M || n >= p.N) continue;
+        int4 sum = make_int4(0, 0, 0, 0);
+        for (int j = 0; j < S; ++j) {
+          const int4 v = red4[(j * ngl + gl) * kRows + row];
+          sum.x += v.x;
+          sum.y += v.y;
+          sum.z += v.z;
+          sum.w += v.w;
+        }
+        const int32_t sv[4] = {sum.x, sum.y, sum.z, sum.w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int m = m0 + 4 * g + q;
+          if (m < p.M) {
+            const float sa = SINK != static_cast<int>(GemmSink::kS32) ? __ldg(p.s_a + m) : 0.0f;
+            store_output<SINK>(p, m, n, sv[q], sa, sw, bv);
+          }
+        }
+      }
     }
   }
 
@@ -520,12 +465,52 @@ cudaError_t launch_sink(const CUtensorMap& tw, const CUtensorMap& tx, const PPar
   cfg.blockDim = dim3(kPThreads, 1, 1);
   cfg.dynamicSmemBytes = static_cast<size_t>(t.smem_bytes);
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchAttribute attr[2];
+  int nattr = 0;
+  attr[nattr].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[nattr].val.programmaticStreamSerializationAllowed = 1;
+  ++nattr;
+  if (t.splits > 1) {
+    attr[nattr].id = cudaLaunchAttributeClusterDimension;
+    attr[nattr].val.clusterDim.x = static_cast<unsigned>(t.splits);
+    attr[nattr].val.clusterDim.y = 1;
+    attr[nattr].val.clusterDim.z = 1;
+    ++nattr;
+  }
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = nattr;
   return note_cuda(cudaLaunchKernelEx(&cfg, w4a4_tc_gemm_kernel<SINK>, tw, tx, prm), "w4a4_gemm: launch");
+}
+
+// Clusters of S CTAs (one CTA per SM) that can be resident at once on the
+// current device; a conservative estimate when it cannot be queried.
+int max_active_clusters(int S, int num_sms) {
+  static int cache[64][9] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64 || S < 1 || S > 8) return num_sms / (2 * S);
+  if (cache[dev][S] > 0) return cache[dev][S];
+  static int smem_cache[64] = {0};
+  const int smem = 200 * 1024;
+  const void* kfn = reinterpret_cast<const void*>(w4a4_tc_gemm_kernel<0>);
+  int n = 0;
+  if (ensure_dynamic_smem(kfn, smem, smem_cache) == cudaSuccess) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(S * 64), 1, 1);
+    cfg.blockDim = dim3(kPThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = static_cast<unsigned>(S);
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaOccupancyMaxActiveClusters(&n, w4a4_tc_gemm_kernel<0>, &cfg) != cudaSuccess) n = 0;
+  }
+  cudaGetLastError();  // a failed query is not an error of the caller
+  if (n <= 0) n = num_sms / (2 * S);
+  cache[dev][S] = n;
+  return n;
 }
 
 // Estimated cycles of the whole-tile schedule for a token tile of BT: rounds
@@ -544,15 +529,21 @@ long persistent_cost(int M, int N, int K, int BT, int num_sms) {
 
 namespace {
 
-// Stages of BT-token units that fit the shared memory of one CTA, and the
+// Bytes of the split-K receive buffer: S partials of ceil(BT / 4 / S) 4-token
+// groups x 128 rows x 16 bytes.
+int red_bytes(int BT, int S) { return S > 1 ? S * ((BT / 4 + S - 1) / S) * kRows * 16 : 0; }
+
+// Stages of BT-token units that fit the shared memory of one CTA next to the
+// header (1 KB), the s_a staging (1.5 KB) and the split-K buffer, and the
 // dynamic shared memory for them (padded so that one CTA, which owns all of
 // tensor memory, occupies an SM).
 void set_stages(GemmTiling& t) {
   const int stage = kWTileBytes + t.BT * kKB;
-  int ns = (220 * 1024 - 4096) / stage;
+  const int rb = red_bytes(t.BT, t.splits);
+  int ns = (220 * 1024 - 4096 - rb) / stage;
   if (ns > kMaxStages) ns = kMaxStages;
   t.nstages = ns;
-  t.smem_bytes = 1024 + ns * stage + 1024 + 2 * 192 * 4;
+  t.smem_bytes = 1024 + ns * stage + 2560 + rb;
   if (t.smem_bytes < 120 * 1024) t.smem_bytes = 120 * 1024;
   // Tensor memory: two accumulators of BT (rounded up to 32) columns, then
   // 64-column A slots in the rest of the 512.
@@ -563,44 +554,12 @@ void set_stages(GemmTiling& t) {
 
 }  // namespace
 
-// Stream-K grid: the number of CTAs g (at most one per SM) with the lowest
-// modelled time.  The weights stream at the lower of the HBM rate and what g
-// SMs pull (kSmBps each); a split tile then costs its last CTA one round of
-// L2 loads (kRoundSec) per 32 tokens for every two other contributors.
-int streamk_grid(int units, int kbn, int BT, int max_grid) {
-  constexpr double kHbmBps = 6.0e12, kSmBps = 150e9, kRoundSec = 0.4e-6;
-  const double unit_w = kWTileBytes, unit_all = kWTileBytes + static_cast<double>(BT) * kKB;
-  double best = 0;
-  int best_g = 1;
-  const int gmax = units < max_grid ? units : max_grid;
-  for (int g = 1; g <= gmax; ++g) {
-    const int most = (units + g - 1) / g, least = units / g;
-    int parts = 1;  // contributors of the most split tile
-    if (!(units % g == 0 && least % kbn == 0)) {
-      parts = (kbn + least - 1) / least + 1;
-      if (units % g == 0 && kbn % least == 0) parts = kbn / least;
-    }
-    const double t_stream = std::max(units * unit_w / kHbmBps, most * unit_all / kSmBps);
-    const double t_red = ((parts - 1 + 1) / 2) * ((BT + 31) / 32) * kRoundSec;
-    const double t = t_stream + t_red;
-    if (g == 1 || t < best * 0.999) {
-      best = t;
-      best_g = g;
-    }
-  }
-  return best_g;
-}
-
-size_t streamk_scratch_bytes(const GemmTiling& t) {
-  if (!t.stream_k) return 0;
-  return static_cast<size_t>(2 * kMaxGemmGrid) * static_cast<size_t>(t.BT) * kRows * sizeof(int32_t);
-}
-
 GemmTiling choose_tiling(int M, int N, int K, int num_sms) {
   GemmTiling t{};
   const int kbn = K / kKB;
   const int G = num_sms < kMaxGemmGrid ? num_sms : kMaxGemmGrid;
   t.n_tiles = (N + kRows - 1) / kRows;
+  t.splits = 1;
   // Large M: whole tiles, with the token tile BT (multiple of 16, <= 192) of
   // the lowest estimated cost, when it yields at least half as many tiles as
   // SMs.
@@ -617,32 +576,38 @@ GemmTiling choose_tiling(int M, int N, int K, int num_sms) {
       }
     }
     if (best_bt > 0) {
-      t.stream_k = false;
       t.BT = best_bt;
       t.m_tiles = (M + best_bt - 1) / best_bt;
-      t.units = t.m_tiles * t.n_tiles * kbn;
       const int tiles = t.m_tiles * t.n_tiles;
       t.grid = tiles < G ? tiles : G;
       set_stages(t);
       return t;
     }
   }
-  // Small M (or few tiles): stream-K over tiles of BT = M rounded up to 16
-  // (at most 128) tokens.
+  // Small M (or few tiles): tiles of BT = M rounded up to 16 (at most 128)
+  // tokens, K split over a cluster of S CTAs when that is estimated faster:
+  // per wave of CTAs, its start-up (kWaveSec: first loads in flight) plus its
+  // units per CTA x kUnitSec, and kSplitSec for the exchange of partial tiles
+  // when S > 1 (constants measured on B200).
   int bt = M <= 128 ? ((M + 15) / 16) * 16 : 128;
   if (bt < 16) bt = 16;
   t.BT = bt;
   t.m_tiles = (M + bt - 1) / bt;
   const int tiles = t.m_tiles * t.n_tiles;
-  t.units = tiles * kbn;
-  if (tiles > kMaxSplitTiles) {
-    // More tiles than counters (N > 128 * 1024): whole tiles balance anyway.
-    t.stream_k = false;
-    t.grid = tiles < G ? tiles : G;
-  } else {
-    t.stream_k = true;
-    t.grid = streamk_grid(t.units, kbn, bt, G);
+  constexpr double kUnitSec = 0.5e-6, kSplitSec = 1.0e-6, kWaveSec = 3.0e-6;
+  double best = 0;
+  for (int S = 1; S <= 8; S *= 2) {
+    if (S > kbn) break;
+    const int conc = S == 1 ? G : max_active_clusters(S, num_sms);  // tiles in flight at once
+    if (conc < 1) continue;
+    const int waves = (tiles + conc - 1) / conc;
+    const double c = waves * (kWaveSec + ((kbn + S - 1) / S) * kUnitSec) + (S > 1 ? kSplitSec : 0.0);
+    if (S == 1 || c < best * 0.999) {
+      best = c;
+      t.splits = S;
+    }
   }
+  t.grid = t.splits > 1 ? tiles * t.splits : (tiles < G ? tiles : G);
   set_stages(t);
   return t;
 }
@@ -655,8 +620,8 @@ cudaError_t launch_w4a4_gemm(const GemmArgs& a, GemmSink sink, const GemmTiling&
   if (!make_map_u8(&tx, a.xs8, static_cast<uint64_t>(a.M), static_cast<uint64_t>(a.K), static_cast<uint32_t>(t.BT),
                    kXBox, CU_TENSOR_MAP_SWIZZLE_128B))
     return note_cuda(cudaErrorInvalidValue, "w4a4_gemm: activation tensor map");
-  if (t.grid < 1 || t.grid > kMaxGemmGrid || (t.stream_k && (!a.ctr || !a.slots)) || t.a_slots < 2 ||
-      t.nstages < 1 || t.nstages > kMaxStages)
+  if (t.grid < 1 || (t.splits == 1 && t.grid > kMaxGemmGrid) || t.splits < 1 || t.splits > 8 ||
+      t.splits > a.K / kKB || t.a_slots < 2 || t.nstages < 1 || t.nstages > kMaxStages)
     return note_cuda(cudaErrorInvalidValue, "w4a4_gemm: tiling");
   PParams pp{};
   pp.s_a = a.s_a;
@@ -673,17 +638,14 @@ cudaError_t launch_w4a4_gemm(const GemmArgs& a, GemmSink sink, const GemmTiling&
   pp.kbn = a.K / kKB;
   pp.acc_stride = t.acc_stride;
   pp.a_slots = t.a_slots;
-  pp.stream_k = t.stream_k ? 1 : 0;
-  pp.units = t.units;
-  pp.ctr = a.ctr;
-  pp.slots = a.slots;
+  pp.splits = t.splits;
   cudaError_t e;
   switch (sink) {
     case GemmSink::kBF16: e = launch_sink<0>(tw, tx, pp, t, stream); break;
     case GemmSink::kF32: e = launch_sink<1>(tw, tx, pp, t, stream); break;
     default: e = launch_sink<2>(tw, tx, pp, t, stream); break;
   }
-  count_dispatch(t.stream_k ? 3 : 2);
+  count_dispatch(t.splits > 1 ? 3 : 2);
   return e;
 }
 

@@ -18,30 +18,23 @@ struct RotateQuantOut {
   uint8_t* packed;  // [M, K/2] two codes per byte, or null
   int8_t* s8;       // [M, K] codes as signed bytes in chunk order (0,2,4,6,1,3,5,7), or null
   float* scale;     // [M]
-  uint32_t* zero;   // [nzero] words set to zero (the GEMM's tile counters), or null
-  int nzero;
 };
 
 cudaError_t launch_rotate_quant(const uint16_t* x, int M, int K, RotateQuantOut out, cudaStream_t stream);
 
 // Packed codes [M, K/2] -> signed-byte operand layout [M, K].
-// Also sets zero[0 .. nzero) to zero (the GEMM's tile counters) when non-null.
-cudaError_t launch_unpack_codes(const uint8_t* packed, int M, int K, int8_t* s8, uint32_t* zero, int nzero,
-                                cudaStream_t stream);
+cudaError_t launch_unpack_codes(const uint8_t* packed, int M, int K, int8_t* s8, cudaStream_t stream);
 
 enum class GemmSink : int { kBF16 = 0, kF32 = 1, kS32 = 2 };
 
-// Limits of the stream-K scratch reserved in the workspace.
-constexpr int kMaxGemmGrid = 160;     // CTAs (one per SM); two partial-tile slots each
-constexpr int kMaxSplitTiles = 1024;  // per-tile arrival counters
+constexpr int kMaxGemmGrid = 160;  // whole-tile CTAs (one per SM)
 
 struct GemmTiling {
-  bool stream_k;    // stream-K ranges of K-block units (small M) vs whole tiles round-robin (large M)
-  int grid;         // CTAs launched, at most one per SM
+  int splits;       // 1: whole tiles round-robin; S in {2,4,8}: a cluster of S CTAs splits each tile's K
+  int grid;         // CTAs launched
   int BT;           // tokens per tile (MMA N), multiple of 16 in [16, 192]
   int m_tiles;      // ceil(M / BT)
   int n_tiles;      // ceil(N / 128)
-  int units;        // m_tiles * n_tiles * K / 128
   int nstages;      // depth of the shared-memory TMA ring
   int smem_bytes;   // dynamic shared memory per CTA
   int acc_stride;   // tensor-memory columns per accumulator
@@ -49,9 +42,6 @@ struct GemmTiling {
 };
 
 GemmTiling choose_tiling(int M, int N, int K, int num_sms);
-
-// Bytes of partial-tile slots a tiling needs (0 for whole tiles).
-size_t streamk_scratch_bytes(const GemmTiling& t);
 
 struct GemmArgs {
   const int8_t* xs8;      // [M, K] activation codes (operand layout)
@@ -61,8 +51,6 @@ struct GemmArgs {
   const uint16_t* bias;   // [N] or null
   void* out;              // [M, N] bf16 / f32 / s32
   int M, N, K;
-  uint32_t* ctr;          // [kMaxSplitTiles] tile counters, zero on entry (stream-K)
-  int32_t* slots;         // streamk_scratch_bytes of partial tiles (stream-K)
 };
 
 // Builds the tensor maps and launches the tensor-core GEMM.

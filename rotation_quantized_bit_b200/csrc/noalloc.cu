@@ -66,7 +66,6 @@ extern "C" convrot_status_t convrot_w4a4_linear_noalloc(const uint16_t* x, const
     g_scratch_ptr[dev] = p;
   }
   // Nothing in the scratch needs to start at zero: the first kernel writes
-  // every code and scale that the second one reads and zeroes the GEMM's
-  // tile counters.
+  // every code and scale that the second one reads.
   return convrot_w4a4_linear(x, Wq, s_w, bias, M, N, K, y, g_scratch_ptr[dev], kNoAllocScratchBytes, stream);
 }

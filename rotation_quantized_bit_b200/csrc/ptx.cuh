@@ -60,13 +60,10 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Wait until the phase with the given parity has completed.  Bounded: returns
-// false (and records kErrTimeout) after kWaitLimitNs.  Once any wait in the
-// grid has failed, later waits give up immediately so that the whole grid
-// drains quickly.
-__device__ __forceinline__ bool mbar_wait_for(uint64_t* bar, uint32_t parity, unsigned long long limit_ns) {
-  const uint32_t a = smem_u32(bar);
-  if (mbar_try_wait(a, parity)) return true;
+// The waiting part of mbar_wait_for, kept out of line so that the common case
+// (the phase has already completed) costs one try_wait and no loop in the
+// caller.
+static __device__ __noinline__ bool mbar_wait_slow(uint32_t a, uint32_t parity, unsigned long long limit_ns) {
   const unsigned long long t0 = globaltimer_ns();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(a, parity)) return true;
@@ -78,6 +75,16 @@ __device__ __forceinline__ bool mbar_wait_for(uint64_t* bar, uint32_t parity, un
       }
     }
   }
+}
+
+// Wait until the phase with the given parity has completed.  Bounded: returns
+// false (and records kErrTimeout) after limit_ns.  Once any wait in the grid
+// has failed, later waits give up within 16 polls so that the whole grid
+// drains quickly.
+__device__ __forceinline__ bool mbar_wait_for(uint64_t* bar, uint32_t parity, unsigned long long limit_ns) {
+  const uint32_t a = smem_u32(bar);
+  if (__builtin_expect(mbar_try_wait(a, parity), 1)) return true;
+  return mbar_wait_slow(a, parity, limit_ns);
 }
 
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {

@@ -193,8 +193,6 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) rotate_quant_kernel(const _
   };
 
   for (int i = threadIdx.x; i < 2 * 128; i += blockDim.x) (&row_amax[0][0])[i] = 0u;
-  if (blockIdx.x == 0 && p.out.zero)
-    for (int i = threadIdx.x; i < p.out.nzero; i += blockDim.x) p.out.zero[i] = 0u;
   __syncthreads();
 
   int it = 0;
@@ -352,9 +350,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) rotate_quant_kernel(const _
 // nibbles (1,3,5,7).  u = nibble ^ 8 = q + 8 in [0, 15]; the signed byte is
 // (u + 0x78) ^ 0x80 = u - 8 (mod 256), with no carry between bytes.
 __global__ void __launch_bounds__(256) unpack_codes_kernel(const uint8_t* __restrict__ packed, int M, int K,
-                                                           int8_t* __restrict__ s8, uint32_t* zero, int nzero) {
-  if (blockIdx.x == 0 && zero)
-    for (int i = threadIdx.x; i < nzero; i += blockDim.x) zero[i] = 0u;
+                                                           int8_t* __restrict__ s8) {
   const int lane = threadIdx.x & 31;
   const int warps_per_block = blockDim.x / 32;
   const int nword = K >> 3;
@@ -452,12 +448,11 @@ cudaError_t launch_rotate_quant(const uint16_t* x, int M, int K, RotateQuantOut 
   return note_cuda(cudaGetLastError(), "rotate_quant: launch");
 }
 
-cudaError_t launch_unpack_codes(const uint8_t* packed, int M, int K, int8_t* s8, uint32_t* zero, int nzero,
-                                cudaStream_t stream) {
+cudaError_t launch_unpack_codes(const uint8_t* packed, int M, int K, int8_t* s8, cudaStream_t stream) {
   const int per_block = 8;
   int grid = (M + per_block - 1) / per_block;
   if (grid > num_sms_cached() * 8) grid = num_sms_cached() * 8;
-  unpack_codes_kernel<<<grid, 256, 0, stream>>>(packed, M, K, s8, zero, nzero);
+  unpack_codes_kernel<<<grid, 256, 0, stream>>>(packed, M, K, s8);
   count_dispatch(1);
   return note_cuda(cudaGetLastError(), "unpack_codes: launch");
 }
