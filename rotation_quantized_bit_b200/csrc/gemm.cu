@@ -73,6 +73,21 @@ __device__ __forceinline__ void unpack_row_to_tmem(const uint8_t* wstage, int ro
   }
 }
 
+// int32 -> fp32 without the conversion unit: for |i| < 2^22 the float with
+// bits 0x4B400000 + i is exactly 1.5 * 2^23 + i, and subtracting 1.5 * 2^23
+// leaves exactly i (the value a correctly rounded conversion gives, since i
+// is representable).  |acc| <= 64 K <= 2^21 here.
+__device__ __forceinline__ float int_to_float_exact(int32_t i) {
+  return __fsub_rn(__int_as_float(0x4B400000 + i), 12582912.0f);
+}
+
+// fp32 -> bf16 bits, round to nearest even, with integer operations (finite
+// values and infinities; the epilogue produces no NaN from finite inputs).
+__device__ __forceinline__ uint16_t bf16_bits_rne(float y) {
+  const uint32_t u = __float_as_uint(y);
+  return static_cast<uint16_t>((u + 0x7FFFu + ((u >> 16) & 1u)) >> 16);
+}
+
 // One output element from the MMA sum (16 * acc): scales and bias already
 // loaded by the caller.
 template <int SINK, class P>
@@ -84,12 +99,12 @@ __device__ __forceinline__ void store_output(const P& p, int m, int n, int32_t d
     static_cast<int32_t*>(p.out)[idx] = acc;
     return;
   }
-  float y = __fmul_rn(__fmul_rn(__int2float_rn(acc), sa), sw);
+  float y = __fmul_rn(__fmul_rn(int_to_float_exact(acc), sa), sw);
   if (p.bias) y = __fadd_rn(y, bv);
   if (SINK == static_cast<int>(GemmSink::kF32)) {
     static_cast<float*>(p.out)[idx] = y;
   } else {
-    static_cast<uint16_t*>(p.out)[idx] = __bfloat16_as_ushort(__float2bfloat16_rn(y));
+    static_cast<uint16_t*>(p.out)[idx] = bf16_bits_rne(y);
   }
 }
 
@@ -109,13 +124,15 @@ __device__ __forceinline__ void store_output(const P& p, int m, int n, int32_t d
 //   warp 0      TMA producer (ring of `nstages` shared-memory stages)
 //   warp 1      TMEM allocation (all 512 columns) and the MMA-issuing thread
 //   warps 2..5  weight unpack into 64-column A slots of tensor memory
-//   warps 6..9  epilogue, draining one of two accumulators while the MMA
-//               fills the other
+//   warps 6..13 epilogue, draining one of two accumulators while the MMA
+//               fills the other (two warps per tensor-memory lane quadrant,
+//               each taking every other 16-column chunk)
 // The MMA thread commits once per unit, to done[unit % 32]; that one
 // completion frees both the unit's shared-memory stage (for the TMA producer)
 // and its A slot (for the unpack warps).  A unit of 256 K values is 8 MMAs,
 // so the waits and the commit of the issuing thread are spread over 8.
-constexpr int kPThreads = 320;
+constexpr int kPThreads = 448;
+constexpr int kEpiThreads = 256;  // warps 6..13
 
 struct PParams {
   const float* s_a;
@@ -184,7 +201,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
     for (int a = 0; a < nas; ++a) mbar_init(&hdr->a_full[a], 4);      // one arrive per unpack warp
     for (int b = 0; b < 2; ++b) {
       mbar_init(&hdr->acc_full[b], 1);
-      mbar_init(&hdr->acc_empty[b], 4);  // one arrive per epilogue warp
+      mbar_init(&hdr->acc_empty[b], kEpiThreads / 32);  // one arrive per epilogue warp
     }
     fence_mbarrier_init();
     prefetch_tmap(&tm_w);
@@ -303,10 +320,11 @@ __global__ void __launch_bounds__(kPThreads, 1)
     }
   } else {
     // ------------------------------------------------ epilogue
-    const int quad = warp & 3;
+    const int quad = warp & 3;             // tensor-memory lane quadrant (warp id mod 4)
+    const int half = (warp - 6) >> 2;      // which 16-column chunks: 16 * half + 32 k
     const int row = quad * 32 + lane;
     const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
-    const int et = threadIdx.x - 192;  // 0..127
+    const int et = threadIdx.x - 192;  // 0 .. kEpiThreads - 1
     pdl_wait();  // s_a comes from the preceding kernel
     int seg = 0, tile = tile0, kb = kb0;
     for (int i = 0; i < total; ++i, unit_next(p, tile, kb)) {
@@ -323,11 +341,11 @@ __global__ void __launch_bounds__(kPThreads, 1)
       if (p.splits == 1) {
         float* sa = sa_buf + 192 * b;
         if (SINK != static_cast<int>(GemmSink::kS32))
-          for (int c = et; c < BT; c += 128) sa[c] = (m0 + c < p.M) ? __ldg(p.s_a + m0 + c) : 0.0f;
-        named_barrier(1, 128);  // s_a staged; all warps are done with segment seg - 2
+          for (int c = et; c < BT; c += kEpiThreads) sa[c] = (m0 + c < p.M) ? __ldg(p.s_a + m0 + c) : 0.0f;
+        named_barrier(1, kEpiThreads);  // s_a staged; all warps are done with segment seg - 2
         const float sw = (SINK != static_cast<int>(GemmSink::kS32) && n < p.N) ? __ldg(p.s_w + n) : 0.0f;
         const float bv = (p.bias && n < p.N) ? __uint_as_float(static_cast<uint32_t>(__ldg(p.bias + n)) << 16) : 0.0f;
-        for (int c = 0; ok && c < BT; c += 16) {
+        for (int c = 16 * half; ok && c < BT; c += 32) {
           uint32_t v[16];
           tmem_ld_32x32b_x16(acc + static_cast<uint32_t>(c), v);
           tmem_wait_ld();
@@ -347,7 +365,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
         const int ngl = (BT / 4 + S - 1) / S;
         const uint32_t me = cluster_ctarank();
         const uint32_t red_base = smem_u32(red);
-        for (int c = 0; c < BT; c += 16) {
+        for (int c = 16 * half; c < BT; c += 32) {
           uint32_t v[16];
           if (ok) {
             tmem_ld_32x32b_x16(acc + static_cast<uint32_t>(c), v);
@@ -380,6 +398,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
       // the barrier, so none has to wait before exiting.
       const int S = p.splits;
       const int ngl = (BT / 4 + S - 1) / S;
+      const int half = (warp - 6) >> 2;
       const int row = (warp & 3) * 32 + lane;
       const int n = (tile0 / p.m_tiles) * kRows + row;
       const int m0 = (tile0 % p.m_tiles) * BT;
@@ -387,7 +406,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
       const float sw = (SINK != static_cast<int>(GemmSink::kS32) && n < p.N) ? __ldg(p.s_w + n) : 0.0f;
       const float bv = (p.bias && n < p.N) ? __uint_as_float(static_cast<uint32_t>(__ldg(p.bias + n)) << 16) : 0.0f;
       const int4* red4 = reinterpret_cast<const int4*>(red);
-      for (int gl = 0; gl < ngl; ++gl) {
+      for (int gl = half; gl < ngl; gl += 2) {
         const int g = gl * S + rank;
         if (g >= BT / 4 || m0 + 4 * g >= p.M || n >= p.N) continue;
         int4 sum = make_int4(0, 0, 0, 0);
