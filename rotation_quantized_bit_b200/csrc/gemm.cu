@@ -108,6 +108,41 @@ __device__ __forceinline__ void store_output(const P& p, int m, int n, int32_t d
   }
 }
 
+// Outputs of one 32-token chunk of one output channel n: tokens m .. m +
+// count - 1 (count <= 32), accumulators v (16 * acc), token scales sa[0..31]
+// (16-byte aligned in shared memory).
+template <int SINK, class P>
+__device__ __forceinline__ void store_chunk(const P& p, int m, int n, const uint32_t (&v)[32], const float* sa,
+                                            float sw, float bv, int count) {
+  const size_t ld = static_cast<size_t>(p.N);
+  const size_t base = static_cast<size_t>(m) * ld + static_cast<size_t>(n);
+  if (SINK == static_cast<int>(GemmSink::kS32)) {
+    int32_t* o = static_cast<int32_t*>(p.out) + base;
+#pragma unroll
+    for (int j = 0; j < 32; ++j)
+      if (j < count) o[j * ld] = static_cast<int32_t>(v[j]) >> 4;
+    return;
+  }
+  const float4* sa4 = reinterpret_cast<const float4*>(sa);
+#pragma unroll
+  for (int q = 0; q < 8; ++q) {
+    const float4 s4 = sa4[q];
+    const float sv[4] = {s4.x, s4.y, s4.z, s4.w};
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      const int j = 4 * q + r;
+      if (j < count) {
+        float y = __fmul_rn(__fmul_rn(int_to_float_exact(static_cast<int32_t>(v[j]) >> 4), sv[r]), sw);
+        if (p.bias) y = __fadd_rn(y, bv);
+        if (SINK == static_cast<int>(GemmSink::kF32))
+          static_cast<float*>(p.out)[base + j * ld] = y;
+        else
+          static_cast<uint16_t*>(p.out)[base + j * ld] = bf16_bits_rne(y);
+      }
+    }
+  }
+}
+
 // ---------------------------------------------------------------- the kernel
 //
 // A unit is one 256-wide K block of one output tile (BT tokens x 128 output
@@ -126,7 +161,7 @@ __device__ __forceinline__ void store_output(const P& p, int m, int n, int32_t d
 //   warps 2..5  weight unpack into 64-column A slots of tensor memory
 //   warps 6..13 epilogue, draining one of two accumulators while the MMA
 //               fills the other (two warps per tensor-memory lane quadrant,
-//               each taking every other 16-column chunk)
+//               each taking every other 32-column chunk)
 // The MMA thread commits once per unit, to done[unit % 32]; that one
 // completion frees both the unit's shared-memory stage (for the TMA producer)
 // and its A slot (for the unpack warps).  A unit of 256 K values is 8 MMAs,
@@ -147,7 +182,8 @@ struct PParams {
 };
 
 struct PHeader {
-  uint64_t full[kMaxStages];
+  uint64_t full[kMaxStages];    // stage landed (CTA pair: the activation halves of both CTAs, leader only)
+  uint64_t w_full[kMaxStages];  // CTA pair: this CTA's weight tile of the stage landed
   uint64_t done[kDoneRing];     // unit i's MMAs have completed (its stage and A slot are free)
   uint64_t a_full[kMaxASlots];
   uint64_t acc_full[2];
@@ -155,36 +191,41 @@ struct PHeader {
   uint32_t tmem_base;
 };
 
-// This CTA's first unit (tile, K block) and number of units.
+// This CTA's first unit (tile, K block) and number of units.  A CTA pair
+// (PAIR) shares its tiles: both CTAs of pair q walk tiles q, q + pairs, ...
+template <bool PAIR>
 __device__ __forceinline__ void unit_range(const PParams& p, int& tile, int& kb, int& count) {
-  if (p.splits > 1) {
+  if (!PAIR && p.splits > 1) {
     const int j = static_cast<int>(blockIdx.x) % p.splits;  // rank in the cluster
     tile = static_cast<int>(blockIdx.x) / p.splits;
     kb = (j * p.kbn) / p.splits;
     count = ((j + 1) * p.kbn) / p.splits - kb;
   } else {
-    tile = static_cast<int>(blockIdx.x);
+    const int walkers = static_cast<int>(gridDim.x) / (PAIR ? 2 : 1);
+    tile = static_cast<int>(blockIdx.x) / (PAIR ? 2 : 1);
     kb = 0;
-    count = (p.num_tiles - tile + static_cast<int>(gridDim.x) - 1) / static_cast<int>(gridDim.x) * p.kbn;
+    count = (p.num_tiles - tile + walkers - 1) / walkers * p.kbn;
   }
 }
 // The unit after (tile, kb) in this CTA's list.
+template <bool PAIR>
 __device__ __forceinline__ void unit_next(const PParams& p, int& tile, int& kb) {
   if (++kb == p.kbn) {
     kb = 0;
-    tile += static_cast<int>(gridDim.x);
+    tile += static_cast<int>(gridDim.x) / (PAIR ? 2 : 1);
   }
 }
 
-template <int SINK>
+template <int SINK, bool PAIR>
 __global__ void __launch_bounds__(kPThreads, 1)
     w4a4_tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_x,
                         const __grid_constant__ PParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int BT = p.BT;
+  const int XT = PAIR ? BT / 2 : BT;  // token rows of activations this CTA loads per unit
   const int ns = p.nstages;
-  const int stage_bytes = kWTileBytes + BT * kKB;
+  const int stage_bytes = kWTileBytes + XT * kKB;
   const int nas = p.a_slots;
   const uint32_t a_col0 = 2u * static_cast<uint32_t>(p.acc_stride);
   PHeader* hdr = reinterpret_cast<PHeader*>(smem + ns * stage_bytes);
@@ -192,74 +233,106 @@ __global__ void __launch_bounds__(kPThreads, 1)
   int32_t* red = reinterpret_cast<int32_t*>(reinterpret_cast<uint8_t*>(hdr) + 2560);  // split-K partials
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int kbn = p.kbn;
+  // CTA pair: rank 0 leads (issues the MMAs and owns the pair's barriers).
+  const int rank = PAIR ? static_cast<int>(blockIdx.x & 1u) : 0;
   int tile0, kb0, total;
-  unit_range(p, tile0, kb0, total);
+  unit_range<PAIR>(p, tile0, kb0, total);
+  // First weight row and first token row this CTA loads for a tile.
+  auto w_row = [&](int tile) { return (tile / p.m_tiles) * (PAIR ? 2 * kRows : kRows) + rank * kRows; };
+  auto x_row = [&](int tile) { return (tile % p.m_tiles) * BT + rank * XT; };
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < ns; ++s) mbar_init(&hdr->full[s], 1);
-    for (int r = 0; r < kDoneRing; ++r) mbar_init(&hdr->done[r], 1);  // one MMA commit
-    for (int a = 0; a < nas; ++a) mbar_init(&hdr->a_full[a], 4);      // one arrive per unpack warp
+    for (int s = 0; s < ns; ++s) {
+      mbar_init(&hdr->full[s], 1);
+      if (PAIR) mbar_init(&hdr->w_full[s], 1);
+    }
+    for (int r = 0; r < kDoneRing; ++r) mbar_init(&hdr->done[r], 1);      // one MMA commit
+    for (int a = 0; a < nas; ++a) mbar_init(&hdr->a_full[a], PAIR ? 8 : 4);  // one arrive per unpack warp
     for (int b = 0; b < 2; ++b) {
       mbar_init(&hdr->acc_full[b], 1);
-      mbar_init(&hdr->acc_empty[b], kEpiThreads / 32);  // one arrive per epilogue warp
+      mbar_init(&hdr->acc_empty[b], (PAIR ? 2 : 1) * kEpiThreads / 32);  // one arrive per epilogue warp
     }
     fence_mbarrier_init();
     prefetch_tmap(&tm_w);
     prefetch_tmap(&tm_x);
   }
   if (warp == 1) {
-    tmem_alloc(&hdr->tmem_base, 512u);
-    tmem_relinquish();
+    if (PAIR) {
+      tmem_alloc_pair(&hdr->tmem_base, 512u);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(&hdr->tmem_base, 512u);
+      tmem_relinquish();
+    }
   }
   tc_fence_before();
-  __syncthreads();
+  if (PAIR) {
+    __syncwarp();
+    cluster_sync();  // both CTAs' barriers exist before any remote arrive or load targets them
+  } else {
+    __syncthreads();
+  }
   tc_fence_after();
   const uint32_t tmem = hdr->tmem_base;
 
   if (warp == 0) {
     // ------------------------------------------------ TMA producer
+    // Single CTA: weights and activations of a stage complete on full[s].
+    // CTA pair: the weight tile completes on this CTA's w_full[s] (read by
+    // its unpack warps); both CTAs' activation halves complete on the
+    // leader's full[s] (read by the leader's MMA).
     if (lane == 0) {
-      const uint32_t bytes = static_cast<uint32_t>(stage_bytes);
+      const uint32_t wbytes = PAIR ? static_cast<uint32_t>(kWTileBytes) : static_cast<uint32_t>(stage_bytes);
+      auto wbar = [&](int s) { return PAIR ? &hdr->w_full[s] : &hdr->full[s]; };
+      auto load_x = [&](int s, int tile, int kb) {
+        uint8_t* xs = smem + s * stage_bytes + kWTileBytes;
+        if (PAIR) {
+          if (rank == 0) mbar_arrive_expect_tx(&hdr->full[s], static_cast<uint32_t>(BT * kKB));
+          const uint32_t bar = map_shared_rank(smem_u32(&hdr->full[s]), 0);
+          tma_load_2d_pair(xs, &tm_x, bar, kb * kKB, x_row(tile));
+          tma_load_2d_pair(xs + XT * kXBox, &tm_x, bar, kb * kKB + kXBox, x_row(tile));
+        } else {
+          tma_load_2d(xs, &tm_x, &hdr->full[s], kb * kKB, x_row(tile));
+          tma_load_2d(xs + XT * kXBox, &tm_x, &hdr->full[s], kb * kKB + kXBox, x_row(tile));
+        }
+      };
       // Weight tiles of the first stages do not depend on the preceding
       // prologue kernel: request them before waiting for it.
       const int prime = total < ns ? total : ns;
       int tile = tile0, kb = kb0;
-      for (int i = 0; i < prime; ++i, unit_next(p, tile, kb)) {
-        mbar_arrive_expect_tx(&hdr->full[i], bytes);
-        tma_load_2d(smem + i * stage_bytes, &tm_w, &hdr->full[i], kb * (kKB / 2), (tile / p.m_tiles) * kRows);
+      for (int i = 0; i < prime; ++i, unit_next<PAIR>(p, tile, kb)) {
+        mbar_arrive_expect_tx(wbar(i), wbytes);
+        tma_load_2d(smem + i * stage_bytes, &tm_w, wbar(i), kb * (kKB / 2), w_row(tile));
       }
       pdl_wait();
       tile = tile0;
       kb = kb0;
-      for (int i = 0; i < prime; ++i, unit_next(p, tile, kb)) {
-        uint8_t* xs = smem + i * stage_bytes + kWTileBytes;
-        tma_load_2d(xs, &tm_x, &hdr->full[i], kb * kKB, (tile % p.m_tiles) * BT);
-        tma_load_2d(xs + BT * kXBox, &tm_x, &hdr->full[i], kb * kKB + kXBox, (tile % p.m_tiles) * BT);
-      }
+      for (int i = 0; i < prime; ++i, unit_next<PAIR>(p, tile, kb)) load_x(i, tile, kb);
       int it = prime, s = prime % ns;  // stage of unit `it`
-      for (; it < total; ++it, unit_next(p, tile, kb)) {
+      for (; it < total; ++it, unit_next<PAIR>(p, tile, kb)) {
         const int w = it - ns;  // the unit that last used stage s
         if (!mbar_wait(&hdr->done[w % kDoneRing], (w / kDoneRing) & 1)) break;
-        uint8_t* st = smem + s * stage_bytes;
-        mbar_arrive_expect_tx(&hdr->full[s], bytes);
-        tma_load_2d(st, &tm_w, &hdr->full[s], kb * (kKB / 2), (tile / p.m_tiles) * kRows);
-        tma_load_2d(st + kWTileBytes, &tm_x, &hdr->full[s], kb * kKB, (tile % p.m_tiles) * BT);
-        tma_load_2d(st + kWTileBytes + BT * kXBox, &tm_x, &hdr->full[s], kb * kKB + kXBox, (tile % p.m_tiles) * BT);
+        mbar_arrive_expect_tx(wbar(s), wbytes);
+        tma_load_2d(smem + s * stage_bytes, &tm_w, wbar(s), kb * (kKB / 2), w_row(tile));
+        load_x(s, tile, kb);
         if (++s == ns) s = 0;
       }
-      // Drain: every issued load has landed before the block may exit.
-      for (int i = (it > ns ? it - ns : 0); i < it; ++i) mbar_wait(&hdr->full[i % ns], (i / ns) & 1);
+      // Drain: every issued load into this CTA has landed before it may exit
+      // (a CTA pair's activation halves are covered by the final cluster
+      // barrier: the leader's MMAs have consumed them).
+      for (int i = (it > ns ? it - ns : 0); i < it; ++i) mbar_wait(wbar(i % ns), (i / ns) & 1);
     }
   } else if (warp == 1) {
     // ------------------------------------------------ MMA issuer
     // The unpack warps arrive on a_full only after they have seen the unit's
-    // stage complete (weights and activations landed), so a_full alone says
-    // both operands are in place.  The loop over a segment's units is kept
-    // free of branches other than its own back edge: a branch between
-    // tcgen05.mma groups costs about as much as an MMA.
-    if (lane == 0) {
-      const uint32_t idesc = umma_idesc_i8(kRows, BT, /*a_signed=*/true, /*b_signed=*/true);
-      const uint32_t x1 = static_cast<uint32_t>(BT * kXBox);  // second activation box of a stage
+    // operands land (a pair's leader warps also wait for both CTAs'
+    // activation halves on full[s]), so a_full alone says the MMAs may go.
+    // The loop over a segment's units is kept free of branches other than
+    // its own back edge: a branch between tcgen05.mma groups costs about as
+    // much as an MMA.
+    if (lane == 0 && rank == 0) {
+      const uint32_t idesc = umma_idesc_i8(PAIR ? 2 * kRows : kRows, BT, /*a_signed=*/true, /*b_signed=*/true);
+      const uint32_t x1 = static_cast<uint32_t>(XT * kXBox);  // second activation box of a stage
       int kb = kb0, seg = 0, s = 0, a = 0;
       uint32_t aph = 0;
       bool ok = true;
@@ -280,16 +353,27 @@ __global__ void __launch_bounds__(kPThreads, 1)
           const uint32_t at = tmem + a_col0 + 64u * static_cast<uint32_t>(a);
           const uint32_t acc0 = j > 0 ? 1u : 0u;
 #pragma unroll
-          for (int kk = 0; kk < kKB / 32; ++kk)
-            umma_i8_ts(d_tmem, at + 8 * kk, (kk < 4 ? bd0 : bd1) + 2 * (kk & 3), idesc, kk == 0 ? acc0 : 1u);
-          umma_commit(&hdr->done[i & (kDoneRing - 1)]);
+          for (int kk = 0; kk < kKB / 32; ++kk) {
+            const uint64_t bd = (kk < 4 ? bd0 : bd1) + 2 * (kk & 3);
+            if (PAIR)
+              umma_i8_ts_pair(d_tmem, at + 8 * kk, bd, idesc, kk == 0 ? acc0 : 1u);
+            else
+              umma_i8_ts(d_tmem, at + 8 * kk, bd, idesc, kk == 0 ? acc0 : 1u);
+          }
+          if (PAIR)
+            umma_commit_pair_mc(&hdr->done[i & (kDoneRing - 1)], 3);
+          else
+            umma_commit(&hdr->done[i & (kDoneRing - 1)]);
           s = (s + 1 == ns) ? 0 : s + 1;
           const bool wrap = a + 1 == nas;
           a = wrap ? 0 : a + 1;
           aph ^= wrap ? 1u : 0u;
         }
         if (!ok) break;
-        umma_commit(&hdr->acc_full[b]);  // the segment's accumulator is complete
+        if (PAIR)
+          umma_commit_pair_mc(&hdr->acc_full[b], 3);  // the segment's accumulator is complete (both CTAs)
+        else
+          umma_commit(&hdr->acc_full[b]);
         ++seg;
         kb = 0;
       }
@@ -300,7 +384,8 @@ __global__ void __launch_bounds__(kPThreads, 1)
     const int row = quad * 32 + lane;
     const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
     for (int it = 0, s = 0, ph = 0, a = 0; it < total; ++it) {
-      bool w = mbar_wait(&hdr->full[s], ph & 1);
+      bool w = mbar_wait(PAIR ? &hdr->w_full[s] : &hdr->full[s], ph & 1);
+      if (PAIR && rank == 0 && w) w = mbar_wait(&hdr->full[s], ph & 1);  // both activation halves landed
       if (w && it >= nas) {
         const int u = it - nas;  // the unit that last used A slot a
         w = mbar_wait(&hdr->done[u % kDoneRing], (u / kDoneRing) & 1);
@@ -311,7 +396,12 @@ __global__ void __launch_bounds__(kPThreads, 1)
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&hdr->a_full[a]);
+      if (lane == 0) {
+        if (PAIR)
+          mbar_arrive_cluster(map_shared_rank(smem_u32(&hdr->a_full[a]), 0));
+        else
+          mbar_arrive(&hdr->a_full[a]);
+      }
       if (++s == ns) {
         s = 0;
         ++ph;
@@ -321,17 +411,17 @@ __global__ void __launch_bounds__(kPThreads, 1)
   } else {
     // ------------------------------------------------ epilogue
     const int quad = warp & 3;             // tensor-memory lane quadrant (warp id mod 4)
-    const int half = (warp - 6) >> 2;      // which 16-column chunks: 16 * half + 32 k
+    const int half = (warp - 6) >> 2;      // which chunks of the accumulator this warp drains
     const int row = quad * 32 + lane;
     const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
     const int et = threadIdx.x - 192;  // 0 .. kEpiThreads - 1
     pdl_wait();  // s_a comes from the preceding kernel
     int seg = 0, tile = tile0, kb = kb0;
-    for (int i = 0; i < total; ++i, unit_next(p, tile, kb)) {
+    for (int i = 0; i < total; ++i, unit_next<PAIR>(p, tile, kb)) {
       if (!(i == total - 1 || kb == kbn - 1)) continue;
       // Segment `seg` (this CTA's units of `tile`) ends at unit i.
       const int b = seg & 1;
-      const int m0 = (tile % p.m_tiles) * BT, n0 = (tile / p.m_tiles) * kRows;
+      const int m0 = (tile % p.m_tiles) * BT, n0 = w_row(tile);
       const int n = n0 + row;
       // On a failed wait the warp skips the segment's data but keeps taking
       // part in the named and cluster barriers, so no peer is left waiting.
@@ -345,17 +435,14 @@ __global__ void __launch_bounds__(kPThreads, 1)
         named_barrier(1, kEpiThreads);  // s_a staged; all warps are done with segment seg - 2
         const float sw = (SINK != static_cast<int>(GemmSink::kS32) && n < p.N) ? __ldg(p.s_w + n) : 0.0f;
         const float bv = (p.bias && n < p.N) ? __uint_as_float(static_cast<uint32_t>(__ldg(p.bias + n)) << 16) : 0.0f;
-        for (int c = 16 * half; ok && c < BT; c += 32) {
-          uint32_t v[16];
-          tmem_ld_32x32b_x16(acc + static_cast<uint32_t>(c), v);
+        // 32-column chunks (the accumulator stride is BT rounded up to 32, so
+        // the last chunk's extra columns exist and are simply not stored).
+        for (int c = 32 * half; ok && c < BT; c += 64) {
+          uint32_t v[32];
+          tmem_ld_32x32b_x32(acc + static_cast<uint32_t>(c), v);
           tmem_wait_ld();
-          if (n < p.N) {
-#pragma unroll
-            for (int j = 0; j < 16; ++j) {
-              const int m = m0 + c + j;
-              if (m < p.M) store_output<SINK>(p, m, n, static_cast<int32_t>(v[j]), sa[c + j], sw, bv);
-            }
-          }
+          const int count = min(min(32, BT - c), p.M - (m0 + c));
+          if (n < p.N && count > 0) store_chunk<SINK>(p, m0 + c, n, v, sa + c, sw, bv, count);
         }
       } else {
         // Push the partial tile to its owners: 4-token group g belongs to CTA
@@ -384,12 +471,17 @@ __global__ void __launch_bounds__(kPThreads, 1)
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&hdr->acc_empty[b]);
+      if (lane == 0) {
+        if (PAIR)
+          mbar_arrive_cluster(map_shared_rank(smem_u32(&hdr->acc_empty[b]), 0));
+        else
+          mbar_arrive(&hdr->acc_empty[b]);
+      }
       ++seg;
     }
   }
 
-  if (p.splits > 1) {
+  if (!PAIR && p.splits > 1) {
     __syncwarp();    // the cluster barrier below is .aligned: reconverge first
     cluster_sync();  // every partial has reached its owner's shared memory
     if (warp >= 6) {
@@ -431,11 +523,22 @@ __global__ void __launch_bounds__(kPThreads, 1)
   }
 
   tc_fence_before();
-  __syncthreads();
+  if (PAIR) {
+    // Both CTAs' epilogues have seen their last accumulator, so every MMA of
+    // the pair (which writes into both CTAs' tensor memory and reads both
+    // CTAs' shared memory) has completed.
+    __syncwarp();
+    cluster_sync();
+  } else {
+    __syncthreads();
+  }
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();
-    tmem_dealloc(tmem, 512u);
+    if (PAIR)
+      tmem_dealloc_pair(tmem, 512u);
+    else
+      tmem_dealloc(tmem, 512u);
   }
 }
 
@@ -472,11 +575,11 @@ bool make_map_u8(CUtensorMap* map, const void* base, uint64_t rows, uint64_t col
   return r == CUDA_SUCCESS;
 }
 
-template <int SINK>
+template <int SINK, bool PAIR>
 cudaError_t launch_sink(const CUtensorMap& tw, const CUtensorMap& tx, const PParams& prm, const GemmTiling& t,
                         cudaStream_t stream) {
   static int cache[64] = {0};
-  const void* kfn = reinterpret_cast<const void*>(w4a4_tc_gemm_kernel<SINK>);
+  const void* kfn = reinterpret_cast<const void*>(w4a4_tc_gemm_kernel<SINK, PAIR>);
   cudaError_t e = ensure_dynamic_smem(kfn, t.smem_bytes, cache);
   if (e != cudaSuccess) return note_cuda(e, "w4a4_gemm: dynamic shared memory attribute");
   cudaLaunchConfig_t cfg = {};
@@ -489,16 +592,16 @@ cudaError_t launch_sink(const CUtensorMap& tw, const CUtensorMap& tx, const PPar
   attr[nattr].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[nattr].val.programmaticStreamSerializationAllowed = 1;
   ++nattr;
-  if (t.splits > 1) {
+  if (PAIR || t.splits > 1) {
     attr[nattr].id = cudaLaunchAttributeClusterDimension;
-    attr[nattr].val.clusterDim.x = static_cast<unsigned>(t.splits);
+    attr[nattr].val.clusterDim.x = PAIR ? 2u : static_cast<unsigned>(t.splits);
     attr[nattr].val.clusterDim.y = 1;
     attr[nattr].val.clusterDim.z = 1;
     ++nattr;
   }
   cfg.attrs = attr;
   cfg.numAttrs = nattr;
-  return note_cuda(cudaLaunchKernelEx(&cfg, w4a4_tc_gemm_kernel<SINK>, tw, tx, prm), "w4a4_gemm: launch");
+  return note_cuda(cudaLaunchKernelEx(&cfg, w4a4_tc_gemm_kernel<SINK, PAIR>, tw, tx, prm), "w4a4_gemm: launch");
 }
 
 // Clusters of S CTAs (one CTA per SM) that can be resident at once on the
@@ -510,7 +613,7 @@ int max_active_clusters(int S, int num_sms) {
   if (cache[dev][S] > 0) return cache[dev][S];
   static int smem_cache[64] = {0};
   const int smem = 200 * 1024;
-  const void* kfn = reinterpret_cast<const void*>(w4a4_tc_gemm_kernel<0>);
+  const void* kfn = reinterpret_cast<const void*>(w4a4_tc_gemm_kernel<0, false>);
   int n = 0;
   if (ensure_dynamic_smem(kfn, smem, smem_cache) == cudaSuccess) {
     cudaLaunchConfig_t cfg = {};
@@ -524,7 +627,7 @@ int max_active_clusters(int S, int num_sms) {
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (cudaOccupancyMaxActiveClusters(&n, w4a4_tc_gemm_kernel<0>, &cfg) != cudaSuccess) n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, w4a4_tc_gemm_kernel<0, false>, &cfg) != cudaSuccess) n = 0;
   }
   cudaGetLastError();  // a failed query is not an error of the caller
   if (n <= 0) n = num_sms / (2 * S);
@@ -533,14 +636,19 @@ int max_active_clusters(int S, int num_sms) {
 }
 
 // Estimated cycles of the whole-tile schedule for a token tile of BT: rounds
-// of tiles per SM x units x the slower of the MMA (4 * BT cycles per 256-K
-// unit at 8192 int8 MACs/clk) and a per-unit floor of 640 cycles that every
-// unit costs whatever BT is (issuing its 8 MMAs and commit, and the 16 KB
-// weight tile fetched and unpacked into tensor memory).
-long persistent_cost(int M, int N, int K, int BT, int num_sms) {
-  const long tiles = static_cast<long>((M + BT - 1) / BT) * ((N + kRows - 1) / kRows);
-  const long rounds = (tiles + num_sms - 1) / num_sms;
-  const long per_unit = 4L * BT > 640 ? 4L * BT : 640;
+// of tiles per SM (per CTA pair) x units x the slower of the MMA (4 * BT
+// cycles per 256-K unit on each SM at 8192 int8 MACs/clk) and a per-unit
+// floor that every unit costs whatever BT is (issuing 8 MMAs and a commit,
+// fetching and unpacking the 16 KB weight tile): about 900 cycles measured
+// for one CTA, less for a pair, whose leader issues for two SMs and whose
+// CTAs each load half the activations.
+long persistent_cost(int M, int N, int K, int BT, int num_sms, bool pair) {
+  const int rows = pair ? 2 * kRows : kRows;  // output channels per tile
+  const long tiles = static_cast<long>((M + BT - 1) / BT) * ((N + rows - 1) / rows);
+  const int walkers = pair ? num_sms / 2 : num_sms;
+  const long rounds = (tiles + walkers - 1) / walkers;
+  const long floor_cycles = pair ? 640 : 900;
+  const long per_unit = 4L * BT > floor_cycles ? 4L * BT : floor_cycles;
   return rounds * (K / kKB) * per_unit;
 }
 
@@ -557,12 +665,16 @@ int red_bytes(int BT, int S) { return S > 1 ? S * ((BT / 4 + S - 1) / S) * kRows
 // dynamic shared memory for them (padded so that one CTA, which owns all of
 // tensor memory, occupies an SM).
 void set_stages(GemmTiling& t) {
-  const int stage = kWTileBytes + t.BT * kKB;
+  const int stage = kWTileBytes + (t.pair ? t.BT / 2 : t.BT) * kKB;
   const int rb = red_bytes(t.BT, t.splits);
-  int ns = (220 * 1024 - 4096 - rb) / stage;
+  int ns = (220 * 1024 - 4096 - rb - (t.pair ? (t.BT / 2) * kXBox : 0)) / stage;
   if (ns > kMaxStages) ns = kMaxStages;
   t.nstages = ns;
   t.smem_bytes = 1024 + ns * stage + 2560 + rb;
+  // A pair's MMA reads its half of the activation tile from each CTA; keep
+  // one more half of slack behind the last stage so that the reads of the
+  // last stage never reach the end of the allocation.
+  if (t.pair) t.smem_bytes += (t.BT / 2) * kXBox;
   if (t.smem_bytes < 120 * 1024) t.smem_bytes = 120 * 1024;
   // Tensor memory: two accumulators of BT (rounded up to 32) columns, then
   // 64-column A slots in the rest of the 512.
@@ -582,23 +694,35 @@ GemmTiling choose_tiling(int M, int N, int K, int num_sms) {
   // Large M: whole tiles, with the token tile BT (multiple of 16, <= 192) of
   // the lowest estimated cost, when it yields at least half as many tiles as
   // SMs.
+  // A CTA pair takes tiles of 256 channels with BT a multiple of 32.
   if (M > 128) {
-    int best_bt = 0;
+    int best_bt = 0, best_pair = 0;
     long best = -1;
-    for (int bt = 192; bt >= 64; bt -= 16) {
-      const long tiles = static_cast<long>((M + bt - 1) / bt) * t.n_tiles;
-      if (2 * tiles < G) continue;
-      const long c = persistent_cost(M, N, K, bt, G);
-      if (best < 0 || c < best) {
-        best = c;
-        best_bt = bt;
+    for (int pair = 0; pair < 1; ++pair) {  // CTA pairs measured slower; not selected
+      for (int bt = 192; bt >= 64; bt -= (pair ? 32 : 16)) {
+        const int rows = pair ? 2 * kRows : kRows;
+        const long tiles = static_cast<long>((M + bt - 1) / bt) * ((N + rows - 1) / rows);
+        if ((pair ? 4 : 2) * tiles < G) continue;
+        const long c = persistent_cost(M, N, K, bt, G, pair != 0);
+        if (best < 0 || c < best) {
+          best = c;
+          best_bt = bt;
+          best_pair = pair;
+        }
       }
     }
     if (best_bt > 0) {
+      t.pair = best_pair;
       t.BT = best_bt;
+      t.n_tiles = (N + (best_pair ? 2 * kRows : kRows) - 1) / (best_pair ? 2 * kRows : kRows);
       t.m_tiles = (M + best_bt - 1) / best_bt;
       const int tiles = t.m_tiles * t.n_tiles;
-      t.grid = tiles < G ? tiles : G;
+      int walkers = G;
+      if (best_pair) {
+        walkers = max_active_clusters(2, num_sms);  // pairs resident at once
+        if (walkers < 1 || walkers > G / 2) walkers = G / 2;
+      }
+      t.grid = (tiles < walkers ? tiles : walkers) * (best_pair ? 2 : 1);
       set_stages(t);
       return t;
     }
@@ -636,11 +760,12 @@ cudaError_t launch_w4a4_gemm(const GemmArgs& a, GemmSink sink, const GemmTiling&
   if (!make_map_u8(&tw, a.Wq, static_cast<uint64_t>(a.N), static_cast<uint64_t>(a.K / 2), kRows, kKB / 2,
                    CU_TENSOR_MAP_SWIZZLE_128B))
     return note_cuda(cudaErrorInvalidValue, "w4a4_gemm: weight tensor map");
-  if (!make_map_u8(&tx, a.xs8, static_cast<uint64_t>(a.M), static_cast<uint64_t>(a.K), static_cast<uint32_t>(t.BT),
-                   kXBox, CU_TENSOR_MAP_SWIZZLE_128B))
+  if (!make_map_u8(&tx, a.xs8, static_cast<uint64_t>(a.M), static_cast<uint64_t>(a.K),
+                   static_cast<uint32_t>(t.pair ? t.BT / 2 : t.BT), kXBox, CU_TENSOR_MAP_SWIZZLE_128B))
     return note_cuda(cudaErrorInvalidValue, "w4a4_gemm: activation tensor map");
   if (t.grid < 1 || (t.splits == 1 && t.grid > kMaxGemmGrid) || t.splits < 1 || t.splits > 8 ||
-      t.splits > a.K / kKB || t.a_slots < 2 || t.nstages < 1 || t.nstages > kMaxStages)
+      t.splits > a.K / kKB || t.a_slots < 2 || t.nstages < 1 || t.nstages > kMaxStages ||
+      (t.pair && (t.splits != 1 || t.grid % 2 != 0 || t.BT % 32 != 0)))
     return note_cuda(cudaErrorInvalidValue, "w4a4_gemm: tiling");
   PParams pp{};
   pp.s_a = a.s_a;
@@ -659,10 +784,18 @@ cudaError_t launch_w4a4_gemm(const GemmArgs& a, GemmSink sink, const GemmTiling&
   pp.a_slots = t.a_slots;
   pp.splits = t.splits;
   cudaError_t e;
-  switch (sink) {
-    case GemmSink::kBF16: e = launch_sink<0>(tw, tx, pp, t, stream); break;
-    case GemmSink::kF32: e = launch_sink<1>(tw, tx, pp, t, stream); break;
-    default: e = launch_sink<2>(tw, tx, pp, t, stream); break;
+  if (t.pair) {
+    switch (sink) {
+      case GemmSink::kBF16: e = launch_sink<0, true>(tw, tx, pp, t, stream); break;
+      case GemmSink::kF32: e = launch_sink<1, true>(tw, tx, pp, t, stream); break;
+      default: e = launch_sink<2, true>(tw, tx, pp, t, stream); break;
+    }
+  } else {
+    switch (sink) {
+      case GemmSink::kBF16: e = launch_sink<0, false>(tw, tx, pp, t, stream); break;
+      case GemmSink::kF32: e = launch_sink<1, false>(tw, tx, pp, t, stream); break;
+      default: e = launch_sink<2, false>(tw, tx, pp, t, stream); break;
+    }
   }
   count_dispatch(t.splits > 1 ? 3 : 2);
   return e;
