@@ -182,8 +182,7 @@ struct PParams {
 };
 
 struct PHeader {
-  uint64_t full[kMaxStages];    // stage landed (CTA pair: the activation halves of both CTAs, leader only)
-  uint64_t w_full[kMaxStages];  // CTA pair: this CTA's weight tile of the stage landed
+  uint64_t full[kMaxStages];    // the stage's weight and activation tiles landed
   uint64_t done[kDoneRing];     // unit i's MMAs have completed (its stage and A slot are free)
   uint64_t a_full[kMaxASlots];
   uint64_t acc_full[2];
@@ -191,41 +190,36 @@ struct PHeader {
   uint32_t tmem_base;
 };
 
-// This CTA's first unit (tile, K block) and number of units.  A CTA pair
-// (PAIR) shares its tiles: both CTAs of pair q walk tiles q, q + pairs, ...
-template <bool PAIR>
+// This CTA's first unit (tile, K block) and number of units.
 __device__ __forceinline__ void unit_range(const PParams& p, int& tile, int& kb, int& count) {
-  if (!PAIR && p.splits > 1) {
+  if (p.splits > 1) {
     const int j = static_cast<int>(blockIdx.x) % p.splits;  // rank in the cluster
     tile = static_cast<int>(blockIdx.x) / p.splits;
     kb = (j * p.kbn) / p.splits;
     count = ((j + 1) * p.kbn) / p.splits - kb;
   } else {
-    const int walkers = static_cast<int>(gridDim.x) / (PAIR ? 2 : 1);
-    tile = static_cast<int>(blockIdx.x) / (PAIR ? 2 : 1);
+    tile = static_cast<int>(blockIdx.x);
     kb = 0;
-    count = (p.num_tiles - tile + walkers - 1) / walkers * p.kbn;
+    count = (p.num_tiles - tile + static_cast<int>(gridDim.x) - 1) / static_cast<int>(gridDim.x) * p.kbn;
   }
 }
 // The unit after (tile, kb) in this CTA's list.
-template <bool PAIR>
 __device__ __forceinline__ void unit_next(const PParams& p, int& tile, int& kb) {
   if (++kb == p.kbn) {
     kb = 0;
-    tile += static_cast<int>(gridDim.x) / (PAIR ? 2 : 1);
+    tile += static_cast<int>(gridDim.x);
   }
 }
 
-template <int SINK, bool PAIR>
+template <int SINK>
 __global__ void __launch_bounds__(kPThreads, 1)
     w4a4_tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_x,
                         const __grid_constant__ PParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int BT = p.BT;
-  const int XT = PAIR ? BT / 2 : BT;  // token rows of activations this CTA loads per unit
   const int ns = p.nstages;
-  const int stage_bytes = kWTileBytes + XT * kKB;
+  const int stage_bytes = kWTileBytes + BT * kKB;
   const int nas = p.a_slots;
   const uint32_t a_col0 = 2u * static_cast<uint32_t>(p.acc_stride);
   PHeader* hdr = reinterpret_cast<PHeader*>(smem + ns * stage_bytes);
@@ -233,83 +227,58 @@ __global__ void __launch_bounds__(kPThreads, 1)
   int32_t* red = reinterpret_cast<int32_t*>(reinterpret_cast<uint8_t*>(hdr) + 2560);  // split-K partials
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int kbn = p.kbn;
-  // CTA pair: rank 0 leads (issues the MMAs and owns the pair's barriers).
-  const int rank = PAIR ? static_cast<int>(blockIdx.x & 1u) : 0;
   int tile0, kb0, total;
-  unit_range<PAIR>(p, tile0, kb0, total);
-  // First weight row and first token row this CTA loads for a tile.
-  auto w_row = [&](int tile) { return (tile / p.m_tiles) * (PAIR ? 2 * kRows : kRows) + rank * kRows; };
-  auto x_row = [&](int tile) { return (tile % p.m_tiles) * BT + rank * XT; };
+  unit_range(p, tile0, kb0, total);
+  // First weight row and first token row of a tile.
+  auto w_row = [&](int tile) { return (tile / p.m_tiles) * kRows; };
+  auto x_row = [&](int tile) { return (tile % p.m_tiles) * BT; };
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < ns; ++s) {
-      mbar_init(&hdr->full[s], 1);
-      if (PAIR) mbar_init(&hdr->w_full[s], 1);
-    }
-    for (int r = 0; r < kDoneRing; ++r) mbar_init(&hdr->done[r], 1);      // one MMA commit
-    for (int a = 0; a < nas; ++a) mbar_init(&hdr->a_full[a], PAIR ? 8 : 4);  // one arrive per unpack warp
+    for (int s = 0; s < ns; ++s) mbar_init(&hdr->full[s], 1);
+    for (int r = 0; r < kDoneRing; ++r) mbar_init(&hdr->done[r], 1);  // one MMA commit
+    for (int a = 0; a < nas; ++a) mbar_init(&hdr->a_full[a], 4);      // one arrive per unpack warp
     for (int b = 0; b < 2; ++b) {
       mbar_init(&hdr->acc_full[b], 1);
-      mbar_init(&hdr->acc_empty[b], (PAIR ? 2 : 1) * kEpiThreads / 32);  // one arrive per epilogue warp
+      mbar_init(&hdr->acc_empty[b], kEpiThreads / 32);  // one arrive per epilogue warp
     }
     fence_mbarrier_init();
     prefetch_tmap(&tm_w);
     prefetch_tmap(&tm_x);
   }
   if (warp == 1) {
-    if (PAIR) {
-      tmem_alloc_pair(&hdr->tmem_base, 512u);
-      tmem_relinquish_pair();
-    } else {
-      tmem_alloc(&hdr->tmem_base, 512u);
-      tmem_relinquish();
-    }
+    tmem_alloc(&hdr->tmem_base, 512u);
+    tmem_relinquish();
   }
   tc_fence_before();
-  if (PAIR) {
-    __syncwarp();
-    cluster_sync();  // both CTAs' barriers exist before any remote arrive or load targets them
-  } else {
-    __syncthreads();
-  }
+  __syncthreads();
   tc_fence_after();
   const uint32_t tmem = hdr->tmem_base;
 
   if (warp == 0) {
     // ------------------------------------------------ TMA producer
-    // Single CTA: weights and activations of a stage complete on full[s].
-    // CTA pair: the weight tile completes on this CTA's w_full[s] (read by
-    // its unpack warps); both CTAs' activation halves complete on the
-    // leader's full[s] (read by the leader's MMA).
+    // The weight and activation tiles of a stage complete on full[s].
     if (lane == 0) {
-      const uint32_t wbytes = PAIR ? static_cast<uint32_t>(kWTileBytes) : static_cast<uint32_t>(stage_bytes);
-      auto wbar = [&](int s) { return PAIR ? &hdr->w_full[s] : &hdr->full[s]; };
+      const uint32_t wbytes = static_cast<uint32_t>(stage_bytes);
+      auto wbar = [&](int s) { return &hdr->full[s]; };
       auto load_x = [&](int s, int tile, int kb) {
         uint8_t* xs = smem + s * stage_bytes + kWTileBytes;
-        if (PAIR) {
-          if (rank == 0) mbar_arrive_expect_tx(&hdr->full[s], static_cast<uint32_t>(BT * kKB));
-          const uint32_t bar = map_shared_rank(smem_u32(&hdr->full[s]), 0);
-          tma_load_2d_pair(xs, &tm_x, bar, kb * kKB, x_row(tile));
-          tma_load_2d_pair(xs + XT * kXBox, &tm_x, bar, kb * kKB + kXBox, x_row(tile));
-        } else {
-          tma_load_2d(xs, &tm_x, &hdr->full[s], kb * kKB, x_row(tile));
-          tma_load_2d(xs + XT * kXBox, &tm_x, &hdr->full[s], kb * kKB + kXBox, x_row(tile));
-        }
+        tma_load_2d(xs, &tm_x, &hdr->full[s], kb * kKB, x_row(tile));
+        tma_load_2d(xs + BT * kXBox, &tm_x, &hdr->full[s], kb * kKB + kXBox, x_row(tile));
       };
       // Weight tiles of the first stages do not depend on the preceding
       // prologue kernel: request them before waiting for it.
       const int prime = total < ns ? total : ns;
       int tile = tile0, kb = kb0;
-      for (int i = 0; i < prime; ++i, unit_next<PAIR>(p, tile, kb)) {
+      for (int i = 0; i < prime; ++i, unit_next(p, tile, kb)) {
         mbar_arrive_expect_tx(wbar(i), wbytes);
         tma_load_2d(smem + i * stage_bytes, &tm_w, wbar(i), kb * (kKB / 2), w_row(tile));
       }
       pdl_wait();
       tile = tile0;
       kb = kb0;
-      for (int i = 0; i < prime; ++i, unit_next<PAIR>(p, tile, kb)) load_x(i, tile, kb);
+      for (int i = 0; i < prime; ++i, unit_next(p, tile, kb)) load_x(i, tile, kb);
       int it = prime, s = prime % ns;  // stage of unit `it`
-      for (; it < total; ++it, unit_next<PAIR>(p, tile, kb)) {
+      for (; it < total; ++it, unit_next(p, tile, kb)) {
         const int w = it - ns;  // the unit that last used stage s
         if (!mbar_wait(&hdr->done[w % kDoneRing], (w / kDoneRing) & 1)) break;
         mbar_arrive_expect_tx(wbar(s), wbytes);
@@ -317,22 +286,20 @@ __global__ void __launch_bounds__(kPThreads, 1)
         load_x(s, tile, kb);
         if (++s == ns) s = 0;
       }
-      // Drain: every issued load into this CTA has landed before it may exit
-      // (a CTA pair's activation halves are covered by the final cluster
-      // barrier: the leader's MMAs have consumed them).
+      // Drain: every issued load has landed before the block may exit.
       for (int i = (it > ns ? it - ns : 0); i < it; ++i) mbar_wait(wbar(i % ns), (i / ns) & 1);
     }
   } else if (warp == 1) {
     // ------------------------------------------------ MMA issuer
     // The unpack warps arrive on a_full only after they have seen the unit's
-    // operands land (a pair's leader warps also wait for both CTAs'
-    // activation halves on full[s]), so a_full alone says the MMAs may go.
+    // stage land (weights and activations), so a_full alone says the MMAs
+    // may go.
     // The loop over a segment's units is kept free of branches other than
     // its own back edge: a branch between tcgen05.mma groups costs about as
     // much as an MMA.
-    if (lane == 0 && rank == 0) {
-      const uint32_t idesc = umma_idesc_i8(PAIR ? 2 * kRows : kRows, BT, /*a_signed=*/true, /*b_signed=*/true);
-      const uint32_t x1 = static_cast<uint32_t>(XT * kXBox);  // second activation box of a stage
+    if (lane == 0) {
+      const uint32_t idesc = umma_idesc_i8(kRows, BT, /*a_signed=*/true, /*b_signed=*/true);
+      const uint32_t x1 = static_cast<uint32_t>(BT * kXBox);  // second activation box of a stage
       int kb = kb0, seg = 0, s = 0, a = 0;
       uint32_t aph = 0;
       bool ok = true;
@@ -353,27 +320,16 @@ __global__ void __launch_bounds__(kPThreads, 1)
           const uint32_t at = tmem + a_col0 + 64u * static_cast<uint32_t>(a);
           const uint32_t acc0 = j > 0 ? 1u : 0u;
 #pragma unroll
-          for (int kk = 0; kk < kKB / 32; ++kk) {
-            const uint64_t bd = (kk < 4 ? bd0 : bd1) + 2 * (kk & 3);
-            if (PAIR)
-              umma_i8_ts_pair(d_tmem, at + 8 * kk, bd, idesc, kk == 0 ? acc0 : 1u);
-            else
-              umma_i8_ts(d_tmem, at + 8 * kk, bd, idesc, kk == 0 ? acc0 : 1u);
-          }
-          if (PAIR)
-            umma_commit_pair_mc(&hdr->done[i & (kDoneRing - 1)], 3);
-          else
-            umma_commit(&hdr->done[i & (kDoneRing - 1)]);
+          for (int kk = 0; kk < kKB / 32; ++kk)
+            umma_i8_ts(d_tmem, at + 8 * kk, (kk < 4 ? bd0 : bd1) + 2 * (kk & 3), idesc, kk == 0 ? acc0 : 1u);
+          umma_commit(&hdr->done[i & (kDoneRing - 1)]);
           s = (s + 1 == ns) ? 0 : s + 1;
           const bool wrap = a + 1 == nas;
           a = wrap ? 0 : a + 1;
           aph ^= wrap ? 1u : 0u;
         }
         if (!ok) break;
-        if (PAIR)
-          umma_commit_pair_mc(&hdr->acc_full[b], 3);  // the segment's accumulator is complete (both CTAs)
-        else
-          umma_commit(&hdr->acc_full[b]);
+        umma_commit(&hdr->acc_full[b]);  // the segment's accumulator is complete
         ++seg;
         kb = 0;
       }
@@ -384,8 +340,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
     const int row = quad * 32 + lane;
     const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
     for (int it = 0, s = 0, ph = 0, a = 0; it < total; ++it) {
-      bool w = mbar_wait(PAIR ? &hdr->w_full[s] : &hdr->full[s], ph & 1);
-      if (PAIR && rank == 0 && w) w = mbar_wait(&hdr->full[s], ph & 1);  // both activation halves landed
+      bool w = mbar_wait(&hdr->full[s], ph & 1);
       if (w && it >= nas) {
         const int u = it - nas;  // the unit that last used A slot a
         w = mbar_wait(&hdr->done[u % kDoneRing], (u / kDoneRing) & 1);
@@ -396,12 +351,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) {
-        if (PAIR)
-          mbar_arrive_cluster(map_shared_rank(smem_u32(&hdr->a_full[a]), 0));
-        else
-          mbar_arrive(&hdr->a_full[a]);
-      }
+      if (lane == 0) mbar_arrive(&hdr->a_full[a]);
       if (++s == ns) {
         s = 0;
         ++ph;
@@ -417,7 +367,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
     const int et = threadIdx.x - 192;  // 0 .. kEpiThreads - 1
     pdl_wait();  // s_a comes from the preceding kernel
     int seg = 0, tile = tile0, kb = kb0;
-    for (int i = 0; i < total; ++i, unit_next<PAIR>(p, tile, kb)) {
+    for (int i = 0; i < total; ++i, unit_next(p, tile, kb)) {
       if (!(i == total - 1 || kb == kbn - 1)) continue;
       // Segment `seg` (this CTA's units of `tile`) ends at unit i.
       const int b = seg & 1;
@@ -471,17 +421,12 @@ __global__ void __launch_bounds__(kPThreads, 1)
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) {
-        if (PAIR)
-          mbar_arrive_cluster(map_shared_rank(smem_u32(&hdr->acc_empty[b]), 0));
-        else
-          mbar_arrive(&hdr->acc_empty[b]);
-      }
+      if (lane == 0) mbar_arrive(&hdr->acc_empty[b]);
       ++seg;
     }
   }
 
-  if (!PAIR && p.splits > 1) {
+  if (p.splits > 1) {
     __syncwarp();    // the cluster barrier below is .aligned: reconverge first
     cluster_sync();  // every partial has reached its owner's shared memory
     if (warp >= 6) {
@@ -523,22 +468,11 @@ __global__ void __launch_bounds__(kPThreads, 1)
   }
 
   tc_fence_before();
-  if (PAIR) {
-    // Both CTAs' epilogues have seen their last accumulator, so every MMA of
-    // the pair (which writes into both CTAs' tensor memory and reads both
-    // CTAs' shared memory) has completed.
-    __syncwarp();
-    cluster_sync();
-  } else {
-    __syncthreads();
-  }
+  __syncthreads();
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();
-    if (PAIR)
-      tmem_dealloc_pair(tmem, 512u);
-    else
-      tmem_dealloc(tmem, 512u);
+    tmem_dealloc(tmem, 512u);
   }
 }
 
@@ -575,11 +509,11 @@ bool make_map_u8(CUtensorMap* map, const void* base, uint64_t rows, uint64_t col
   return r == CUDA_SUCCESS;
 }
 
-template <int SINK, bool PAIR>
+template <int SINK>
 cudaError_t launch_sink(const CUtensorMap& tw, const CUtensorMap& tx, const PParams& prm, const GemmTiling& t,
                         cudaStream_t stream) {
   static int cache[64] = {0};
-  const void* kfn = reinterpret_cast<const void*>(w4a4_tc_gemm_kernel<SINK, PAIR>);
+  const void* kfn = reinterpret_cast<const void*>(w4a4_tc_gemm_kernel<SINK>);
   cudaError_t e = ensure_dynamic_smem(kfn, t.smem_bytes, cache);
   if (e != cudaSuccess) return note_cuda(e, "w4a4_gemm: dynamic shared memory attribute");
   cudaLaunchConfig_t cfg = {};
@@ -592,16 +526,16 @@ cudaError_t launch_sink(const CUtensorMap& tw, const CUtensorMap& tx, const PPar
   attr[nattr].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[nattr].val.programmaticStreamSerializationAllowed = 1;
   ++nattr;
-  if (PAIR || t.splits > 1) {
+  if (t.splits > 1) {
     attr[nattr].id = cudaLaunchAttributeClusterDimension;
-    attr[nattr].val.clusterDim.x = PAIR ? 2u : static_cast<unsigned>(t.splits);
+    attr[nattr].val.clusterDim.x = static_cast<unsigned>(t.splits);
     attr[nattr].val.clusterDim.y = 1;
     attr[nattr].val.clusterDim.z = 1;
     ++nattr;
   }
   cfg.attrs = attr;
   cfg.numAttrs = nattr;
-  return note_cuda(cudaLaunchKernelEx(&cfg, w4a4_tc_gemm_kernel<SINK, PAIR>, tw, tx, prm), "w4a4_gemm: launch");
+  return note_cuda(cudaLaunchKernelEx(&cfg, w4a4_tc_gemm_kernel<SINK>, tw, tx, prm), "w4a4_gemm: launch");
 }
 
 // Clusters of S CTAs (one CTA per SM) that can be resident at once on the
@@ -613,7 +547,7 @@ int max_active_clusters(int S, int num_sms) {
   if (cache[dev][S] > 0) return cache[dev][S];
   static int smem_cache[64] = {0};
   const int smem = 200 * 1024;
-  const void* kfn = reinterpret_cast<const void*>(w4a4_tc_gemm_kernel<0, false>);
+  const void* kfn = reinterpret_cast<const void*>(w4a4_tc_gemm_kernel<0>);
   int n = 0;
   if (ensure_dynamic_smem(kfn, smem, smem_cache) == cudaSuccess) {
     cudaLaunchConfig_t cfg = {};
@@ -627,7 +561,7 @@ int max_active_clusters(int S, int num_sms) {
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (cudaOccupancyMaxActiveClusters(&n, w4a4_tc_gemm_kernel<0, false>, &cfg) != cudaSuccess) n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, w4a4_tc_gemm_kernel<0>, &cfg) != cudaSuccess) n = 0;
   }
   cudaGetLastError();  // a failed query is not an error of the caller
   if (n <= 0) n = num_sms / (2 * S);
@@ -636,19 +570,14 @@ int max_active_clusters(int S, int num_sms) {
 }
 
 // Estimated cycles of the whole-tile schedule for a token tile of BT: rounds
-// of tiles per SM (per CTA pair) x units x the slower of the MMA (4 * BT
-// cycles per 256-K unit on each SM at 8192 int8 MACs/clk) and a per-unit
-// floor that every unit costs whatever BT is (issuing 8 MMAs and a commit,
-// fetching and unpacking the 16 KB weight tile): about 900 cycles measured
-// for one CTA, less for a pair, whose leader issues for two SMs and whose
-// CTAs each load half the activations.
-long persistent_cost(int M, int N, int K, int BT, int num_sms, bool pair) {
-  const int rows = pair ? 2 * kRows : kRows;  // output channels per tile
-  const long tiles = static_cast<long>((M + BT - 1) / BT) * ((N + rows - 1) / rows);
-  const int walkers = pair ? num_sms / 2 : num_sms;
-  const long rounds = (tiles + walkers - 1) / walkers;
-  const long floor_cycles = pair ? 640 : 900;
-  const long per_unit = 4L * BT > floor_cycles ? 4L * BT : floor_cycles;
+// of tiles per SM x units x the slower of the MMA (4 * BT cycles per 256-K
+// unit at 8192 int8 MACs/clk) and a per-unit floor of about 900 cycles
+// (measured) that every unit costs whatever BT is: issuing 8 MMAs and a
+// commit, fetching and unpacking the 16 KB weight tile.
+long persistent_cost(int M, int N, int K, int BT, int num_sms) {
+  const long tiles = static_cast<long>((M + BT - 1) / BT) * ((N + kRows - 1) / kRows);
+  const long rounds = (tiles + num_sms - 1) / num_sms;
+  const long per_unit = 4L * BT > 900 ? 4L * BT : 900;
   return rounds * (K / kKB) * per_unit;
 }
 
@@ -665,16 +594,12 @@ int red_bytes(int BT, int S) { return S > 1 ? S * ((BT / 4 + S - 1) / S) * kRows
 // dynamic shared memory for them (padded so that one CTA, which owns all of
 // tensor memory, occupies an SM).
 void set_stages(GemmTiling& t) {
-  const int stage = kWTileBytes + (t.pair ? t.BT / 2 : t.BT) * kKB;
+  const int stage = kWTileBytes + t.BT * kKB;
   const int rb = red_bytes(t.BT, t.splits);
-  int ns = (220 * 1024 - 4096 - rb - (t.pair ? (t.BT / 2) * kXBox : 0)) / stage;
+  int ns = (220 * 1024 - 4096 - rb) / stage;
   if (ns > kMaxStages) ns = kMaxStages;
   t.nstages = ns;
   t.smem_bytes = 1024 + ns * stage + 2560 + rb;
-  // A pair's MMA reads its half of the activation tile from each CTA; keep
-  // one more half of slack behind the last stage so that the reads of the
-  // last stage never reach the end of the allocation.
-  if (t.pair) t.smem_bytes += (t.BT / 2) * kXBox;
   if (t.smem_bytes < 120 * 1024) t.smem_bytes = 120 * 1024;
   // Tensor memory: two accumulators of BT (rounded up to 32) columns, then
   // 64-column A slots in the rest of the 512.
@@ -694,35 +619,23 @@ GemmTiling choose_tiling(int M, int N, int K, int num_sms) {
   // Large M: whole tiles, with the token tile BT (multiple of 16, <= 192) of
   // the lowest estimated cost, when it yields at least half as many tiles as
   // SMs.
-  // A CTA pair takes tiles of 256 channels with BT a multiple of 32.
   if (M > 128) {
-    int best_bt = 0, best_pair = 0;
+    int best_bt = 0;
     long best = -1;
-    for (int pair = 0; pair < 1; ++pair) {  // CTA pairs measured slower; not selected
-      for (int bt = 192; bt >= 64; bt -= (pair ? 32 : 16)) {
-        const int rows = pair ? 2 * kRows : kRows;
-        const long tiles = static_cast<long>((M + bt - 1) / bt) * ((N + rows - 1) / rows);
-        if ((pair ? 4 : 2) * tiles < G) continue;
-        const long c = persistent_cost(M, N, K, bt, G, pair != 0);
-        if (best < 0 || c < best) {
-          best = c;
-          best_bt = bt;
-          best_pair = pair;
-        }
+    for (int bt = 192; bt >= 64; bt -= 16) {
+      const long tiles = static_cast<long>((M + bt - 1) / bt) * t.n_tiles;
+      if (2 * tiles < G) continue;
+      const long c = persistent_cost(M, N, K, bt, G);
+      if (best < 0 || c < best) {
+        best = c;
+        best_bt = bt;
       }
     }
     if (best_bt > 0) {
-      t.pair = best_pair;
       t.BT = best_bt;
-      t.n_tiles = (N + (best_pair ? 2 * kRows : kRows) - 1) / (best_pair ? 2 * kRows : kRows);
       t.m_tiles = (M + best_bt - 1) / best_bt;
       const int tiles = t.m_tiles * t.n_tiles;
-      int walkers = G;
-      if (best_pair) {
-        walkers = max_active_clusters(2, num_sms);  // pairs resident at once
-        if (walkers < 1 || walkers > G / 2) walkers = G / 2;
-      }
-      t.grid = (tiles < walkers ? tiles : walkers) * (best_pair ? 2 : 1);
+      t.grid = tiles < G ? tiles : G;
       set_stages(t);
       return t;
     }
@@ -761,11 +674,10 @@ cudaError_t launch_w4a4_gemm(const GemmArgs& a, GemmSink sink, const GemmTiling&
                    CU_TENSOR_MAP_SWIZZLE_128B))
     return note_cuda(cudaErrorInvalidValue, "w4a4_gemm: weight tensor map");
   if (!make_map_u8(&tx, a.xs8, static_cast<uint64_t>(a.M), static_cast<uint64_t>(a.K),
-                   static_cast<uint32_t>(t.pair ? t.BT / 2 : t.BT), kXBox, CU_TENSOR_MAP_SWIZZLE_128B))
+                   static_cast<uint32_t>(t.BT), kXBox, CU_TENSOR_MAP_SWIZZLE_128B))
     return note_cuda(cudaErrorInvalidValue, "w4a4_gemm: activation tensor map");
   if (t.grid < 1 || (t.splits == 1 && t.grid > kMaxGemmGrid) || t.splits < 1 || t.splits > 8 ||
-      t.splits > a.K / kKB || t.a_slots < 2 || t.nstages < 1 || t.nstages > kMaxStages ||
-      (t.pair && (t.splits != 1 || t.grid % 2 != 0 || t.BT % 32 != 0)))
+      t.splits > a.K / kKB || t.a_slots < 2 || t.nstages < 1 || t.nstages > kMaxStages)
     return note_cuda(cudaErrorInvalidValue, "w4a4_gemm: tiling");
   PParams pp{};
   pp.s_a = a.s_a;
@@ -784,18 +696,10 @@ cudaError_t launch_w4a4_gemm(const GemmArgs& a, GemmSink sink, const GemmTiling&
   pp.a_slots = t.a_slots;
   pp.splits = t.splits;
   cudaError_t e;
-  if (t.pair) {
-    switch (sink) {
-      case GemmSink::kBF16: e = launch_sink<0, true>(tw, tx, pp, t, stream); break;
-      case GemmSink::kF32: e = launch_sink<1, true>(tw, tx, pp, t, stream); break;
-      default: e = launch_sink<2, true>(tw, tx, pp, t, stream); break;
-    }
-  } else {
-    switch (sink) {
-      case GemmSink::kBF16: e = launch_sink<0, false>(tw, tx, pp, t, stream); break;
-      case GemmSink::kF32: e = launch_sink<1, false>(tw, tx, pp, t, stream); break;
-      default: e = launch_sink<2, false>(tw, tx, pp, t, stream); break;
-    }
+  switch (sink) {
+    case GemmSink::kBF16: e = launch_sink<0>(tw, tx, pp, t, stream); break;
+    case GemmSink::kF32: e = launch_sink<1>(tw, tx, pp, t, stream); break;
+    default: e = launch_sink<2>(tw, tx, pp, t, stream); break;
   }
   count_dispatch(t.splits > 1 ? 3 : 2);
   return e;

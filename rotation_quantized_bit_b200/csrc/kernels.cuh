@@ -30,7 +30,6 @@ enum class GemmSink : int { kBF16 = 0, kF32 = 1, kS32 = 2 };
 constexpr int kMaxGemmGrid = 160;  // whole-tile CTAs (one per SM)
 
 struct GemmTiling {
-  int pair;         // 1: CTA pairs (cta_group::2) on tiles of 256 output channels
   int splits;       // 1: whole tiles round-robin; S in {2,4,8}: a cluster of S CTAs splits each tile's K
   int grid;         // CTAs launched
   int BT;           // tokens per tile (MMA N), multiple of 16 in [16, 192]
