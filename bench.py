@@ -62,6 +62,9 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--only", default=None, help="restrict the workload to the linear with this name")
     ap.add_argument("--no-graph", action="store_true", help="launch the step eagerly instead of replaying a CUDA graph")
+    ap.add_argument("--flush", choices=["write+read", "write"], default="write+read",
+                    help="L2 flush between timed steps: a 256 MiB write, then (default) a 256 MiB read of a "
+                         "second buffer so that the write-back of the dirty lines is not charged to the step")
     return ap.parse_args()
 
 
@@ -83,6 +86,22 @@ def load_peaks():
                 "bf16_tflops_sustained": float(p.get("bf16_tflops_sustained", p["bf16_tflops"])),
                 "source": "measured"}
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def make_flusher(torch, dev, mode):
+    """L2 flush between timed steps.  A write of a buffer larger than L2 evicts
+    every input; with mode "write+read" a read of a second such buffer then
+    replaces the (dirty) written lines with clean ones, so that their
+    write-back to HBM is not charged to the next timed step."""
+    wbuf = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    rbuf = torch.zeros(L2_FLUSH_BYTES // 4, dtype=torch.int32, device=dev) if mode == "write+read" else None
+
+    def flush():
+        wbuf.zero_()
+        if rbuf is not None:
+            torch.amax(rbuf)
+
+    return flush
 
 
 # ------------------------------------------------------------------ clocks
@@ -188,7 +207,9 @@ def main():
             raise SystemExit(f"no linear named {args.only!r} in workload {args.workload}")
     config = {"workload": args.workload, "description": WORKLOAD_DESC[args.workload],
               "linears": [f"{s.name}:M{s.M}xK{s.K}xN{s.N}" for s in shapes],
-              "l2": "flushed between timed steps (256 MiB write, outside the events)",
+              "l2": ("flushed between timed steps, outside the events: 256 MiB write, then 256 MiB read of a second "
+                     "buffer (inputs cold, no dirty lines left in L2)") if args.flush == "write+read"
+                    else "flushed between timed steps, outside the events: 256 MiB write",
               "launch": "each step replayed from a CUDA graph (2 kernels per linear)" if not args.no_graph
                         else "eager launches",
               "parallelism": f"replicas x{max(world, args.gpus)}" if max(world, args.gpus) > 1 else "single GPU",
@@ -211,6 +232,10 @@ def main():
         torch.cuda.set_device(0)
     dev = torch.device("cuda", torch.cuda.current_device())
     rq.load_library()
+    # Dense int8 tensor-core rate of this GPU from the library's own no-memory
+    # tcgen05.mma.kind::i8 loop (128 x 256 x 32, all SMs), reported beside the
+    # roofline; the roofline's peak itself is the measured bf16 rate x 2.
+    mma_i8_tops, _ = rq.convrot_measure_mma_i8(256, False, 4096)
 
     # ---- inputs (untimed): activations per (M, K), packed weights per linear
     xs = {}
@@ -229,7 +254,7 @@ def main():
         del wd
     ws_bytes = max(rq.convrot_w4a4_workspace_size(s.M, s.N, s.K) for s in shapes)
     ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
-    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    flush = make_flusher(torch, dev, args.flush)
     stream = torch.cuda.current_stream()
     torch.cuda.synchronize()
 
@@ -251,7 +276,7 @@ def main():
                 evs[i][2].record(cur)
 
     for _ in range(max(args.warmup, 3)):
-        flush.zero_()
+        flush()
         run_step()
     torch.cuda.synchronize()
 
@@ -276,7 +301,7 @@ def main():
                 run_step(kern_events[k], per_kernel=True)
             kgraphs.append(g2)
         for g in (graphs[0], kgraphs[0]):  # one untimed replay of each
-            flush.zero_()
+            flush()
             g.replay()
         torch.cuda.synchronize()
     stream = torch.cuda.current_stream()
@@ -289,7 +314,7 @@ def main():
     if sampler:
         sampler.start()
     for k in range(args.steps):
-        flush.zero_()  # L2 flush, outside the step's events
+        flush()  # L2 flush, outside the step's events
         if graphs:
             graphs[k].replay()
         else:
@@ -302,7 +327,7 @@ def main():
     # Per-kernel breakdown (for the roofline of the dominant kernel): the same
     # step with the two launches of each linear separated by an event.
     for k in range(args.steps):
-        flush.zero_()
+        flush()
         if kgraphs:
             kgraphs[k].replay()
         else:
@@ -383,6 +408,9 @@ def main():
     roof["peak_source"] = (f"{peaks['source']} bf16 dense burst {peaks['bf16_tflops']} TFLOP/s x {INT8_PER_BF16} "
                            "(nominal int8:bf16)" if roof["bound"] == "tensor" else f"{peaks['source']} HBM copy")
     roof["share_of_breakdown"] = float(tsum / (t_quant.sum() + t_gemm.sum()))
+    if roof["bound"] == "tensor":
+        roof["int8_mma_measured_tops"] = round(mma_i8_tops, 1)
+        roof["frac_of_int8_mma_measured"] = roof["achieved"] / mma_i8_tops
     roof["traffic"] = committed_traffic(kname, s)
 
     e2e = None
@@ -450,14 +478,14 @@ def end_to_end(args, rq, torch, dev, stream, shapes, xs, layers, ws, flush, worl
             hy.copy_(y, non_blocking=True)
 
     for _ in range(max(args.warmup, 3)):
-        flush.zero_()
+        flush()
         step()
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     total = 0.0
     for _ in range(args.steps):
-        flush.zero_()
+        flush()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
         step()

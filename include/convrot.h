@@ -206,6 +206,22 @@ void convrot_dispatch_counts(uint64_t *counts, int n);
  * the next failing call on the same thread. */
 const char *convrot_last_error(void);
 
+/* Measurement of the dense int8 tensor-core rate of the current device (the
+ * denominator of the GEMM's roofline fraction; the pages quote no B200
+ * figure).  Launches one CTA per SM; one thread per CTA issues 16 * iters
+ * back-to-back tcgen05.mma.kind::i8 of shape 128 x N x 32 (s8 x s8 -> s32)
+ * whose operands stay on chip: B in shared memory, A in shared memory
+ * (a_in_tmem == 0) or in tensor memory (a_in_tmem != 0, the form the W4A4
+ * GEMM issues).  No global memory is touched except a per-CTA cycle count.
+ *   N       16 .. 256, a multiple of 16
+ *   iters   1 .. 2^20
+ *   tops    (output) 2 * 128 * N * 32 * MMAs / wall time (CUDA events), 1e12/s
+ *   cycles_per_mma (output) mean SM cycles per MMA of one CTA
+ * Runs on the legacy default stream and synchronizes it (a host-blocking
+ * diagnostic, not for use inside stream capture). */
+convrot_status_t convrot_measure_mma_i8(int N, int a_in_tmem, int iters, double *tops,
+                                        double *cycles_per_mma);
+
 /* Library build identifier (static string). */
 const char *convrot_version(void);
 

@@ -40,6 +40,7 @@ EXPORTS = [
     "w4a4_gemm", "w4a4_gemm_s32", "w4a4_gemm_f32", "convrot_w4a4_workspace_size", "convrot_w4a4_linear",
     "convrot_w4a4_linear_f32", "convrot_w4a4_linear_noalloc", "convrot_w4a4_quantize", "convrot_w4a4_gemm_quantized", "convrot_device_error",
     "convrot_dispatch_counts", "convrot_last_error", "convrot_selftest_timeout", "convrot_version",
+    "convrot_measure_mma_i8",
 ]
 
 
@@ -86,6 +87,7 @@ def load_library():
     lib.convrot_selftest_timeout.argtypes = [ctypes.c_uint, P]
     lib.convrot_dispatch_counts.argtypes = [ctypes.POINTER(ctypes.c_uint64), I]
     lib.convrot_dispatch_counts.restype = None
+    lib.convrot_measure_mma_i8.argtypes = [I, I, I, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_double)]
     for name in lib_status_fns():
         getattr(lib, name).restype = I
     _lib = lib
@@ -95,7 +97,8 @@ def load_library():
 def lib_status_fns():
     return ["convrot_pack_weight", "convrot_rotate_quant", "w4a4_gemm", "w4a4_gemm_s32", "w4a4_gemm_f32",
             "convrot_w4a4_linear", "convrot_w4a4_linear_f32", "convrot_w4a4_linear_noalloc", "convrot_w4a4_quantize",
-            "convrot_w4a4_gemm_quantized", "convrot_device_error", "convrot_selftest_timeout"]
+            "convrot_w4a4_gemm_quantized", "convrot_device_error", "convrot_selftest_timeout",
+            "convrot_measure_mma_i8"]
 
 
 def _check(fn: str, rc: int):
@@ -293,6 +296,15 @@ def convrot_dispatch_counts():
     arr = (ctypes.c_uint64 * 4)()
     lib.convrot_dispatch_counts(arr, 4)
     return {"rotate_quant": arr[0], "unpack_codes": arr[1], "tc_gemm": arr[2], "tc_gemm_splitk": arr[3]}
+
+
+def convrot_measure_mma_i8(N: int = 256, a_in_tmem: bool = False, iters: int = 4096):
+    """Dense int8 tensor-core rate of this GPU (see include/convrot.h):
+    returns (TOPS, SM cycles per 128 x N x 32 MMA).  Blocks the host."""
+    tops, cyc = ctypes.c_double(0.0), ctypes.c_double(0.0)
+    _check("convrot_measure_mma_i8", load_library().convrot_measure_mma_i8(
+        int(N), 1 if a_in_tmem else 0, int(iters), ctypes.byref(tops), ctypes.byref(cyc)))
+    return float(tops.value), float(cyc.value)
 
 
 def convrot_version() -> str:

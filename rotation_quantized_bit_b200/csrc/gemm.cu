@@ -162,10 +162,17 @@ __device__ __forceinline__ void store_chunk(const P& p, int m, int n, const uint
 //   warps 6..13 epilogue, draining one of two accumulators while the MMA
 //               fills the other (two warps per tensor-memory lane quadrant,
 //               each taking every other 32-column chunk)
-// The MMA thread commits once per unit, to done[unit % 32]; that one
-// completion frees both the unit's shared-memory stage (for the TMA producer)
-// and its A slot (for the unpack warps).  A unit of 256 K values is 8 MMAs,
-// so the waits and the commit of the issuing thread are spread over 8.
+// A stage's weight tile lands on wfull[s]; ready[s] completes when its
+// activation tile has landed and all four unpack warps have written the
+// unit's weights to tensor memory, so the MMA thread waits on ready alone.
+// Weight tiles do not depend on the preceding prologue kernel: the first
+// stages are requested, and their weights unpacked, before the grid waits
+// for that kernel.  The MMA thread issues the units of a tile two at a time
+// (16 MMAs between waits: at small token counts an MMA takes ~45 cycles and
+// each wait, commit or branch between MMA groups costs about as much), then
+// commits once per unit, to done[unit % 32]; that completion frees both the
+// unit's shared-memory stage (for the TMA producer) and its A slot (for the
+// unpack warps).
 constexpr int kPThreads = 448;
 constexpr int kEpiThreads = 256;  // warps 6..13
 
@@ -179,12 +186,13 @@ struct PParams {
   int acc_stride;   // tensor-memory columns per accumulator (BT rounded up to 32)
   int a_slots;      // A slots of 64 columns after the two accumulators
   int splits;       // 1: whole tiles; S > 1: the cluster of S CTAs splits one tile's K
+  int pair;         // the MMA thread issues two units per group
 };
 
 struct PHeader {
-  uint64_t full[kMaxStages];    // the stage's weight and activation tiles landed
+  uint64_t wfull[kMaxStages];   // the stage's weight tile landed
+  uint64_t ready[kMaxStages];   // the stage's activation tile landed and its weights are in tensor memory
   uint64_t done[kDoneRing];     // unit i's MMAs have completed (its stage and A slot are free)
-  uint64_t a_full[kMaxASlots];
   uint64_t acc_full[2];
   uint64_t acc_empty[2];
   uint32_t tmem_base;
@@ -234,9 +242,11 @@ __global__ void __launch_bounds__(kPThreads, 1)
   auto x_row = [&](int tile) { return (tile % p.m_tiles) * BT; };
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < ns; ++s) mbar_init(&hdr->full[s], 1);
+    for (int s = 0; s < ns; ++s) {
+      mbar_init(&hdr->wfull[s], 1);
+      mbar_init(&hdr->ready[s], 5);  // the producer (with the activation bytes) + one arrive per unpack warp
+    }
     for (int r = 0; r < kDoneRing; ++r) mbar_init(&hdr->done[r], 1);  // one MMA commit
-    for (int a = 0; a < nas; ++a) mbar_init(&hdr->a_full[a], 4);      // one arrive per unpack warp
     for (int b = 0; b < 2; ++b) {
       mbar_init(&hdr->acc_full[b], 1);
       mbar_init(&hdr->acc_empty[b], kEpiThreads / 32);  // one arrive per epilogue warp
@@ -256,23 +266,25 @@ __global__ void __launch_bounds__(kPThreads, 1)
 
   if (warp == 0) {
     // ------------------------------------------------ TMA producer
-    // The weight and activation tiles of a stage complete on full[s].
+    // A stage's weight tile completes on wfull[s]; its activation tile on
+    // ready[s] (the producer's arrival, together with the unpack warps').
     if (lane == 0) {
-      const uint32_t wbytes = static_cast<uint32_t>(stage_bytes);
-      auto wbar = [&](int s) { return &hdr->full[s]; };
+      const uint32_t xbytes = static_cast<uint32_t>(BT * kKB);
+      auto load_w = [&](int s, int tile, int kb) {
+        mbar_arrive_expect_tx(&hdr->wfull[s], static_cast<uint32_t>(kWTileBytes));
+        tma_load_2d(smem + s * stage_bytes, &tm_w, &hdr->wfull[s], kb * (kKB / 2), w_row(tile));
+      };
       auto load_x = [&](int s, int tile, int kb) {
         uint8_t* xs = smem + s * stage_bytes + kWTileBytes;
-        tma_load_2d(xs, &tm_x, &hdr->full[s], kb * kKB, x_row(tile));
-        tma_load_2d(xs + BT * kXBox, &tm_x, &hdr->full[s], kb * kKB + kXBox, x_row(tile));
+        mbar_arrive_expect_tx(&hdr->ready[s], xbytes);
+        tma_load_2d(xs, &tm_x, &hdr->ready[s], kb * kKB, x_row(tile));
+        tma_load_2d(xs + BT * kXBox, &tm_x, &hdr->ready[s], kb * kKB + kXBox, x_row(tile));
       };
       // Weight tiles of the first stages do not depend on the preceding
       // prologue kernel: request them before waiting for it.
       const int prime = total < ns ? total : ns;
       int tile = tile0, kb = kb0;
-      for (int i = 0; i < prime; ++i, unit_next(p, tile, kb)) {
-        mbar_arrive_expect_tx(wbar(i), wbytes);
-        tma_load_2d(smem + i * stage_bytes, &tm_w, wbar(i), kb * (kKB / 2), w_row(tile));
-      }
+      for (int i = 0; i < prime; ++i, unit_next(p, tile, kb)) load_w(i, tile, kb);
       pdl_wait();
       tile = tile0;
       kb = kb0;
@@ -281,55 +293,96 @@ __global__ void __launch_bounds__(kPThreads, 1)
       for (; it < total; ++it, unit_next(p, tile, kb)) {
         const int w = it - ns;  // the unit that last used stage s
         if (!mbar_wait(&hdr->done[w % kDoneRing], (w / kDoneRing) & 1)) break;
-        mbar_arrive_expect_tx(wbar(s), wbytes);
-        tma_load_2d(smem + s * stage_bytes, &tm_w, wbar(s), kb * (kKB / 2), w_row(tile));
+        load_w(s, tile, kb);
         load_x(s, tile, kb);
         if (++s == ns) s = 0;
       }
-      // Drain: every issued load has landed before the block may exit.
-      for (int i = (it > ns ? it - ns : 0); i < it; ++i) mbar_wait(wbar(i % ns), (i / ns) & 1);
+      // Drain: every issued load has landed before the block may exit.  In
+      // the normal case the last stages' barriers have completed; after a
+      // failed wait (anywhere in the grid) the weight tiles are awaited with a
+      // time limit that ignores the error word, and the activation tiles,
+      // whose barrier also needs the unpack warps, are given a fixed 100 us.
+      bool clean = true;
+      for (int i = (it > ns ? it - ns : 0); i < it; ++i) {
+        if (clean) clean = mbar_wait(&hdr->wfull[i % ns], (i / ns) & 1) && mbar_wait(&hdr->ready[i % ns], (i / ns) & 1);
+        if (!clean) (void)mbar_drain(&hdr->wfull[i % ns], (i / ns) & 1, 100000000ull);
+      }
+      if (!clean || it < total) {
+        const unsigned long long t0 = globaltimer_ns();
+        while (globaltimer_ns() - t0 < 100000ull) {
+        }
+      }
     }
   } else if (warp == 1) {
     // ------------------------------------------------ MMA issuer
-    // The unpack warps arrive on a_full only after they have seen the unit's
-    // stage land (weights and activations), so a_full alone says the MMAs
-    // may go.
-    // The loop over a segment's units is kept free of branches other than
-    // its own back edge: a branch between tcgen05.mma groups costs about as
-    // much as an MMA.
-    if (lane == 0) {
+    // The whole warp runs the loop, so that the operand descriptors are
+    // warp-uniform values; lane 0 issues the MMAs and commits.  ready[s]
+    // says both operands of the stage's unit are in place.
+    {
+      const bool leader = lane == 0;
       const uint32_t idesc = umma_idesc_i8(kRows, BT, /*a_signed=*/true, /*b_signed=*/true);
       const uint32_t x1 = static_cast<uint32_t>(BT * kXBox);  // second activation box of a stage
-      int kb = kb0, seg = 0, s = 0, a = 0;
-      uint32_t aph = 0;
+      const uint32_t smem0 = smem_u32(smem) + static_cast<uint32_t>(kWTileBytes);
+      int kb = kb0, seg = 0, s = 0, a = 0, sph = 0;
       bool ok = true;
-      for (int i = 0; i < total && ok;) {
-        const int len = min(total - i, kbn - kb);  // units of this segment
-        const int b = seg & 1;
-        if (seg >= 2 && !mbar_wait(&hdr->acc_empty[b], ((seg / 2) - 1) & 1)) break;
-        tc_fence_after();
-        const uint32_t d_tmem = tmem + static_cast<uint32_t>(b * p.acc_stride);
-        for (int j = 0; j < len; ++j, ++i) {
-          if (!mbar_wait(&hdr->a_full[a], aph)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t xs = smem_u32(smem + s * stage_bytes + kWTileBytes);
-          const uint64_t bd0 = umma_desc_k_sw128(xs), bd1 = umma_desc_k_sw128(xs + x1);
-          const uint32_t at = tmem + a_col0 + 64u * static_cast<uint32_t>(a);
-          const uint32_t acc0 = j > 0 ? 1u : 0u;
+      // The 8 MMAs of the unit in stage s / A slot a (acc0: accumulate into
+      // the existing sum for the first of them).
+      auto issue_unit = [&](uint32_t d_tmem, uint32_t acc0) {
+        const uint32_t xs = smem0 + static_cast<uint32_t>(s * stage_bytes);
+        const uint64_t bd0 = umma_desc_k_sw128(xs), bd1 = umma_desc_k_sw128(xs + x1);
+        const uint32_t at = tmem + a_col0 + 64u * static_cast<uint32_t>(a);
+        if (leader) {
 #pragma unroll
           for (int kk = 0; kk < kKB / 32; ++kk)
             umma_i8_ts(d_tmem, at + 8 * kk, (kk < 4 ? bd0 : bd1) + 2 * (kk & 3), idesc, kk == 0 ? acc0 : 1u);
-          umma_commit(&hdr->done[i & (kDoneRing - 1)]);
-          s = (s + 1 == ns) ? 0 : s + 1;
-          const bool wrap = a + 1 == nas;
-          a = wrap ? 0 : a + 1;
-          aph ^= wrap ? 1u : 0u;
+        }
+      };
+      auto advance = [&]() {
+        if (++s == ns) {
+          s = 0;
+          sph ^= 1;
+        }
+        if (++a == nas) a = 0;
+      };
+      for (int i = 0; i < total && ok;) {
+        const int len = min(total - i, kbn - kb);  // units of this segment
+        const int b = seg & 1;
+        if (seg >= 2 && !__all_sync(0xffffffffu, mbar_wait(&hdr->acc_empty[b], ((seg / 2) - 1) & 1))) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem + static_cast<uint32_t>(b * p.acc_stride);
+        int j = 0;
+        // Two units per group when the MMAs are short (small token tiles,
+        // enough stages and A slots to prepare two units ahead).
+        if (p.pair) {
+          for (; j + 1 < len; j += 2, i += 2) {
+            const int s1 = s + 1 == ns ? 0 : s + 1;
+            const int ph1 = s + 1 == ns ? sph ^ 1 : sph;
+            ok = __all_sync(0xffffffffu, mbar_wait(&hdr->ready[s], sph) & mbar_wait(&hdr->ready[s1], ph1));
+            if (!ok) break;
+            tc_fence_after();
+            issue_unit(d_tmem, j > 0 ? 1u : 0u);
+            advance();
+            issue_unit(d_tmem, 1u);
+            advance();
+            if (leader) {
+              umma_commit(&hdr->done[i & (kDoneRing - 1)]);
+              umma_commit(&hdr->done[(i + 1) & (kDoneRing - 1)]);
+            }
+            __syncwarp();
+          }
+        }
+        for (; ok && j < len; ++j, ++i) {
+          ok = __all_sync(0xffffffffu, mbar_wait(&hdr->ready[s], sph));
+          if (!ok) break;
+          tc_fence_after();
+          issue_unit(d_tmem, j > 0 ? 1u : 0u);
+          advance();
+          if (leader) umma_commit(&hdr->done[i & (kDoneRing - 1)]);
+          __syncwarp();
         }
         if (!ok) break;
-        umma_commit(&hdr->acc_full[b]);  // the segment's accumulator is complete
+        if (leader) umma_commit(&hdr->acc_full[b]);  // the segment's accumulator is complete
+        __syncwarp();
         ++seg;
         kb = 0;
       }
@@ -340,7 +393,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
     const int row = quad * 32 + lane;
     const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
     for (int it = 0, s = 0, ph = 0, a = 0; it < total; ++it) {
-      bool w = mbar_wait(&hdr->full[s], ph & 1);
+      bool w = mbar_wait(&hdr->wfull[s], ph & 1);
       if (w && it >= nas) {
         const int u = it - nas;  // the unit that last used A slot a
         w = mbar_wait(&hdr->done[u % kDoneRing], (u / kDoneRing) & 1);
@@ -351,7 +404,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&hdr->a_full[a]);
+      if (lane == 0) mbar_arrive(&hdr->ready[s]);
       if (++s == ns) {
         s = 0;
         ++ph;
@@ -373,18 +426,23 @@ __global__ void __launch_bounds__(kPThreads, 1)
       const int b = seg & 1;
       const int m0 = (tile % p.m_tiles) * BT, n0 = w_row(tile);
       const int n = n0 + row;
+      // The segment's scales and bias are fetched before its accumulator is
+      // waited for, so their latency hides behind the MMAs.
+      float* sa = sa_buf + 192 * b;
+      float sw = 0.0f, bv = 0.0f;
+      if (p.splits == 1) {
+        if (SINK != static_cast<int>(GemmSink::kS32))
+          for (int c = et; c < BT; c += kEpiThreads) sa[c] = (m0 + c < p.M) ? __ldg(p.s_a + m0 + c) : 0.0f;
+        sw = (SINK != static_cast<int>(GemmSink::kS32) && n < p.N) ? __ldg(p.s_w + n) : 0.0f;
+        bv = (p.bias && n < p.N) ? __uint_as_float(static_cast<uint32_t>(__ldg(p.bias + n)) << 16) : 0.0f;
+        named_barrier(1, kEpiThreads);  // s_a staged; all warps are done with segment seg - 2
+      }
       // On a failed wait the warp skips the segment's data but keeps taking
       // part in the named and cluster barriers, so no peer is left waiting.
       const bool ok = __all_sync(0xffffffffu, mbar_wait(&hdr->acc_full[b], (seg / 2) & 1));
       tc_fence_after();
       const uint32_t acc = tmem + lane_base + static_cast<uint32_t>(b * p.acc_stride);
       if (p.splits == 1) {
-        float* sa = sa_buf + 192 * b;
-        if (SINK != static_cast<int>(GemmSink::kS32))
-          for (int c = et; c < BT; c += kEpiThreads) sa[c] = (m0 + c < p.M) ? __ldg(p.s_a + m0 + c) : 0.0f;
-        named_barrier(1, kEpiThreads);  // s_a staged; all warps are done with segment seg - 2
-        const float sw = (SINK != static_cast<int>(GemmSink::kS32) && n < p.N) ? __ldg(p.s_w + n) : 0.0f;
-        const float bv = (p.bias && n < p.N) ? __uint_as_float(static_cast<uint32_t>(__ldg(p.bias + n)) << 16) : 0.0f;
         // 32-column chunks (the accumulator stride is BT rounded up to 32, so
         // the last chunk's extra columns exist and are simply not stored).
         for (int c = 32 * half; ok && c < BT; c += 64) {
@@ -427,6 +485,18 @@ __global__ void __launch_bounds__(kPThreads, 1)
   }
 
   if (p.splits > 1) {
+    // Scales and bias of this CTA's rows and channels, fetched before the
+    // cluster barrier (tokens into sa_buf, made visible by the barrier).
+    float sw_red = 0.0f, bv_red = 0.0f;
+    if (warp >= 6) {
+      const int n = (tile0 / p.m_tiles) * kRows + (warp & 3) * 32 + lane;
+      const int m0 = (tile0 % p.m_tiles) * BT;
+      if (SINK != static_cast<int>(GemmSink::kS32)) {
+        for (int c = threadIdx.x - 192; c < BT; c += kEpiThreads) sa_buf[c] = (m0 + c < p.M) ? __ldg(p.s_a + m0 + c) : 0.0f;
+        sw_red = n < p.N ? __ldg(p.s_w + n) : 0.0f;
+      }
+      bv_red = (p.bias && n < p.N) ? __uint_as_float(static_cast<uint32_t>(__ldg(p.bias + n)) << 16) : 0.0f;
+    }
     __syncwarp();    // the cluster barrier below is .aligned: reconverge first
     cluster_sync();  // every partial has reached its owner's shared memory
     if (warp >= 6) {
@@ -440,8 +510,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
       const int n = (tile0 / p.m_tiles) * kRows + row;
       const int m0 = (tile0 % p.m_tiles) * BT;
       const int rank = static_cast<int>(cluster_ctarank());
-      const float sw = (SINK != static_cast<int>(GemmSink::kS32) && n < p.N) ? __ldg(p.s_w + n) : 0.0f;
-      const float bv = (p.bias && n < p.N) ? __uint_as_float(static_cast<uint32_t>(__ldg(p.bias + n)) << 16) : 0.0f;
+      const float sw = sw_red, bv = bv_red;
       const int4* red4 = reinterpret_cast<const int4*>(red);
       for (int gl = half; gl < ngl; gl += 2) {
         const int g = gl * S + rank;
@@ -459,7 +528,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
         for (int q = 0; q < 4; ++q) {
           const int m = m0 + 4 * g + q;
           if (m < p.M) {
-            const float sa = SINK != static_cast<int>(GemmSink::kS32) ? __ldg(p.s_a + m) : 0.0f;
+            const float sa = SINK != static_cast<int>(GemmSink::kS32) ? sa_buf[m - m0] : 0.0f;
             store_output<SINK>(p, m, n, sv[q], sa, sw, bv);
           }
         }
@@ -695,6 +764,7 @@ cudaError_t launch_w4a4_gemm(const GemmArgs& a, GemmSink sink, const GemmTiling&
   pp.acc_stride = t.acc_stride;
   pp.a_slots = t.a_slots;
   pp.splits = t.splits;
+  pp.pair = (t.BT <= 128 && t.a_slots >= 4 && t.nstages >= 4) ? 1 : 0;
   cudaError_t e;
   switch (sink) {
     case GemmSink::kBF16: e = launch_sink<0>(tw, tx, pp, t, stream); break;

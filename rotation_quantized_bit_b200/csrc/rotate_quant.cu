@@ -11,22 +11,34 @@
 //
 // Bit-exact contract.  The butterflies use the fixed stage order (stride 1,
 // 4, 16, 64) and association (p=a+b, q=a-b, r=c+d, t=c-d -> p+t, p-t, q+r,
-// r-q), every add is a correctly rounded fp32 add (packed f32x2 or scalar, no
-// contraction), the 1/16 is one multiply, the scale is an IEEE division, and
-// each code equals rint(fl(x' / s)) with ties to even, so codes and scales are
-// identical bit for bit to any plain fp32 evaluation of that definition.
+// r-q), every add is a correctly rounded fp32 add (no contraction), the 1/16
+// is one multiply, the scale is an IEEE division, and each code equals
+// rint(fl(x' / s)) with ties to even, so codes and scales are identical bit
+// for bit to any plain fp32 evaluation of that definition.
 //
-// Layout.  A lane owns one half (128 channels) of a 256-channel group and
-// keeps it in registers as 64 fp32 pairs; pair i holds channels i and i + 64
-// of the half, so the radix-4 stages on channel bits (0,1), (2,3), (4,5) are
-// packed f32x2 butterflies, and the stage on bits (6,7) combines the two
-// members of a pair and the two halves held by the lane pair (lane ^ 1), one
-// shuffle per two channels.  Input is staged through shared memory: a warp
-// copies its 8 KB tile (16 groups) with coalesced 16-byte cp.async into
-// XOR-swizzled slots, so both the copy and each lane's 16 reads of its own
-// 256 bytes are free of bank conflicts.  The next row block is prefetched
-// while the current one is computed.  Codes leave through the same buffer
-// and coalesced 16-byte stores.
+// Layout.  A 256-channel group is one task of 16 lanes (half a warp); each
+// lane holds 16 channels of each of two tasks (two groups, from the same row
+// or not) as fp32 pairs (task 0, task 1), so that every operation of the path
+// is one packed f32x2 instruction for both tasks.  Channel index bits 0-3
+// are first the register index and bits 4-7 the lane (lane l holds channels
+// 16 l .. 16 l + 15), so the stages on bits (0,1) and (2,3) run in registers.
+// A transpose of the pairs through the half-warp's shared-memory tile then
+// swaps the roles (lane l holds channels l, 16 + l, ..., 240 + l) and the
+// stages on bits (4,5) and (6,7) run in registers as well.  The tile's rows
+// are 16 pairs (128 bytes) with the 16-byte chunks XOR-swizzled by the row,
+// so the eight 16-byte stores of a lane and its sixteen 8-byte loads are free
+// of bank conflicts.  A block owns blocks of R whole rows (R * G tasks, G = K
+// / 256) in turn, so the per-row amax is a shuffle reduction within each
+// task plus one shared-memory atomic max per task.  Each lane then quantizes
+// its channels; the code bytes go back to row order through the same tile
+// (byte stores at their final positions, one 16-byte load per task) and
+// leave with coalesced stores.
+//
+// Input staging.  The blocks are persistent: one thread keeps a ring of S
+// row blocks in flight with 1-D bulk copies (the TMA engine, one contiguous
+// copy of R * K bf16 per row block, completion on an mbarrier), so HBM reads
+// run ahead of the arithmetic without holding registers.  A stage is
+// refilled right after the block barrier that ends its readers' use of it.
 //
 // Quantization.  The code is rint(q) with q the correctly rounded quotient
 // x' / s.  q is formed without a division by Markstein's correction (P.
@@ -40,26 +52,29 @@
 // the remainders and products clear of underflow, which holds for every scale
 // s >= 2^-100 wherever the code can be nonzero; rows with a smaller scale (zero
 // included) take the IEEE division.  rint is the addition of 1.5 * 2^23, whose
-// low byte is then the two's-complement code.
+// low byte is then the two's-complement code (|x'/s| <= 7 up to rounding, so
+// no clamp is needed on this path).
 #include <cuda_runtime.h>
 
 #include <cstdint>
 
 #include "kernels.cuh"
+#include "ptx.cuh"
 
 namespace convrot {
 
 namespace {
 
+constexpr float kMagic = 12582912.0f;           // 1.5 * 2^23: x + kMagic rounds x to an integer, ties to even
+constexpr float kMinScale = 7.88860905e-31f;    // 2^-100: below it, codes by division
+constexpr int kTileBytes = 2048;                // per-half-warp transpose tile: 16 x 16 fp32 pairs
+constexpr int kMaxRows = 64;                    // rows per row block (K = 256 -> 64 tasks)
+constexpr int kMaxThreads = 1024;
+
 typedef unsigned long long u64;
 
-constexpr int kTileBytes = 8192;          // 16 groups x 256 bf16 per warp
-constexpr int kMaxWarps = 8;              // at most 128 groups per row block
-constexpr float kMagic = 12582912.0f;     // 1.5 * 2^23: x + kMagic rounds x to an integer, ties to even
-constexpr float kMinScale = 7.88860905e-31f;           // 2^-100: below it, codes by division
-
-// ---------------------------------------------------------------- helpers
-
+// Packed fp32 pairs: f2(lo, hi), and correctly rounded f32x2 arithmetic (no
+// contraction).
 __device__ __forceinline__ u64 f2(float lo, float hi) {
   u64 d;
   asm("mov.b64 %0, {%1, %2};" : "=l"(d) : "f"(lo), "f"(hi));
@@ -88,38 +103,14 @@ __device__ __forceinline__ u64 f2_fma(u64 a, u64 b, u64 c) {
   asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
   return d;
 }
-__device__ __forceinline__ float max3(float a, float b, float c) {
-  float d;
-  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
-  return d;
-}
 
-// One radix-4 butterfly on packed pairs: (a,b,c,d) -> (p+t, p-t, q+r, r-q).
+// One radix-4 butterfly on pairs: (a,b,c,d) -> (p+t, p-t, q+r, r-q).
 __device__ __forceinline__ void bfly4(u64& a, u64& b, u64& c, u64& d) {
   const u64 p = f2_add(a, b), q = f2_sub(a, b), r = f2_add(c, d), t = f2_sub(c, d);
   a = f2_add(p, t);
   b = f2_sub(p, t);
   c = f2_add(q, r);
   d = f2_sub(r, q);
-}
-
-__device__ __forceinline__ uint32_t smem_addr(const void* p) {
-  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, bool valid) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(valid ? 16 : 0) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
-
-// Byte 0 of four words -> one word (the code bytes of four rounded floats).
-__device__ __forceinline__ uint32_t gather_b0(uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
-  const uint32_t ab = __byte_perm(a, b, 0x0040);  // [a0, b0, .., ..]
-  const uint32_t cd = __byte_perm(c, d, 0x0040);  // [c0, d0, .., ..]
-  return __byte_perm(ab, cd, 0x5410);             // [a0, b0, c0, d0]
 }
 
 // Eight codes as bytes (natural order, two words) -> packed nibbles, even index low.
@@ -129,219 +120,226 @@ __device__ __forceinline__ uint32_t pack_nibbles(uint32_t lo4, uint32_t hi4) {
   return __byte_perm(a2, b2, 0x6420);
 }
 
-// Sixteen codes of two chunks (8 + 8, natural order) -> staging.  s8 layout:
-// per chunk the operand order (0,2,4,6,1,3,5,7), 16 bytes per chunk pair in
-// slot (pair ^ (region & 7)) of the lane's 128-byte region.  Packed layout: 4
-// bytes per chunk, 8 bytes per chunk pair, at region * 64 + 8 * pair.
-template <bool PACKED>
-__device__ __forceinline__ void stage_chunk_pair(uint8_t* stage, int region, int pair, const uint32_t (&c)[16]) {
-  if (PACKED) {
-    const uint32_t w0 = pack_nibbles(gather_b0(c[0], c[1], c[2], c[3]), gather_b0(c[4], c[5], c[6], c[7]));
-    const uint32_t w1 = pack_nibbles(gather_b0(c[8], c[9], c[10], c[11]), gather_b0(c[12], c[13], c[14], c[15]));
-    *reinterpret_cast<uint2*>(stage + 64 * region + 8 * pair) = make_uint2(w0, w1);
-  } else {
-    uint4 o;
-    o.x = gather_b0(c[0], c[2], c[4], c[6]);
-    o.y = gather_b0(c[1], c[3], c[5], c[7]);
-    o.z = gather_b0(c[8], c[10], c[12], c[14]);
-    o.w = gather_b0(c[9], c[11], c[13], c[15]);
-    *reinterpret_cast<uint4*>(stage + 128 * region + 16 * (pair ^ (region & 7))) = o;
-  }
-}
-
 struct RQParams {
   const uint16_t* x;
   int M, K;
   int G;        // groups of 256 per row
-  int R;        // rows per block
+  int R;        // rows per row block
   int nblocks;  // ceil(M / R)
+  int S;        // stages of the input ring
   RotateQuantOut out;
 };
 
-// Shared-memory slot of logical 16-byte chunk c = 16 * region + k of the input
-// tile: k XOR the region's low three bits.
-__device__ __forceinline__ int in_slot(int c) { return (c & ~15) | ((c & 15) ^ ((c >> 4) & 7)); }
+// Byte position of channel c's code within its 16-byte run of the output
+// row: natural order for packed output; for the s8 operand layout each
+// 8-channel chunk is stored in the order (0, 2, 4, 6, 1, 3, 5, 7).
+template <bool PACKED>
+__device__ __forceinline__ int code_pos(int c) {
+  if (PACKED) return c & 15;
+  const int e = c & 7;
+  return (c & 8) | ((e & 1) ? 4 + (e >> 1) : (e >> 1));
+}
+
+// Dynamic shared memory: S input stages of R * K bf16, then one transpose tile
+// per half-warp, then S mbarriers.
+__host__ __device__ constexpr int rq_stage_bytes(int R, int K) { return R * K * 2; }
+__host__ __device__ constexpr int rq_smem_bytes(int R, int K, int S, int threads) {
+  return S * rq_stage_bytes(R, K) + (threads / 16) * kTileBytes + 8 * S;
+}
 
 template <bool PACKED>
-__global__ void __launch_bounds__(kMaxWarps * 32, 1) rotate_quant_kernel(const __grid_constant__ RQParams p) {
-  extern __shared__ __align__(16) uint8_t smem[];
-  __shared__ uint32_t row_amax[2][128];
+__global__ void __launch_bounds__(kMaxThreads) rotate_quant_kernel(const __grid_constant__ RQParams p) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  __shared__ uint32_t row_amax[3][kMaxRows];
   // Let the dependent GEMM launch now: it streams its weights meanwhile and
   // waits (griddepcontrol.wait) for this grid before reading codes or scales.
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  uint8_t* const wbuf0 = smem + (2 * warp) * kTileBytes;
-  uint8_t* const wbuf1 = smem + (2 * warp + 1) * kTileBytes;
-  const int groups_per_block = p.R * p.G;
-  const size_t row_bytes = static_cast<size_t>(p.K) * 2;
-  const size_t total_bytes = static_cast<size_t>(p.M) * row_bytes;
-  const uint8_t* xb = reinterpret_cast<const uint8_t*>(p.x);
+  const int hw = threadIdx.x >> 4, l = threadIdx.x & 15;
+  const int nhw = blockDim.x >> 4;
+  const int S = p.S;
+  const int stage_bytes = rq_stage_bytes(p.R, p.K);
+  uint8_t* const stages = smem;
+  uint8_t* const tile = smem + S * stage_bytes + hw * kTileBytes;
+  // Byte tiles of the two tasks inside the pair tile; odd half-warps start 16
+  // bytes later so that the two half-warps of a warp hit different banks.
+  uint8_t* const btile0 = tile + 16 * (hw & 1);
+  uint8_t* const btile1 = btile0 + 256;
+  uint64_t* const full = reinterpret_cast<uint64_t*>(smem + S * stage_bytes + nhw * kTileBytes);
+  const int tasks = p.R * p.G;
+  const int iters =
+      static_cast<int>(blockIdx.x) < p.nblocks ? (p.nblocks - 1 - static_cast<int>(blockIdx.x)) / gridDim.x + 1 : 0;
 
-  // Coalesced copy of this warp's tile of row block b into buffer `buf`.
-  auto prefetch = [&](int b, int buf) {
-    const size_t base = static_cast<size_t>(b) * p.R * row_bytes + static_cast<size_t>(warp) * kTileBytes;
-    const size_t block_end = min(static_cast<size_t>(b + 1) * p.R * row_bytes, total_bytes);
-    const uint32_t s0 = smem_addr(buf ? wbuf1 : wbuf0);
-#pragma unroll
-    for (int i = 0; i < kTileBytes / 512; ++i) {
-      const int c = 32 * i + lane;
-      const size_t g = base + 16 * static_cast<size_t>(c);
-      const bool valid = g < block_end;
-      cp_async16(s0 + 16 * in_slot(c), valid ? xb + g : xb, valid);
-    }
-    cp_async_commit();
+  // Thread 0: the bulk copy of this block's row block number `it`.
+  auto issue = [&](int it) {
+    const int b = static_cast<int>(blockIdx.x) + it * static_cast<int>(gridDim.x);
+    const int rows = min(p.R, p.M - b * p.R);
+    const uint32_t bytes = static_cast<uint32_t>(rows) * static_cast<uint32_t>(p.K) * 2u;
+    uint64_t* bar = &full[it % S];
+    mbar_arrive_expect_tx(bar, bytes);
+    bulk_load(stages + (it % S) * stage_bytes, p.x + static_cast<size_t>(b) * p.R * p.K, bytes, bar);
   };
-
-  for (int i = threadIdx.x; i < 2 * 128; i += blockDim.x) (&row_amax[0][0])[i] = 0u;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) mbar_init(&full[s], 1);
+    fence_mbarrier_init();
+    for (int it = 0; it < S && it < iters; ++it) issue(it);
+  }
+  for (int i = threadIdx.x; i < 3 * kMaxRows; i += blockDim.x) (&row_amax[0][0])[i] = 0u;
   __syncthreads();
 
+  // The lane's two tasks: hw and hw + nhw.
+  const int task0 = hw, task1 = hw + nhw;
+  const int rloc0 = task0 < tasks ? task0 / p.G : 0, rloc1 = task1 < tasks ? task1 / p.G : 0;
+  const int g0 = task0 - rloc0 * p.G, g1 = task1 - rloc1 * p.G;
+
   int it = 0;
-  if (static_cast<int>(blockIdx.x) < p.nblocks) prefetch(blockIdx.x, 0);
-  for (int b = blockIdx.x; b < p.nblocks; b += gridDim.x, ++it) {
-    const int buf = it & 1;
-    uint8_t* const tile = buf ? wbuf1 : wbuf0;
-    uint32_t* const amax_slot = row_amax[it & 1];
-    const int nb = b + gridDim.x;
-    if (nb < p.nblocks) {
-      prefetch(nb, buf ^ 1);
-      cp_async_wait<1>();
-    } else {
-      cp_async_wait<0>();
-    }
-    __syncwarp();
+  for (; it < iters; ++it) {
+    const int row0 = (static_cast<int>(blockIdx.x) + it * static_cast<int>(gridDim.x)) * p.R;
+    const int slot = it % 3;
+    const bool ok = mbar_wait(&full[it % S], (it / S) & 1);
+    const uint8_t* stage = stages + (it % S) * stage_bytes;
+    const bool live0 = ok && task0 < tasks && row0 + rloc0 < p.M;
+    const bool live1 = ok && task1 < tasks && row0 + rloc1 < p.M;
 
-    // This lane's half-group.
-    const int f = 16 * warp + (lane >> 1);  // group index within the block
-    const int h = lane & 1;                 // which half of the group
-    const bool active = f < groups_per_block;
-    const int rloc = active ? f / p.G : 0;
-    const int row = b * p.R + rloc;
-    const bool live = active && row < p.M;
-
-    // ---- 128 bf16 -> 64 fp32 pairs: pair i = (channel i, channel i + 64)
-    u64 P[64];
-#pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      const uint4 lo = *reinterpret_cast<const uint4*>(tile + 16 * ((lane << 4) | (k ^ (lane & 7))));
-      const uint4 hi = *reinterpret_cast<const uint4*>(tile + 16 * ((lane << 4) | ((k + 8) ^ (lane & 7))));
-      const uint32_t w0[4] = {lo.x, lo.y, lo.z, lo.w};
-      const uint32_t w1[4] = {hi.x, hi.y, hi.z, hi.w};
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        P[8 * k + 2 * e] = f2(__uint_as_float(w0[e] << 16), __uint_as_float(w1[e] << 16));
-        P[8 * k + 2 * e + 1] = f2(__uint_as_float(w0[e] & 0xFFFF0000u), __uint_as_float(w1[e] & 0xFFFF0000u));
-      }
-    }
-    __syncwarp();  // the tile buffer becomes the output staging area below
-
-    // ---- rotation: stages on channel bits (0,1), (2,3), (4,5), packed
-#pragma unroll
-    for (int s = 0; s < 3; ++s) {
-      const int st = 1 << (2 * s);
-#pragma unroll
-      for (int i = 0; i < 64; ++i)
-        if (((i >> (2 * s)) & 3) == 0) bfly4(P[i], P[i + st], P[i + 2 * st], P[i + 3 * st]);
-    }
-    // stage on bits (6,7): bit 6 within the pair, bit 7 across the lane pair.
-    // Lane h=0 holds (a, b), lane h=1 holds (c, d); u = own sum, w = own
-    // difference; the partner's w completes (p+t, p-t) resp. (q+r, r-q).
-#pragma unroll
-    for (int i = 0; i < 64; ++i) {
-      float a, c;
-      f2_split(P[i], a, c);
-      const float u = __fadd_rn(a, c), w = __fsub_rn(a, c);
-      const float r = __shfl_xor_sync(0xffffffffu, w, 1);
-      P[i] = f2(__fadd_rn(u, r), __fsub_rn(u, r));
-    }
-    // x' = v * 1/16, and the lane's amax
-    const u64 sixteenth = f2(0.0625f, 0.0625f);
-    float m = 0.0f;
-#pragma unroll
-    for (int i = 0; i < 64; ++i) {
-      P[i] = f2_mul(P[i], sixteenth);
-      float a, c;
-      f2_split(P[i], a, c);
-      m = max3(m, fabsf(a), fabsf(c));
-    }
-    if (live) atomicMax(&amax_slot[rloc], __float_as_uint(m));
-    __syncthreads();
-    const float scale = __fdiv_rn(__uint_as_float(amax_slot[rloc]), 7.0f);
-    // The other slot is free now (its last readers finished before this
-    // barrier): clear it for the next block.
-    if (static_cast<int>(threadIdx.x) < 128) row_amax[(it + 1) & 1][threadIdx.x] = 0u;
-
-    // ---- quantize into the staging area (region `lane` of `tile`)
-    if (scale >= kMinScale) {
-      const float rcp = __frcp_rn(scale);
-      const u64 rr = f2(rcp, rcp), ns = f2(-scale, -scale), mg = f2(kMagic, kMagic);
-#pragma unroll
-      for (int k = 0; k < 8; k += 2) {
-        // pairs 8k .. 8k+15 hold chunks k, k+1 (.x) and k+8, k+9 (.y)
-        uint32_t cx[16], cy[16];
-#pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const u64 x = P[8 * k + e];
-          u64 q = f2_mul(x, rr);
-          q = f2_fma(f2_fma(ns, q, x), rr, q);  // faithful
-          q = f2_fma(f2_fma(ns, q, x), rr, q);  // RN(x / s)
-          float tx, ty;
-          f2_split(f2_add(q, mg), tx, ty);
-          cx[e] = __float_as_uint(tx);
-          cy[e] = __float_as_uint(ty);
-        }
-        stage_chunk_pair<PACKED>(tile, lane, k >> 1, cx);
-        stage_chunk_pair<PACKED>(tile, lane, (k + 8) >> 1, cy);
-      }
-    } else {
-      // Zero or tiny scale (a whole row takes this branch): IEEE division,
-      // in a rolled loop over a local copy to keep the code small.
-      float v[128];
-#pragma unroll
-      for (int i = 0; i < 64; ++i) f2_split(P[i], v[i], v[i + 64]);
-#pragma unroll 1
-      for (int k = 0; k < 16; ++k) {  // chunk k: channels 8k .. 8k+7 of the half
-        uint32_t q[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const int qq = scale != 0.0f ? __float2int_rn(__fdiv_rn(v[8 * k + e], scale)) : 0;
-          q[e] = static_cast<uint32_t>(min(7, max(-8, qq)));
-        }
-        if (PACKED) {
-          uint32_t w = 0;
-#pragma unroll
-          for (int e = 0; e < 8; ++e) w |= (q[e] & 0xFu) << (4 * e);
-          *reinterpret_cast<uint32_t*>(tile + 64 * lane + 4 * k) = w;
-        } else {
-          const uint2 o = make_uint2(gather_b0(q[0], q[2], q[4], q[6]), gather_b0(q[1], q[3], q[5], q[7]));
-          *reinterpret_cast<uint2*>(tile + 128 * lane + 16 * ((k >> 1) ^ (lane & 7)) + 8 * (k & 1)) = o;
-        }
-      }
-    }
-    if (live && h == 0 && f % p.G == 0) p.out.scale[row] = scale;
-    __syncwarp();
-
-    // ---- coalesced copy-out of the warp's codes (16 groups x 256 codes)
+    // ---- lane l: channels 16 l .. 16 l + 15 of both tasks, as pairs
+    u64 P[16];
     {
-      constexpr int kOutTile = kTileBytes / (PACKED ? 4 : 2);  // 2 KB packed, 4 KB as bytes
-      const size_t code_row = PACKED ? static_cast<size_t>(p.K) / 2 : static_cast<size_t>(p.K);
-      const size_t block_end = min(static_cast<size_t>(b + 1) * p.R * code_row, static_cast<size_t>(p.M) * code_row);
-      const size_t base = static_cast<size_t>(b) * p.R * code_row + static_cast<size_t>(warp) * kOutTile;
-      uint8_t* dst = PACKED ? p.out.packed : reinterpret_cast<uint8_t*>(p.out.s8);
+      uint4 a0 = make_uint4(0, 0, 0, 0), a1 = a0, b0 = a0, b1 = a0;
+      if (live0) {
+        const uint8_t* src = stage + (static_cast<size_t>(rloc0) * p.K + g0 * 256 + l * 16) * 2;
+        a0 = *reinterpret_cast<const uint4*>(src);
+        a1 = *reinterpret_cast<const uint4*>(src + 16);
+      }
+      if (live1) {
+        const uint8_t* src = stage + (static_cast<size_t>(rloc1) * p.K + g1 * 256 + l * 16) * 2;
+        b0 = *reinterpret_cast<const uint4*>(src);
+        b1 = *reinterpret_cast<const uint4*>(src + 16);
+      }
+      const uint32_t wa[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+      const uint32_t wb[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
 #pragma unroll
-      for (int i = 0; i < kOutTile / 512; ++i) {
-        const int c = 32 * i + lane;
-        uint4 v;
-        if (PACKED) {
-          v = *reinterpret_cast<const uint4*>(tile + 16 * c);
-        } else {
-          const int region = c >> 3, k = c & 7;
-          v = *reinterpret_cast<const uint4*>(tile + 128 * region + 16 * (k ^ (region & 7)));
-        }
-        const size_t g = base + 16 * static_cast<size_t>(c);
-        if (g < block_end) *reinterpret_cast<uint4*>(dst + g) = v;
+      for (int e = 0; e < 8; ++e) {
+        P[2 * e] = f2(__uint_as_float(wa[e] << 16), __uint_as_float(wb[e] << 16));
+        P[2 * e + 1] = f2(__uint_as_float(wa[e] & 0xFFFF0000u), __uint_as_float(wb[e] & 0xFFFF0000u));
       }
     }
+    // stage on channel bits (0,1): stride 1
+#pragma unroll
+    for (int i = 0; i < 16; i += 4) bfly4(P[i], P[i + 1], P[i + 2], P[i + 3]);
+    // stage on bits (2,3): stride 4
+#pragma unroll
+    for (int i = 0; i < 4; ++i) bfly4(P[i], P[i + 4], P[i + 8], P[i + 12]);
+    // transpose: row l of the tile <- channels 16 l + i; 16-byte chunk c (pairs
+    // 2c, 2c + 1) of row r sits at chunk c ^ (r & 7)
+#pragma unroll
+    for (int c = 0; c < 8; ++c)
+      *reinterpret_cast<ulonglong2*>(tile + 128 * l + 16 * (c ^ (l & 7))) = make_ulonglong2(P[2 * c], P[2 * c + 1]);
     __syncwarp();
+#pragma unroll
+    for (int i = 0; i < 16; ++i)
+      P[i] = *reinterpret_cast<const u64*>(tile + 128 * i + 16 * ((l >> 1) ^ (i & 7)) + 8 * (l & 1));
+    __syncwarp();
+    // now P[i] = channel 16 i + l.  stage on bits (4,5): stride 16
+#pragma unroll
+    for (int i = 0; i < 16; i += 4) bfly4(P[i], P[i + 1], P[i + 2], P[i + 3]);
+    // stage on bits (6,7): stride 64
+#pragma unroll
+    for (int i = 0; i < 4; ++i) bfly4(P[i], P[i + 4], P[i + 8], P[i + 12]);
+    // x' = v * 1/16, and the two tasks' amax
+    float m0 = 0.0f, m1 = 0.0f;
+    {
+      const u64 sixteenth = f2(0.0625f, 0.0625f);
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        P[i] = f2_mul(P[i], sixteenth);
+        float x0, x1;
+        f2_split(P[i], x0, x1);
+        m0 = fmaxf(m0, fabsf(x0));
+        m1 = fmaxf(m1, fabsf(x1));
+      }
+    }
+    // ---- per-row amax: within each task (16 lanes), then across the row's tasks
+#pragma unroll
+    for (int o = 8; o >= 1; o >>= 1) {
+      m0 = fmaxf(m0, __shfl_xor_sync(0xffffffffu, m0, o));
+      m1 = fmaxf(m1, __shfl_xor_sync(0xffffffffu, m1, o));
+    }
+    if (l == 0 && live0) atomicMax(&row_amax[slot][rloc0], __float_as_uint(m0));
+    if (l == 0 && live1) atomicMax(&row_amax[slot][rloc1], __float_as_uint(m1));
+    // Every read of this iteration's stage and every amax contribution is
+    // done after this barrier; a failed wait anywhere ends the loop for all.
+    if (!__syncthreads_and(ok)) break;
+    if (threadIdx.x == 0 && it + S < iters) {
+      fence_proxy_async_smem();
+      issue(it + S);
+    }
+    // Slot (it + 2) % 3 was last read in iteration it - 1 and is next written
+    // in iteration it + 2, after one more barrier.
+    if (threadIdx.x < kMaxRows) row_amax[(it + 2) % 3][threadIdx.x] = 0u;
+
+    // ---- quantize
+    const float scale0 = __fdiv_rn(__uint_as_float(row_amax[slot][rloc0]), 7.0f);
+    const float scale1 = __fdiv_rn(__uint_as_float(row_amax[slot][rloc1]), 7.0f);
+    uint32_t c0[16], c1[16];  // code bytes (low byte) of channel 16 i + l
+    if (scale0 >= kMinScale && scale1 >= kMinScale) {
+      const u64 rr = f2(__frcp_rn(scale0), __frcp_rn(scale1)), ns = f2(-scale0, -scale1);
+      const u64 mg = f2(kMagic, kMagic);
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const u64 x = P[i];
+        u64 q = f2_mul(x, rr);
+        q = f2_fma(f2_fma(ns, q, x), rr, q);  // faithful
+        q = f2_fma(f2_fma(ns, q, x), rr, q);  // RN(x / s)
+        float t0, t1;
+        f2_split(f2_add(q, mg), t0, t1);      // low byte = rint(q)
+        c0[i] = __float_as_uint(t0);
+        c1[i] = __float_as_uint(t1);
+      }
+    } else {
+      // A zero or tiny scale (a whole row takes this branch): IEEE division.
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        float x0, x1;
+        f2_split(P[i], x0, x1);
+        const int q0 = scale0 != 0.0f ? __float2int_rn(__fdiv_rn(x0, scale0)) : 0;
+        const int q1 = scale1 != 0.0f ? __float2int_rn(__fdiv_rn(x1, scale1)) : 0;
+        c0[i] = static_cast<uint32_t>(min(7, max(-8, q0)));
+        c1[i] = static_cast<uint32_t>(min(7, max(-8, q1)));
+      }
+    }
+    // ---- back to row order through the byte tiles, store
+    const int pos = code_pos<PACKED>(l);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      btile0[16 * i + pos] = static_cast<uint8_t>(c0[i]);
+      btile1[16 * i + pos] = static_cast<uint8_t>(c1[i]);
+    }
+    __syncwarp();
+    const uint4 o0 = *reinterpret_cast<const uint4*>(btile0 + 16 * l);  // channels 16 l .. 16 l + 15
+    const uint4 o1 = *reinterpret_cast<const uint4*>(btile1 + 16 * l);
+    __syncwarp();
+    if (live0) {
+      const int row = row0 + rloc0;
+      if (PACKED)
+        *reinterpret_cast<uint2*>(p.out.packed + static_cast<size_t>(row) * (p.K / 2) + g0 * 128 + l * 8) =
+            make_uint2(pack_nibbles(o0.x, o0.y), pack_nibbles(o0.z, o0.w));
+      else
+        *reinterpret_cast<uint4*>(p.out.s8 + static_cast<size_t>(row) * p.K + g0 * 256 + l * 16) = o0;
+      if (g0 == 0 && l == 0) p.out.scale[row] = scale0;
+    }
+    if (live1) {
+      const int row = row0 + rloc1;
+      if (PACKED)
+        *reinterpret_cast<uint2*>(p.out.packed + static_cast<size_t>(row) * (p.K / 2) + g1 * 128 + l * 8) =
+            make_uint2(pack_nibbles(o1.x, o1.y), pack_nibbles(o1.z, o1.w));
+      else
+        *reinterpret_cast<uint4*>(p.out.s8 + static_cast<size_t>(row) * p.K + g1 * 256 + l * 16) = o1;
+      if (g1 == 0 && l == 0) p.out.scale[row] = scale1;
+    }
+  }
+  if (it < iters && threadIdx.x == 0) {
+    // A wait gave up: let the copies still in flight land before the block
+    // exits (their stages are it .. min(it + S, iters) - 1).
+    for (int k = it; k < it + S && k < iters; ++k) (void)mbar_drain(&full[k % S], (k / S) & 1, 100000000ull);
   }
 }
 
@@ -378,6 +376,23 @@ int num_sms_cached() {
   return n[dev];
 }
 
+template <bool PACKED>
+cudaError_t launch_rq(const RQParams& p, int threads, cudaStream_t stream) {
+  static int cache[64] = {0};
+  const int smem = rq_smem_bytes(p.R, p.K, p.S, threads);
+  const void* kfn = reinterpret_cast<const void*>(rotate_quant_kernel<PACKED>);
+  cudaError_t e = ensure_dynamic_smem(kfn, smem, cache);
+  if (e != cudaSuccess) return note_cuda(e, "rotate_quant: dynamic shared memory attribute");
+  int per_sm = 0;
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, rotate_quant_kernel<PACKED>, threads, smem);
+  if (e != cudaSuccess) return note_cuda(e, "rotate_quant: occupancy query");
+  if (per_sm < 1) per_sm = 1;
+  int grid = num_sms_cached() * per_sm;
+  if (grid > p.nblocks) grid = p.nblocks;
+  rotate_quant_kernel<PACKED><<<grid, threads, smem, stream>>>(p);
+  return note_cuda(cudaGetLastError(), "rotate_quant: launch");
+}
+
 }  // namespace
 
 cudaError_t launch_rotate_quant(const uint16_t* x, int M, int K, RotateQuantOut out, cudaStream_t stream) {
@@ -386,66 +401,51 @@ cudaError_t launch_rotate_quant(const uint16_t* x, int M, int K, RotateQuantOut 
   p.M = M;
   p.K = K;
   p.G = K / 256;
-  // Rows per block R: a block holds R*G half-group pairs (at most 128 groups,
-  // 8 warps).  Pick the R with the fewest waves of blocks over the SMs and,
-  // among those, the fewest warps on the busiest SM.
+  p.out = out;
   const int sms = num_sms_cached();
-  const bool packed_out = out.packed != nullptr;
-  const void* kfn_sel = packed_out ? reinterpret_cast<const void*>(rotate_quant_kernel<true>)
-                                   : reinterpret_cast<const void*>(rotate_quant_kernel<false>);
-  static int regs_cache[2][64] = {{0}};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 0 || dev >= 64) dev = 0;
-  int& regs = regs_cache[packed_out ? 1 : 0][dev];
-  if (regs == 0) {
-    cudaFuncAttributes fa;
-    regs = (cudaFuncGetAttributes(&fa, kfn_sel) == cudaSuccess && fa.numRegs > 0) ? fa.numRegs : 255;
+  // One task (16 lanes) per group, two tasks per half-warp.  Rows per row
+  // block R: up to 32 tasks, and no more rows than leave about two row blocks
+  // per SM, so that small M spreads its rows over the SMs.
+  int R = 1;
+  if (p.G <= 32) {
+    const int by_tasks = 32 / p.G;
+    const int by_spread = (M + 2 * sms - 1) / (2 * sms);
+    R = by_tasks < by_spread ? by_tasks : by_spread;
+    if (R < 1) R = 1;
+    if (R > kMaxRows) R = kMaxRows;
   }
-  const int warp_regs = ((regs * 32 + 255) / 256) * 256;
-  int best_R = 1;
-  long best_key = -1;
-  for (int R = 1; R <= 128 / p.G; ++R) {
-    const int nb = (M + R - 1) / R;
-    const int w = (R * p.G + 15) / 16;
-    int per_sm = 65536 / (warp_regs * w);
-    per_sm = min(per_sm, (228 * 1024) / (w * 2 * kTileBytes + 2048));
-    per_sm = min(per_sm, 64 / w);
-    if (per_sm < 1) continue;
-    const long slots = static_cast<long>(sms) * per_sm;
-    const long waves = (nb + slots - 1) / slots;
-    const long busiest = static_cast<long>((nb + sms - 1) / sms) * w;  // warps on the busiest SM per wave
-    const long key = waves * 100000 + (waves > 1 ? 0 : busiest);
-    if (best_key < 0 || key < best_key || (key == best_key && R > best_R)) {
-      best_key = key;
-      best_R = R;
-    }
-    if (R > M) break;
-  }
-  const int R = best_R;
   p.R = R;
   p.nblocks = (M + R - 1) / R;
-  p.out = out;
-  const int warps = (R * p.G + 15) / 16;
-  const int smem = warps * 2 * kTileBytes;
-  const bool packed = out.packed != nullptr;
-  const void* kfn = packed ? reinterpret_cast<const void*>(rotate_quant_kernel<true>)
-                           : reinterpret_cast<const void*>(rotate_quant_kernel<false>);
-  static int cache_packed[64] = {0}, cache_s8[64] = {0};
-  cudaError_t e = ensure_dynamic_smem(kfn, smem, packed ? cache_packed : cache_s8);
-  if (e != cudaSuccess) return note_cuda(e, "rotate_quant: dynamic shared memory attribute");
-  int per_sm = 0;
-  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kfn, warps * 32, smem);
-  if (e != cudaSuccess) return note_cuda(e, "rotate_quant: occupancy query");
+  const int hws = (R * p.G + 1) / 2;
+  const int threads = ((hws * 16 + 31) / 32) * 32;
+  if (threads > kMaxThreads) return note_cuda(cudaErrorInvalidValue, "rotate_quant: block shape");
+  // Blocks per SM by threads and registers (up to 64 per thread); then the
+  // input ring: about 128 KB of row blocks in flight per SM, at least 2
+  // stages where they fit next to the transpose tiles (fewer blocks per SM
+  // otherwise), never more stages than a block has row blocks.
+  int per_sm = 65536 / (threads * 64);
+  if (per_sm > 2048 / threads) per_sm = 2048 / threads;
+  if (per_sm > 8) per_sm = 8;
   if (per_sm < 1) per_sm = 1;
-  int grid = sms * per_sm;
-  if (grid > p.nblocks) grid = p.nblocks;
-  if (packed)
-    rotate_quant_kernel<true><<<grid, warps * 32, smem, stream>>>(p);
-  else
-    rotate_quant_kernel<false><<<grid, warps * 32, smem, stream>>>(p);
+  const int stage = rq_stage_bytes(R, K);
+  const int fixed = rq_smem_bytes(R, K, 0, threads) + 64;
+  int s_fit = 0;
+  for (;;) {
+    s_fit = (220 * 1024 / per_sm - fixed) / stage;
+    if (s_fit >= 2 || per_sm == 1) break;
+    --per_sm;
+  }
+  int S = (128 * 1024 + per_sm * stage - 1) / (per_sm * stage);
+  if (S < 2) S = 2;
+  if (S > 8) S = 8;
+  if (S > s_fit) S = s_fit;
+  const int most_iters = (p.nblocks + sms * per_sm - 1) / (sms * per_sm);
+  if (S > most_iters) S = most_iters;
+  if (S < 1) S = 1;
+  p.S = S;
+  cudaError_t e = out.packed != nullptr ? launch_rq<true>(p, threads, stream) : launch_rq<false>(p, threads, stream);
   count_dispatch(0);
-  return note_cuda(cudaGetLastError(), "rotate_quant: launch");
+  return e;
 }
 
 cudaError_t launch_unpack_codes(const uint8_t* packed, int M, int K, int8_t* s8, cudaStream_t stream) {
