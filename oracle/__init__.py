@@ -50,6 +50,9 @@ def _load():
         lib.oracle_linear_rows.argtypes = [P, P, P, P, I, I, I, I, I, P, P]
         lib.oracle_pack_codes.argtypes = [P, ctypes.c_int64, P]
         lib.oracle_unpack_codes.argtypes = [P, ctypes.c_int64, P]
+        lib.oracle_quant8.argtypes = [P, I, I, I, I, P, P]
+        lib.oracle_gemm8_s64_rows.argtypes = [P, P, I, I, I, I, I, P]
+        lib.oracle_linear8_rows.argtypes = [P, P, P, P, I, I, I, I, I, I, I, P, P]
         lib.oracle_f32_to_bf16.argtypes = [ctypes.c_float]
         lib.oracle_f32_to_bf16.restype = ctypes.c_uint16
         lib.oracle_bf16_to_f32.argtypes = [ctypes.c_uint16]
@@ -149,6 +152,51 @@ def linear(x_bits, wq, s_w, bias_bits, K: int, rows=None):
     y16 = np.empty((m1 - m0, N), np.uint16)
     _check(_load().oracle_linear_rows(_ptr(x), _ptr(wq), _ptr(s_w), _ptr(b), M, N, K, m0, m1, _ptr(y32), _ptr(y16)),
            "linear")
+    return y32, y16
+
+
+# ---- int8 formats: int8_tensorwise (group 0, one scale per tensor) and
+# ConvRot INT8 row-scaled (group 256, one scale per row)
+
+TENSORWISE = (0, False)
+CONVROT_ROW = (256, True)
+
+
+def quant8(x_bits, group: int = 0, per_row: bool = False):
+    """bf16 bits [M, K] -> (int8 codes [M, K], scales fp32: [M] per row, [1] per tensor)."""
+    x = _c(x_bits, np.uint16)
+    M, K = x.shape
+    codes = np.empty((M, K), np.int8)
+    s = np.empty((M if per_row else 1,), np.float32)
+    _check(_load().oracle_quant8(_ptr(x), M, K, group, 1 if per_row else 0, _ptr(codes), _ptr(s)), "quant8")
+    return codes, s
+
+
+def gemm8_s64(x8, w8, rows=None):
+    """int64 acc[m, n] = sum_k x8[m,k] w8[n,k]; ``rows=(m0, m1)`` limits the rows."""
+    x8 = _c(x8, np.int8)
+    w8 = _c(w8, np.int8)
+    M, K = x8.shape
+    N = w8.shape[0]
+    m0, m1 = rows if rows is not None else (0, M)
+    acc = np.empty((m1 - m0, N), np.int64)
+    _check(_load().oracle_gemm8_s64_rows(_ptr(x8), _ptr(w8), M, N, K, m0, m1, _ptr(acc)), "gemm8_s64")
+    return acc
+
+
+def linear8(x_bits, w8, s_w, bias_bits, group: int = 0, per_row: bool = False, rows=None):
+    """The int8 Linear: returns (y32 fp32, y bf16 bits) for rows ``rows=(m0, m1)``."""
+    x = _c(x_bits, np.uint16)
+    w8 = _c(w8, np.int8)
+    s_w = _c(s_w, np.float32)
+    b = None if bias_bits is None else _c(bias_bits, np.uint16)
+    M, K = x.shape
+    N = w8.shape[0]
+    m0, m1 = rows if rows is not None else (0, M)
+    y32 = np.empty((m1 - m0, N), np.float32)
+    y16 = np.empty((m1 - m0, N), np.uint16)
+    _check(_load().oracle_linear8_rows(_ptr(x), _ptr(w8), _ptr(s_w), _ptr(b), M, N, K, group, 1 if per_row else 0,
+                                       m0, m1, _ptr(y32), _ptr(y16)), "linear8")
     return y32, y16
 
 

@@ -39,6 +39,21 @@
  *  - GEMM: acc[m,n] = sum_k q_a[m,k] * q_w[n,k] in int64.
  *  - Epilogue: y32 = ((float)acc * s_a[m]) * s_w[n] + (float)bias[n], each op
  *    one fp32 RN op; y = bf16 round-to-nearest-even of y32.
+ *
+ * The int8 formats the pages use next to W4A4 (a W8A8 path: int8 weights,
+ * int8 activations, int32 accumulation, the same rank-one rescale):
+ *  - "Qwen-Image-Edit-2511 -- INT4 tensorwise W4A4 (+ConvRot, mixed int8
+ *    fallback)", intro: the sensitive layers (attention value/output
+ *    projections) are stock "int8_tensorwise" -- read as one scale for the
+ *    whole weight tensor and one dynamic scale for the whole activation
+ *    tensor, no rotation.
+ *  - "rockerBOO/qwen3-4b-nvfp4-convrot", file table and notes: "ConvRot INT8
+ *    (row-scaled)" -- the group-256 rotation, then int8 with one scale per
+ *    weight row; read here with one dynamic scale per activation row (token).
+ *  Readings for both: s = amax / 127 (IEEE fp32 divide), q = clamp(rint(v /
+ *  s), -127, 127) with a true division and round half to even, s = 0 gives
+ *  q = 0; the epilogue is the same rank-one rescale (a per-tensor scale is a
+ *  constant vector).
  */
 #include <math.h>
 #include <stdint.h>
@@ -272,4 +287,103 @@ int oracle_linear_rows(const uint16_t *x, const uint8_t *Wq, const float *s_w, c
 int oracle_linear(const uint16_t *x, const uint8_t *Wq, const float *s_w, const uint16_t *bias,
                   int M, int N, int K, float *y32, uint16_t *y16) {
   return oracle_linear_rows(x, Wq, s_w, bias, M, N, K, 0, M, y32, y16);
+}
+
+/* ---- int8 formats (int8_tensorwise; ConvRot INT8 row-scaled) -------------- */
+
+/* bf16 x[M, K] -> int8 codes [M, K] and scales.  group = 0: no rotation,
+ * group = 256 (or 64, 16): the ConvRot rotation of each group first.
+ * per_row = 0: one scale for the whole tensor (scale[0]); per_row = 1: one
+ * scale per row (scale[M]).  s = amax / 127, q = clamp(rint(v / s), -127, 127). */
+int oracle_quant8(const uint16_t *x, int M, int K, int group, int per_row, int8_t *codes, float *scale) {
+  int S = group == 0 ? 0 : group_log4(group);
+  if (S < 0 || M < 0 || K <= 0 || (group != 0 && K % group != 0)) return ORACLE_ERR_SHAPE;
+  float *v = (float *)malloc(sizeof(float) * (size_t)(M > 0 ? M : 1) * (size_t)K);
+  if (!v) return ORACLE_ERR_NOMEM;
+  for (size_t i = 0; i < (size_t)M * (size_t)K; ++i) v[i] = bf16_bits_to_f32(x[i]); /* widen */
+  if (group != 0)
+    for (int m = 0; m < M; ++m)
+      for (int g = 0; g < K / group; ++g) rotate_group(v + (size_t)m * K + (size_t)g * group, S);
+  float tensor_amax = 0.0f;
+  if (!per_row)
+    for (size_t i = 0; i < (size_t)M * (size_t)K; ++i) {
+      float a = fabsf(v[i]);
+      if (a > tensor_amax) tensor_amax = a;
+    }
+  for (int m = 0; m < M; ++m) {
+    const float *row = v + (size_t)m * K;
+    float amax = tensor_amax;
+    if (per_row) {
+      amax = 0.0f;
+      for (int k = 0; k < K; ++k) {
+        float a = fabsf(row[k]);
+        if (a > amax) amax = a;
+      }
+    }
+    float s = amax / 127.0f;
+    for (int k = 0; k < K; ++k) {
+      int c = 0;
+      if (s != 0.0f) {
+        float qv = rintf(row[k] / s);
+        if (qv < -127.0f) qv = -127.0f;
+        if (qv > 127.0f) qv = 127.0f;
+        c = (int)qv;
+      }
+      codes[(size_t)m * K + k] = (int8_t)c;
+    }
+    if (per_row) scale[m] = s;
+    else if (m == 0) scale[0] = s;
+  }
+  if (!per_row && M == 0) scale[0] = 0.0f;
+  free(v);
+  return ORACLE_OK;
+}
+
+/* acc[m, n] = sum_k x8[m, k] * w8[n, k] in int64, rows [m0, m1). */
+int oracle_gemm8_s64_rows(const int8_t *x8, const int8_t *w8, int M, int N, int K, int m0, int m1,
+                          int64_t *acc) {
+  if (M < 0 || N < 0 || K <= 0 || m0 < 0 || m1 > M || m0 > m1) return ORACLE_ERR_SHAPE;
+  for (int m = m0; m < m1; ++m)
+    for (int n = 0; n < N; ++n) {
+      const int8_t *a = x8 + (size_t)m * K, *w = w8 + (size_t)n * K;
+      int64_t s = 0;
+      for (int k = 0; k < K; ++k) s += (int64_t)a[k] * (int64_t)w[k];
+      acc[(size_t)(m - m0) * N + n] = s;
+    }
+  return ORACLE_OK;
+}
+
+/* The int8 Linear: x quantized with (group, per_row) as above, times the int8
+ * weights w8[N, K] with their scales s_w (N of them when per_row, else one),
+ * then the rank-one epilogue; rows [m0, m1) of y.  With one scale per tensor
+ * the activation scale depends on every row of x, so all M rows are
+ * quantized. */
+int oracle_linear8_rows(const uint16_t *x, const int8_t *w8, const float *s_w, const uint16_t *bias, int M,
+                        int N, int K, int group, int per_row, int m0, int m1, float *y32, uint16_t *y16) {
+  if (M < 0 || N <= 0 || K <= 0 || m0 < 0 || m1 > M || m0 > m1) return ORACLE_ERR_SHAPE;
+  int rows = m1 - m0;
+  int qrows = per_row ? rows : M;
+  const uint16_t *xq_src = per_row ? x + (size_t)m0 * K : x;
+  int8_t *x8 = (int8_t *)malloc((size_t)(qrows > 0 ? qrows : 1) * (size_t)K);
+  float *sx = (float *)malloc(sizeof(float) * (size_t)(qrows > 0 ? qrows : 1));
+  float *sa = (float *)malloc(sizeof(float) * (size_t)(rows > 0 ? rows : 1));
+  float *sw = (float *)malloc(sizeof(float) * (size_t)N);
+  int64_t *acc = (int64_t *)malloc(sizeof(int64_t) * (size_t)(rows > 0 ? rows : 1) * (size_t)N);
+  int rc = ORACLE_ERR_NOMEM;
+  if (x8 && sx && sa && sw && acc) {
+    rc = oracle_quant8(xq_src, qrows, K, group, per_row, x8, sx);
+    if (rc == ORACLE_OK) {
+      for (int r = 0; r < rows; ++r) sa[r] = per_row ? sx[r] : sx[0];
+      for (int n = 0; n < N; ++n) sw[n] = per_row ? s_w[n] : s_w[0];
+      int off = per_row ? 0 : m0;
+      rc = oracle_gemm8_s64_rows(x8, w8, qrows, N, K, off, off + rows, acc);
+    }
+    if (rc == ORACLE_OK) rc = oracle_epilogue(acc, sa, sw, bias, rows, N, y32, y16);
+  }
+  free(x8);
+  free(sx);
+  free(sa);
+  free(sw);
+  free(acc);
+  return rc;
 }
