@@ -210,8 +210,8 @@ def main():
               "l2": ("flushed between timed steps, outside the events: 256 MiB write, then 256 MiB read of a second "
                      "buffer (inputs cold, no dirty lines left in L2)") if args.flush == "write+read"
                     else "flushed between timed steps, outside the events: 256 MiB write",
-              "launch": "each step replayed from a CUDA graph (2 kernels per linear)" if not args.no_graph
-                        else "eager launches",
+              "launch": ("each step replayed from a CUDA graph" if not args.no_graph else "eager launches")
+                        + ": per input tensor one rotate+quantize launch, then one GEMM launch per linear reading it",
               "parallelism": f"replicas x{max(world, args.gpus)}" if max(world, args.gpus) > 1 else "single GPU",
               "codes": "s4 packed weights, s4 activations widened to s8 for tcgen05 kind::i8, int32 accumulate, "
                        "fp32 epilogue, bf16 out"}
@@ -237,21 +237,31 @@ def main():
     # roofline; the roofline's peak itself is the measured bf16 rate x 2.
     mma_i8_tops, _ = rq.convrot_measure_mma_i8(256, False, 4096)
 
-    # ---- inputs (untimed): activations per (M, K), packed weights per linear
+    # ---- inputs (untimed): one activation tensor per source (linears of a
+    # layer that read the same tensor share it), packed weights per linear
     xs = {}
     for s in shapes:
-        if (s.M, s.K) not in xs:
-            xb = synthetic.activations(args.workload, s.M, s.K)
-            xs[(s.M, s.K)] = torch.from_numpy(xb.view(np.int16)).view(torch.bfloat16).to(dev)
+        if s.source not in xs:
+            xb = synthetic.activations(args.workload, s.M, s.K, seed_extra=synthetic.source_seed(s.source))
+            xs[s.source] = torch.from_numpy(xb.view(np.int16)).view(torch.bfloat16).to(dev)
     layers = []
     for s in shapes:
-        w, b = synthetic.weights(args.workload, s.N, s.K)
+        w, b = synthetic.weights(args.workload, s.N, s.K, seed_extra=synthetic.source_seed(s.name))
         wd = torch.from_numpy(w.view(np.int16)).view(torch.bfloat16).to(dev)
         wq, s_w = rq.convrot_pack_weight(wd)
         bias = torch.from_numpy(b.view(np.int16)).view(torch.bfloat16).to(dev)
         y = torch.empty((s.M, s.N), dtype=torch.bfloat16, device=dev)
         layers.append((s, wq, s_w, bias, y))
         del wd
+    # groups of linears that read one source, in order of first use
+    groups = []
+    for i, (s, *_r) in enumerate(layers):
+        for g in groups:
+            if g[0] == s.source:
+                g[1].append(i)
+                break
+        else:
+            groups.append((s.source, [i]))
     ws_bytes = max(rq.convrot_w4a4_workspace_size(s.M, s.N, s.K) for s in shapes)
     ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
     flush = make_flusher(torch, dev, args.flush)
@@ -259,21 +269,27 @@ def main():
     torch.cuda.synchronize()
 
     nlin = len(layers)
+    ngrp = len(groups)
 
     def run_step(evs=None, per_kernel=False):
-        """One step.  With per_kernel, an event sits between the two launches of
-        each linear (which serialises them); otherwise events only bracket each
-        linear, so the GEMM's programmatic launch overlaps the prologue."""
+        """One step: per source, one rotate + quantize, then the GEMM of every
+        linear that reads it.  evs[g] = [start, after quantize, after each
+        GEMM]; in the timed step only the group's start and end are recorded
+        (so the GEMMs' programmatic launches overlap what precedes them), in
+        the per-kernel breakdown every boundary is."""
         cur = torch.cuda.current_stream()  # the capture stream while a graph is being captured
-        for i, (s, wq, s_w, bias, y) in enumerate(layers):
-            if evs is not None:
-                evs[i][0].record(cur)
-            rq.convrot_w4a4_quantize(xs[(s.M, s.K)], ws)
-            if evs is not None and per_kernel:
-                evs[i][1].record(cur)
-            rq.convrot_w4a4_gemm_quantized(ws, s.M, wq, s_w, bias, out=y)
-            if evs is not None:
-                evs[i][2].record(cur)
+        for gi, (src, idx) in enumerate(groups):
+            ev = evs[gi] if evs is not None else None
+            if ev is not None:
+                ev[0].record(cur)
+            rq.convrot_w4a4_quantize(xs[src], ws)
+            if ev is not None and per_kernel:
+                ev[1].record(cur)
+            for j, i in enumerate(idx):
+                s, wq, s_w, bias, y = layers[i]
+                rq.convrot_w4a4_gemm_quantized(ws, s.M, wq, s_w, bias, out=y)
+                if ev is not None and (per_kernel or j == len(idx) - 1):
+                    ev[2 + j].record(cur)
 
     for _ in range(max(args.warmup, 3)):
         flush()
@@ -285,8 +301,8 @@ def main():
     # recorded inside a capture they become event-record nodes timestamped on
     # every replay.
     def make_events():
-        return [[[torch.cuda.Event(enable_timing=True, external=True) for _ in range(3)] for _ in range(nlin)]
-                for _ in range(args.steps)]
+        return [[[torch.cuda.Event(enable_timing=True, external=True) for _ in range(2 + len(idx))]
+                 for (_src, idx) in groups] for _ in range(args.steps)]
 
     step_events, kern_events = make_events(), make_events()
     graphs, kgraphs = [], []
@@ -325,7 +341,7 @@ def main():
     clocks = sampler.stop() if sampler else None
     counts1 = rq.convrot_dispatch_counts()
     # Per-kernel breakdown (for the roofline of the dominant kernel): the same
-    # step with the two launches of each linear separated by an event.
+    # step with an event between every two launches.
     for k in range(args.steps):
         flush()
         if kgraphs:
@@ -337,23 +353,25 @@ def main():
     if err:
         raise RuntimeError(f"device error word {err:#x}: a bounded wait expired")
     if graphs:  # launches of a replayed graph are not seen by the host counters
-        launches = 2 * nlin * args.steps
+        launches = (ngrp + nlin) * args.steps
     else:
         launches = (counts1["rotate_quant"] - counts0["rotate_quant"]) + (counts1["tc_gemm"] - counts0["tc_gemm"]) + \
                    (counts1["tc_gemm_splitk"] - counts0["tc_gemm_splitk"])
 
-    # per-linear times of the timed steps, and per-kernel times of the breakdown
-    # steps (ms), summed over the K steps
-    t_lin = np.zeros(nlin)
-    t_quant = np.zeros(nlin)
+    # per-group times of the timed steps, and per-kernel times of the
+    # breakdown steps (ms), summed over the K steps
+    t_grp = np.zeros(ngrp)
+    t_quant = np.zeros(ngrp)
     t_gemm = np.zeros(nlin)
     for k in range(args.steps):
-        for i in range(nlin):
-            t_lin[i] += step_events[k][i][0].elapsed_time(step_events[k][i][2])
-            e0, e1, e2 = kern_events[k][i]
-            t_quant[i] += e0.elapsed_time(e1)
-            t_gemm[i] += e1.elapsed_time(e2)
-    total_ms = float(t_lin.sum())
+        for gi, (_src, idx) in enumerate(groups):
+            ev = step_events[k][gi]
+            t_grp[gi] += ev[0].elapsed_time(ev[1 + len(idx)])
+            kv = kern_events[k][gi]
+            t_quant[gi] += kv[0].elapsed_time(kv[1])
+            for j, i in enumerate(idx):
+                t_gemm[i] += kv[1 + j].elapsed_time(kv[2 + j])
+    total_ms = float(t_grp.sum())
     if world > 1:
         t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
@@ -366,29 +384,30 @@ def main():
     peaks = load_peaks()
     int8_peak = peaks["bf16_tflops"] * INT8_PER_BF16
     detail = []
-    for i, (s, *_rest) in enumerate(layers):
-        tq, tg = t_quant[i] / args.steps, t_gemm[i] / args.steps
-        op = 2.0 * s.M * s.N * s.K
-        gemm_bytes = s.N * s.K // 2 + s.M * s.K + 4 * s.M + 6 * s.N + 2 * s.M * s.N
-        tl = t_lin[i] / args.steps
-        detail.append({
-            "linear": s.name, "M": s.M, "K": s.K, "N": s.N,
-            "us_linear": round(tl * 1e3, 2), "us_prologue": round(tq * 1e3, 2), "us_gemm": round(tg * 1e3, 2),
-            "tops_fused": round(op / (tl * 1e-3) / 1e12, 1),
-            "gemm_tops": round(op / (tg * 1e-3) / 1e12, 1),
-            "gemm_frac_int8_peak": round(op / (tg * 1e-3) / 1e12 / int8_peak, 3),
-            "gemm_hbm_gbs": round(gemm_bytes / (tg * 1e-3) / 1e9, 1),
-            "prologue_hbm_gbs": round((2.5 * s.M * s.K + 4 * s.M) / (tq * 1e-3) / 1e9, 1),
-        })
-    # dominant kernel = the single launch class with the largest share of the step
-    cand = []
-    for i, (s, *_r) in enumerate(layers):
-        cand.append(("gemm", i, t_gemm[i]))
-        cand.append(("prologue", i, t_quant[i]))
+    for gi, (src, idx) in enumerate(groups):
+        s0 = layers[idx[0]][0]
+        tq, tgrp = t_quant[gi] / args.steps, t_grp[gi] / args.steps
+        gops = sum(2.0 * layers[i][0].M * layers[i][0].N * layers[i][0].K for i in idx)
+        entry = {"input": src, "M": s0.M, "K": s0.K, "us_group": round(tgrp * 1e3, 2),
+                 "tops_group": round(gops / (tgrp * 1e-3) / 1e12, 1), "us_prologue": round(tq * 1e3, 2),
+                 "prologue_hbm_gbs": round((3.0 * s0.M * s0.K + 4 * s0.M) / (tq * 1e-3) / 1e9, 1), "linears": []}
+        for i in idx:
+            s = layers[i][0]
+            tg = t_gemm[i] / args.steps
+            op = 2.0 * s.M * s.N * s.K
+            gemm_bytes = s.N * s.K // 2 + s.M * s.K + 4 * s.M + 6 * s.N + 2 * s.M * s.N
+            entry["linears"].append({
+                "linear": s.name, "N": s.N, "us_gemm": round(tg * 1e3, 2),
+                "gemm_tops": round(op / (tg * 1e-3) / 1e12, 1),
+                "gemm_frac_int8_peak": round(op / (tg * 1e-3) / 1e12 / int8_peak, 3),
+                "gemm_hbm_gbs": round(gemm_bytes / (tg * 1e-3) / 1e9, 1)})
+        detail.append(entry)
+    # dominant kernel = the single launch with the largest share of the step
+    cand = [("gemm", i, t_gemm[i]) for i in range(nlin)] + [("prologue", gi, t_quant[gi]) for gi in range(ngrp)]
     kind, idx, tsum = max(cand, key=lambda c: c[2])
-    s = layers[idx][0]
     t_launch = tsum / args.steps * 1e-3  # seconds per launch
     if kind == "gemm":
+        s = layers[idx][0]
         ridge = int8_peak * 1e12 / (peaks["hbm_gbs"] * 1e9)
         gemm_bytes = s.N * s.K // 2 + s.M * s.K + 4 * s.M + 6 * s.N + 2 * s.M * s.N
         intensity = 2.0 * s.M * s.N * s.K / gemm_bytes
@@ -398,13 +417,15 @@ def main():
         else:
             roof = {"bound": "hbm", "achieved": gemm_bytes / t_launch / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s"}
         kname = "w4a4_tc_gemm_kernel"
+        roof["launch"] = f"{s.name} M{s.M} K{s.K} N{s.N}"
     else:
-        roof = {"bound": "hbm", "achieved": (2.5 * s.M * s.K + 4 * s.M) / t_launch / 1e9,
+        s = layers[groups[idx][1][0]][0]
+        roof = {"bound": "hbm", "achieved": (3.0 * s.M * s.K + 4 * s.M) / t_launch / 1e9,
                 "peak": peaks["hbm_gbs"], "unit": "GB/s"}
         kname = "rotate_quant_kernel"
+        roof["launch"] = f"prologue of {groups[idx][0]} M{s.M} K{s.K}"
     roof["frac"] = roof["achieved"] / roof["peak"]
     roof["kernel"] = kname
-    roof["launch"] = f"{s.name} M{s.M} K{s.K} N{s.N}"
     roof["peak_source"] = (f"{peaks['source']} bf16 dense burst {peaks['bf16_tflops']} TFLOP/s x {INT8_PER_BF16} "
                            "(nominal int8:bf16)" if roof["bound"] == "tensor" else f"{peaks['source']} HBM copy")
     roof["share_of_breakdown"] = float(tsum / (t_quant.sum() + t_gemm.sum()))
@@ -415,7 +436,7 @@ def main():
 
     e2e = None
     if not args.no_e2e:
-        e2e = end_to_end(args, rq, torch, dev, stream, shapes, xs, layers, ws, flush, world, dist)
+        e2e = end_to_end(args, rq, torch, dev, stream, shapes, xs, layers, groups, ws, flush, world, dist)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -461,9 +482,11 @@ def source_sha(kernel):
         return hashlib.sha256(f.read()).hexdigest()
 
 
-def end_to_end(args, rq, torch, dev, stream, shapes, xs, layers, ws, flush, world, dist):
-    """Same step through the public fused call, with the step's inputs copied
-    from pinned host memory and every output read back, inside the timing."""
+def end_to_end(args, rq, torch, dev, stream, shapes, xs, layers, groups, ws, flush, world, dist):
+    """Same step through the public C-ABI calls (convrot_w4a4_quantize once per
+    source, convrot_w4a4_gemm_quantized per linear; convrot_w4a4_linear when a
+    source feeds one linear), with the step's inputs copied from pinned host
+    memory and every output read back, inside the timing."""
     host_x = {k: v.cpu().pin_memory() for k, v in xs.items()}
     host_y = [torch.empty(y.shape, dtype=y.dtype).pin_memory() for (_, _, _, _, y) in layers]
     h2d = sum(v.numel() * 2 for v in host_x.values())
@@ -472,8 +495,15 @@ def end_to_end(args, rq, torch, dev, stream, shapes, xs, layers, ws, flush, worl
     def step():
         for k, v in host_x.items():
             xs[k].copy_(v, non_blocking=True)
-        for (s, wq, s_w, bias, y) in layers:
-            rq.convrot_w4a4_linear(xs[(s.M, s.K)], wq, s_w, bias, out=y, workspace=ws)
+        for src, idx in groups:
+            if len(idx) == 1:
+                s, wq, s_w, bias, y = layers[idx[0]]
+                rq.convrot_w4a4_linear(xs[src], wq, s_w, bias, out=y, workspace=ws)
+                continue
+            rq.convrot_w4a4_quantize(xs[src], ws)
+            for i in idx:
+                s, wq, s_w, bias, y = layers[i]
+                rq.convrot_w4a4_gemm_quantized(ws, s.M, wq, s_w, bias, out=y)
         for (s, wq, s_w, bias, y), hy in zip(layers, host_y):
             hy.copy_(y, non_blocking=True)
 
@@ -500,7 +530,8 @@ def end_to_end(args, rq, torch, dev, stream, shapes, xs, layers, ws, flush, worl
     return {"value": round(n_rep * step_ops(shapes) * args.steps / (total * 1e-3) / 1e12, 2), "unit": UNIT,
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
             "ms_per_step": round(total / args.steps, 4),
-            "api": "convrot_w4a4_linear (C ABI) per linear, pinned host->device x, device->host y"}
+            "api": "C ABI: convrot_w4a4_quantize per source + convrot_w4a4_gemm_quantized per linear "
+                   "(convrot_w4a4_linear for single-linear sources); pinned host->device x, device->host y"}
 
 
 def reference_arm(args, shapes, config, world, rank):

@@ -25,9 +25,9 @@
 // A transpose of the pairs through the half-warp's shared-memory tile then
 // swaps the roles (lane l holds channels l, 16 + l, ..., 240 + l) and the
 // stages on bits (4,5) and (6,7) run in registers as well.  The tile's rows
-// are 16 pairs (128 bytes) with the 16-byte chunks XOR-swizzled by the row,
-// so the eight 16-byte stores of a lane and its sixteen 8-byte loads are free
-// of bank conflicts.  A block owns blocks of R whole rows (R * G tasks, G = K
+// are 16 pairs (128 bytes) padded to 144 bytes, so the eight 16-byte stores
+// of a lane (a row) and its sixteen 8-byte loads (a column) are free of bank
+// conflicts and every address is a per-lane base plus a constant.  A block owns blocks of R whole rows (R * G tasks, G = K
 // / 256) in turn, so the per-row amax is a shuffle reduction within each
 // task plus one shared-memory atomic max per task.  Each lane then quantizes
 // its channels; the code bytes go back to row order through the same tile
@@ -67,7 +67,8 @@ namespace {
 
 constexpr float kMagic = 12582912.0f;           // 1.5 * 2^23: x + kMagic rounds x to an integer, ties to even
 constexpr float kMinScale = 7.88860905e-31f;    // 2^-100: below it, codes by division
-constexpr int kTileBytes = 2048;                // per-half-warp transpose tile: 16 x 16 fp32 pairs
+constexpr int kTileRow = 144;                   // bytes per transpose-tile row: 16 fp32 pairs + 16 of padding
+constexpr int kTileBytes = 16 * kTileRow;       // per-half-warp transpose tile
 constexpr int kMaxRows = 64;                    // rows per row block (K = 256 -> 64 tasks)
 constexpr int kMaxThreads = 1024;
 
@@ -104,6 +105,12 @@ __device__ __forceinline__ u64 f2_fma(u64 a, u64 b, u64 c) {
   return d;
 }
 
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
 // One radix-4 butterfly on pairs: (a,b,c,d) -> (p+t, p-t, q+r, r-q).
 __device__ __forceinline__ void bfly4(u64& a, u64& b, u64& c, u64& d) {
   const u64 p = f2_add(a, b), q = f2_sub(a, b), r = f2_add(c, d), t = f2_sub(c, d);
@@ -130,12 +137,19 @@ struct RQParams {
   RotateQuantOut out;
 };
 
+// Output formats of the prologue:
+//   kPacked4  4-bit codes, two per byte (convrot_rotate_quant, weight packing)
+//   kOperand4 4-bit codes as signed bytes in the W4A4 GEMM's operand order
+//   kInt8     8-bit codes (amax / 127, clamp [-127, 127]) in natural order:
+//             the ConvRot INT8 row-scaled format
+enum : int { kPacked4 = 0, kOperand4 = 1, kInt8 = 2 };
+
 // Byte position of channel c's code within its 16-byte run of the output
-// row: natural order for packed output; for the s8 operand layout each
-// 8-channel chunk is stored in the order (0, 2, 4, 6, 1, 3, 5, 7).
-template <bool PACKED>
+// row: natural order, except the W4A4 operand layout, which stores each
+// 8-channel chunk in the order (0, 2, 4, 6, 1, 3, 5, 7).
+template <int MODE>
 __device__ __forceinline__ int code_pos(int c) {
-  if (PACKED) return c & 15;
+  if (MODE != kOperand4) return c & 15;
   const int e = c & 7;
   return (c & 8) | ((e & 1) ? 4 + (e >> 1) : (e >> 1));
 }
@@ -147,36 +161,47 @@ __host__ __device__ constexpr int rq_smem_bytes(int R, int K, int S, int threads
   return S * rq_stage_bytes(R, K) + (threads / 16) * kTileBytes + 8 * S;
 }
 
-template <bool PACKED>
+template <int MODE>
 __global__ void __launch_bounds__(kMaxThreads) rotate_quant_kernel(const __grid_constant__ RQParams p) {
+  constexpr bool PACKED = MODE == kPacked4;
+  constexpr float kQMax = MODE == kInt8 ? 127.0f : 7.0f;
+  constexpr int kQLo = MODE == kInt8 ? -127 : -8, kQHi = MODE == kInt8 ? 127 : 7;
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ uint32_t row_amax[3][kMaxRows];
   // Let the dependent GEMM launch now: it streams its weights meanwhile and
   // waits (griddepcontrol.wait) for this grid before reading codes or scales.
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  // Parameters in registers (the inline-asm memory clobbers below would
+  // otherwise reload them).
+  const int M = p.M, K = p.K, G = p.G, R = p.R, S = p.S;
+  const uint16_t* const x = p.x;
+  const RotateQuantOut out = p.out;
   const int hw = threadIdx.x >> 4, l = threadIdx.x & 15;
   const int nhw = blockDim.x >> 4;
-  const int S = p.S;
-  const int stage_bytes = rq_stage_bytes(p.R, p.K);
+  const int stage_bytes = rq_stage_bytes(R, K);
   uint8_t* const stages = smem;
   uint8_t* const tile = smem + S * stage_bytes + hw * kTileBytes;
+  uint8_t* const tile_w = tile + kTileRow * l;  // this lane's row
+  const uint8_t* const tile_r = tile + 8 * l;   // this lane's column
   // Byte tiles of the two tasks inside the pair tile; odd half-warps start 16
   // bytes later so that the two half-warps of a warp hit different banks.
   uint8_t* const btile0 = tile + 16 * (hw & 1);
   uint8_t* const btile1 = btile0 + 256;
+  uint8_t* const bw0 = btile0 + code_pos<MODE>(l);
+  uint8_t* const bw1 = btile1 + code_pos<MODE>(l);
   uint64_t* const full = reinterpret_cast<uint64_t*>(smem + S * stage_bytes + nhw * kTileBytes);
-  const int tasks = p.R * p.G;
-  const int iters =
-      static_cast<int>(blockIdx.x) < p.nblocks ? (p.nblocks - 1 - static_cast<int>(blockIdx.x)) / gridDim.x + 1 : 0;
+  const int tasks = R * G;
+  const int nb = p.nblocks;
+  const int iters = static_cast<int>(blockIdx.x) < nb ? (nb - 1 - static_cast<int>(blockIdx.x)) / gridDim.x + 1 : 0;
 
   // Thread 0: the bulk copy of this block's row block number `it`.
   auto issue = [&](int it) {
     const int b = static_cast<int>(blockIdx.x) + it * static_cast<int>(gridDim.x);
-    const int rows = min(p.R, p.M - b * p.R);
-    const uint32_t bytes = static_cast<uint32_t>(rows) * static_cast<uint32_t>(p.K) * 2u;
+    const int rows = min(R, M - b * R);
+    const uint32_t bytes = static_cast<uint32_t>(rows) * static_cast<uint32_t>(K) * 2u;
     uint64_t* bar = &full[it % S];
     mbar_arrive_expect_tx(bar, bytes);
-    bulk_load(stages + (it % S) * stage_bytes, p.x + static_cast<size_t>(b) * p.R * p.K, bytes, bar);
+    bulk_load(stages + (it % S) * stage_bytes, x + static_cast<size_t>(b) * R * K, bytes, bar);
   };
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) mbar_init(&full[s], 1);
@@ -186,34 +211,34 @@ __global__ void __launch_bounds__(kMaxThreads) rotate_quant_kernel(const __grid_
   for (int i = threadIdx.x; i < 3 * kMaxRows; i += blockDim.x) (&row_amax[0][0])[i] = 0u;
   __syncthreads();
 
-  // The lane's two tasks: hw and hw + nhw.
+  // The lane's two tasks: hw and hw + nhw (a task past the end computes on
+  // row 0, group 0 of the stage and is never stored).
   const int task0 = hw, task1 = hw + nhw;
-  const int rloc0 = task0 < tasks ? task0 / p.G : 0, rloc1 = task1 < tasks ? task1 / p.G : 0;
-  const int g0 = task0 - rloc0 * p.G, g1 = task1 - rloc1 * p.G;
+  const bool have0 = task0 < tasks, have1 = task1 < tasks;
+  const int rloc0 = have0 ? task0 / G : 0, rloc1 = have1 ? task1 / G : 0;
+  const int g0 = have0 ? task0 - rloc0 * G : 0, g1 = have1 ? task1 - rloc1 * G : 0;
+  const int in0 = (rloc0 * K + g0 * 256 + l * 16) * 2, in1 = (rloc1 * K + g1 * 256 + l * 16) * 2;
+  const size_t code_row = PACKED ? static_cast<size_t>(K / 2) : static_cast<size_t>(K);
+  const size_t out0 = static_cast<size_t>(rloc0) * code_row + (PACKED ? g0 * 128 + l * 8 : g0 * 256 + l * 16);
+  const size_t out1 = static_cast<size_t>(rloc1) * code_row + (PACKED ? g1 * 128 + l * 8 : g1 * 256 + l * 16);
+  uint8_t* const codes = PACKED ? out.packed : reinterpret_cast<uint8_t*>(out.s8);
 
   int it = 0;
   for (; it < iters; ++it) {
-    const int row0 = (static_cast<int>(blockIdx.x) + it * static_cast<int>(gridDim.x)) * p.R;
+    const int row0 = (static_cast<int>(blockIdx.x) + it * static_cast<int>(gridDim.x)) * R;
     const int slot = it % 3;
     const bool ok = mbar_wait(&full[it % S], (it / S) & 1);
     const uint8_t* stage = stages + (it % S) * stage_bytes;
-    const bool live0 = ok && task0 < tasks && row0 + rloc0 < p.M;
-    const bool live1 = ok && task1 < tasks && row0 + rloc1 < p.M;
+    const bool live0 = ok && have0 && row0 + rloc0 < M;
+    const bool live1 = ok && have1 && row0 + rloc1 < M;
 
     // ---- lane l: channels 16 l .. 16 l + 15 of both tasks, as pairs
     u64 P[16];
     {
-      uint4 a0 = make_uint4(0, 0, 0, 0), a1 = a0, b0 = a0, b1 = a0;
-      if (live0) {
-        const uint8_t* src = stage + (static_cast<size_t>(rloc0) * p.K + g0 * 256 + l * 16) * 2;
-        a0 = *reinterpret_cast<const uint4*>(src);
-        a1 = *reinterpret_cast<const uint4*>(src + 16);
-      }
-      if (live1) {
-        const uint8_t* src = stage + (static_cast<size_t>(rloc1) * p.K + g1 * 256 + l * 16) * 2;
-        b0 = *reinterpret_cast<const uint4*>(src);
-        b1 = *reinterpret_cast<const uint4*>(src + 16);
-      }
+      const uint4 a0 = *reinterpret_cast<const uint4*>(stage + in0);
+      const uint4 a1 = *reinterpret_cast<const uint4*>(stage + in0 + 16);
+      const uint4 b0 = *reinterpret_cast<const uint4*>(stage + in1);
+      const uint4 b1 = *reinterpret_cast<const uint4*>(stage + in1 + 16);
       const uint32_t wa[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
       const uint32_t wb[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
 #pragma unroll
@@ -228,15 +253,12 @@ __global__ void __launch_bounds__(kMaxThreads) rotate_quant_kernel(const __grid_
     // stage on bits (2,3): stride 4
 #pragma unroll
     for (int i = 0; i < 4; ++i) bfly4(P[i], P[i + 4], P[i + 8], P[i + 12]);
-    // transpose: row l of the tile <- channels 16 l + i; 16-byte chunk c (pairs
-    // 2c, 2c + 1) of row r sits at chunk c ^ (r & 7)
+    // transpose: row l of the tile <- channels 16 l + i
 #pragma unroll
-    for (int c = 0; c < 8; ++c)
-      *reinterpret_cast<ulonglong2*>(tile + 128 * l + 16 * (c ^ (l & 7))) = make_ulonglong2(P[2 * c], P[2 * c + 1]);
+    for (int c = 0; c < 8; ++c) *reinterpret_cast<ulonglong2*>(tile_w + 16 * c) = make_ulonglong2(P[2 * c], P[2 * c + 1]);
     __syncwarp();
 #pragma unroll
-    for (int i = 0; i < 16; ++i)
-      P[i] = *reinterpret_cast<const u64*>(tile + 128 * i + 16 * ((l >> 1) ^ (i & 7)) + 8 * (l & 1));
+    for (int i = 0; i < 16; ++i) P[i] = *reinterpret_cast<const u64*>(tile_r + kTileRow * i);
     __syncwarp();
     // now P[i] = channel 16 i + l.  stage on bits (4,5): stride 16
 #pragma unroll
@@ -249,12 +271,14 @@ __global__ void __launch_bounds__(kMaxThreads) rotate_quant_kernel(const __grid_
     {
       const u64 sixteenth = f2(0.0625f, 0.0625f);
 #pragma unroll
-      for (int i = 0; i < 16; ++i) {
+      for (int i = 0; i < 16; i += 2) {
         P[i] = f2_mul(P[i], sixteenth);
-        float x0, x1;
+        P[i + 1] = f2_mul(P[i + 1], sixteenth);
+        float x0, x1, y0, y1;
         f2_split(P[i], x0, x1);
-        m0 = fmaxf(m0, fabsf(x0));
-        m1 = fmaxf(m1, fabsf(x1));
+        f2_split(P[i + 1], y0, y1);
+        m0 = max3(m0, fabsf(x0), fabsf(y0));
+        m1 = max3(m1, fabsf(x1), fabsf(y1));
       }
     }
     // ---- per-row amax: within each task (16 lanes), then across the row's tasks
@@ -277,20 +301,20 @@ __global__ void __launch_bounds__(kMaxThreads) rotate_quant_kernel(const __grid_
     if (threadIdx.x < kMaxRows) row_amax[(it + 2) % 3][threadIdx.x] = 0u;
 
     // ---- quantize
-    const float scale0 = __fdiv_rn(__uint_as_float(row_amax[slot][rloc0]), 7.0f);
-    const float scale1 = __fdiv_rn(__uint_as_float(row_amax[slot][rloc1]), 7.0f);
+    const float scale0 = __fdiv_rn(__uint_as_float(row_amax[slot][rloc0]), kQMax);
+    const float scale1 = __fdiv_rn(__uint_as_float(row_amax[slot][rloc1]), kQMax);
     uint32_t c0[16], c1[16];  // code bytes (low byte) of channel 16 i + l
     if (scale0 >= kMinScale && scale1 >= kMinScale) {
       const u64 rr = f2(__frcp_rn(scale0), __frcp_rn(scale1)), ns = f2(-scale0, -scale1);
       const u64 mg = f2(kMagic, kMagic);
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
-        const u64 x = P[i];
-        u64 q = f2_mul(x, rr);
-        q = f2_fma(f2_fma(ns, q, x), rr, q);  // faithful
-        q = f2_fma(f2_fma(ns, q, x), rr, q);  // RN(x / s)
+        const u64 xv = P[i];
+        u64 q = f2_mul(xv, rr);
+        q = f2_fma(f2_fma(ns, q, xv), rr, q);  // faithful
+        q = f2_fma(f2_fma(ns, q, xv), rr, q);  // RN(x / s)
         float t0, t1;
-        f2_split(f2_add(q, mg), t0, t1);      // low byte = rint(q)
+        f2_split(f2_add(q, mg), t0, t1);       // low byte = rint(q)
         c0[i] = __float_as_uint(t0);
         c1[i] = __float_as_uint(t1);
       }
@@ -302,38 +326,34 @@ __global__ void __launch_bounds__(kMaxThreads) rotate_quant_kernel(const __grid_
         f2_split(P[i], x0, x1);
         const int q0 = scale0 != 0.0f ? __float2int_rn(__fdiv_rn(x0, scale0)) : 0;
         const int q1 = scale1 != 0.0f ? __float2int_rn(__fdiv_rn(x1, scale1)) : 0;
-        c0[i] = static_cast<uint32_t>(min(7, max(-8, q0)));
-        c1[i] = static_cast<uint32_t>(min(7, max(-8, q1)));
+        c0[i] = static_cast<uint32_t>(min(kQHi, max(kQLo, q0)));
+        c1[i] = static_cast<uint32_t>(min(kQHi, max(kQLo, q1)));
       }
     }
     // ---- back to row order through the byte tiles, store
-    const int pos = code_pos<PACKED>(l);
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
-      btile0[16 * i + pos] = static_cast<uint8_t>(c0[i]);
-      btile1[16 * i + pos] = static_cast<uint8_t>(c1[i]);
+      bw0[16 * i] = static_cast<uint8_t>(c0[i]);
+      bw1[16 * i] = static_cast<uint8_t>(c1[i]);
     }
     __syncwarp();
     const uint4 o0 = *reinterpret_cast<const uint4*>(btile0 + 16 * l);  // channels 16 l .. 16 l + 15
     const uint4 o1 = *reinterpret_cast<const uint4*>(btile1 + 16 * l);
     __syncwarp();
+    const size_t obase = static_cast<size_t>(row0) * code_row;
     if (live0) {
-      const int row = row0 + rloc0;
       if (PACKED)
-        *reinterpret_cast<uint2*>(p.out.packed + static_cast<size_t>(row) * (p.K / 2) + g0 * 128 + l * 8) =
-            make_uint2(pack_nibbles(o0.x, o0.y), pack_nibbles(o0.z, o0.w));
+        *reinterpret_cast<uint2*>(codes + obase + out0) = make_uint2(pack_nibbles(o0.x, o0.y), pack_nibbles(o0.z, o0.w));
       else
-        *reinterpret_cast<uint4*>(p.out.s8 + static_cast<size_t>(row) * p.K + g0 * 256 + l * 16) = o0;
-      if (g0 == 0 && l == 0) p.out.scale[row] = scale0;
+        *reinterpret_cast<uint4*>(codes + obase + out0) = o0;
+      if (g0 == 0 && l == 0) out.scale[row0 + rloc0] = scale0;
     }
     if (live1) {
-      const int row = row0 + rloc1;
       if (PACKED)
-        *reinterpret_cast<uint2*>(p.out.packed + static_cast<size_t>(row) * (p.K / 2) + g1 * 128 + l * 8) =
-            make_uint2(pack_nibbles(o1.x, o1.y), pack_nibbles(o1.z, o1.w));
+        *reinterpret_cast<uint2*>(codes + obase + out1) = make_uint2(pack_nibbles(o1.x, o1.y), pack_nibbles(o1.z, o1.w));
       else
-        *reinterpret_cast<uint4*>(p.out.s8 + static_cast<size_t>(row) * p.K + g1 * 256 + l * 16) = o1;
-      if (g1 == 0 && l == 0) p.out.scale[row] = scale1;
+        *reinterpret_cast<uint4*>(codes + obase + out1) = o1;
+      if (g1 == 0 && l == 0) out.scale[row0 + rloc1] = scale1;
     }
   }
   if (it < iters && threadIdx.x == 0) {
@@ -376,20 +396,20 @@ int num_sms_cached() {
   return n[dev];
 }
 
-template <bool PACKED>
+template <int MODE>
 cudaError_t launch_rq(const RQParams& p, int threads, cudaStream_t stream) {
   static int cache[64] = {0};
   const int smem = rq_smem_bytes(p.R, p.K, p.S, threads);
-  const void* kfn = reinterpret_cast<const void*>(rotate_quant_kernel<PACKED>);
+  const void* kfn = reinterpret_cast<const void*>(rotate_quant_kernel<MODE>);
   cudaError_t e = ensure_dynamic_smem(kfn, smem, cache);
   if (e != cudaSuccess) return note_cuda(e, "rotate_quant: dynamic shared memory attribute");
   int per_sm = 0;
-  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, rotate_quant_kernel<PACKED>, threads, smem);
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, rotate_quant_kernel<MODE>, threads, smem);
   if (e != cudaSuccess) return note_cuda(e, "rotate_quant: occupancy query");
   if (per_sm < 1) per_sm = 1;
   int grid = num_sms_cached() * per_sm;
   if (grid > p.nblocks) grid = p.nblocks;
-  rotate_quant_kernel<PACKED><<<grid, threads, smem, stream>>>(p);
+  rotate_quant_kernel<MODE><<<grid, threads, smem, stream>>>(p);
   return note_cuda(cudaGetLastError(), "rotate_quant: launch");
 }
 
@@ -443,7 +463,9 @@ cudaError_t launch_rotate_quant(const uint16_t* x, int M, int K, RotateQuantOut 
   if (S > most_iters) S = most_iters;
   if (S < 1) S = 1;
   p.S = S;
-  cudaError_t e = out.packed != nullptr ? launch_rq<true>(p, threads, stream) : launch_rq<false>(p, threads, stream);
+  cudaError_t e = out.packed != nullptr ? launch_rq<kPacked4>(p, threads, stream)
+                  : out.int8      ? launch_rq<kInt8>(p, threads, stream)
+                                  : launch_rq<kOperand4>(p, threads, stream);
   count_dispatch(0);
   return e;
 }

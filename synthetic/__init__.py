@@ -153,6 +153,14 @@ class LinearShape:
     M: int
     K: int
     N: int
+    # The activation tensor the linear reads: linears of one layer that read
+    # the same tensor (q/k/v; gate/up) share it, and one rotate + quantize
+    # of it serves all of them.
+    input: str = ""
+
+    @property
+    def source(self) -> str:
+        return self.input or self.name
 
 
 _ACT = {
@@ -170,19 +178,21 @@ def workload_shapes(workload: str) -> list[LinearShape]:
     if workload == "small":
         return [LinearShape("linear", 32, 512, 256)]
     if workload == "qwen3_4b":
-        lin = [("q_proj", 2560, 4096), ("k_proj", 2560, 1024), ("v_proj", 2560, 1024),
-               ("o_proj", 2560, 2560), ("gate_proj", 2560, 9728), ("up_proj", 2560, 9728),
-               ("down_proj", 9728, 2560)]
-        return [LinearShape(f"{n}@{M}", M, K, N) for M in (76, 1220) for (n, K, N) in lin]
+        lin = [("q_proj", 2560, 4096, "attn_in"), ("k_proj", 2560, 1024, "attn_in"), ("v_proj", 2560, 1024, "attn_in"),
+               ("o_proj", 2560, 2560, "attn_out"), ("gate_proj", 2560, 9728, "mlp_in"),
+               ("up_proj", 2560, 9728, "mlp_in"), ("down_proj", 9728, 2560, "mlp_act")]
+        return [LinearShape(f"{n}@{M}", M, K, N, f"{src}@{M}") for M in (76, 1220) for (n, K, N, src) in lin]
     if workload == "dit6b":
         M = 4096 + 128
-        lin = [("qkv", 3840, 3 * 3840), ("out", 3840, 3840), ("ffn_up", 3840, 10240), ("ffn_down", 10240, 3840)]
-        return [LinearShape(n, M, K, N) for (n, K, N) in lin]
+        lin = [("qkv", 3840, 3 * 3840, "attn_in"), ("out", 3840, 3840, "attn_out"),
+               ("ffn_up", 3840, 10240, "mlp_in"), ("ffn_down", 10240, 3840, "mlp_act")]
+        return [LinearShape(n, M, K, N, src) for (n, K, N, src) in lin]
     if workload == "edit20b":
         M = 8192 + 512
-        lin = [("to_q", 3072, 3072), ("to_k", 3072, 3072), ("to_v", 3072, 3072), ("to_out", 3072, 3072),
-               ("mlp_up", 3072, 12288), ("mlp_down", 12288, 3072)]
-        return [LinearShape(n, M, K, N) for (n, K, N) in lin]
+        lin = [("to_q", 3072, 3072, "attn_in"), ("to_k", 3072, 3072, "attn_in"), ("to_v", 3072, 3072, "attn_in"),
+               ("to_out", 3072, 3072, "attn_out"), ("mlp_up", 3072, 12288, "mlp_in"),
+               ("mlp_down", 12288, 3072, "mlp_act")]
+        return [LinearShape(n, M, K, N, src) for (n, K, N, src) in lin]
     if workload == "small_m":
         kn = [(2560, 9728), (9728, 2560), (3072, 12288), (12288, 3072)]
         return [LinearShape(f"k{K}_n{N}@{M}", M, K, N) for M in (1, 8, 16, 64, 128) for (K, N) in kn]
@@ -193,6 +203,14 @@ def activations(workload: str, M: int, K: int, seed_extra: int = 0) -> np.ndarra
     """bf16 bits [M, K] drawn with the workload's activation recipe."""
     seed = derive_seed(_BASE_SEED[workload] ^ seed_extra, "x", M, K)
     return _ACT[workload](seed, M, K)
+
+
+def source_seed(source: str) -> int:
+    """seed_extra of a named activation tensor (a fixed hash of its name)."""
+    h = 0
+    for ch in source.encode():
+        h = (h * 131 + ch) & 0xFFFFFFFF
+    return h
 
 
 def weights(workload: str, N: int, K: int, seed_extra: int = 0):
