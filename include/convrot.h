@@ -177,6 +177,71 @@ convrot_status_t convrot_w4a4_gemm_quantized(const uint8_t *Wq, const float *s_w
                                              uint16_t *y, const void *workspace,
                                              size_t workspace_bytes, void *stream);
 
+/* ---- int8 W8A8 formats -------------------------------------------------------
+ * The pages store their quality-sensitive layers in int8 next to the W4A4
+ * ones, and both run on the same integer tensor-core path:
+ *   W8A8_INT8_TENSORWISE  stock "int8_tensorwise" ("Qwen-Image-Edit-2511 --
+ *     INT4 tensorwise W4A4 (+ConvRot, mixed int8 fallback)", intro: the
+ *     attention value/output projections and adaLN Linears): no rotation, one
+ *     scale for the whole weight tensor and one dynamic scale for the whole
+ *     activation tensor.
+ *   W8A8_CONVROT_INT8_ROW  "ConvRot INT8 (row-scaled)" ("rockerBOO/qwen3-4b-
+ *     nvfp4-convrot", file table: the attention projections): the group-256
+ *     rotation R above, one scale per weight row and one dynamic scale per
+ *     activation row (token).
+ * Codes: s = amax / 127 (one fp32 IEEE division), q = clamp(rint(v / s),
+ * -127, 127) with a true division and round half to even, s == 0 -> q = 0;
+ * int8 [rows, K] row-major, natural order.  Linear: acc = sum_k q_x q_w
+ * (exact int32), y = acc * s_x[m] * s_w[n] + bias[n] -> bf16 (a per-tensor
+ * scale is used for every m / n).  Same shape rules as above (K % 256 == 0,
+ * N % 8 == 0, 16-byte-aligned pointers). */
+typedef enum { W8A8_INT8_TENSORWISE = 0, W8A8_CONVROT_INT8_ROW = 1 } w8a8_format_t;
+
+/* Bytes of workspace w8a8_quantize / w8a8_pack_weight / w8a8_linear* need
+ * for (M, N, K) in `format` (0 for an invalid shape or format): the int8
+ * activation codes (M * K), the activation scales and 4 bytes of reduction
+ * scratch, each part rounded up to 256 bytes. */
+size_t w8a8_workspace_size(int M, int N, int K, int format);
+
+/* Quantize x [M, K] bf16 to int8 codes x8 [M, K] and scales s_x ([1] for
+ * int8_tensorwise, [M] for ConvRot INT8 row-scaled).  workspace: at least
+ * w8a8_workspace_size(M, 8, K, format) bytes of device scratch (only its
+ * reduction scratch is used). */
+convrot_status_t w8a8_quantize(const uint16_t *x, int M, int K, int format, int8_t *x8, float *s_x,
+                               void *workspace, size_t workspace_bytes, void *stream);
+
+/* Offline weight preparation: the same quantizer on W [N, K] bf16 -> Wq8
+ * [N, K] int8 and s_w ([1] tensorwise, [N] row-scaled). */
+convrot_status_t w8a8_pack_weight(const uint16_t *W, int N, int K, int format, int8_t *Wq8, float *s_w,
+                                  void *workspace, size_t workspace_bytes, void *stream);
+
+/* Integer GEMM with the rank-one epilogue on int8 codes: y [M, N] bf16 from
+ * x8 [M, K], s_x, Wq8 [N, K], s_w (per `format`), bias [N] or NULL. */
+convrot_status_t w8a8_gemm(const int8_t *x8, const float *s_x, const int8_t *Wq8, const float *s_w,
+                           const uint16_t *bias, int M, int N, int K, int format, uint16_t *y,
+                           void *stream);
+
+/* Same kernel, fp32 sink y32 [M, N] before the bf16 rounding (parity). */
+convrot_status_t w8a8_gemm_f32(const int8_t *x8, const float *s_x, const int8_t *Wq8, const float *s_w,
+                               const uint16_t *bias, int M, int N, int K, int format, float *y32,
+                               void *stream);
+
+/* Same kernel, the exact int32 accumulator acc [M, N] (parity). */
+convrot_status_t w8a8_gemm_s32(const int8_t *x8, const int8_t *Wq8, int M, int N, int K, int32_t *acc,
+                               void *stream);
+
+/* The fused int8 Linear: x [M, K] bf16 quantized online (per `format`), times
+ * Wq8 / s_w from w8a8_pack_weight, plus bias -> y [M, N] bf16.  workspace:
+ * >= w8a8_workspace_size(M, N, K, format) bytes. */
+convrot_status_t w8a8_linear(const uint16_t *x, const int8_t *Wq8, const float *s_w, const uint16_t *bias,
+                             int M, int N, int K, int format, uint16_t *y, void *workspace,
+                             size_t workspace_bytes, void *stream);
+
+/* The fused int8 Linear with an fp32 sink (parity). */
+convrot_status_t w8a8_linear_f32(const uint16_t *x, const int8_t *Wq8, const float *s_w,
+                                 const uint16_t *bias, int M, int N, int K, int format, float *y32,
+                                 void *workspace, size_t workspace_bytes, void *stream);
+
 /* Device-side error word of the current device: bit 0 = a bounded wait
  * inside a kernel expired (the kernel skipped its remaining work and
  * returned; its outputs are invalid).  Synchronizes `stream`, copies the word

@@ -41,7 +41,13 @@ EXPORTS = [
     "convrot_w4a4_linear_f32", "convrot_w4a4_linear_noalloc", "convrot_w4a4_quantize", "convrot_w4a4_gemm_quantized", "convrot_device_error",
     "convrot_dispatch_counts", "convrot_last_error", "convrot_selftest_timeout", "convrot_version",
     "convrot_measure_mma_i8",
+    "w8a8_workspace_size", "w8a8_quantize", "w8a8_pack_weight", "w8a8_gemm", "w8a8_gemm_f32", "w8a8_gemm_s32",
+    "w8a8_linear", "w8a8_linear_f32",
 ]
+
+# int8 formats (include/convrot.h, w8a8_format_t)
+W8A8_INT8_TENSORWISE = 0
+W8A8_CONVROT_INT8_ROW = 1
 
 
 class ConvRotError(RuntimeError):
@@ -88,6 +94,15 @@ def load_library():
     lib.convrot_dispatch_counts.argtypes = [ctypes.POINTER(ctypes.c_uint64), I]
     lib.convrot_dispatch_counts.restype = None
     lib.convrot_measure_mma_i8.argtypes = [I, I, I, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_double)]
+    lib.w8a8_workspace_size.argtypes = [I, I, I, I]
+    lib.w8a8_workspace_size.restype = Z
+    lib.w8a8_quantize.argtypes = [P, I, I, I, P, P, P, Z, P]
+    lib.w8a8_pack_weight.argtypes = [P, I, I, I, P, P, P, Z, P]
+    lib.w8a8_gemm.argtypes = [P, P, P, P, P, I, I, I, I, P, P]
+    lib.w8a8_gemm_f32.argtypes = [P, P, P, P, P, I, I, I, I, P, P]
+    lib.w8a8_gemm_s32.argtypes = [P, P, I, I, I, P, P]
+    lib.w8a8_linear.argtypes = [P, P, P, P, I, I, I, I, P, P, Z, P]
+    lib.w8a8_linear_f32.argtypes = [P, P, P, P, I, I, I, I, P, P, Z, P]
     for name in lib_status_fns():
         getattr(lib, name).restype = I
     _lib = lib
@@ -98,7 +113,8 @@ def lib_status_fns():
     return ["convrot_pack_weight", "convrot_rotate_quant", "w4a4_gemm", "w4a4_gemm_s32", "w4a4_gemm_f32",
             "convrot_w4a4_linear", "convrot_w4a4_linear_f32", "convrot_w4a4_linear_noalloc", "convrot_w4a4_quantize",
             "convrot_w4a4_gemm_quantized", "convrot_device_error", "convrot_selftest_timeout",
-            "convrot_measure_mma_i8"]
+            "convrot_measure_mma_i8", "w8a8_quantize", "w8a8_pack_weight", "w8a8_gemm", "w8a8_gemm_f32",
+            "w8a8_gemm_s32", "w8a8_linear", "w8a8_linear_f32"]
 
 
 def _check(fn: str, rc: int):
@@ -305,6 +321,101 @@ def convrot_measure_mma_i8(N: int = 256, a_in_tmem: bool = False, iters: int = 4
     _check("convrot_measure_mma_i8", load_library().convrot_measure_mma_i8(
         int(N), 1 if a_in_tmem else 0, int(iters), ctypes.byref(tops), ctypes.byref(cyc)))
     return float(tops.value), float(cyc.value)
+
+
+# ---- int8 W8A8 formats (int8_tensorwise, ConvRot INT8 row-scaled)
+
+def w8a8_workspace_size(M: int, N: int, K: int, fmt: int) -> int:
+    return int(load_library().w8a8_workspace_size(M, N, K, int(fmt)))
+
+
+def _n_scales(rows, fmt):
+    return rows if fmt == W8A8_CONVROT_INT8_ROW else 1
+
+
+def w8a8_quantize(x, fmt, x8=None, s_x=None, workspace=None, stream=None):
+    """x [M, K] bf16 -> (int8 codes [M, K], scales fp32 [M] row-scaled / [1] tensorwise)."""
+    M, K = x.shape
+    _need(x, "x", torch.bfloat16)
+    x8 = torch.empty((M, K), dtype=torch.int8, device=x.device) if x8 is None else x8
+    s_x = torch.empty((_n_scales(M, fmt),), dtype=torch.float32, device=x.device) if s_x is None else s_x
+    _need(x8, "x8", torch.int8, (M, K))
+    _need(s_x, "s_x", torch.float32, (_n_scales(M, fmt),))
+    ws = _workspace(workspace, w8a8_workspace_size(M, 8, K, fmt), x.device)
+    _check("w8a8_quantize", load_library().w8a8_quantize(_ptr(x), M, K, int(fmt), _ptr(x8), _ptr(s_x), _ptr(ws),
+                                                         ws.numel(), _stream(stream)))
+    return x8, s_x
+
+
+def w8a8_pack_weight(W, fmt, Wq8=None, s_w=None, workspace=None, stream=None):
+    """W [N, K] bf16 -> (int8 codes [N, K], scales fp32 [N] row-scaled / [1] tensorwise)."""
+    N, K = W.shape
+    _need(W, "W", torch.bfloat16)
+    Wq8 = torch.empty((N, K), dtype=torch.int8, device=W.device) if Wq8 is None else Wq8
+    s_w = torch.empty((_n_scales(N, fmt),), dtype=torch.float32, device=W.device) if s_w is None else s_w
+    _need(Wq8, "Wq8", torch.int8, (N, K))
+    _need(s_w, "s_w", torch.float32, (_n_scales(N, fmt),))
+    ws = _workspace(workspace, w8a8_workspace_size(N, 8, K, fmt), W.device)
+    _check("w8a8_pack_weight", load_library().w8a8_pack_weight(_ptr(W), N, K, int(fmt), _ptr(Wq8), _ptr(s_w),
+                                                               _ptr(ws), ws.numel(), _stream(stream)))
+    return Wq8, s_w
+
+
+def _gemm8(fn_name, out_dtype, x8, s_x, Wq8, s_w, bias, fmt, out, stream):
+    M, K = x8.shape
+    N = Wq8.shape[0]
+    _need(x8, "x8", torch.int8)
+    _need(Wq8, "Wq8", torch.int8, (N, K))
+    _need(s_x, "s_x", torch.float32, (_n_scales(M, fmt),))
+    _need(s_w, "s_w", torch.float32, (_n_scales(N, fmt),))
+    _need(bias, "bias", torch.bfloat16, (N,))
+    out = torch.empty((M, N), dtype=out_dtype, device=x8.device) if out is None else out
+    _need(out, "out", out_dtype, (M, N))
+    _check(fn_name, getattr(load_library(), fn_name)(_ptr(x8), _ptr(s_x), _ptr(Wq8), _ptr(s_w), _ptr(bias), M, N, K,
+                                                     int(fmt), _ptr(out), _stream(stream)))
+    return out
+
+
+def w8a8_gemm(x8, s_x, Wq8, s_w, bias=None, fmt=W8A8_INT8_TENSORWISE, out=None, stream=None):
+    return _gemm8("w8a8_gemm", torch.bfloat16, x8, s_x, Wq8, s_w, bias, fmt, out, stream)
+
+
+def w8a8_gemm_f32(x8, s_x, Wq8, s_w, bias=None, fmt=W8A8_INT8_TENSORWISE, out=None, stream=None):
+    return _gemm8("w8a8_gemm_f32", torch.float32, x8, s_x, Wq8, s_w, bias, fmt, out, stream)
+
+
+def w8a8_gemm_s32(x8, Wq8, out=None, stream=None):
+    M, K = x8.shape
+    N = Wq8.shape[0]
+    _need(x8, "x8", torch.int8)
+    _need(Wq8, "Wq8", torch.int8, (N, K))
+    out = torch.empty((M, N), dtype=torch.int32, device=x8.device) if out is None else out
+    _need(out, "out", torch.int32, (M, N))
+    _check("w8a8_gemm_s32", load_library().w8a8_gemm_s32(_ptr(x8), _ptr(Wq8), M, N, K, _ptr(out), _stream(stream)))
+    return out
+
+
+def _linear8(fn_name, out_dtype, x, Wq8, s_w, bias, fmt, out, workspace, stream):
+    M, K = x.shape
+    N = Wq8.shape[0]
+    _need(x, "x", torch.bfloat16)
+    _need(Wq8, "Wq8", torch.int8, (N, K))
+    _need(s_w, "s_w", torch.float32, (_n_scales(N, fmt),))
+    _need(bias, "bias", torch.bfloat16, (N,))
+    out = torch.empty((M, N), dtype=out_dtype, device=x.device) if out is None else out
+    _need(out, "out", out_dtype, (M, N))
+    ws = _workspace(workspace, w8a8_workspace_size(M, N, K, fmt), x.device)
+    _check(fn_name, getattr(load_library(), fn_name)(_ptr(x), _ptr(Wq8), _ptr(s_w), _ptr(bias), M, N, K, int(fmt),
+                                                     _ptr(out), _ptr(ws), ws.numel(), _stream(stream)))
+    return out
+
+
+def w8a8_linear(x, Wq8, s_w, bias=None, fmt=W8A8_INT8_TENSORWISE, out=None, workspace=None, stream=None):
+    return _linear8("w8a8_linear", torch.bfloat16, x, Wq8, s_w, bias, fmt, out, workspace, stream)
+
+
+def w8a8_linear_f32(x, Wq8, s_w, bias=None, fmt=W8A8_INT8_TENSORWISE, out=None, workspace=None, stream=None):
+    return _linear8("w8a8_linear_f32", torch.float32, x, Wq8, s_w, bias, fmt, out, workspace, stream)
 
 
 def convrot_version() -> str:

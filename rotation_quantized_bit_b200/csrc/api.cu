@@ -146,6 +146,76 @@ convrot_status_t linear_common(const uint16_t* x, const uint8_t* Wq, const float
   return gemm_quantized_common(Wq, s_w, bias, M, N, K, out, sink, ws, ws_bytes, stream);
 }
 
+// ---- int8 W8A8 formats
+
+bool valid_format(int format) { return format == W8A8_INT8_TENSORWISE || format == W8A8_CONVROT_INT8_ROW; }
+
+// Workspace of the int8 path: codes [M*K], scales [M] (or [1]), 4 bytes of
+// reduction scratch; each on a 256-byte boundary.
+size_t w8_scales_offset(int M, int K) { return codes_bytes(M, K); }
+size_t w8_scratch_offset(int M, int K) { return w8_scales_offset(M, K) + round_up(static_cast<size_t>(M) * 4, 256); }
+size_t w8_workspace_bytes(int M, int K) { return w8_scratch_offset(M, K) + 256; }
+
+// Quantize rows of a bf16 [rows, K] matrix into int8 codes and scales.
+convrot_status_t quant8_common(const uint16_t* x, int rows, int K, int format, int8_t* codes, float* scales,
+                               void* ws, size_t ws_bytes, void* stream) {
+  if (!x || !codes || !scales) return CONVROT_ERR_NULL;
+  if (!valid_format(format)) return CONVROT_ERR_SHAPE;
+  convrot_status_t st = check_mk(rows, K);
+  if (st != CONVROT_OK) return st;
+  if (!aligned16(x) || !aligned16(codes) || !aligned16(scales)) return CONVROT_ERR_ALIGN;
+  st = check_device(nullptr);
+  if (st != CONVROT_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (format == W8A8_CONVROT_INT8_ROW) {
+    RotateQuantOut o{nullptr, codes, scales};
+    o.int8 = true;
+    return from_cuda(launch_rotate_quant(x, rows, K, o, s));
+  }
+  if (!ws || ws_bytes < 4) return CONVROT_ERR_WORKSPACE;
+  if (!aligned16(ws)) return CONVROT_ERR_ALIGN;
+  return from_cuda(launch_quant8_tensorwise(x, static_cast<size_t>(rows) * static_cast<size_t>(K), codes, scales,
+                                            static_cast<uint32_t*>(ws), s));
+}
+
+convrot_status_t gemm8_common(const int8_t* x8, const float* s_x, const int8_t* Wq8, const float* s_w,
+                              const uint16_t* bias, int M, int N, int K, int format, void* out, GemmSink sink,
+                              void* stream) {
+  if (!x8 || !Wq8 || !out) return CONVROT_ERR_NULL;
+  if (sink != GemmSink::kS32 && (!s_x || !s_w)) return CONVROT_ERR_NULL;
+  if (!valid_format(format)) return CONVROT_ERR_SHAPE;
+  convrot_status_t st = check_mnk(M, N, K);
+  if (st != CONVROT_OK) return st;
+  if (!aligned16(x8) || !aligned16(Wq8) || !aligned16(out) || (s_x && !aligned16(s_x)) ||
+      (s_w && !aligned16(s_w)) || (bias && !aligned16(bias)))
+    return CONVROT_ERR_ALIGN;
+  int sms = 0;
+  st = check_device(&sms);
+  if (st != CONVROT_OK) return st;
+  GemmArgs a{x8, s_x, reinterpret_cast<const uint8_t*>(Wq8), s_w, bias, out, M, N, K};
+  a.w8 = 1;
+  a.sa_stride = format == W8A8_CONVROT_INT8_ROW ? 1 : 0;
+  a.sw_stride = format == W8A8_CONVROT_INT8_ROW ? 1 : 0;
+  return from_cuda(launch_w4a4_gemm(a, sink, choose_tiling(M, N, K, sms, true), static_cast<cudaStream_t>(stream)));
+}
+
+convrot_status_t linear8_common(const uint16_t* x, const int8_t* Wq8, const float* s_w, const uint16_t* bias, int M,
+                                int N, int K, int format, void* out, GemmSink sink, void* ws, size_t ws_bytes,
+                                void* stream) {
+  if (!x || !Wq8 || !s_w || !out) return CONVROT_ERR_NULL;
+  if (!valid_format(format)) return CONVROT_ERR_SHAPE;
+  convrot_status_t st = check_mnk(M, N, K);
+  if (st != CONVROT_OK) return st;
+  if (!ws || ws_bytes < w8_workspace_bytes(M, K)) return CONVROT_ERR_WORKSPACE;
+  if (!aligned16(ws)) return CONVROT_ERR_ALIGN;
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  int8_t* codes = reinterpret_cast<int8_t*>(base);
+  float* scales = reinterpret_cast<float*>(base + w8_scales_offset(M, K));
+  st = quant8_common(x, M, K, format, codes, scales, base + w8_scratch_offset(M, K), 256, stream);
+  if (st != CONVROT_OK) return st;
+  return gemm8_common(codes, scales, Wq8, s_w, bias, M, N, K, format, out, sink, stream);
+}
+
 }  // namespace
 
 void count_dispatch(int which) {
@@ -309,6 +379,62 @@ convrot_status_t convrot_device_error(void* stream, uint32_t* code) {
 void convrot_dispatch_counts(uint64_t* counts, int n) {
   if (!counts) return;
   for (int i = 0; i < n && i < 4; ++i) counts[i] = g_counts[i].load(std::memory_order_relaxed);
+}
+
+}  // extern "C"
+
+extern "C" {
+
+size_t w8a8_workspace_size(int M, int N, int K, int format) {
+  if (!valid_format(format) || check_mnk(M, N, K) != CONVROT_OK) return 0;
+  return w8_workspace_bytes(M, K);
+}
+
+convrot_status_t w8a8_quantize(const uint16_t* x, int M, int K, int format, int8_t* x8, float* s_x, void* workspace,
+                               size_t workspace_bytes, void* stream) {
+  uint8_t* scratch = nullptr;
+  size_t scratch_bytes = 0;
+  if (workspace && check_mk(M, K) == CONVROT_OK && workspace_bytes >= w8_workspace_bytes(M, K)) {
+    scratch = static_cast<uint8_t*>(workspace) + w8_scratch_offset(M, K);
+    scratch_bytes = 256;
+  }
+  if (format == W8A8_INT8_TENSORWISE && !scratch && check_mk(M, K) == CONVROT_OK && x && x8 && s_x)
+    return CONVROT_ERR_WORKSPACE;
+  return quant8_common(x, M, K, format, x8, s_x, scratch, scratch_bytes, stream);
+}
+
+convrot_status_t w8a8_pack_weight(const uint16_t* W, int N, int K, int format, int8_t* Wq8, float* s_w,
+                                  void* workspace, size_t workspace_bytes, void* stream) {
+  return w8a8_quantize(W, N, K, format, Wq8, s_w, workspace, workspace_bytes, stream);
+}
+
+convrot_status_t w8a8_gemm(const int8_t* x8, const float* s_x, const int8_t* Wq8, const float* s_w,
+                           const uint16_t* bias, int M, int N, int K, int format, uint16_t* y, void* stream) {
+  return gemm8_common(x8, s_x, Wq8, s_w, bias, M, N, K, format, y, GemmSink::kBF16, stream);
+}
+
+convrot_status_t w8a8_gemm_f32(const int8_t* x8, const float* s_x, const int8_t* Wq8, const float* s_w,
+                               const uint16_t* bias, int M, int N, int K, int format, float* y32, void* stream) {
+  return gemm8_common(x8, s_x, Wq8, s_w, bias, M, N, K, format, y32, GemmSink::kF32, stream);
+}
+
+convrot_status_t w8a8_gemm_s32(const int8_t* x8, const int8_t* Wq8, int M, int N, int K, int32_t* acc,
+                               void* stream) {
+  return gemm8_common(x8, nullptr, Wq8, nullptr, nullptr, M, N, K, W8A8_CONVROT_INT8_ROW, acc, GemmSink::kS32,
+                      stream);
+}
+
+convrot_status_t w8a8_linear(const uint16_t* x, const int8_t* Wq8, const float* s_w, const uint16_t* bias, int M,
+                             int N, int K, int format, uint16_t* y, void* workspace, size_t workspace_bytes,
+                             void* stream) {
+  return linear8_common(x, Wq8, s_w, bias, M, N, K, format, y, GemmSink::kBF16, workspace, workspace_bytes, stream);
+}
+
+convrot_status_t w8a8_linear_f32(const uint16_t* x, const int8_t* Wq8, const float* s_w, const uint16_t* bias,
+                                 int M, int N, int K, int format, float* y32, void* workspace,
+                                 size_t workspace_bytes, void* stream) {
+  return linear8_common(x, Wq8, s_w, bias, M, N, K, format, y32, GemmSink::kF32, workspace, workspace_bytes,
+                        stream);
 }
 
 }  // extern "C"

@@ -25,6 +25,10 @@
 //     chunk order, so the contraction pairs the right codes;
 //   * the accumulator is exactly 16 * acc (|16 acc| <= 1024 K < 2^31), and
 //     the epilogue shifts it right by 4.
+// The W8A8 formats (int8 weights [N, K]) use the same kernel with W8 = true:
+// the weight tile goes by TMA straight into shared memory as the MMA's A
+// operand (no unpack, no tensor-memory A slots), the accumulator is the
+// integer product itself, and per-tensor scales are read with stride 0.
 // Work is cut into units of one 256-wide K block of one output tile; see
 // the kernel below for the two schedules (whole tiles, and K split over a
 // thread-block cluster when there are few tiles) and the exact reduction of
@@ -90,16 +94,23 @@ __device__ __forceinline__ uint16_t bf16_bits_rne(float y) {
 
 // One output element from the MMA sum (16 * acc): scales and bias already
 // loaded by the caller.
-template <int SINK, class P>
+// The accumulator as a float: the W4A4 sum (|acc| <= 2^21) by the exact
+// bit trick, the W8A8 sum (up to 127^2 K) by a correctly rounded conversion.
+template <bool W8>
+__device__ __forceinline__ float acc_to_float(int32_t acc) {
+  return W8 ? __int2float_rn(acc) : int_to_float_exact(acc);
+}
+
+template <int SINK, bool W8, class P>
 __device__ __forceinline__ void store_output(const P& p, int m, int n, int32_t dsum, float sa, float sw,
                                              float bv) {
-  const int32_t acc = dsum >> 4;  // the weights entered the MMA as 16 * q_w
+  const int32_t acc = W8 ? dsum : dsum >> 4;  // 4-bit weights entered the MMA as 16 * q_w
   const size_t idx = static_cast<size_t>(m) * p.N + n;
   if (SINK == static_cast<int>(GemmSink::kS32)) {
     static_cast<int32_t*>(p.out)[idx] = acc;
     return;
   }
-  float y = __fmul_rn(__fmul_rn(int_to_float_exact(acc), sa), sw);
+  float y = __fmul_rn(__fmul_rn(acc_to_float<W8>(acc), sa), sw);
   if (p.bias) y = __fadd_rn(y, bv);
   if (SINK == static_cast<int>(GemmSink::kF32)) {
     static_cast<float*>(p.out)[idx] = y;
@@ -111,7 +122,7 @@ __device__ __forceinline__ void store_output(const P& p, int m, int n, int32_t d
 // Outputs of one 32-token chunk of one output channel n: tokens m .. m +
 // count - 1 (count <= 32), accumulators v (16 * acc), token scales sa[0..31]
 // (16-byte aligned in shared memory).
-template <int SINK, class P>
+template <int SINK, bool W8, class P>
 __device__ __forceinline__ void store_chunk(const P& p, int m, int n, const uint32_t (&v)[32], const float* sa,
                                             float sw, float bv, int count) {
   const size_t ld = static_cast<size_t>(p.N);
@@ -120,7 +131,7 @@ __device__ __forceinline__ void store_chunk(const P& p, int m, int n, const uint
     int32_t* o = static_cast<int32_t*>(p.out) + base;
 #pragma unroll
     for (int j = 0; j < 32; ++j)
-      if (j < count) o[j * ld] = static_cast<int32_t>(v[j]) >> 4;
+      if (j < count) o[j * ld] = W8 ? static_cast<int32_t>(v[j]) : static_cast<int32_t>(v[j]) >> 4;
     return;
   }
   const float4* sa4 = reinterpret_cast<const float4*>(sa);
@@ -132,7 +143,8 @@ __device__ __forceinline__ void store_chunk(const P& p, int m, int n, const uint
     for (int r = 0; r < 4; ++r) {
       const int j = 4 * q + r;
       if (j < count) {
-        float y = __fmul_rn(__fmul_rn(int_to_float_exact(static_cast<int32_t>(v[j]) >> 4), sv[r]), sw);
+        const int32_t acc = W8 ? static_cast<int32_t>(v[j]) : static_cast<int32_t>(v[j]) >> 4;
+        float y = __fmul_rn(__fmul_rn(acc_to_float<W8>(acc), sv[r]), sw);
         if (p.bias) y = __fadd_rn(y, bv);
         if (SINK == static_cast<int>(GemmSink::kF32))
           static_cast<float*>(p.out)[base + j * ld] = y;
@@ -187,6 +199,8 @@ struct PParams {
   int a_slots;      // A slots of 64 columns after the two accumulators
   int splits;       // 1: whole tiles; S > 1: the cluster of S CTAs splits one tile's K
   int pair;         // the MMA thread issues two units per group
+  int sa_stride;    // 0: one activation scale for every row
+  int sw_stride;    // 0: one weight scale for every output channel
 };
 
 struct PHeader {
@@ -219,7 +233,7 @@ __device__ __forceinline__ void unit_next(const PParams& p, int& tile, int& kb) 
   }
 }
 
-template <int SINK>
+template <int SINK, bool W8>
 __global__ void __launch_bounds__(kPThreads, 1)
     w4a4_tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_x,
                         const __grid_constant__ PParams p) {
@@ -227,7 +241,8 @@ __global__ void __launch_bounds__(kPThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int BT = p.BT;
   const int ns = p.nstages;
-  const int stage_bytes = kWTileBytes + BT * kKB;
+  constexpr int kWBytes = W8 ? 2 * kWTileBytes : kWTileBytes;  // weight bytes of a unit
+  const int stage_bytes = kWBytes + BT * kKB;
   const int nas = p.a_slots;
   const uint32_t a_col0 = 2u * static_cast<uint32_t>(p.acc_stride);
   PHeader* hdr = reinterpret_cast<PHeader*>(smem + ns * stage_bytes);
@@ -244,7 +259,9 @@ __global__ void __launch_bounds__(kPThreads, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < ns; ++s) {
       mbar_init(&hdr->wfull[s], 1);
-      mbar_init(&hdr->ready[s], 5);  // the producer (with the activation bytes) + one arrive per unpack warp
+      // W4: the producer (with the activation bytes) + one arrive per unpack
+      // warp; W8: the producer twice (weight bytes, activation bytes).
+      mbar_init(&hdr->ready[s], W8 ? 2 : 5);
     }
     for (int r = 0; r < kDoneRing; ++r) mbar_init(&hdr->done[r], 1);  // one MMA commit
     for (int b = 0; b < 2; ++b) {
@@ -271,11 +288,17 @@ __global__ void __launch_bounds__(kPThreads, 1)
     if (lane == 0) {
       const uint32_t xbytes = static_cast<uint32_t>(BT * kKB);
       auto load_w = [&](int s, int tile, int kb) {
-        mbar_arrive_expect_tx(&hdr->wfull[s], static_cast<uint32_t>(kWTileBytes));
-        tma_load_2d(smem + s * stage_bytes, &tm_w, &hdr->wfull[s], kb * (kKB / 2), w_row(tile));
+        if (W8) {
+          mbar_arrive_expect_tx(&hdr->ready[s], static_cast<uint32_t>(kWBytes));
+          tma_load_2d(smem + s * stage_bytes, &tm_w, &hdr->ready[s], kb * kKB, w_row(tile));
+          tma_load_2d(smem + s * stage_bytes + kWTileBytes, &tm_w, &hdr->ready[s], kb * kKB + kXBox, w_row(tile));
+        } else {
+          mbar_arrive_expect_tx(&hdr->wfull[s], static_cast<uint32_t>(kWTileBytes));
+          tma_load_2d(smem + s * stage_bytes, &tm_w, &hdr->wfull[s], kb * (kKB / 2), w_row(tile));
+        }
       };
       auto load_x = [&](int s, int tile, int kb) {
-        uint8_t* xs = smem + s * stage_bytes + kWTileBytes;
+        uint8_t* xs = smem + s * stage_bytes + kWBytes;
         mbar_arrive_expect_tx(&hdr->ready[s], xbytes);
         tma_load_2d(xs, &tm_x, &hdr->ready[s], kb * kKB, x_row(tile));
         tma_load_2d(xs + BT * kXBox, &tm_x, &hdr->ready[s], kb * kKB + kXBox, x_row(tile));
@@ -304,8 +327,9 @@ __global__ void __launch_bounds__(kPThreads, 1)
       // whose barrier also needs the unpack warps, are given a fixed 100 us.
       bool clean = true;
       for (int i = (it > ns ? it - ns : 0); i < it; ++i) {
-        if (clean) clean = mbar_wait(&hdr->wfull[i % ns], (i / ns) & 1) && mbar_wait(&hdr->ready[i % ns], (i / ns) & 1);
-        if (!clean) (void)mbar_drain(&hdr->wfull[i % ns], (i / ns) & 1, 100000000ull);
+        if (clean)
+          clean = (W8 || mbar_wait(&hdr->wfull[i % ns], (i / ns) & 1)) && mbar_wait(&hdr->ready[i % ns], (i / ns) & 1);
+        if (!clean && !W8) (void)mbar_drain(&hdr->wfull[i % ns], (i / ns) & 1, 100000000ull);
       }
       if (!clean || it < total) {
         const unsigned long long t0 = globaltimer_ns();
@@ -322,7 +346,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
       const bool leader = lane == 0;
       const uint32_t idesc = umma_idesc_i8(kRows, BT, /*a_signed=*/true, /*b_signed=*/true);
       const uint32_t x1 = static_cast<uint32_t>(BT * kXBox);  // second activation box of a stage
-      const uint32_t smem0 = smem_u32(smem) + static_cast<uint32_t>(kWTileBytes);
+      const uint32_t smem0 = smem_u32(smem) + static_cast<uint32_t>(kWBytes);
       int kb = kb0, seg = 0, s = 0, a = 0, sph = 0;
       bool ok = true;
       // The 8 MMAs of the unit in stage s / A slot a (acc0: accumulate into
@@ -330,11 +354,22 @@ __global__ void __launch_bounds__(kPThreads, 1)
       auto issue_unit = [&](uint32_t d_tmem, uint32_t acc0) {
         const uint32_t xs = smem0 + static_cast<uint32_t>(s * stage_bytes);
         const uint64_t bd0 = umma_desc_k_sw128(xs), bd1 = umma_desc_k_sw128(xs + x1);
-        const uint32_t at = tmem + a_col0 + 64u * static_cast<uint32_t>(a);
-        if (leader) {
+        if (W8) {
+          const uint32_t ws = xs - static_cast<uint32_t>(kWBytes);
+          const uint64_t ad0 = umma_desc_k_sw128(ws), ad1 = umma_desc_k_sw128(ws + kWTileBytes);
+          if (leader) {
 #pragma unroll
-          for (int kk = 0; kk < kKB / 32; ++kk)
-            umma_i8_ts(d_tmem, at + 8 * kk, (kk < 4 ? bd0 : bd1) + 2 * (kk & 3), idesc, kk == 0 ? acc0 : 1u);
+            for (int kk = 0; kk < kKB / 32; ++kk)
+              umma_i8_ss(d_tmem, (kk < 4 ? ad0 : ad1) + 2 * (kk & 3), (kk < 4 ? bd0 : bd1) + 2 * (kk & 3), idesc,
+                         kk == 0 ? acc0 : 1u);
+          }
+        } else {
+          const uint32_t at = tmem + a_col0 + 64u * static_cast<uint32_t>(a);
+          if (leader) {
+#pragma unroll
+            for (int kk = 0; kk < kKB / 32; ++kk)
+              umma_i8_ts(d_tmem, at + 8 * kk, (kk < 4 ? bd0 : bd1) + 2 * (kk & 3), idesc, kk == 0 ? acc0 : 1u);
+          }
         }
       };
       auto advance = [&]() {
@@ -388,11 +423,11 @@ __global__ void __launch_bounds__(kPThreads, 1)
       }
     }
   } else if (warp < 6) {
-    // ------------------------------------------------ weight unpack
+    // ------------------------------------------------ weight unpack (4-bit weights only)
     const int quad = warp & 3;
     const int row = quad * 32 + lane;
     const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
-    for (int it = 0, s = 0, ph = 0, a = 0; it < total; ++it) {
+    for (int it = 0, s = 0, ph = 0, a = 0; !W8 && it < total; ++it) {
       bool w = mbar_wait(&hdr->wfull[s], ph & 1);
       if (w && it >= nas) {
         const int u = it - nas;  // the unit that last used A slot a
@@ -432,8 +467,9 @@ __global__ void __launch_bounds__(kPThreads, 1)
       float sw = 0.0f, bv = 0.0f;
       if (p.splits == 1) {
         if (SINK != static_cast<int>(GemmSink::kS32))
-          for (int c = et; c < BT; c += kEpiThreads) sa[c] = (m0 + c < p.M) ? __ldg(p.s_a + m0 + c) : 0.0f;
-        sw = (SINK != static_cast<int>(GemmSink::kS32) && n < p.N) ? __ldg(p.s_w + n) : 0.0f;
+          for (int c = et; c < BT; c += kEpiThreads)
+            sa[c] = (m0 + c < p.M) ? __ldg(p.s_a + (m0 + c) * p.sa_stride) : 0.0f;
+        sw = (SINK != static_cast<int>(GemmSink::kS32) && n < p.N) ? __ldg(p.s_w + n * p.sw_stride) : 0.0f;
         bv = (p.bias && n < p.N) ? __uint_as_float(static_cast<uint32_t>(__ldg(p.bias + n)) << 16) : 0.0f;
         named_barrier(1, kEpiThreads);  // s_a staged; all warps are done with segment seg - 2
       }
@@ -450,7 +486,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
           tmem_ld_32x32b_x32(acc + static_cast<uint32_t>(c), v);
           tmem_wait_ld();
           const int count = min(min(32, BT - c), p.M - (m0 + c));
-          if (n < p.N && count > 0) store_chunk<SINK>(p, m0 + c, n, v, sa + c, sw, bv, count);
+          if (n < p.N && count > 0) store_chunk<SINK, W8>(p, m0 + c, n, v, sa + c, sw, bv, count);
         }
       } else {
         // Push the partial tile to its owners: 4-token group g belongs to CTA
@@ -492,8 +528,9 @@ __global__ void __launch_bounds__(kPThreads, 1)
       const int n = (tile0 / p.m_tiles) * kRows + (warp & 3) * 32 + lane;
       const int m0 = (tile0 % p.m_tiles) * BT;
       if (SINK != static_cast<int>(GemmSink::kS32)) {
-        for (int c = threadIdx.x - 192; c < BT; c += kEpiThreads) sa_buf[c] = (m0 + c < p.M) ? __ldg(p.s_a + m0 + c) : 0.0f;
-        sw_red = n < p.N ? __ldg(p.s_w + n) : 0.0f;
+        for (int c = threadIdx.x - 192; c < BT; c += kEpiThreads)
+          sa_buf[c] = (m0 + c < p.M) ? __ldg(p.s_a + (m0 + c) * p.sa_stride) : 0.0f;
+        sw_red = n < p.N ? __ldg(p.s_w + n * p.sw_stride) : 0.0f;
       }
       bv_red = (p.bias && n < p.N) ? __uint_as_float(static_cast<uint32_t>(__ldg(p.bias + n)) << 16) : 0.0f;
     }
@@ -529,7 +566,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
           const int m = m0 + 4 * g + q;
           if (m < p.M) {
             const float sa = SINK != static_cast<int>(GemmSink::kS32) ? sa_buf[m - m0] : 0.0f;
-            store_output<SINK>(p, m, n, sv[q], sa, sw, bv);
+            store_output<SINK, W8>(p, m, n, sv[q], sa, sw, bv);
           }
         }
       }
@@ -578,11 +615,11 @@ bool make_map_u8(CUtensorMap* map, const void* base, uint64_t rows, uint64_t col
   return r == CUDA_SUCCESS;
 }
 
-template <int SINK>
+template <int SINK, bool W8>
 cudaError_t launch_sink(const CUtensorMap& tw, const CUtensorMap& tx, const PParams& prm, const GemmTiling& t,
                         cudaStream_t stream) {
   static int cache[64] = {0};
-  const void* kfn = reinterpret_cast<const void*>(w4a4_tc_gemm_kernel<SINK>);
+  const void* kfn = reinterpret_cast<const void*>(w4a4_tc_gemm_kernel<SINK, W8>);
   cudaError_t e = ensure_dynamic_smem(kfn, t.smem_bytes, cache);
   if (e != cudaSuccess) return note_cuda(e, "w4a4_gemm: dynamic shared memory attribute");
   cudaLaunchConfig_t cfg = {};
@@ -604,7 +641,7 @@ cudaError_t launch_sink(const CUtensorMap& tw, const CUtensorMap& tx, const PPar
   }
   cfg.attrs = attr;
   cfg.numAttrs = nattr;
-  return note_cuda(cudaLaunchKernelEx(&cfg, w4a4_tc_gemm_kernel<SINK>, tw, tx, prm), "w4a4_gemm: launch");
+  return note_cuda(cudaLaunchKernelEx(&cfg, w4a4_tc_gemm_kernel<SINK, W8>, tw, tx, prm), "w4a4_gemm: launch");
 }
 
 // Clusters of S CTAs (one CTA per SM) that can be resident at once on the
@@ -616,7 +653,7 @@ int max_active_clusters(int S, int num_sms) {
   if (cache[dev][S] > 0) return cache[dev][S];
   static int smem_cache[64] = {0};
   const int smem = 200 * 1024;
-  const void* kfn = reinterpret_cast<const void*>(w4a4_tc_gemm_kernel<0>);
+  const void* kfn = reinterpret_cast<const void*>(w4a4_tc_gemm_kernel<0, false>);
   int n = 0;
   if (ensure_dynamic_smem(kfn, smem, smem_cache) == cudaSuccess) {
     cudaLaunchConfig_t cfg = {};
@@ -630,7 +667,7 @@ int max_active_clusters(int S, int num_sms) {
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (cudaOccupancyMaxActiveClusters(&n, w4a4_tc_gemm_kernel<0>, &cfg) != cudaSuccess) n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, w4a4_tc_gemm_kernel<0, false>, &cfg) != cudaSuccess) n = 0;
   }
   cudaGetLastError();  // a failed query is not an error of the caller
   if (n <= 0) n = num_sms / (2 * S);
@@ -662,8 +699,8 @@ int red_bytes(int BT, int S) { return S > 1 ? S * ((BT / 4 + S - 1) / S) * kRows
 // header (1 KB), the s_a staging (1.5 KB) and the split-K buffer, and the
 // dynamic shared memory for them (padded so that one CTA, which owns all of
 // tensor memory, occupies an SM).
-void set_stages(GemmTiling& t) {
-  const int stage = kWTileBytes + t.BT * kKB;
+void set_stages(GemmTiling& t, bool w8) {
+  const int stage = (w8 ? 2 : 1) * kWTileBytes + t.BT * kKB;
   const int rb = red_bytes(t.BT, t.splits);
   int ns = (220 * 1024 - 4096 - rb) / stage;
   if (ns > kMaxStages) ns = kMaxStages;
@@ -679,7 +716,7 @@ void set_stages(GemmTiling& t) {
 
 }  // namespace
 
-GemmTiling choose_tiling(int M, int N, int K, int num_sms) {
+GemmTiling choose_tiling(int M, int N, int K, int num_sms, bool w8) {
   GemmTiling t{};
   const int kbn = K / kKB;
   const int G = num_sms < kMaxGemmGrid ? num_sms : kMaxGemmGrid;
@@ -705,7 +742,7 @@ GemmTiling choose_tiling(int M, int N, int K, int num_sms) {
       t.m_tiles = (M + best_bt - 1) / best_bt;
       const int tiles = t.m_tiles * t.n_tiles;
       t.grid = tiles < G ? tiles : G;
-      set_stages(t);
+      set_stages(t, w8);
       return t;
     }
   }
@@ -733,14 +770,14 @@ GemmTiling choose_tiling(int M, int N, int K, int num_sms) {
     }
   }
   t.grid = t.splits > 1 ? tiles * t.splits : (tiles < G ? tiles : G);
-  set_stages(t);
+  set_stages(t, w8);
   return t;
 }
 
 cudaError_t launch_w4a4_gemm(const GemmArgs& a, GemmSink sink, const GemmTiling& t, cudaStream_t stream) {
   CUtensorMap tw, tx;
-  if (!make_map_u8(&tw, a.Wq, static_cast<uint64_t>(a.N), static_cast<uint64_t>(a.K / 2), kRows, kKB / 2,
-                   CU_TENSOR_MAP_SWIZZLE_128B))
+  if (!make_map_u8(&tw, a.Wq, static_cast<uint64_t>(a.N), static_cast<uint64_t>(a.w8 ? a.K : a.K / 2), kRows,
+                   a.w8 ? kXBox : kKB / 2, CU_TENSOR_MAP_SWIZZLE_128B))
     return note_cuda(cudaErrorInvalidValue, "w4a4_gemm: weight tensor map");
   if (!make_map_u8(&tx, a.xs8, static_cast<uint64_t>(a.M), static_cast<uint64_t>(a.K),
                    static_cast<uint32_t>(t.BT), kXBox, CU_TENSOR_MAP_SWIZZLE_128B))
@@ -764,12 +801,22 @@ cudaError_t launch_w4a4_gemm(const GemmArgs& a, GemmSink sink, const GemmTiling&
   pp.acc_stride = t.acc_stride;
   pp.a_slots = t.a_slots;
   pp.splits = t.splits;
-  pp.pair = (t.BT <= 128 && t.a_slots >= 4 && t.nstages >= 4) ? 1 : 0;
+  pp.pair = (t.BT <= 128 && (a.w8 || t.a_slots >= 4) && t.nstages >= 4) ? 1 : 0;
+  pp.sa_stride = a.sa_stride;
+  pp.sw_stride = a.sw_stride;
   cudaError_t e;
-  switch (sink) {
-    case GemmSink::kBF16: e = launch_sink<0>(tw, tx, pp, t, stream); break;
-    case GemmSink::kF32: e = launch_sink<1>(tw, tx, pp, t, stream); break;
-    default: e = launch_sink<2>(tw, tx, pp, t, stream); break;
+  if (a.w8) {
+    switch (sink) {
+      case GemmSink::kBF16: e = launch_sink<0, true>(tw, tx, pp, t, stream); break;
+      case GemmSink::kF32: e = launch_sink<1, true>(tw, tx, pp, t, stream); break;
+      default: e = launch_sink<2, true>(tw, tx, pp, t, stream); break;
+    }
+  } else {
+    switch (sink) {
+      case GemmSink::kBF16: e = launch_sink<0, false>(tw, tx, pp, t, stream); break;
+      case GemmSink::kF32: e = launch_sink<1, false>(tw, tx, pp, t, stream); break;
+      default: e = launch_sink<2, false>(tw, tx, pp, t, stream); break;
+    }
   }
   count_dispatch(t.splits > 1 ? 3 : 2);
   return e;

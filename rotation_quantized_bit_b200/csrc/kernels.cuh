@@ -18,7 +18,14 @@ struct RotateQuantOut {
   uint8_t* packed;  // [M, K/2] two codes per byte, or null
   int8_t* s8;       // [M, K] codes as signed bytes in chunk order (0,2,4,6,1,3,5,7), or null
   float* scale;     // [M]
+  bool int8 = false;  // s8 holds 8-bit codes (amax / 127) in natural order instead
 };
+
+// The int8_tensorwise quantizer: one scale s = amax|x| / 127 for the whole
+// [rows, K] tensor, codes clamp(rint(x / s), -127, 127), no rotation.
+// scratch: 4 bytes of device memory (the amax while it is reduced).
+cudaError_t launch_quant8_tensorwise(const uint16_t* x, size_t n, int8_t* codes, float* scale, uint32_t* scratch,
+                                     cudaStream_t stream);
 
 cudaError_t launch_rotate_quant(const uint16_t* x, int M, int K, RotateQuantOut out, cudaStream_t stream);
 
@@ -41,16 +48,21 @@ struct GemmTiling {
   int a_slots;      // 64-column tensor-memory slots for unpacked weights
 };
 
-GemmTiling choose_tiling(int M, int N, int K, int num_sms);
+// w8: the weights are int8 codes [N, K] (the W8A8 formats) instead of packed
+// 4-bit codes [N, K/2].
+GemmTiling choose_tiling(int M, int N, int K, int num_sms, bool w8 = false);
 
 struct GemmArgs {
-  const int8_t* xs8;      // [M, K] activation codes (operand layout)
-  const float* s_a;       // [M]   (ignored by the s32 sink)
-  const uint8_t* Wq;      // [N, K/2] packed weight codes
-  const float* s_w;       // [N]
+  const int8_t* xs8;      // [M, K] activation codes (operand layout; natural order with w8)
+  const float* s_a;       // [M], or [1] with sa_stride 0 (ignored by the s32 sink)
+  const uint8_t* Wq;      // [N, K/2] packed weight codes, or [N, K] int8 codes with w8
+  const float* s_w;       // [N], or [1] with sw_stride 0
   const uint16_t* bias;   // [N] or null
   void* out;              // [M, N] bf16 / f32 / s32
   int M, N, K;
+  int w8 = 0;             // 1: int8 weights (W8A8)
+  int sa_stride = 1;      // 0: one activation scale for every row
+  int sw_stride = 1;      // 0: one weight scale for every output channel
 };
 
 // Builds the tensor maps and launches the tensor-core GEMM.
