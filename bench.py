@@ -46,7 +46,11 @@ WORKLOAD_DESC = {
     "edit20b": "20B image-edit DiT linears (to_q/k/v/out, mlp up/down; hidden 3072), M=8704",
     "small_m": "small-M sweep, M in {1,8,16,64,128} x (K,N) in {(2560,9728),(9728,2560),(3072,12288),(12288,3072)}",
     "small": "single linear M=32, K=512, N=256",
+    "edit20b_int8": "20B image-edit DiT value/output projections (3072x3072) in int8_tensorwise W8A8, M=8704",
+    "qwen3_4b_mixed": "Qwen3-4B layer at M=76 and M=1220: q,k,v,o in ConvRot INT8 (row-scaled) W8A8, "
+                      "gate,up,down in ConvRot W4A4",
 }
+FORMAT_ID = {"int8_tensorwise": 0, "convrot_int8": 1}  # w8a8_format_t
 L2_FLUSH_BYTES = 256 << 20
 INT8_PER_BF16 = 2.0  # nominal dense int8 : bf16 tensor throughput (4.5 : 2.25 PFLOP/s)
 
@@ -72,9 +76,20 @@ def step_ops(shapes):
     return sum(2.0 * s.M * s.N * s.K for s in shapes)
 
 
+def weight_bytes(s):
+    """Bytes of the stored weight codes: 4-bit packed, or int8."""
+    return s.N * s.K // 2 if s.fmt == "w4a4" else s.N * s.K
+
+
 def alg_bytes(s):
-    """Algorithmic HBM bytes of one fused linear: x, packed W, s_w, bias, y."""
-    return 2 * s.M * s.K + s.N * s.K // 2 + 4 * s.N + 2 * s.N + 2 * s.M * s.N
+    """Algorithmic HBM bytes of one fused linear: x, W codes, s_w, bias, y."""
+    return 2 * s.M * s.K + weight_bytes(s) + 4 * s.N + 2 * s.N + 2 * s.M * s.N
+
+
+def gemm_alg_bytes(s):
+    """Algorithmic bytes of the GEMM launch: W codes, activation codes as bytes,
+    scales, bias, y."""
+    return weight_bytes(s) + s.M * s.K + 4 * s.M + 6 * s.N + 2 * s.M * s.N
 
 
 def load_peaks():
@@ -164,24 +179,40 @@ class ClockSampler:
 
 # ------------------------------------------------------------------ the oracle leg
 
+def oracle_inputs(oracle, workload, s):
+    """(shape, x, weight codes, weight scales, bias) for the oracle, prepared
+    in the linear's format (weight preparation is not timed)."""
+    x = synthetic.activations(workload, s.M, s.K, seed_extra=synthetic.source_seed(s.source))
+    w, b = synthetic.weights(workload, s.N, s.K, seed_extra=synthetic.source_seed(s.name))
+    if s.fmt == "w4a4":
+        wq, s_w = oracle.pack_weight(w)
+    else:
+        wq, s_w = oracle.quant8(w, *ORACLE_FORMAT[s.fmt])
+    return s, x, wq, s_w, b
+
+
+ORACLE_FORMAT = {"int8_tensorwise": (0, False), "convrot_int8": (256, True)}  # (group, per_row)
+
+
+def oracle_linear(oracle, s, x, wq, s_w, b):
+    if s.fmt == "w4a4":
+        return oracle.linear(x, wq, s_w, b, s.K)
+    return oracle.linear8(x, wq, s_w, b, *ORACLE_FORMAT[s.fmt])
+
+
 def cpu_baseline(shapes, workload, budget_s=15.0):
     """Time the CPU oracle (single thread, as it stands) on a bounded sample:
     the first ``r`` rows of each linear of the step, r grown until the run
     takes about ``budget_s``; throughput in the metric's unit (TOPS)."""
     import oracle
-    inputs = []
-    for s in shapes:
-        x = synthetic.activations(workload, s.M, s.K)
-        w, b = synthetic.weights(workload, s.N, s.K)
-        wq, s_w = oracle.pack_weight(w)
-        inputs.append((s, x, wq, s_w, b))
+    inputs = [oracle_inputs(oracle, workload, s) for s in shapes]
     rows = 1
     while True:
         t0 = time.perf_counter()
         ops = 0.0
         for s, x, wq, s_w, b in inputs:
             r = min(rows, s.M)
-            oracle.linear(x[:r], wq, s_w, b, s.K)
+            oracle_linear(oracle, s, x[:r], wq, s_w, b)
             ops += 2.0 * r * s.N * s.K
         dt = time.perf_counter() - t0
         if dt >= budget_s / 3 or rows >= max(s.M for s in shapes):
@@ -248,7 +279,10 @@ def main():
     for s in shapes:
         w, b = synthetic.weights(args.workload, s.N, s.K, seed_extra=synthetic.source_seed(s.name))
         wd = torch.from_numpy(w.view(np.int16)).view(torch.bfloat16).to(dev)
-        wq, s_w = rq.convrot_pack_weight(wd)
+        if s.fmt == "w4a4":
+            wq, s_w = rq.convrot_pack_weight(wd)
+        else:
+            wq, s_w = rq.w8a8_pack_weight(wd, FORMAT_ID[s.fmt])
         bias = torch.from_numpy(b.view(np.int16)).view(torch.bfloat16).to(dev)
         y = torch.empty((s.M, s.N), dtype=torch.bfloat16, device=dev)
         layers.append((s, wq, s_w, bias, y))
@@ -262,8 +296,15 @@ def main():
                 break
         else:
             groups.append((s.source, [i]))
-    ws_bytes = max(rq.convrot_w4a4_workspace_size(s.M, s.N, s.K) for s in shapes)
+    ws_bytes = max(rq.convrot_w4a4_workspace_size(s.M, s.N, s.K) if s.fmt == "w4a4"
+                   else rq.w8a8_workspace_size(s.M, s.N, s.K, FORMAT_ID[s.fmt]) for s in shapes)
     ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    # int8 formats: the activation codes and scales of each source
+    q8 = {}
+    for s in shapes:
+        if s.fmt != "w4a4" and s.source not in q8:
+            q8[s.source] = (torch.empty((s.M, s.K), dtype=torch.int8, device=dev),
+                            torch.empty((s.M if s.fmt == "convrot_int8" else 1,), dtype=torch.float32, device=dev))
     flush = make_flusher(torch, dev, args.flush)
     stream = torch.cuda.current_stream()
     torch.cuda.synchronize()
@@ -282,12 +323,19 @@ def main():
             ev = evs[gi] if evs is not None else None
             if ev is not None:
                 ev[0].record(cur)
-            rq.convrot_w4a4_quantize(xs[src], ws)
+            fmt = layers[idx[0]][0].fmt
+            if fmt == "w4a4":
+                rq.convrot_w4a4_quantize(xs[src], ws)
+            else:
+                rq.w8a8_quantize(xs[src], FORMAT_ID[fmt], x8=q8[src][0], s_x=q8[src][1], workspace=ws)
             if ev is not None and per_kernel:
                 ev[1].record(cur)
             for j, i in enumerate(idx):
                 s, wq, s_w, bias, y = layers[i]
-                rq.convrot_w4a4_gemm_quantized(ws, s.M, wq, s_w, bias, out=y)
+                if fmt == "w4a4":
+                    rq.convrot_w4a4_gemm_quantized(ws, s.M, wq, s_w, bias, out=y)
+                else:
+                    rq.w8a8_gemm(q8[src][0], q8[src][1], wq, s_w, bias, FORMAT_ID[fmt], out=y)
                 if ev is not None and (per_kernel or j == len(idx) - 1):
                     ev[2 + j].record(cur)
 
@@ -388,14 +436,14 @@ def main():
         s0 = layers[idx[0]][0]
         tq, tgrp = t_quant[gi] / args.steps, t_grp[gi] / args.steps
         gops = sum(2.0 * layers[i][0].M * layers[i][0].N * layers[i][0].K for i in idx)
-        entry = {"input": src, "M": s0.M, "K": s0.K, "us_group": round(tgrp * 1e3, 2),
+        entry = {"input": src, "format": s0.fmt, "M": s0.M, "K": s0.K, "us_group": round(tgrp * 1e3, 2),
                  "tops_group": round(gops / (tgrp * 1e-3) / 1e12, 1), "us_prologue": round(tq * 1e3, 2),
                  "prologue_hbm_gbs": round((3.0 * s0.M * s0.K + 4 * s0.M) / (tq * 1e-3) / 1e9, 1), "linears": []}
         for i in idx:
             s = layers[i][0]
             tg = t_gemm[i] / args.steps
             op = 2.0 * s.M * s.N * s.K
-            gemm_bytes = s.N * s.K // 2 + s.M * s.K + 4 * s.M + 6 * s.N + 2 * s.M * s.N
+            gemm_bytes = gemm_alg_bytes(s)
             entry["linears"].append({
                 "linear": s.name, "N": s.N, "us_gemm": round(tg * 1e3, 2),
                 "gemm_tops": round(op / (tg * 1e-3) / 1e12, 1),
@@ -409,7 +457,7 @@ def main():
     if kind == "gemm":
         s = layers[idx][0]
         ridge = int8_peak * 1e12 / (peaks["hbm_gbs"] * 1e9)
-        gemm_bytes = s.N * s.K // 2 + s.M * s.K + 4 * s.M + 6 * s.N + 2 * s.M * s.N
+        gemm_bytes = gemm_alg_bytes(s)
         intensity = 2.0 * s.M * s.N * s.K / gemm_bytes
         if intensity >= ridge:
             roof = {"bound": "tensor", "achieved": 2.0 * s.M * s.N * s.K / t_launch / 1e12,
@@ -496,14 +544,24 @@ def end_to_end(args, rq, torch, dev, stream, shapes, xs, layers, groups, ws, flu
         for k, v in host_x.items():
             xs[k].copy_(v, non_blocking=True)
         for src, idx in groups:
+            fmt = layers[idx[0]][0].fmt
             if len(idx) == 1:
                 s, wq, s_w, bias, y = layers[idx[0]]
-                rq.convrot_w4a4_linear(xs[src], wq, s_w, bias, out=y, workspace=ws)
+                if fmt == "w4a4":
+                    rq.convrot_w4a4_linear(xs[src], wq, s_w, bias, out=y, workspace=ws)
+                else:
+                    rq.w8a8_linear(xs[src], wq, s_w, bias, FORMAT_ID[fmt], out=y, workspace=ws)
                 continue
-            rq.convrot_w4a4_quantize(xs[src], ws)
+            if fmt == "w4a4":
+                rq.convrot_w4a4_quantize(xs[src], ws)
+            else:
+                x8, sx = rq.w8a8_quantize(xs[src], FORMAT_ID[fmt], workspace=ws)
             for i in idx:
                 s, wq, s_w, bias, y = layers[i]
-                rq.convrot_w4a4_gemm_quantized(ws, s.M, wq, s_w, bias, out=y)
+                if fmt == "w4a4":
+                    rq.convrot_w4a4_gemm_quantized(ws, s.M, wq, s_w, bias, out=y)
+                else:
+                    rq.w8a8_gemm(x8, sx, wq, s_w, bias, FORMAT_ID[fmt], out=y)
         for (s, wq, s_w, bias, y), hy in zip(layers, host_y):
             hy.copy_(y, non_blocking=True)
 
@@ -539,19 +597,14 @@ def reference_arm(args, shapes, config, world, rank):
     if rank != 0:
         return
     import oracle
-    inputs = []
-    for s in shapes:
-        x = synthetic.activations(args.workload, s.M, s.K)
-        w, b = synthetic.weights(args.workload, s.N, s.K)
-        wq, s_w = oracle.pack_weight(w)
-        inputs.append((s, x, wq, s_w, b))
+    inputs = [oracle_inputs(oracle, args.workload, s) for s in shapes]
     rows = 2  # rows per linear per step: keeps a step near a few seconds
 
     def step():
         ops = 0.0
         for s, x, wq, s_w, b in inputs:
             r = min(rows, s.M)
-            oracle.linear(x[:r], wq, s_w, b, s.K)
+            oracle_linear(oracle, s, x[:r], wq, s_w, b)
             ops += 2.0 * r * s.N * s.K
         return ops
 

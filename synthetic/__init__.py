@@ -157,6 +157,9 @@ class LinearShape:
     # the same tensor (q/k/v; gate/up) share it, and one rotate + quantize
     # of it serves all of them.
     input: str = ""
+    # Weight/activation format: "w4a4" (ConvRot W4A4), "int8_tensorwise" or
+    # "convrot_int8" (the int8 W8A8 formats the pages mix with W4A4).
+    fmt: str = "w4a4"
 
     @property
     def source(self) -> str:
@@ -169,8 +172,11 @@ _ACT = {
     "dit6b": act_laplace_lognormal,
     "edit20b": act_t4_outliers,
     "small_m": act_t4_outliers,
+    "edit20b_int8": act_t4_outliers,
+    "qwen3_4b_mixed": act_t4_outliers,
 }
-_BASE_SEED = {"small": 0, "qwen3_4b": 1, "dit6b": 2, "edit20b": 3, "small_m": 4}
+_BASE_SEED = {"small": 0, "qwen3_4b": 1, "dit6b": 2, "edit20b": 3, "small_m": 4, "edit20b_int8": 3,
+              "qwen3_4b_mixed": 1}
 
 
 def workload_shapes(workload: str) -> list[LinearShape]:
@@ -193,6 +199,19 @@ def workload_shapes(workload: str) -> list[LinearShape]:
                ("to_out", 3072, 3072, "attn_out"), ("mlp_up", 3072, 12288, "mlp_in"),
                ("mlp_down", 12288, 3072, "mlp_act")]
         return [LinearShape(n, M, K, N, src) for (n, K, N, src) in lin]
+    if workload == "edit20b_int8":
+        # the value / output projections of the 20B edit DiT in stock int8_tensorwise
+        M = 8192 + 512
+        return [LinearShape("to_v", M, 3072, 3072, "attn_in", "int8_tensorwise"),
+                LinearShape("to_out", M, 3072, 3072, "attn_out", "int8_tensorwise")]
+    if workload == "qwen3_4b_mixed":
+        # the Qwen3-4B layer with its attention projections in ConvRot INT8
+        # (row-scaled) and its MLP in W4A4
+        out = []
+        for s in workload_shapes("qwen3_4b"):
+            fmt = "convrot_int8" if s.name.split("@")[0] in ("q_proj", "k_proj", "v_proj", "o_proj") else "w4a4"
+            out.append(dataclasses.replace(s, fmt=fmt))
+        return out
     if workload == "small_m":
         kn = [(2560, 9728), (9728, 2560), (3072, 12288), (12288, 3072)]
         return [LinearShape(f"k{K}_n{N}@{M}", M, K, N) for M in (1, 8, 16, 64, 128) for (K, N) in kn]
