@@ -239,6 +239,11 @@ __global__ void __launch_bounds__(kPThreads, 1)
                         const __grid_constant__ PParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  // The next kernel on the stream (launched with programmatic stream
+  // serialization: another GEMM, or a prologue) may start now and prepare
+  // what does not depend on this grid; it waits for this grid's completion
+  // (griddepcontrol.wait) before touching anything this grid reads or writes.
+  pdl_launch_dependents();
   const int BT = p.BT;
   const int ns = p.nstages;
   constexpr int kWBytes = W8 ? 2 * kWTileBytes : kWTileBytes;  // weight bytes of a unit
@@ -677,14 +682,16 @@ int max_active_clusters(int S, int num_sms) {
 
 // Estimated cycles of the whole-tile schedule for a token tile of BT: rounds
 // of tiles per SM x units x the slower of the MMA (4 * BT cycles per 256-K
-// unit at 8192 int8 MACs/clk) and a per-unit floor of about 900 cycles
-// (measured) that every unit costs whatever BT is: issuing 8 MMAs and a
-// commit, fetching and unpacking the 16 KB weight tile.
-long persistent_cost(int M, int N, int K, int BT, int num_sms) {
+// unit at 8192 int8 MACs/clk) and the unit's operand delivery into shared
+// memory plus the unit's fixed costs, fitted to measured runs of this kernel
+// as about 700 + 3.2 * BT cycles (the BT-dependent part is the BT x 256
+// activation bytes); with int8 weights the weight tile is twice as large.
+long persistent_cost(int M, int N, int K, int BT, int num_sms, bool w8) {
   const long tiles = static_cast<long>((M + BT - 1) / BT) * ((N + kRows - 1) / kRows);
   const long rounds = (tiles + num_sms - 1) / num_sms;
-  const long per_unit = 4L * BT > 900 ? 4L * BT : 900;
-  return rounds * (K / kKB) * per_unit;
+  const long mma = 4L * BT;
+  const long data = (w8 ? 1030L : 700L) + (32L * BT) / 10;
+  return rounds * (K / kKB) * (mma > data ? mma : data);
 }
 
 }  // namespace
@@ -731,7 +738,7 @@ GemmTiling choose_tiling(int M, int N, int K, int num_sms, bool w8) {
     for (int bt = 192; bt >= 64; bt -= 16) {
       const long tiles = static_cast<long>((M + bt - 1) / bt) * t.n_tiles;
       if (2 * tiles < G) continue;
-      const long c = persistent_cost(M, N, K, bt, G);
+      const long c = persistent_cost(M, N, K, bt, G, w8);
       if (best < 0 || c < best) {
         best = c;
         best_bt = bt;

@@ -170,7 +170,10 @@ __global__ void __launch_bounds__(kMaxThreads) rotate_quant_kernel(const __grid_
   __shared__ uint32_t row_amax[3][kMaxRows];
   // Let the dependent GEMM launch now: it streams its weights meanwhile and
   // waits (griddepcontrol.wait) for this grid before reading codes or scales.
+  // This grid itself may have been launched before the preceding kernel
+  // finished: wait for it before reading x or writing any output.
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   // Parameters in registers (the inline-asm memory clobbers below would
   // otherwise reload them).
   const int M = p.M, K = p.K, G = p.G, R = p.R, S = p.S;
@@ -194,19 +197,19 @@ __global__ void __launch_bounds__(kMaxThreads) rotate_quant_kernel(const __grid_
   const int nb = p.nblocks;
   const int iters = static_cast<int>(blockIdx.x) < nb ? (nb - 1 - static_cast<int>(blockIdx.x)) / gridDim.x + 1 : 0;
 
-  // Thread 0: the bulk copy of this block's row block number `it`.
-  auto issue = [&](int it) {
+  // Thread 0: the bulk copy of this block's row block number `it` into
+  // stage `st` (= it mod S).
+  auto issue = [&](int it, int st) {
     const int b = static_cast<int>(blockIdx.x) + it * static_cast<int>(gridDim.x);
     const int rows = min(R, M - b * R);
     const uint32_t bytes = static_cast<uint32_t>(rows) * static_cast<uint32_t>(K) * 2u;
-    uint64_t* bar = &full[it % S];
-    mbar_arrive_expect_tx(bar, bytes);
-    bulk_load(stages + (it % S) * stage_bytes, x + static_cast<size_t>(b) * R * K, bytes, bar);
+    mbar_arrive_expect_tx(&full[st], bytes);
+    bulk_load(stages + st * stage_bytes, x + static_cast<size_t>(b) * R * K, bytes, &full[st]);
   };
   if (threadIdx.x == 0) {
-    for (int s = 0; s < S; ++s) mbar_init(&full[s], 1);
+    for (int st = 0; st < S; ++st) mbar_init(&full[st], 1);
     fence_mbarrier_init();
-    for (int it = 0; it < S && it < iters; ++it) issue(it);
+    for (int it = 0; it < S && it < iters; ++it) issue(it, it);
   }
   for (int i = threadIdx.x; i < 3 * kMaxRows; i += blockDim.x) (&row_amax[0][0])[i] = 0u;
   __syncthreads();
@@ -223,12 +226,15 @@ __global__ void __launch_bounds__(kMaxThreads) rotate_quant_kernel(const __grid_
   const size_t out1 = static_cast<size_t>(rloc1) * code_row + (PACKED ? g1 * 128 + l * 8 : g1 * 256 + l * 16);
   uint8_t* const codes = PACKED ? out.packed : reinterpret_cast<uint8_t*>(out.s8);
 
-  int it = 0;
+  // Loop counters kept incrementally (no division by runtime values): the
+  // stage st = it mod S with its phase parity ph, the amax slot = it mod 3,
+  // and the first row of the row block.
+  int it = 0, st = 0, ph = 0, slot = 0;
+  int row0 = static_cast<int>(blockIdx.x) * R;
+  const int row_step = static_cast<int>(gridDim.x) * R;
   for (; it < iters; ++it) {
-    const int row0 = (static_cast<int>(blockIdx.x) + it * static_cast<int>(gridDim.x)) * R;
-    const int slot = it % 3;
-    const bool ok = mbar_wait(&full[it % S], (it / S) & 1);
-    const uint8_t* stage = stages + (it % S) * stage_bytes;
+    const bool ok = mbar_wait(&full[st], ph);
+    const uint8_t* stage = stages + st * stage_bytes;
     const bool live0 = ok && have0 && row0 + rloc0 < M;
     const bool live1 = ok && have1 && row0 + rloc1 < M;
 
@@ -294,18 +300,29 @@ __global__ void __launch_bounds__(kMaxThreads) rotate_quant_kernel(const __grid_
     if (!__syncthreads_and(ok)) break;
     if (threadIdx.x == 0 && it + S < iters) {
       fence_proxy_async_smem();
-      issue(it + S);
+      issue(it + S, st);
     }
     // Slot (it + 2) % 3 was last read in iteration it - 1 and is next written
     // in iteration it + 2, after one more barrier.
-    if (threadIdx.x < kMaxRows) row_amax[(it + 2) % 3][threadIdx.x] = 0u;
+    if (threadIdx.x < kMaxRows) row_amax[slot == 0 ? 2 : slot - 1][threadIdx.x] = 0u;
 
-    // ---- quantize
-    const float scale0 = __fdiv_rn(__uint_as_float(row_amax[slot][rloc0]), kQMax);
-    const float scale1 = __fdiv_rn(__uint_as_float(row_amax[slot][rloc1]), kQMax);
+    // ---- quantize: lane 0 of the task forms the scale (one IEEE division)
+    // and its reciprocal; the half-warp shares them.
+    float scale0 = 0.0f, scale1 = 0.0f, rcp0 = 0.0f, rcp1 = 0.0f;
+    if (l == 0) {
+      scale0 = __fdiv_rn(__uint_as_float(row_amax[slot][rloc0]), kQMax);
+      scale1 = __fdiv_rn(__uint_as_float(row_amax[slot][rloc1]), kQMax);
+      rcp0 = __frcp_rn(scale0);
+      rcp1 = __frcp_rn(scale1);
+    }
+    const int src = threadIdx.x & 16;  // lane 0 of this half-warp
+    scale0 = __shfl_sync(0xffffffffu, scale0, src);
+    scale1 = __shfl_sync(0xffffffffu, scale1, src);
+    rcp0 = __shfl_sync(0xffffffffu, rcp0, src);
+    rcp1 = __shfl_sync(0xffffffffu, rcp1, src);
     uint32_t c0[16], c1[16];  // code bytes (low byte) of channel 16 i + l
     if (scale0 >= kMinScale && scale1 >= kMinScale) {
-      const u64 rr = f2(__frcp_rn(scale0), __frcp_rn(scale1)), ns = f2(-scale0, -scale1);
+      const u64 rr = f2(rcp0, rcp1), ns = f2(-scale0, -scale1);
       const u64 mg = f2(kMagic, kMagic);
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
@@ -355,6 +372,12 @@ __global__ void __launch_bounds__(kMaxThreads) rotate_quant_kernel(const __grid_
         *reinterpret_cast<uint4*>(codes + obase + out1) = o1;
       if (g1 == 0 && l == 0) out.scale[row0 + rloc1] = scale1;
     }
+    if (++st == S) {
+      st = 0;
+      ph ^= 1;
+    }
+    slot = slot == 2 ? 0 : slot + 1;
+    row0 += row_step;
   }
   if (it < iters && threadIdx.x == 0) {
     // A wait gave up: let the copies still in flight land before the block
@@ -409,8 +432,19 @@ cudaError_t launch_rq(const RQParams& p, int threads, cudaStream_t stream) {
   if (per_sm < 1) per_sm = 1;
   int grid = num_sms_cached() * per_sm;
   if (grid > p.nblocks) grid = p.nblocks;
-  rotate_quant_kernel<MODE><<<grid, threads, smem, stream>>>(p);
-  return note_cuda(cudaGetLastError(), "rotate_quant: launch");
+  // Programmatic stream serialization: the kernel may launch while the
+  // preceding one finishes (it waits for it with griddepcontrol.wait).
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid, 1, 1);
+  cfg.blockDim = dim3(threads, 1, 1);
+  cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return note_cuda(cudaLaunchKernelEx(&cfg, rotate_quant_kernel<MODE>, p), "rotate_quant: launch");
 }
 
 }  // namespace
