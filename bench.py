@@ -66,6 +66,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--only", default=None, help="restrict the workload to the linear with this name")
     ap.add_argument("--no-graph", action="store_true", help="launch the step eagerly instead of replaying a CUDA graph")
+    ap.add_argument("--group", type=int, default=256, choices=[256, 64, 16],
+                    help="ConvRot rotation group of the W4A4 linears (the convrot_groupsize variants)")
     ap.add_argument("--flush", choices=["write+read", "write"], default="write+read",
                     help="L2 flush between timed steps: a 256 MiB write, then (default) a 256 MiB read of a "
                          "second buffer so that the write-back of the dirty lines is not charged to the step")
@@ -236,7 +238,7 @@ def main():
         shapes = [s for s in shapes if s.name == args.only]
         if not shapes:
             raise SystemExit(f"no linear named {args.only!r} in workload {args.workload}")
-    config = {"workload": args.workload, "description": WORKLOAD_DESC[args.workload],
+    config = {"workload": args.workload, "description": WORKLOAD_DESC[args.workload], "convrot_group": args.group,
               "linears": [f"{s.name}:M{s.M}xK{s.K}xN{s.N}" for s in shapes],
               "l2": ("flushed between timed steps, outside the events: 256 MiB write, then 256 MiB read of a second "
                      "buffer (inputs cold, no dirty lines left in L2)") if args.flush == "write+read"
@@ -280,7 +282,7 @@ def main():
         w, b = synthetic.weights(args.workload, s.N, s.K, seed_extra=synthetic.source_seed(s.name))
         wd = torch.from_numpy(w.view(np.int16)).view(torch.bfloat16).to(dev)
         if s.fmt == "w4a4":
-            wq, s_w = rq.convrot_pack_weight(wd)
+            wq, s_w = rq.convrot_pack_weight_g(wd, args.group)
         else:
             wq, s_w = rq.w8a8_pack_weight(wd, FORMAT_ID[s.fmt])
         bias = torch.from_numpy(b.view(np.int16)).view(torch.bfloat16).to(dev)
@@ -325,7 +327,7 @@ def main():
                 ev[0].record(cur)
             fmt = layers[idx[0]][0].fmt
             if fmt == "w4a4":
-                rq.convrot_w4a4_quantize(xs[src], ws)
+                rq.convrot_w4a4_quantize_g(xs[src], ws, args.group)
             else:
                 rq.w8a8_quantize(xs[src], FORMAT_ID[fmt], x8=q8[src][0], s_x=q8[src][1], workspace=ws)
             if ev is not None and per_kernel:
@@ -548,12 +550,12 @@ def end_to_end(args, rq, torch, dev, stream, shapes, xs, layers, groups, ws, flu
             if len(idx) == 1:
                 s, wq, s_w, bias, y = layers[idx[0]]
                 if fmt == "w4a4":
-                    rq.convrot_w4a4_linear(xs[src], wq, s_w, bias, out=y, workspace=ws)
+                    rq.convrot_w4a4_linear_g(xs[src], wq, s_w, bias, args.group, out=y, workspace=ws)
                 else:
                     rq.w8a8_linear(xs[src], wq, s_w, bias, FORMAT_ID[fmt], out=y, workspace=ws)
                 continue
             if fmt == "w4a4":
-                rq.convrot_w4a4_quantize(xs[src], ws)
+                rq.convrot_w4a4_quantize_g(xs[src], ws, args.group)
             else:
                 x8, sx = rq.w8a8_quantize(xs[src], FORMAT_ID[fmt], workspace=ws)
             for i in idx:
@@ -588,8 +590,9 @@ def end_to_end(args, rq, torch, dev, stream, shapes, xs, layers, groups, ws, flu
     return {"value": round(n_rep * step_ops(shapes) * args.steps / (total * 1e-3) / 1e12, 2), "unit": UNIT,
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
             "ms_per_step": round(total / args.steps, 4),
-            "api": "C ABI: convrot_w4a4_quantize per source + convrot_w4a4_gemm_quantized per linear "
-                   "(convrot_w4a4_linear for single-linear sources); pinned host->device x, device->host y"}
+            "api": "C ABI: convrot_w4a4_quantize_g per source + convrot_w4a4_gemm_quantized per linear "
+                   "(convrot_w4a4_linear_g for single-linear sources; w8a8_* for the int8 formats); "
+                   "pinned host->device x, device->host y"}
 
 
 def reference_arm(args, shapes, config, world, rank):

@@ -177,6 +177,31 @@ convrot_status_t convrot_w4a4_gemm_quantized(const uint8_t *Wq, const float *s_w
                                              uint16_t *y, const void *workspace,
                                              size_t workspace_bytes, void *stream);
 
+/* ---- rotation group-size variants ---------------------------------------------
+ * "JoaoZaokk/Z-Image-Turbo-W4A4-ConvRot", "Where Z-Image sits": the
+ * convrot_groupsize ablation runs groups of 256, 64 and 16 (a rotation of size
+ * N spreads each outlier over N channels).  These entry points are the ones
+ * above with the group as a parameter: each group of `group` (256, 64 or 16)
+ * channels is multiplied by H4 Kronecker'd log4(group) times, evaluated as
+ * the first log4(group) butterfly stages of R (strides 1, 4, 16), then by
+ * 2^-log4(group); the per-token scale, the codes, the packing and the GEMM are
+ * unchanged.  group == 256 is exactly the default path.  Other groups give
+ * CONVROT_ERR_SHAPE; K % 256 == 0 as everywhere. */
+convrot_status_t convrot_rotate_quant_g(const uint16_t *x, int M, int K, int group, uint8_t *xq,
+                                        float *s_a, void *stream);
+convrot_status_t convrot_pack_weight_g(const uint16_t *W, int N, int K, int group, uint8_t *Wq,
+                                       float *s_w, void *stream);
+convrot_status_t convrot_w4a4_quantize_g(const uint16_t *x, int M, int K, int group, void *workspace,
+                                         size_t workspace_bytes, void *stream);
+convrot_status_t convrot_w4a4_linear_g(const uint16_t *x, const uint8_t *Wq, const float *s_w,
+                                       const uint16_t *bias, int M, int N, int K, int group,
+                                       uint16_t *y, void *workspace, size_t workspace_bytes,
+                                       void *stream);
+convrot_status_t convrot_w4a4_linear_g_f32(const uint16_t *x, const uint8_t *Wq, const float *s_w,
+                                           const uint16_t *bias, int M, int N, int K, int group,
+                                           float *y32, void *workspace, size_t workspace_bytes,
+                                           void *stream);
+
 /* ---- int8 W8A8 formats -------------------------------------------------------
  * The pages store their quality-sensitive layers in int8 next to the W4A4
  * ones, and both run on the same integer tensor-core path:

@@ -43,6 +43,8 @@ EXPORTS = [
     "convrot_measure_mma_i8",
     "w8a8_workspace_size", "w8a8_quantize", "w8a8_pack_weight", "w8a8_gemm", "w8a8_gemm_f32", "w8a8_gemm_s32",
     "w8a8_linear", "w8a8_linear_f32",
+    "convrot_rotate_quant_g", "convrot_pack_weight_g", "convrot_w4a4_linear_g", "convrot_w4a4_linear_g_f32",
+    "convrot_w4a4_quantize_g",
 ]
 
 # int8 formats (include/convrot.h, w8a8_format_t)
@@ -94,6 +96,11 @@ def load_library():
     lib.convrot_dispatch_counts.argtypes = [ctypes.POINTER(ctypes.c_uint64), I]
     lib.convrot_dispatch_counts.restype = None
     lib.convrot_measure_mma_i8.argtypes = [I, I, I, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_double)]
+    lib.convrot_rotate_quant_g.argtypes = [P, I, I, I, P, P, P]
+    lib.convrot_w4a4_quantize_g.argtypes = [P, I, I, I, P, Z, P]
+    lib.convrot_pack_weight_g.argtypes = [P, I, I, I, P, P, P]
+    lib.convrot_w4a4_linear_g.argtypes = [P, P, P, P, I, I, I, I, P, P, Z, P]
+    lib.convrot_w4a4_linear_g_f32.argtypes = [P, P, P, P, I, I, I, I, P, P, Z, P]
     lib.w8a8_workspace_size.argtypes = [I, I, I, I]
     lib.w8a8_workspace_size.restype = Z
     lib.w8a8_quantize.argtypes = [P, I, I, I, P, P, P, Z, P]
@@ -114,7 +121,8 @@ def lib_status_fns():
             "convrot_w4a4_linear", "convrot_w4a4_linear_f32", "convrot_w4a4_linear_noalloc", "convrot_w4a4_quantize",
             "convrot_w4a4_gemm_quantized", "convrot_device_error", "convrot_selftest_timeout",
             "convrot_measure_mma_i8", "w8a8_quantize", "w8a8_pack_weight", "w8a8_gemm", "w8a8_gemm_f32",
-            "w8a8_gemm_s32", "w8a8_linear", "w8a8_linear_f32"]
+            "w8a8_gemm_s32", "w8a8_linear", "w8a8_linear_f32", "convrot_rotate_quant_g", "convrot_pack_weight_g",
+            "convrot_w4a4_linear_g", "convrot_w4a4_linear_g_f32", "convrot_w4a4_quantize_g"]
 
 
 def _check(fn: str, rc: int):
@@ -321,6 +329,67 @@ def convrot_measure_mma_i8(N: int = 256, a_in_tmem: bool = False, iters: int = 4
     _check("convrot_measure_mma_i8", load_library().convrot_measure_mma_i8(
         int(N), 1 if a_in_tmem else 0, int(iters), ctypes.byref(tops), ctypes.byref(cyc)))
     return float(tops.value), float(cyc.value)
+
+
+# ---- rotation group-size variants (256, 64, 16)
+
+def convrot_rotate_quant_g(x, group, xq=None, s_a=None, stream=None):
+    """convrot_rotate_quant with rotation group ``group`` (256, 64 or 16)."""
+    M, K = x.shape
+    _need(x, "x", torch.bfloat16)
+    xq = torch.empty((M, K // 2), dtype=torch.uint8, device=x.device) if xq is None else xq
+    s_a = torch.empty((M,), dtype=torch.float32, device=x.device) if s_a is None else s_a
+    _need(xq, "xq", torch.uint8, (M, K // 2))
+    _need(s_a, "s_a", torch.float32, (M,))
+    _check("convrot_rotate_quant_g", load_library().convrot_rotate_quant_g(_ptr(x), M, K, int(group), _ptr(xq),
+                                                                           _ptr(s_a), _stream(stream)))
+    return xq, s_a
+
+
+def convrot_pack_weight_g(W, group, Wq=None, s_w=None, stream=None):
+    """convrot_pack_weight with rotation group ``group`` (256, 64 or 16)."""
+    N, K = W.shape
+    _need(W, "W", torch.bfloat16)
+    Wq = torch.empty((N, K // 2), dtype=torch.uint8, device=W.device) if Wq is None else Wq
+    s_w = torch.empty((N,), dtype=torch.float32, device=W.device) if s_w is None else s_w
+    _need(Wq, "Wq", torch.uint8, (N, K // 2))
+    _need(s_w, "s_w", torch.float32, (N,))
+    _check("convrot_pack_weight_g", load_library().convrot_pack_weight_g(_ptr(W), N, K, int(group), _ptr(Wq),
+                                                                         _ptr(s_w), _stream(stream)))
+    return Wq, s_w
+
+
+def convrot_w4a4_quantize_g(x, workspace, group, stream=None):
+    """convrot_w4a4_quantize with rotation group ``group`` (256, 64 or 16)."""
+    M, K = x.shape
+    _need(x, "x", torch.bfloat16)
+    _need(workspace, "workspace", torch.uint8)
+    _check("convrot_w4a4_quantize_g", load_library().convrot_w4a4_quantize_g(
+        _ptr(x), M, K, int(group), _ptr(workspace), workspace.numel(), _stream(stream)))
+    return workspace
+
+
+def _linear_g(fn_name, out_dtype, x, Wq, s_w, bias, group, out, workspace, stream):
+    M, K = x.shape
+    N = Wq.shape[0]
+    _need(x, "x", torch.bfloat16)
+    _need(Wq, "Wq", torch.uint8, (N, K // 2))
+    _need(s_w, "s_w", torch.float32, (N,))
+    _need(bias, "bias", torch.bfloat16, (N,))
+    out = torch.empty((M, N), dtype=out_dtype, device=x.device) if out is None else out
+    _need(out, "out", out_dtype, (M, N))
+    ws = _workspace(workspace, convrot_w4a4_workspace_size(M, N, K), x.device)
+    _check(fn_name, getattr(load_library(), fn_name)(_ptr(x), _ptr(Wq), _ptr(s_w), _ptr(bias), M, N, K, int(group),
+                                                     _ptr(out), _ptr(ws), ws.numel(), _stream(stream)))
+    return out
+
+
+def convrot_w4a4_linear_g(x, Wq, s_w, bias=None, group=256, out=None, workspace=None, stream=None):
+    return _linear_g("convrot_w4a4_linear_g", torch.bfloat16, x, Wq, s_w, bias, group, out, workspace, stream)
+
+
+def convrot_w4a4_linear_g_f32(x, Wq, s_w, bias=None, group=256, out=None, workspace=None, stream=None):
+    return _linear_g("convrot_w4a4_linear_g_f32", torch.float32, x, Wq, s_w, bias, group, out, workspace, stream)
 
 
 # ---- int8 W8A8 formats (int8_tensorwise, ConvRot INT8 row-scaled)

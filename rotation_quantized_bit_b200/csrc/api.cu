@@ -100,7 +100,10 @@ convrot_status_t gemm_common(const uint8_t* xq, const float* s_a, const uint8_t*
   return from_cuda(launch_w4a4_gemm(a, sink, choose_tiling(M, N, K, sms), s));
 }
 
-convrot_status_t quantize_common(const uint16_t* x, int M, int K, void* ws, size_t ws_bytes, void* stream) {
+bool valid_group(int group) { return group == 256 || group == 64 || group == 16; }
+
+convrot_status_t quantize_common(const uint16_t* x, int M, int K, void* ws, size_t ws_bytes, void* stream,
+                                 int group = 256) {
   if (!x) return CONVROT_ERR_NULL;
   convrot_status_t st = check_mk(M, K);
   if (st != CONVROT_OK) return st;
@@ -111,6 +114,7 @@ convrot_status_t quantize_common(const uint16_t* x, int M, int K, void* ws, size
   if (st != CONVROT_OK) return st;
   uint8_t* base = static_cast<uint8_t*>(ws);
   RotateQuantOut o{nullptr, reinterpret_cast<int8_t*>(base), reinterpret_cast<float*>(base + sa_offset(M, K))};
+  o.group = group;
   return from_cuda(launch_rotate_quant(x, M, K, o, static_cast<cudaStream_t>(stream)));
 }
 
@@ -133,7 +137,8 @@ convrot_status_t gemm_quantized_common(const uint8_t* Wq, const float* s_w, cons
 }
 
 convrot_status_t linear_common(const uint16_t* x, const uint8_t* Wq, const float* s_w, const uint16_t* bias, int M,
-                               int N, int K, void* out, GemmSink sink, void* ws, size_t ws_bytes, void* stream) {
+                               int N, int K, void* out, GemmSink sink, void* ws, size_t ws_bytes, void* stream,
+                               int group = 256) {
   if (!x || !Wq || !s_w || !out) return CONVROT_ERR_NULL;
   convrot_status_t st = check_mnk(M, N, K);
   if (st != CONVROT_OK) return st;
@@ -141,7 +146,8 @@ convrot_status_t linear_common(const uint16_t* x, const uint8_t* Wq, const float
     return CONVROT_ERR_ALIGN;
   if (!ws || ws_bytes < workspace_bytes_for(M, K)) return CONVROT_ERR_WORKSPACE;
   if (!aligned16(ws)) return CONVROT_ERR_ALIGN;
-  st = quantize_common(x, M, K, ws, ws_bytes, stream);
+  if (!valid_group(group)) return CONVROT_ERR_SHAPE;
+  st = quantize_common(x, M, K, ws, ws_bytes, stream, group);
   if (st != CONVROT_OK) return st;
   return gemm_quantized_common(Wq, s_w, bias, M, N, K, out, sink, ws, ws_bytes, stream);
 }
@@ -435,6 +441,47 @@ convrot_status_t w8a8_linear_f32(const uint16_t* x, const int8_t* Wq8, const flo
                                  size_t workspace_bytes, void* stream) {
   return linear8_common(x, Wq8, s_w, bias, M, N, K, format, y32, GemmSink::kF32, workspace, workspace_bytes,
                         stream);
+}
+
+}  // extern "C"
+
+extern "C" {
+
+convrot_status_t convrot_rotate_quant_g(const uint16_t* x, int M, int K, int group, uint8_t* xq, float* s_a,
+                                        void* stream) {
+  if (!x || !xq || !s_a) return CONVROT_ERR_NULL;
+  if (!valid_group(group)) return CONVROT_ERR_SHAPE;
+  convrot_status_t st = check_mk(M, K);
+  if (st != CONVROT_OK) return st;
+  if (!aligned16(x) || !aligned16(xq) || !aligned16(s_a)) return CONVROT_ERR_ALIGN;
+  st = check_device(nullptr);
+  if (st != CONVROT_OK) return st;
+  RotateQuantOut o{xq, nullptr, s_a};
+  o.group = group;
+  return from_cuda(launch_rotate_quant(x, M, K, o, static_cast<cudaStream_t>(stream)));
+}
+
+convrot_status_t convrot_pack_weight_g(const uint16_t* W, int N, int K, int group, uint8_t* Wq, float* s_w,
+                                       void* stream) {
+  return convrot_rotate_quant_g(W, N, K, group, Wq, s_w, stream);
+}
+
+convrot_status_t convrot_w4a4_quantize_g(const uint16_t* x, int M, int K, int group, void* workspace,
+                                         size_t workspace_bytes, void* stream) {
+  if (!valid_group(group)) return CONVROT_ERR_SHAPE;
+  return quantize_common(x, M, K, workspace, workspace_bytes, stream, group);
+}
+
+convrot_status_t convrot_w4a4_linear_g(const uint16_t* x, const uint8_t* Wq, const float* s_w, const uint16_t* bias,
+                                       int M, int N, int K, int group, uint16_t* y, void* workspace,
+                                       size_t workspace_bytes, void* stream) {
+  return linear_common(x, Wq, s_w, bias, M, N, K, y, GemmSink::kBF16, workspace, workspace_bytes, stream, group);
+}
+
+convrot_status_t convrot_w4a4_linear_g_f32(const uint16_t* x, const uint8_t* Wq, const float* s_w,
+                                           const uint16_t* bias, int M, int N, int K, int group, float* y32,
+                                           void* workspace, size_t workspace_bytes, void* stream) {
+  return linear_common(x, Wq, s_w, bias, M, N, K, y32, GemmSink::kF32, workspace, workspace_bytes, stream, group);
 }
 
 }  // extern "C"

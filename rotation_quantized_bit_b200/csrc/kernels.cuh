@@ -19,6 +19,7 @@ struct RotateQuantOut {
   int8_t* s8;       // [M, K] codes as signed bytes in chunk order (0,2,4,6,1,3,5,7), or null
   float* scale;     // [M]
   bool int8 = false;  // s8 holds 8-bit codes (amax / 127) in natural order instead
+  int group = 256;    // rotation group: 256, 64 or 16 (int8: 256 only)
 };
 
 // The int8_tensorwise quantizer: one scale s = amax|x| / 127 for the whole

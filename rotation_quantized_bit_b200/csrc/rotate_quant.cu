@@ -161,7 +161,11 @@ __host__ __device__ constexpr int rq_smem_bytes(int R, int K, int S, int threads
   return S * rq_stage_bytes(R, K) + (threads / 16) * kTileBytes + 8 * S;
 }
 
-template <int MODE>
+// LOG4G: log4 of the rotation group (4: 256, the default; 3: 64; 2: 16 --
+// the convrot_groupsize variants).  A group of 4^LOG4G channels takes the
+// first LOG4G radix-4 stages and the factor 2^-LOG4G; the per-row scale
+// still spans the whole row.
+template <int MODE, int LOG4G>
 __global__ void __launch_bounds__(kMaxThreads) rotate_quant_kernel(const __grid_constant__ RQParams p) {
   constexpr bool PACKED = MODE == kPacked4;
   constexpr float kQMax = MODE == kInt8 ? 127.0f : 7.0f;
@@ -267,15 +271,20 @@ __global__ void __launch_bounds__(kMaxThreads) rotate_quant_kernel(const __grid_
     for (int i = 0; i < 16; ++i) P[i] = *reinterpret_cast<const u64*>(tile_r + kTileRow * i);
     __syncwarp();
     // now P[i] = channel 16 i + l.  stage on bits (4,5): stride 16
+    if (LOG4G >= 3) {
 #pragma unroll
-    for (int i = 0; i < 16; i += 4) bfly4(P[i], P[i + 1], P[i + 2], P[i + 3]);
+      for (int i = 0; i < 16; i += 4) bfly4(P[i], P[i + 1], P[i + 2], P[i + 3]);
+    }
     // stage on bits (6,7): stride 64
+    if (LOG4G >= 4) {
 #pragma unroll
-    for (int i = 0; i < 4; ++i) bfly4(P[i], P[i + 4], P[i + 8], P[i + 12]);
-    // x' = v * 1/16, and the two tasks' amax
+      for (int i = 0; i < 4; ++i) bfly4(P[i], P[i + 4], P[i + 8], P[i + 12]);
+    }
+    // x' = v * 2^-LOG4G (1/16 for groups of 256), and the two tasks' amax
     float m0 = 0.0f, m1 = 0.0f;
     {
-      const u64 sixteenth = f2(0.0625f, 0.0625f);
+      constexpr float kInvSqrtG = LOG4G == 4 ? 0.0625f : (LOG4G == 3 ? 0.125f : 0.25f);
+      const u64 sixteenth = f2(kInvSqrtG, kInvSqrtG);
 #pragma unroll
       for (int i = 0; i < 16; i += 2) {
         P[i] = f2_mul(P[i], sixteenth);
@@ -419,15 +428,15 @@ int num_sms_cached() {
   return n[dev];
 }
 
-template <int MODE>
+template <int MODE, int LOG4G>
 cudaError_t launch_rq(const RQParams& p, int threads, cudaStream_t stream) {
   static int cache[64] = {0};
   const int smem = rq_smem_bytes(p.R, p.K, p.S, threads);
-  const void* kfn = reinterpret_cast<const void*>(rotate_quant_kernel<MODE>);
+  const void* kfn = reinterpret_cast<const void*>(rotate_quant_kernel<MODE, LOG4G>);
   cudaError_t e = ensure_dynamic_smem(kfn, smem, cache);
   if (e != cudaSuccess) return note_cuda(e, "rotate_quant: dynamic shared memory attribute");
   int per_sm = 0;
-  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, rotate_quant_kernel<MODE>, threads, smem);
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, rotate_quant_kernel<MODE, LOG4G>, threads, smem);
   if (e != cudaSuccess) return note_cuda(e, "rotate_quant: occupancy query");
   if (per_sm < 1) per_sm = 1;
   int grid = num_sms_cached() * per_sm;
@@ -444,7 +453,7 @@ cudaError_t launch_rq(const RQParams& p, int threads, cudaStream_t stream) {
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return note_cuda(cudaLaunchKernelEx(&cfg, rotate_quant_kernel<MODE>, p), "rotate_quant: launch");
+  return note_cuda(cudaLaunchKernelEx(&cfg, rotate_quant_kernel<MODE, LOG4G>, p), "rotate_quant: launch");
 }
 
 }  // namespace
@@ -497,9 +506,20 @@ cudaError_t launch_rotate_quant(const uint16_t* x, int M, int K, RotateQuantOut 
   if (S > most_iters) S = most_iters;
   if (S < 1) S = 1;
   p.S = S;
-  cudaError_t e = out.packed != nullptr ? launch_rq<kPacked4>(p, threads, stream)
-                  : out.int8      ? launch_rq<kInt8>(p, threads, stream)
-                                  : launch_rq<kOperand4>(p, threads, stream);
+  cudaError_t e;
+  if (out.group != 256 && out.group != 64 && out.group != 16) return note_cuda(cudaErrorInvalidValue, "rotate_quant: group");
+  if (out.int8) {
+    if (out.group != 256) return note_cuda(cudaErrorInvalidValue, "rotate_quant: int8 group");
+    e = launch_rq<kInt8, 4>(p, threads, stream);
+  } else if (out.packed != nullptr) {
+    e = out.group == 256 ? launch_rq<kPacked4, 4>(p, threads, stream)
+        : out.group == 64 ? launch_rq<kPacked4, 3>(p, threads, stream)
+                          : launch_rq<kPacked4, 2>(p, threads, stream);
+  } else {
+    e = out.group == 256 ? launch_rq<kOperand4, 4>(p, threads, stream)
+        : out.group == 64 ? launch_rq<kOperand4, 3>(p, threads, stream)
+                          : launch_rq<kOperand4, 2>(p, threads, stream);
+  }
   count_dispatch(0);
   return e;
 }
