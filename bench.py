@@ -74,6 +74,21 @@ def parse():
     return ap.parse_args()
 
 
+def job_time_ms(local_ms, world, dist, torch, device):
+    """The job's time: the maximum over ranks of each rank's device time
+    (every rank runs a full replica of the step)."""
+    if world <= 1:
+        return local_ms
+    t = torch.tensor([local_ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tops(ops_per_step, steps, job_ms, world):
+    """Whole-job throughput: the work of all ranks' replicas over the job time."""
+    return max(world, 1) * ops_per_step * steps / (job_ms * 1e-3) / 1e12
+
+
 def step_ops(shapes):
     return sum(2.0 * s.M * s.N * s.K for s in shapes)
 
@@ -421,15 +436,10 @@ def main():
             t_quant[gi] += kv[0].elapsed_time(kv[1])
             for j, i in enumerate(idx):
                 t_gemm[i] += kv[1 + j].elapsed_time(kv[2 + j])
-    total_ms = float(t_grp.sum())
-    if world > 1:
-        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = job_time_ms(float(t_grp.sum()), world, dist, torch, dev)
     ms_per_step = total_ms / args.steps
     ops = step_ops(shapes)
-    n_rep = world if world > 1 else 1
-    value = n_rep * ops * args.steps / (total_ms * 1e-3) / 1e12
+    value = job_tops(ops, args.steps, total_ms, world)
 
     peaks = load_peaks()
     int8_peak = peaks["bf16_tflops"] * INT8_PER_BF16
@@ -582,12 +592,8 @@ def end_to_end(args, rq, torch, dev, stream, shapes, xs, layers, groups, ws, flu
         e1.record(stream)
         e1.synchronize()
         total += e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([total], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total = float(t.item())
-    n_rep = world if world > 1 else 1
-    return {"value": round(n_rep * step_ops(shapes) * args.steps / (total * 1e-3) / 1e12, 2), "unit": UNIT,
+    total = job_time_ms(total, world, dist, torch, dev)
+    return {"value": round(job_tops(step_ops(shapes), args.steps, total, world), 2), "unit": UNIT,
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
             "ms_per_step": round(total / args.steps, 4),
             "api": "C ABI: convrot_w4a4_quantize_g per source + convrot_w4a4_gemm_quantized per linear "

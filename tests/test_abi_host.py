@@ -98,3 +98,34 @@ def test_dispatch_counters_without_a_gpu(lib):
 
 def test_version(lib):
     assert b"sm_100a" in lib.convrot_version()
+
+
+def test_int8_workspace_sizes(lib):
+    # codes M*K, scales (M floats), 256 bytes of reduction scratch, each 256-aligned
+    assert lib.w8a8_workspace_size(76, 1024, 2560, 0) == _r256(76 * 2560) + _r256(76 * 4) + 256
+    assert lib.w8a8_workspace_size(76, 1024, 2560, 1) == _r256(76 * 2560) + _r256(76 * 4) + 256
+    assert lib.w8a8_workspace_size(76, 1024, 2560, 2) == 0      # unknown format
+    assert lib.w8a8_workspace_size(76, 1024, 300, 0) == 0       # K % 256
+    assert lib.w8a8_workspace_size(76, 1020, 2560, 0) == 0      # N % 8
+
+
+def test_int8_and_group_arguments_rejected_before_any_device_call(lib):
+    P = ctypes.c_void_p
+    buf = ctypes.create_string_buffer(1 << 16)
+    good = P(ctypes.addressof(buf) + (-ctypes.addressof(buf) % 16))
+    null = P(0)
+    # NULL pointers
+    assert lib.w8a8_quantize(null, 4, 256, 0, good, good, good, 4096, null) == 1
+    assert lib.w8a8_gemm(null, good, good, good, null, 4, 8, 256, 0, good, null) == 1
+    assert lib.convrot_rotate_quant_g(null, 4, 256, 64, good, good, null) == 1
+    # bad format / group / shape
+    assert lib.w8a8_quantize(good, 4, 256, 9, good, good, good, 4096, null) == 2
+    assert lib.w8a8_gemm(good, good, good, good, null, 4, 8, 256, 5, good, null) == 2
+    assert lib.w8a8_gemm_s32(good, good, 4, 8, 300, good, null) == 2
+    assert lib.convrot_rotate_quant_g(good, 4, 256, 32, good, good, null) == 2
+    assert lib.convrot_w4a4_quantize_g(good, 4, 256, 128, good, 4096, null) == 2
+    # misaligned pointer
+    bad = P(good.value + 4)
+    assert lib.w8a8_gemm_s32(bad, good, 4, 8, 256, good, null) == 3
+    # a too small workspace for the fused int8 linear
+    assert lib.w8a8_linear(good, good, good, null, 4, 8, 256, 0, good, good, 16, null) == 5
