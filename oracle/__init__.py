@@ -57,6 +57,14 @@ def _load():
         lib.oracle_f32_to_bf16.restype = ctypes.c_uint16
         lib.oracle_bf16_to_f32.argtypes = [ctypes.c_uint16]
         lib.oracle_bf16_to_f32.restype = ctypes.c_float
+        lib.oracle_e4m3_to_f32.argtypes = [ctypes.c_uint8]
+        lib.oracle_e4m3_to_f32.restype = ctypes.c_float
+        lib.oracle_f32_to_e4m3.argtypes = [ctypes.c_float]
+        lib.oracle_f32_to_e4m3.restype = ctypes.c_uint8
+        lib.oracle_asym_decode.argtypes = [P, P, P, I, I, P]
+        lib.oracle_asym_linear_rows.argtypes = [P, P, P, P, P, P, I, I, I, I, I, P, P]
+        lib.oracle_lloyd_max16.argtypes = [P, ctypes.c_int64, I, P]
+        lib.oracle_asym_convert.argtypes = [P, I, I, I, P, P, P, P]
         _lib = lib
     return _lib
 
@@ -220,3 +228,71 @@ def f32_to_bf16(v: float) -> int:
 
 def bf16_to_f32(h: int) -> float:
     return float(_load().oracle_bf16_to_f32(int(h)))
+
+
+# ---- asymmetric W4A8 (asym_w4a8_int8): 4-bit codebook indices, an e4m3 scale
+# per 16 weights along K, one scale per output channel, a 16-level codebook per
+# tensor, the ConvRot INT8 row-scaled activations
+
+def e4m3_to_f32(b):
+    """e4m3fn bytes -> fp32 values (any shape)."""
+    lib = _load()
+    table = np.array([lib.oracle_e4m3_to_f32(i) for i in range(256)], np.float32)
+    return table[np.asarray(b, np.uint8)]
+
+
+def f32_to_e4m3(v):
+    """fp32 values -> e4m3fn bytes, round to nearest even, saturating at 448."""
+    lib = _load()
+    a = np.asarray(v, np.float32)
+    return np.array([lib.oracle_f32_to_e4m3(float(t)) for t in a.reshape(-1)], np.uint8).reshape(a.shape)
+
+
+def asym_decode(idx, s_rel, codebook):
+    """idx u8 [N, K/2], s_rel u8 [N, K/16], codebook fp32 [16] -> int8 weights [N, K]."""
+    idx = _c(idx, np.uint8)
+    s_rel = _c(s_rel, np.uint8)
+    cb = _c(codebook, np.float32)
+    N, K = idx.shape[0], 2 * idx.shape[1]
+    w8 = np.empty((N, K), np.int8)
+    _check(_load().oracle_asym_decode(_ptr(idx), _ptr(s_rel), _ptr(cb), N, K, _ptr(w8)), "asym_decode")
+    return w8
+
+
+def asym_linear(x_bits, idx, s_rel, codebook, s_channel, bias_bits, rows=None):
+    """The asymmetric W4A8 Linear: returns (y32 fp32, y bf16 bits) for rows ``rows=(m0, m1)``."""
+    x = _c(x_bits, np.uint16)
+    idx = _c(idx, np.uint8)
+    s_rel = _c(s_rel, np.uint8)
+    cb = _c(codebook, np.float32)
+    sc = _c(s_channel, np.float32)
+    b = None if bias_bits is None else _c(bias_bits, np.uint16)
+    M, K = x.shape
+    N = idx.shape[0]
+    m0, m1 = rows if rows is not None else (0, M)
+    y32 = np.empty((m1 - m0, N), np.float32)
+    y16 = np.empty((m1 - m0, N), np.uint16)
+    _check(_load().oracle_asym_linear_rows(_ptr(x), _ptr(idx), _ptr(s_rel), _ptr(cb), _ptr(sc), _ptr(b), M, N, K,
+                                           m0, m1, _ptr(y32), _ptr(y16)), "asym_linear")
+    return y32, y16
+
+
+def lloyd_max16(u, iters: int = 100):
+    """16 Lloyd-Max levels (float64) of the values ``u``."""
+    u = _c(u, np.float32).reshape(-1)
+    lv = np.empty(16, np.float64)
+    _check(_load().oracle_lloyd_max16(_ptr(u), u.size, iters, _ptr(lv)), "lloyd_max16")
+    return lv
+
+
+def asym_convert(w_bits, iters: int = 100):
+    """bf16 bits W [N, K] -> (idx u8 [N, K/2], s_rel u8 [N, K/16], s_channel fp32 [N], codebook fp32 [16])."""
+    w = _c(w_bits, np.uint16)
+    N, K = w.shape
+    idx = np.empty((N, K // 2), np.uint8)
+    s_rel = np.empty((N, K // 16), np.uint8)
+    sc = np.empty((N,), np.float32)
+    cb = np.empty((16,), np.float32)
+    _check(_load().oracle_asym_convert(_ptr(w), N, K, iters, _ptr(idx), _ptr(s_rel), _ptr(sc), _ptr(cb)),
+           "asym_convert")
+    return idx, s_rel, sc, cb

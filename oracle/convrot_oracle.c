@@ -54,6 +54,11 @@
  *  s), -127, 127) with a true division and round half to even, s = 0 gives
  *  q = 0; the epilogue is the same rank-one rescale (a per-tensor scale is a
  *  constant vector).
+ *
+ * The asymmetric W4A8 format ("asym_w4a8_int8": 4-bit codebook indices, an
+ * fp8 scale per 16 weights, a per-channel scale, a 16-level codebook per
+ * tensor) is at the end of the file, with its own sources and readings, and
+ * the offline converter that fits the codebook (Lloyd's algorithm).
  */
 #include <math.h>
 #include <stdint.h>
@@ -385,5 +390,195 @@ int oracle_linear8_rows(const uint16_t *x, const int8_t *w8, const float *s_w, c
   free(sa);
   free(sw);
   free(acc);
+  return rc;
+}
+
+/* ---- asymmetric W4A8 ("asym_w4a8_int8") ------------------------------------
+ *
+ * Sources: "Nicolaslas/Rebels_w4a8s" ("What's inside a file": int4 codes two
+ * per byte, an fp8 scale s_rel per group of 16, one scale per output channel,
+ * a 16-level Lloyd-Max codebook fit to the tensor, under a group-256 ConvRot
+ * rotation; the math runs on int8 tensor cores) and
+ * "JoaoZaokk/Qwen3-VL-4B-W4A8-ConvRot" (file table: asym_w4a8_int8, group 16,
+ * convrot_groupsize 256).  Readings (the pages give storage, not arithmetic):
+ *  - fp8 is e4m3 "fn": bias 7, 3 mantissa bits, no infinities, S.1111.111 is
+ *    NaN, largest finite 448.
+ *  - The 4-bit codes are unsigned codebook indices 0..15, low nibble = even k.
+ *  - s_rel[n, g] scales codebook levels onto the int8 grid of the row, so the
+ *    int8 weight the MMA sees is w8 = clamp(rint(codebook[i] * s_rel), -127,
+ *    127): one fp32 multiply, round half to even, NaN -> 0.  The row's real
+ *    weights (rotated basis) are s_channel[n] * w8.
+ *  - Activations: the ConvRot INT8 row-scaled quantizer above (group 256,
+ *    s_a = amax / 127 per token); the epilogue is the rank-one rescale with
+ *    s_w = s_channel. */
+
+/* e4m3fn byte -> fp32, exactly: normal (1 + m/8) 2^(e-7), subnormal m 2^-9. */
+float oracle_e4m3_to_f32(uint8_t b) {
+  int e = (b >> 3) & 15, m = b & 7;
+  if (e == 15 && m == 7) return NAN;
+  double v = e == 0 ? ldexp((double)m, -9) : ldexp(8.0 + (double)m, e - 10);
+  return (float)((b & 0x80) ? -v : v);
+}
+
+/* fp32 -> e4m3fn by exhaustive search: the nearest finite code, a tie going
+ * to the even code (even mantissa); |f| >= 448 saturates to +-448 (reading);
+ * NaN -> 0x7F. */
+uint8_t oracle_f32_to_e4m3(float f) {
+  if (isnan(f)) return 0x7F;
+  uint8_t sign = signbit(f) ? 0x80 : 0x00;
+  double a = fabs((double)f);
+  if (a >= 448.0) return (uint8_t)(sign | 0x7E);
+  int best = 0;
+  double bd = INFINITY;
+  for (int c = 0; c <= 0x7E; ++c) {
+    double d = fabs((double)oracle_e4m3_to_f32((uint8_t)c) - a);
+    if (d < bd || (d == bd && (c & 1) == 0)) {
+      bd = d;
+      best = c;
+    }
+  }
+  return (uint8_t)(sign | best);
+}
+
+/* One decoded weight: codebook level `level` under the group scale byte. */
+static int8_t asym_decode_one(float level, uint8_t s_rel) {
+  float p = level * oracle_e4m3_to_f32(s_rel);
+  if (isnan(p)) return 0;
+  if (p > 127.0f) return 127;
+  if (p < -127.0f) return -127;
+  return (int8_t)rintf(p);
+}
+
+/* idx[N, K/2] (two indices per byte), s_rel[N, K/16], codebook[16] ->
+ * int8 weights w8[N, K]. */
+int oracle_asym_decode(const uint8_t *idx, const uint8_t *s_rel, const float *codebook, int N, int K,
+                       int8_t *w8) {
+  if (N < 0 || K <= 0 || K % 16 != 0) return ORACLE_ERR_SHAPE;
+  for (int n = 0; n < N; ++n)
+    for (int k = 0; k < K; ++k) {
+      uint8_t byte = idx[(size_t)n * (K / 2) + k / 2];
+      int i = (k % 2 == 0) ? (byte & 0xF) : (byte >> 4);
+      w8[(size_t)n * K + k] = asym_decode_one(codebook[i], s_rel[(size_t)n * (K / 16) + k / 16]);
+    }
+  return ORACLE_OK;
+}
+
+/* The asymmetric W4A8 Linear, rows [m0, m1) of y: decode the weights, then
+ * the ConvRot INT8 row-scaled Linear with s_w = s_channel. */
+int oracle_asym_linear_rows(const uint16_t *x, const uint8_t *idx, const uint8_t *s_rel, const float *codebook,
+                            const float *s_channel, const uint16_t *bias, int M, int N, int K, int m0, int m1,
+                            float *y32, uint16_t *y16) {
+  if (M < 0 || N <= 0 || K <= 0 || K % 256 != 0) return ORACLE_ERR_SHAPE;
+  int8_t *w8 = (int8_t *)malloc((size_t)N * (size_t)K);
+  if (!w8) return ORACLE_ERR_NOMEM;
+  int rc = oracle_asym_decode(idx, s_rel, codebook, N, K, w8);
+  if (rc == ORACLE_OK) rc = oracle_linear8_rows(x, w8, s_channel, bias, M, N, K, 256, 1, m0, m1, y32, y16);
+  free(w8);
+  return rc;
+}
+
+/* Index of the level nearest to u (the lower index on a tie). */
+static int nearest_level(const double *c, double u) {
+  int best = 0;
+  double bd = fabs(u - c[0]);
+  for (int j = 1; j < 16; ++j) {
+    double d = fabs(u - c[j]);
+    if (d < bd) {
+      bd = d;
+      best = j;
+    }
+  }
+  return best;
+}
+
+/* Lloyd's algorithm for the 16-level scalar quantizer of the values u[0..n):
+ * levels start at the centres of 16 equal cells of [-1, 1]; each iteration
+ * assigns every value to its nearest level, then moves every level to the
+ * mean of its values (a level without values stays).  It stops when no
+ * assignment changed or after `iters` iterations.  Levels in double. */
+int oracle_lloyd_max16(const float *u, int64_t n, int iters, double *levels) {
+  if (n < 0 || iters < 0) return ORACLE_ERR_SHAPE;
+  for (int j = 0; j < 16; ++j) levels[j] = -1.0 + (2.0 * j + 1.0) / 16.0;
+  int *cell = (int *)malloc(sizeof(int) * (size_t)(n > 0 ? n : 1));
+  if (!cell) return ORACLE_ERR_NOMEM;
+  for (int64_t i = 0; i < n; ++i) cell[i] = -1;
+  for (int it = 0; it < iters; ++it) {
+    int changed = 0;
+    for (int64_t i = 0; i < n; ++i) {
+      int j = nearest_level(levels, (double)u[i]);
+      if (j != cell[i]) changed = 1;
+      cell[i] = j;
+    }
+    if (!changed) break;
+    double sum[16] = {0};
+    int64_t cnt[16] = {0};
+    for (int64_t i = 0; i < n; ++i) {
+      sum[cell[i]] += (double)u[i];
+      cnt[cell[i]] += 1;
+    }
+    for (int j = 0; j < 16; ++j)
+      if (cnt[j] > 0) levels[j] = sum[j] / (double)cnt[j];
+  }
+  free(cell);
+  return ORACLE_OK;
+}
+
+/* Offline conversion of bf16 weights W[N, K] to the asymmetric W4A8 format
+ * (test infrastructure: the pages' converter is not part of the hot path).
+ *   1. rotate each row's 256-groups (the ConvRot rotation above);
+ *   2. s_channel[n] = amax_k |w'[n,k]| / 127;
+ *   3. s_rel[n, g] = e4m3(amax over the 16 values of group g / s_channel[n])
+ *      (0 when s_channel is 0);
+ *   4. u = w' / (s_channel * s_rel), 0 where that product is 0;
+ *   5. codebook = Lloyd-Max levels of all u of the tensor (`iters` at most),
+ *      rounded to fp32;
+ *   6. idx = the nearest fp32 level to each u (the lower index on a tie). */
+int oracle_asym_convert(const uint16_t *W, int N, int K, int iters, uint8_t *idx, uint8_t *s_rel, float *s_channel,
+                        float *codebook) {
+  if (N <= 0 || K <= 0 || K % 256 != 0) return ORACLE_ERR_SHAPE;
+  size_t NK = (size_t)N * (size_t)K;
+  float *v = (float *)malloc(sizeof(float) * NK);
+  float *u = (float *)malloc(sizeof(float) * NK);
+  if (!v || !u) {
+    free(v);
+    free(u);
+    return ORACLE_ERR_NOMEM;
+  }
+  for (size_t i = 0; i < NK; ++i) v[i] = bf16_bits_to_f32(W[i]);
+  for (int n = 0; n < N; ++n)
+    for (int g = 0; g < K / 256; ++g) rotate_group(v + (size_t)n * K + (size_t)g * 256, 4);
+  for (int n = 0; n < N; ++n) {
+    const float *row = v + (size_t)n * K;
+    float amax = 0.0f;
+    for (int k = 0; k < K; ++k)
+      if (fabsf(row[k]) > amax) amax = fabsf(row[k]);
+    float sc = amax / 127.0f;
+    s_channel[n] = sc;
+    for (int g = 0; g < K / 16; ++g) {
+      float ga = 0.0f;
+      for (int k = 16 * g; k < 16 * g + 16; ++k)
+        if (fabsf(row[k]) > ga) ga = fabsf(row[k]);
+      uint8_t sb = sc == 0.0f ? 0 : oracle_f32_to_e4m3(ga / sc);
+      s_rel[(size_t)n * (K / 16) + g] = sb;
+      float d = sc * oracle_e4m3_to_f32(sb);
+      for (int k = 16 * g; k < 16 * g + 16; ++k) u[(size_t)n * K + k] = d == 0.0f ? 0.0f : row[k] / d;
+    }
+  }
+  double lv[16];
+  int rc = oracle_lloyd_max16(u, (int64_t)NK, iters, lv);
+  if (rc == ORACLE_OK) {
+    double c32[16];
+    for (int j = 0; j < 16; ++j) {
+      codebook[j] = (float)lv[j];
+      c32[j] = (double)codebook[j];
+    }
+    memset(idx, 0, NK / 2);
+    for (size_t i = 0; i < NK; ++i) {
+      int j = nearest_level(c32, (double)u[i]);
+      idx[i / 2] |= (uint8_t)((i % 2 == 0) ? j : (j << 4));
+    }
+  }
+  free(v);
+  free(u);
   return rc;
 }
