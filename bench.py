@@ -49,8 +49,14 @@ WORKLOAD_DESC = {
     "edit20b_int8": "20B image-edit DiT value/output projections (3072x3072) in int8_tensorwise W8A8, M=8704",
     "qwen3_4b_mixed": "Qwen3-4B layer at M=76 and M=1220: q,k,v,o in ConvRot INT8 (row-scaled) W8A8, "
                       "gate,up,down in ConvRot W4A4",
+    "qwen3_4b_w4a8": "Qwen3-VL-4B text-encoder layer linears (q,k,v,o,gate,up,down; hidden 2560) in asymmetric "
+                     "W4A8 (4-bit codebook weights, e4m3 group-16 scales), M=76 and M=1220",
+    "small_m_w4a8": "small-M sweep in asymmetric W4A8, M in {1,8,16,64,128} x (K,N) in {(2560,9728),(9728,2560),"
+                    "(3072,12288),(12288,3072)}",
 }
-FORMAT_ID = {"int8_tensorwise": 0, "convrot_int8": 1}  # w8a8_format_t
+# w8a8_format_t of each 8-bit-activation format's quantizer (the asymmetric
+# W4A8 activations are the ConvRot INT8 row-scaled codes)
+FORMAT_ID = {"int8_tensorwise": 0, "convrot_int8": 1, "asym_w4a8": 1}
 L2_FLUSH_BYTES = 256 << 20
 INT8_PER_BF16 = 2.0  # nominal dense int8 : bf16 tensor throughput (4.5 : 2.25 PFLOP/s)
 
@@ -94,7 +100,10 @@ def step_ops(shapes):
 
 
 def weight_bytes(s):
-    """Bytes of the stored weight codes: 4-bit packed, or int8."""
+    """Bytes of the stored weight codes: 4-bit packed, int8, or 4-bit
+    codebook indices plus one e4m3 scale per 16 and the 16-level codebook."""
+    if s.fmt == "asym_w4a8":
+        return s.N * s.K // 2 + s.N * s.K // 16 + 64
     return s.N * s.K // 2 if s.fmt == "w4a4" else s.N * s.K
 
 
@@ -203,6 +212,9 @@ def oracle_inputs(oracle, workload, s):
     w, b = synthetic.weights(workload, s.N, s.K, seed_extra=synthetic.source_seed(s.name))
     if s.fmt == "w4a4":
         wq, s_w = oracle.pack_weight(w)
+    elif s.fmt == "asym_w4a8":
+        idx, s_rel, cb, s_w = synthetic.asym_format(workload, s.N, s.K, seed_extra=synthetic.source_seed(s.name))
+        wq = (idx, s_rel, cb)
     else:
         wq, s_w = oracle.quant8(w, *ORACLE_FORMAT[s.fmt])
     return s, x, wq, s_w, b
@@ -214,6 +226,8 @@ ORACLE_FORMAT = {"int8_tensorwise": (0, False), "convrot_int8": (256, True)}  # 
 def oracle_linear(oracle, s, x, wq, s_w, b):
     if s.fmt == "w4a4":
         return oracle.linear(x, wq, s_w, b, s.K)
+    if s.fmt == "asym_w4a8":
+        return oracle.asym_linear(x, *wq, s_w, b)
     return oracle.linear8(x, wq, s_w, b, *ORACLE_FORMAT[s.fmt])
 
 
@@ -298,6 +312,13 @@ def main():
         wd = torch.from_numpy(w.view(np.int16)).view(torch.bfloat16).to(dev)
         if s.fmt == "w4a4":
             wq, s_w = rq.convrot_pack_weight_g(wd, args.group)
+        elif s.fmt == "asym_w4a8":
+            # weights arrive converted offline (no bf16 -> codebook conversion
+            # runs here): seeded tensors in the storage layout
+            idx, s_rel, cb, sch = synthetic.asym_format(args.workload, s.N, s.K,
+                                                        seed_extra=synthetic.source_seed(s.name))
+            wq = tuple(torch.from_numpy(a).to(dev) for a in (idx, s_rel, cb))
+            s_w = torch.from_numpy(sch).to(dev)
         else:
             wq, s_w = rq.w8a8_pack_weight(wd, FORMAT_ID[s.fmt])
         bias = torch.from_numpy(b.view(np.int16)).view(torch.bfloat16).to(dev)
@@ -314,6 +335,7 @@ def main():
         else:
             groups.append((s.source, [i]))
     ws_bytes = max(rq.convrot_w4a4_workspace_size(s.M, s.N, s.K) if s.fmt == "w4a4"
+                   else rq.asym_w4a8_workspace_size(s.M, s.N, s.K) if s.fmt == "asym_w4a8"
                    else rq.w8a8_workspace_size(s.M, s.N, s.K, FORMAT_ID[s.fmt]) for s in shapes)
     ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
     # int8 formats: the activation codes and scales of each source
@@ -321,7 +343,7 @@ def main():
     for s in shapes:
         if s.fmt != "w4a4" and s.source not in q8:
             q8[s.source] = (torch.empty((s.M, s.K), dtype=torch.int8, device=dev),
-                            torch.empty((s.M if s.fmt == "convrot_int8" else 1,), dtype=torch.float32, device=dev))
+                            torch.empty((s.M if FORMAT_ID[s.fmt] == 1 else 1,), dtype=torch.float32, device=dev))
     flush = make_flusher(torch, dev, args.flush)
     stream = torch.cuda.current_stream()
     torch.cuda.synchronize()
@@ -351,6 +373,8 @@ def main():
                 s, wq, s_w, bias, y = layers[i]
                 if fmt == "w4a4":
                     rq.convrot_w4a4_gemm_quantized(ws, s.M, wq, s_w, bias, out=y)
+                elif fmt == "asym_w4a8":
+                    rq.asym_w4a8_gemm(q8[src][0], q8[src][1], *wq, s_w, bias, out=y)
                 else:
                     rq.w8a8_gemm(q8[src][0], q8[src][1], wq, s_w, bias, FORMAT_ID[fmt], out=y)
                 if ev is not None and (per_kernel or j == len(idx) - 1):
@@ -562,6 +586,8 @@ def end_to_end(args, rq, torch, dev, stream, shapes, xs, layers, groups, ws, flu
             s, wq, s_w, bias, y = layers[idx[0]]
             if fmt == "w4a4":
                 rq.convrot_w4a4_linear_g(xs[src], wq, s_w, bias, args.group, out=y, workspace=ws)
+            elif fmt == "asym_w4a8":
+                rq.asym_w4a8_linear(xs[src], *wq, s_w, bias, out=y, workspace=ws)
             else:
                 rq.w8a8_linear(xs[src], wq, s_w, bias, FORMAT_ID[fmt], out=y, workspace=ws)
             return
@@ -573,6 +599,8 @@ def end_to_end(args, rq, torch, dev, stream, shapes, xs, layers, groups, ws, flu
             s, wq, s_w, bias, y = layers[i]
             if fmt == "w4a4":
                 rq.convrot_w4a4_gemm_quantized(ws, s.M, wq, s_w, bias, out=y)
+            elif fmt == "asym_w4a8":
+                rq.asym_w4a8_gemm(x8, sx, *wq, s_w, bias, out=y)
             else:
                 rq.w8a8_gemm(x8, sx, wq, s_w, bias, FORMAT_ID[fmt], out=y)
 

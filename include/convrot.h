@@ -267,6 +267,65 @@ convrot_status_t w8a8_linear_f32(const uint16_t *x, const int8_t *Wq8, const flo
                                  const uint16_t *bias, int M, int N, int K, int format, float *y32,
                                  void *workspace, size_t workspace_bytes, void *stream);
 
+/* ---- asymmetric W4A8 ("asym_w4a8_int8") ------------------------------------
+ *
+ * The W4A8 layout of "Nicolaslas/Rebels_w4a8s" ("What's inside a file") and
+ * "JoaoZaokk/Qwen3-VL-4B-W4A8-ConvRot" (file table: asym_w4a8_int8, group
+ * 16, convrot_groupsize 256): per Linear W [N, K], in the ConvRot-rotated
+ * basis (group 256),
+ *   idx       [N, K/2]  uint8   4-bit codebook indices 0..15, two per byte,
+ *                               low nibble = even k
+ *   s_rel     [N, K/16] uint8   e4m3 ("fn": bias 7, no infinities) scale of
+ *                               each group of 16 consecutive k
+ *   s_channel [N]       float   per-output-channel scale
+ *   codebook  [16]      float   the tensor's levels
+ * The int8 weight the tensor cores multiply is
+ *   w8[n, k] = clamp(rint(codebook[idx[n, k]] * s_rel[n, k / 16]), -127, 127)
+ * (one fp32 multiply, round half to even, a NaN product -> 0); activations
+ * are the ConvRot INT8 row-scaled codes (w8a8_quantize with
+ * W8A8_CONVROT_INT8_ROW: rotation, s_a = amax / 127 per token); then
+ *   y[m, n] = bf16(((float)acc * s_a[m]) * s_channel[n] + bias[n]),
+ *   acc = sum_k x8[m, k] * w8[n, k] (exact int32).
+ * The decode rule is a reading: the pages give the storage and say that the
+ * arithmetic is int8.  Shapes as for W4A4 (K % 256 == 0, N % 8 == 0, M >= 1);
+ * every pointer 16-byte aligned device memory owned by the caller.  The
+ * weight tensors (converted offline) are inputs; no call here converts bf16
+ * weights to this format. */
+
+/* Bytes of workspace asym_w4a8_linear* need for M tokens (the int8 codes and
+ * scales of the activations). */
+size_t asym_w4a8_workspace_size(int M, int N, int K);
+
+/* x8 [M, K] int8 and s_a [M] from w8a8_quantize(W8A8_CONVROT_INT8_ROW), the
+ * weight tensors above, bias [N] or NULL -> y [M, N] bf16.  The decode runs
+ * inside the GEMM (no int8 weight copy is written). */
+convrot_status_t asym_w4a8_gemm(const int8_t *x8, const float *s_a, const uint8_t *idx, const uint8_t *s_rel,
+                                const float *codebook, const float *s_channel, const uint16_t *bias, int M, int N,
+                                int K, uint16_t *y, void *stream);
+
+/* Same kernel, fp32 sink y32 [M, N] before the bf16 rounding (parity). */
+convrot_status_t asym_w4a8_gemm_f32(const int8_t *x8, const float *s_a, const uint8_t *idx,
+                                    const uint8_t *s_rel, const float *codebook, const float *s_channel,
+                                    const uint16_t *bias, int M, int N, int K, float *y32, void *stream);
+
+/* Same kernel, the exact int32 accumulator acc [M, N] (parity). */
+convrot_status_t asym_w4a8_gemm_s32(const int8_t *x8, const uint8_t *idx, const uint8_t *s_rel,
+                                    const float *codebook, int M, int N, int K, int32_t *acc, void *stream);
+
+/* The fused asymmetric W4A8 Linear: x [M, K] bf16 rotated and quantized
+ * online, then the GEMM above -> y [M, N] bf16.  workspace: >=
+ * asym_w4a8_workspace_size(M, N, K) bytes. */
+convrot_status_t asym_w4a8_linear(const uint16_t *x, const uint8_t *idx, const uint8_t *s_rel,
+                                  const float *codebook, const float *s_channel, const uint16_t *bias, int M,
+                                  int N, int K, uint16_t *y, void *workspace, size_t workspace_bytes,
+                                  void *stream);
+
+/* The fused asymmetric W4A8 Linear with an fp32 sink (parity). */
+convrot_status_t asym_w4a8_linear_f32(const uint16_t *x, const uint8_t *idx, const uint8_t *s_rel,
+                                      const float *codebook, const float *s_channel, const uint16_t *bias,
+                                      int M, int N, int K, float *y32, void *workspace, size_t workspace_bytes,
+                                      void *stream);
+
 /* Device-side error word of the current device: bit 0 = a bounded wait
  * inside a kernel expired (the kernel skipped its remaining work and
  * returned; its outputs are invalid).  Synchronizes `stream`, copies the word

@@ -45,6 +45,8 @@ EXPORTS = [
     "w8a8_linear", "w8a8_linear_f32",
     "convrot_rotate_quant_g", "convrot_pack_weight_g", "convrot_w4a4_linear_g", "convrot_w4a4_linear_g_f32",
     "convrot_w4a4_quantize_g",
+    "asym_w4a8_workspace_size", "asym_w4a8_gemm", "asym_w4a8_gemm_f32", "asym_w4a8_gemm_s32", "asym_w4a8_linear",
+    "asym_w4a8_linear_f32",
 ]
 
 # int8 formats (include/convrot.h, w8a8_format_t)
@@ -110,6 +112,13 @@ def load_library():
     lib.w8a8_gemm_s32.argtypes = [P, P, I, I, I, P, P]
     lib.w8a8_linear.argtypes = [P, P, P, P, I, I, I, I, P, P, Z, P]
     lib.w8a8_linear_f32.argtypes = [P, P, P, P, I, I, I, I, P, P, Z, P]
+    lib.asym_w4a8_workspace_size.argtypes = [I, I, I]
+    lib.asym_w4a8_workspace_size.restype = Z
+    lib.asym_w4a8_gemm.argtypes = [P, P, P, P, P, P, P, I, I, I, P, P]
+    lib.asym_w4a8_gemm_f32.argtypes = [P, P, P, P, P, P, P, I, I, I, P, P]
+    lib.asym_w4a8_gemm_s32.argtypes = [P, P, P, P, I, I, I, P, P]
+    lib.asym_w4a8_linear.argtypes = [P, P, P, P, P, P, I, I, I, P, P, Z, P]
+    lib.asym_w4a8_linear_f32.argtypes = [P, P, P, P, P, P, I, I, I, P, P, Z, P]
     for name in lib_status_fns():
         getattr(lib, name).restype = I
     _lib = lib
@@ -122,7 +131,8 @@ def lib_status_fns():
             "convrot_w4a4_gemm_quantized", "convrot_device_error", "convrot_selftest_timeout",
             "convrot_measure_mma_i8", "w8a8_quantize", "w8a8_pack_weight", "w8a8_gemm", "w8a8_gemm_f32",
             "w8a8_gemm_s32", "w8a8_linear", "w8a8_linear_f32", "convrot_rotate_quant_g", "convrot_pack_weight_g",
-            "convrot_w4a4_linear_g", "convrot_w4a4_linear_g_f32", "convrot_w4a4_quantize_g"]
+            "convrot_w4a4_linear_g", "convrot_w4a4_linear_g_f32", "convrot_w4a4_quantize_g", "asym_w4a8_gemm",
+            "asym_w4a8_gemm_f32", "asym_w4a8_gemm_s32", "asym_w4a8_linear", "asym_w4a8_linear_f32"]
 
 
 def _check(fn: str, rc: int):
@@ -485,6 +495,84 @@ def w8a8_linear(x, Wq8, s_w, bias=None, fmt=W8A8_INT8_TENSORWISE, out=None, work
 
 def w8a8_linear_f32(x, Wq8, s_w, bias=None, fmt=W8A8_INT8_TENSORWISE, out=None, workspace=None, stream=None):
     return _linear8("w8a8_linear_f32", torch.float32, x, Wq8, s_w, bias, fmt, out, workspace, stream)
+
+
+# ---- asymmetric W4A8: idx [N, K/2] uint8, s_rel [N, K/16] uint8 (e4m3 bytes),
+# codebook [16] fp32, s_channel [N] fp32; activations from
+# w8a8_quantize(x, W8A8_CONVROT_INT8_ROW)
+
+def asym_w4a8_workspace_size(M: int, N: int, K: int) -> int:
+    return int(load_library().asym_w4a8_workspace_size(M, N, K))
+
+
+def _need_asym(idx, s_rel, codebook, s_channel, K):
+    N = idx.shape[0]
+    _need(idx, "idx", torch.uint8, (N, K // 2))
+    _need(s_rel, "s_rel", torch.uint8, (N, K // 16))
+    _need(codebook, "codebook", torch.float32, (16,))
+    _need(s_channel, "s_channel", torch.float32, (N,))
+    return N
+
+
+def _gemm_asym(fn_name, out_dtype, x8, s_a, idx, s_rel, codebook, s_channel, bias, out, stream):
+    M, K = x8.shape
+    _need(x8, "x8", torch.int8)
+    N = _need_asym(idx, s_rel, codebook, s_channel, K)
+    _need(s_a, "s_a", torch.float32, (M,))
+    _need(bias, "bias", torch.bfloat16, (N,))
+    out = torch.empty((M, N), dtype=out_dtype, device=x8.device) if out is None else out
+    _need(out, "out", out_dtype, (M, N))
+    _check(fn_name, getattr(load_library(), fn_name)(_ptr(x8), _ptr(s_a), _ptr(idx), _ptr(s_rel), _ptr(codebook),
+                                                     _ptr(s_channel), _ptr(bias), M, N, K, _ptr(out),
+                                                     _stream(stream)))
+    return out
+
+
+def asym_w4a8_gemm(x8, s_a, idx, s_rel, codebook, s_channel, bias=None, out=None, stream=None):
+    return _gemm_asym("asym_w4a8_gemm", torch.bfloat16, x8, s_a, idx, s_rel, codebook, s_channel, bias, out, stream)
+
+
+def asym_w4a8_gemm_f32(x8, s_a, idx, s_rel, codebook, s_channel, bias=None, out=None, stream=None):
+    return _gemm_asym("asym_w4a8_gemm_f32", torch.float32, x8, s_a, idx, s_rel, codebook, s_channel, bias, out,
+                      stream)
+
+
+def asym_w4a8_gemm_s32(x8, idx, s_rel, codebook, out=None, stream=None):
+    M, K = x8.shape
+    _need(x8, "x8", torch.int8)
+    N = idx.shape[0]
+    _need(idx, "idx", torch.uint8, (N, K // 2))
+    _need(s_rel, "s_rel", torch.uint8, (N, K // 16))
+    _need(codebook, "codebook", torch.float32, (16,))
+    out = torch.empty((M, N), dtype=torch.int32, device=x8.device) if out is None else out
+    _need(out, "out", torch.int32, (M, N))
+    _check("asym_w4a8_gemm_s32", load_library().asym_w4a8_gemm_s32(_ptr(x8), _ptr(idx), _ptr(s_rel), _ptr(codebook),
+                                                                   M, N, K, _ptr(out), _stream(stream)))
+    return out
+
+
+def _linear_asym(fn_name, out_dtype, x, idx, s_rel, codebook, s_channel, bias, out, workspace, stream):
+    M, K = x.shape
+    _need(x, "x", torch.bfloat16)
+    N = _need_asym(idx, s_rel, codebook, s_channel, K)
+    _need(bias, "bias", torch.bfloat16, (N,))
+    out = torch.empty((M, N), dtype=out_dtype, device=x.device) if out is None else out
+    _need(out, "out", out_dtype, (M, N))
+    ws = _workspace(workspace, asym_w4a8_workspace_size(M, N, K), x.device)
+    _check(fn_name, getattr(load_library(), fn_name)(_ptr(x), _ptr(idx), _ptr(s_rel), _ptr(codebook), _ptr(s_channel),
+                                                     _ptr(bias), M, N, K, _ptr(out), _ptr(ws), ws.numel(),
+                                                     _stream(stream)))
+    return out
+
+
+def asym_w4a8_linear(x, idx, s_rel, codebook, s_channel, bias=None, out=None, workspace=None, stream=None):
+    return _linear_asym("asym_w4a8_linear", torch.bfloat16, x, idx, s_rel, codebook, s_channel, bias, out, workspace,
+                        stream)
+
+
+def asym_w4a8_linear_f32(x, idx, s_rel, codebook, s_channel, bias=None, out=None, workspace=None, stream=None):
+    return _linear_asym("asym_w4a8_linear_f32", torch.float32, x, idx, s_rel, codebook, s_channel, bias, out,
+                        workspace, stream)
 
 
 def convrot_version() -> str:

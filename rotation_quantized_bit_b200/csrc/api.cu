@@ -199,10 +199,10 @@ convrot_status_t gemm8_common(const int8_t* x8, const float* s_x, const int8_t* 
   st = check_device(&sms);
   if (st != CONVROT_OK) return st;
   GemmArgs a{x8, s_x, reinterpret_cast<const uint8_t*>(Wq8), s_w, bias, out, M, N, K};
-  a.w8 = 1;
+  a.wkind = kWInt8;
   a.sa_stride = format == W8A8_CONVROT_INT8_ROW ? 1 : 0;
   a.sw_stride = format == W8A8_CONVROT_INT8_ROW ? 1 : 0;
-  return from_cuda(launch_w4a4_gemm(a, sink, choose_tiling(M, N, K, sms, true), static_cast<cudaStream_t>(stream)));
+  return from_cuda(launch_w4a4_gemm(a, sink, choose_tiling(M, N, K, sms, kWInt8), static_cast<cudaStream_t>(stream)));
 }
 
 convrot_status_t linear8_common(const uint16_t* x, const int8_t* Wq8, const float* s_w, const uint16_t* bias, int M,
@@ -220,6 +220,45 @@ convrot_status_t linear8_common(const uint16_t* x, const int8_t* Wq8, const floa
   st = quant8_common(x, M, K, format, codes, scales, base + w8_scratch_offset(M, K), 256, stream);
   if (st != CONVROT_OK) return st;
   return gemm8_common(codes, scales, Wq8, s_w, bias, M, N, K, format, out, sink, stream);
+}
+
+// ---- asymmetric W4A8 (codebook weights)
+
+convrot_status_t gemm_cb_common(const int8_t* x8, const float* s_a, const uint8_t* idx, const uint8_t* s_rel,
+                                const float* codebook, const float* s_channel, const uint16_t* bias, int M, int N,
+                                int K, void* out, GemmSink sink, void* stream) {
+  if (!x8 || !idx || !s_rel || !codebook || !out) return CONVROT_ERR_NULL;
+  if (sink != GemmSink::kS32 && (!s_a || !s_channel)) return CONVROT_ERR_NULL;
+  convrot_status_t st = check_mnk(M, N, K);
+  if (st != CONVROT_OK) return st;
+  if (!aligned16(x8) || !aligned16(idx) || !aligned16(s_rel) || !aligned16(codebook) || !aligned16(out) ||
+      (s_a && !aligned16(s_a)) || (s_channel && !aligned16(s_channel)) || (bias && !aligned16(bias)))
+    return CONVROT_ERR_ALIGN;
+  int sms = 0;
+  st = check_device(&sms);
+  if (st != CONVROT_OK) return st;
+  GemmArgs a{x8, s_a, idx, s_channel, bias, out, M, N, K};
+  a.wkind = kWCodebook;
+  a.s_rel = s_rel;
+  a.codebook = codebook;
+  return from_cuda(
+      launch_w4a4_gemm(a, sink, choose_tiling(M, N, K, sms, kWCodebook), static_cast<cudaStream_t>(stream)));
+}
+
+convrot_status_t linear_cb_common(const uint16_t* x, const uint8_t* idx, const uint8_t* s_rel, const float* codebook,
+                                  const float* s_channel, const uint16_t* bias, int M, int N, int K, void* out,
+                                  GemmSink sink, void* ws, size_t ws_bytes, void* stream) {
+  if (!x || !idx || !s_rel || !codebook || !s_channel || !out) return CONVROT_ERR_NULL;
+  convrot_status_t st = check_mnk(M, N, K);
+  if (st != CONVROT_OK) return st;
+  if (!ws || ws_bytes < w8_workspace_bytes(M, K)) return CONVROT_ERR_WORKSPACE;
+  if (!aligned16(ws)) return CONVROT_ERR_ALIGN;
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  int8_t* codes = reinterpret_cast<int8_t*>(base);
+  float* scales = reinterpret_cast<float*>(base + w8_scales_offset(M, K));
+  st = quant8_common(x, M, K, W8A8_CONVROT_INT8_ROW, codes, scales, base + w8_scratch_offset(M, K), 256, stream);
+  if (st != CONVROT_OK) return st;
+  return gemm_cb_common(codes, scales, idx, s_rel, codebook, s_channel, bias, M, N, K, out, sink, stream);
 }
 
 }  // namespace
@@ -482,6 +521,47 @@ convrot_status_t convrot_w4a4_linear_g_f32(const uint16_t* x, const uint8_t* Wq,
                                            const uint16_t* bias, int M, int N, int K, int group, float* y32,
                                            void* workspace, size_t workspace_bytes, void* stream) {
   return linear_common(x, Wq, s_w, bias, M, N, K, y32, GemmSink::kF32, workspace, workspace_bytes, stream, group);
+}
+
+}  // extern "C"
+
+extern "C" {
+
+size_t asym_w4a8_workspace_size(int M, int N, int K) {
+  if (check_mnk(M, N, K) != CONVROT_OK) return 0;
+  return w8_workspace_bytes(M, K);
+}
+
+convrot_status_t asym_w4a8_gemm(const int8_t* x8, const float* s_a, const uint8_t* idx, const uint8_t* s_rel,
+                                const float* codebook, const float* s_channel, const uint16_t* bias, int M, int N,
+                                int K, uint16_t* y, void* stream) {
+  return gemm_cb_common(x8, s_a, idx, s_rel, codebook, s_channel, bias, M, N, K, y, GemmSink::kBF16, stream);
+}
+
+convrot_status_t asym_w4a8_gemm_f32(const int8_t* x8, const float* s_a, const uint8_t* idx, const uint8_t* s_rel,
+                                    const float* codebook, const float* s_channel, const uint16_t* bias, int M,
+                                    int N, int K, float* y32, void* stream) {
+  return gemm_cb_common(x8, s_a, idx, s_rel, codebook, s_channel, bias, M, N, K, y32, GemmSink::kF32, stream);
+}
+
+convrot_status_t asym_w4a8_gemm_s32(const int8_t* x8, const uint8_t* idx, const uint8_t* s_rel,
+                                    const float* codebook, int M, int N, int K, int32_t* acc, void* stream) {
+  return gemm_cb_common(x8, nullptr, idx, s_rel, codebook, nullptr, nullptr, M, N, K, acc, GemmSink::kS32, stream);
+}
+
+convrot_status_t asym_w4a8_linear(const uint16_t* x, const uint8_t* idx, const uint8_t* s_rel, const float* codebook,
+                                  const float* s_channel, const uint16_t* bias, int M, int N, int K, uint16_t* y,
+                                  void* workspace, size_t workspace_bytes, void* stream) {
+  return linear_cb_common(x, idx, s_rel, codebook, s_channel, bias, M, N, K, y, GemmSink::kBF16, workspace,
+                          workspace_bytes, stream);
+}
+
+convrot_status_t asym_w4a8_linear_f32(const uint16_t* x, const uint8_t* idx, const uint8_t* s_rel,
+                                      const float* codebook, const float* s_channel, const uint16_t* bias, int M,
+                                      int N, int K, float* y32, void* workspace, size_t workspace_bytes,
+                                      void* stream) {
+  return linear_cb_common(x, idx, s_rel, codebook, s_channel, bias, M, N, K, y32, GemmSink::kF32, workspace,
+                          workspace_bytes, stream);
 }
 
 }  // extern "C"

@@ -25,10 +25,17 @@
 //     chunk order, so the contraction pairs the right codes;
 //   * the accumulator is exactly 16 * acc (|16 acc| <= 1024 K < 2^31), and
 //     the epilogue shifts it right by 4.
-// The W8A8 formats (int8 weights [N, K]) use the same kernel with W8 = true:
+// The W8A8 formats (int8 weights [N, K]) use the same kernel with WK = kWInt8:
 // the weight tile goes by TMA straight into shared memory as the MMA's A
 // operand (no unpack, no tensor-memory A slots), the accumulator is the
 // integer product itself, and per-tensor scales are read with stride 0.
+// The asymmetric W4A8 format (WK = kWCodebook; "Nicolaslas/Rebels_w4a8s",
+// "What's inside a file") stores 4-bit indices into a 16-level codebook, an
+// e4m3 scale per 16 weights along K and a scale per output channel.  Its
+// weights take the 4-bit path, but the unpack warps decode each index to
+// the int8 weight clamp(rint(level * s_rel), -127, 127) through a per-CTA
+// table (16 levels for each of the 256 scale bytes), in natural K order to
+// match int8 activation codes; the accumulator is the plain integer sum.
 // Work is cut into units of one 256-wide K block of one output tile; see
 // the kernel below for the two schedules (whole tiles, and K split over a
 // thread-block cluster when there are few tiles) and the exact reduction of
@@ -54,6 +61,8 @@ constexpr int kXBox = 128;       // K bytes per activation TMA box (the 128-byte
 constexpr int kMaxStages = 16;   // depth limit of the shared-memory TMA ring
 constexpr int kDoneRing = 32;    // MMA completion barriers, one per unit mod 32 (>= stages, >= A slots)
 constexpr int kMaxASlots = 8;    // tensor-memory A slots (64 columns each)
+constexpr int kSRelTileBytes = kRows * kKB / 16;  // 2 KB of e4m3 group scales per unit (codebook weights)
+constexpr int kLutBytes = 256 * 16;               // decoded levels per scale byte (codebook weights)
 
 // One packed weight row of a unit (128 bytes = 256 codes) -> 64 tensor-memory
 // columns of signed bytes.  The tile landed with the 128-byte TMA swizzle:
@@ -77,6 +86,82 @@ __device__ __forceinline__ void unpack_row_to_tmem(const uint8_t* wstage, int ro
   }
 }
 
+// Byte permute with the sign-replicate mode: byte i of the result is byte
+// (c >> 4i) & 7 of {b, a} (a = bytes 0..3), or, when bit 3 of that selector
+// nibble is set, that byte's top bit copied into all 8 bits.
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t d;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+
+// Four 4-bit indices (the low 16 bits of s, index i in bits 4i..4i+3) -> the
+// four int8 levels lut[index] of the 16-byte row (t0..t3).  Indices 0..7 come
+// from {t1, t0}, 8..15 from {t3, t2}; the per-byte choice is the index's bit
+// 3, turned into a 0x00 / 0xFF byte mask by the sign-replicate mode (the top
+// bit of byte 0 of s << 4 is bit 3 of index 0, of byte 0 of s bit 3 of
+// index 1, and so on: selectors 8, C, 9, D).
+__device__ __forceinline__ uint32_t decode4(uint32_t s, const uint4& t) {
+  const uint32_t sel = s & 0x7777u;
+  const uint32_t lo = prmt(t.x, t.y, sel);
+  const uint32_t hi = prmt(t.z, t.w, sel);
+  const uint32_t mask = prmt(s << 4, s, 0xD9C8u);
+  return (hi & mask) | (lo & ~mask);
+}
+
+// One weight row of a unit in codebook form (128 bytes = 256 indices, the
+// 128-byte TMA swizzle as above; srow: the row's 16 e4m3 scale bytes, one
+// per 16 indices) -> 64 tensor-memory columns of int8 weights in natural K
+// order (column c holds k = 4c .. 4c + 3).  lut[b * 16 + i] is the int8
+// weight of index i under scale byte b.
+__device__ __forceinline__ void decode_row_to_tmem(const uint8_t* wstage, const uint8_t* srow, const uint8_t* lut,
+                                                   int row, uint32_t taddr) {
+  const int sw = row & 7;
+  const uint4 sv = *reinterpret_cast<const uint4*>(srow);
+  const uint32_t sb[4] = {sv.x, sv.y, sv.z, sv.w};
+#pragma unroll
+  for (int qt = 0; qt < 4; ++qt) {  // quarter row: 64 indices -> 16 columns
+    uint32_t cols[16];
+#pragma unroll
+    for (int c2 = 0; c2 < 2; ++c2) {
+      const int cc = 2 * qt + c2;  // 16-byte chunk: indices k = 32 cc .. 32 cc + 31
+      const uint4 v = *reinterpret_cast<const uint4*>(wstage + row * 128 + ((cc ^ sw) << 4));
+      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int gg = 0; gg < 2; ++gg) {
+        const int g = 2 * cc + gg;  // group of 16 indices within the unit
+        const uint32_t b = (sb[g >> 2] >> (8 * (g & 3))) & 0xFFu;
+        const uint4 t = *reinterpret_cast<const uint4*>(lut + 16 * b);
+#pragma unroll
+        for (int jj = 0; jj < 2; ++jj) {
+          const int j = 2 * gg + jj;  // word j of the chunk: indices k = 32 cc + 8j .. + 7
+          cols[8 * c2 + 2 * j] = decode4(w[j], t);
+          cols[8 * c2 + 2 * j + 1] = decode4(w[j] >> 16, t);
+        }
+      }
+    }
+    tmem_st_32x32b_x16(taddr + 16u * qt, cols);
+  }
+}
+
+// e4m3 ("fn": bias 7, no infinities, S.1111.111 = NaN) byte -> fp32, exactly.
+__device__ __forceinline__ float e4m3_to_float(uint32_t b) {
+  const uint32_t e = (b >> 3) & 15u, m = b & 7u;
+  float mag = e == 0 ? __fmul_rn(static_cast<float>(m), 0.001953125f)  // m * 2^-9
+                     : __uint_as_float(((e + 120u) << 23) | (m << 20));
+  if (e == 15u && m == 7u) mag = __uint_as_float(0x7FC00000u);
+  return (b & 0x80u) ? -mag : mag;
+}
+
+// The decoded weight of one level under one scale: rint(level * s) clamped
+// to [-127, 127], NaN -> 0.
+__device__ __forceinline__ int32_t decode_level(float level, float s) {
+  float p = __fmul_rn(level, s);
+  if (p != p) return 0;
+  p = fminf(fmaxf(p, -127.0f), 127.0f);
+  return __float2int_rn(p);
+}
+
 // int32 -> fp32 without the conversion unit: for |i| < 2^22 the float with
 // bits 0x4B400000 + i is exactly 1.5 * 2^23 + i, and subtracting 1.5 * 2^23
 // leaves exactly i (the value a correctly rounded conversion gives, since i
@@ -95,22 +180,24 @@ __device__ __forceinline__ uint16_t bf16_bits_rne(float y) {
 // One output element from the MMA sum (16 * acc): scales and bias already
 // loaded by the caller.
 // The accumulator as a float: the W4A4 sum (|acc| <= 2^21) by the exact
-// bit trick, the W8A8 sum (up to 127^2 K) by a correctly rounded conversion.
-template <bool W8>
+// bit trick, the 8-bit sums (up to 127^2 K) by a correctly rounded
+// conversion.  PLAIN: the MMA sum is the accumulator itself (8-bit weights
+// or decoded codebook weights), not 16 * acc.
+template <bool PLAIN>
 __device__ __forceinline__ float acc_to_float(int32_t acc) {
-  return W8 ? __int2float_rn(acc) : int_to_float_exact(acc);
+  return PLAIN ? __int2float_rn(acc) : int_to_float_exact(acc);
 }
 
-template <int SINK, bool W8, class P>
+template <int SINK, bool PLAIN, class P>
 __device__ __forceinline__ void store_output(const P& p, int m, int n, int32_t dsum, float sa, float sw,
                                              float bv) {
-  const int32_t acc = W8 ? dsum : dsum >> 4;  // 4-bit weights entered the MMA as 16 * q_w
+  const int32_t acc = PLAIN ? dsum : dsum >> 4;  // 4-bit weights entered the MMA as 16 * q_w
   const size_t idx = static_cast<size_t>(m) * p.N + n;
   if (SINK == static_cast<int>(GemmSink::kS32)) {
     static_cast<int32_t*>(p.out)[idx] = acc;
     return;
   }
-  float y = __fmul_rn(__fmul_rn(acc_to_float<W8>(acc), sa), sw);
+  float y = __fmul_rn(__fmul_rn(acc_to_float<PLAIN>(acc), sa), sw);
   if (p.bias) y = __fadd_rn(y, bv);
   if (SINK == static_cast<int>(GemmSink::kF32)) {
     static_cast<float*>(p.out)[idx] = y;
@@ -122,7 +209,7 @@ __device__ __forceinline__ void store_output(const P& p, int m, int n, int32_t d
 // Outputs of one 32-token chunk of one output channel n: tokens m .. m +
 // count - 1 (count <= 32), accumulators v (16 * acc), token scales sa[0..31]
 // (16-byte aligned in shared memory).
-template <int SINK, bool W8, class P>
+template <int SINK, bool PLAIN, class P>
 __device__ __forceinline__ void store_chunk(const P& p, int m, int n, const uint32_t (&v)[32], const float* sa,
                                             float sw, float bv, int count) {
   const size_t ld = static_cast<size_t>(p.N);
@@ -131,7 +218,7 @@ __device__ __forceinline__ void store_chunk(const P& p, int m, int n, const uint
     int32_t* o = static_cast<int32_t*>(p.out) + base;
 #pragma unroll
     for (int j = 0; j < 32; ++j)
-      if (j < count) o[j * ld] = W8 ? static_cast<int32_t>(v[j]) : static_cast<int32_t>(v[j]) >> 4;
+      if (j < count) o[j * ld] = PLAIN ? static_cast<int32_t>(v[j]) : static_cast<int32_t>(v[j]) >> 4;
     return;
   }
   const float4* sa4 = reinterpret_cast<const float4*>(sa);
@@ -143,8 +230,8 @@ __device__ __forceinline__ void store_chunk(const P& p, int m, int n, const uint
     for (int r = 0; r < 4; ++r) {
       const int j = 4 * q + r;
       if (j < count) {
-        const int32_t acc = W8 ? static_cast<int32_t>(v[j]) : static_cast<int32_t>(v[j]) >> 4;
-        float y = __fmul_rn(__fmul_rn(acc_to_float<W8>(acc), sv[r]), sw);
+        const int32_t acc = PLAIN ? static_cast<int32_t>(v[j]) : static_cast<int32_t>(v[j]) >> 4;
+        float y = __fmul_rn(__fmul_rn(acc_to_float<PLAIN>(acc), sv[r]), sw);
         if (p.bias) y = __fadd_rn(y, bv);
         if (SINK == static_cast<int>(GemmSink::kF32))
           static_cast<float*>(p.out)[base + j * ld] = y;
@@ -201,6 +288,8 @@ struct PParams {
   int pair;         // the MMA thread issues two units per group
   int sa_stride;    // 0: one activation scale for every row
   int sw_stride;    // 0: one weight scale for every output channel
+  const float* codebook;  // [16] levels (codebook weights)
+  int lut_off;      // shared-memory offset of the decode table from the header (codebook weights)
 };
 
 struct PHeader {
@@ -233,10 +322,13 @@ __device__ __forceinline__ void unit_next(const PParams& p, int& tile, int& kb) 
   }
 }
 
-template <int SINK, bool W8>
+template <int SINK, int WK>
 __global__ void __launch_bounds__(kPThreads, 1)
     w4a4_tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_x,
-                        const __grid_constant__ PParams p) {
+                        const __grid_constant__ CUtensorMap tm_s, const __grid_constant__ PParams p) {
+  constexpr bool W8 = WK == kWInt8;       // int8 weights: shared-memory A operand, no unpack
+  constexpr bool CB = WK == kWCodebook;   // codebook indices + group scales, decoded by the unpack warps
+  constexpr bool PLAIN = WK != kW4;       // the MMA sum is the accumulator itself
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   // The next kernel on the stream (launched with programmatic stream
@@ -246,7 +338,9 @@ __global__ void __launch_bounds__(kPThreads, 1)
   pdl_launch_dependents();
   const int BT = p.BT;
   const int ns = p.nstages;
-  constexpr int kWBytes = W8 ? 2 * kWTileBytes : kWTileBytes;  // weight bytes of a unit
+  // Weight bytes of a unit: int8 [128 x 256]; packed [128 x 128] (+ the
+  // [128 x 16] e4m3 group scales for codebook weights).
+  constexpr int kWBytes = W8 ? 2 * kWTileBytes : (CB ? kWTileBytes + kSRelTileBytes : kWTileBytes);
   const int stage_bytes = kWBytes + BT * kKB;
   const int nas = p.a_slots;
   const uint32_t a_col0 = 2u * static_cast<uint32_t>(p.acc_stride);
@@ -276,6 +370,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
     fence_mbarrier_init();
     prefetch_tmap(&tm_w);
     prefetch_tmap(&tm_x);
+    if (CB) prefetch_tmap(&tm_s);
   }
   if (warp == 1) {
     tmem_alloc(&hdr->tmem_base, 512u);
@@ -298,8 +393,9 @@ __global__ void __launch_bounds__(kPThreads, 1)
           tma_load_2d(smem + s * stage_bytes, &tm_w, &hdr->ready[s], kb * kKB, w_row(tile));
           tma_load_2d(smem + s * stage_bytes + kWTileBytes, &tm_w, &hdr->ready[s], kb * kKB + kXBox, w_row(tile));
         } else {
-          mbar_arrive_expect_tx(&hdr->wfull[s], static_cast<uint32_t>(kWTileBytes));
+          mbar_arrive_expect_tx(&hdr->wfull[s], static_cast<uint32_t>(kWBytes));
           tma_load_2d(smem + s * stage_bytes, &tm_w, &hdr->wfull[s], kb * (kKB / 2), w_row(tile));
+          if (CB) tma_load_2d(smem + s * stage_bytes + kWTileBytes, &tm_s, &hdr->wfull[s], kb * (kKB / 16), w_row(tile));
         }
       };
       auto load_x = [&](int s, int tile, int kb) {
@@ -432,6 +528,24 @@ __global__ void __launch_bounds__(kPThreads, 1)
     const int quad = warp & 3;
     const int row = quad * 32 + lane;
     const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
+    uint8_t* lut = reinterpret_cast<uint8_t*>(hdr) + p.lut_off;
+    if (CB) {
+      // The decode table: for each e4m3 scale byte b (two per thread), the 16
+      // int8 weights of the codebook levels under that scale.
+      const int ut = threadIdx.x - 64;  // 0 .. 127
+      for (int r = 0; r < 2; ++r) {
+        const uint32_t b = static_cast<uint32_t>(ut + 128 * r);
+        const float sc = e4m3_to_float(b);
+        for (int w = 0; w < 4; ++w) {
+          uint32_t q = 0;
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            q |= (static_cast<uint32_t>(decode_level(__ldg(p.codebook + 4 * w + i), sc)) & 0xFFu) << (8 * i);
+          *reinterpret_cast<uint32_t*>(lut + 16 * b + 4 * w) = q;
+        }
+      }
+      named_barrier(2, 128);  // the four unpack warps
+    }
     for (int it = 0, s = 0, ph = 0, a = 0; !W8 && it < total; ++it) {
       bool w = mbar_wait(&hdr->wfull[s], ph & 1);
       if (w && it >= nas) {
@@ -440,7 +554,11 @@ __global__ void __launch_bounds__(kPThreads, 1)
       }
       if (!__all_sync(0xffffffffu, w)) break;  // tcgen05.st below is warp-collective
       tc_fence_after();
-      unpack_row_to_tmem(smem + s * stage_bytes, row, tmem + lane_base + a_col0 + 64u * static_cast<uint32_t>(a));
+      const uint32_t taddr = tmem + lane_base + a_col0 + 64u * static_cast<uint32_t>(a);
+      if (CB)
+        decode_row_to_tmem(smem + s * stage_bytes, smem + s * stage_bytes + kWTileBytes + 16 * row, lut, row, taddr);
+      else
+        unpack_row_to_tmem(smem + s * stage_bytes, row, taddr);
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
@@ -491,7 +609,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
           tmem_ld_32x32b_x32(acc + static_cast<uint32_t>(c), v);
           tmem_wait_ld();
           const int count = min(min(32, BT - c), p.M - (m0 + c));
-          if (n < p.N && count > 0) store_chunk<SINK, W8>(p, m0 + c, n, v, sa + c, sw, bv, count);
+          if (n < p.N && count > 0) store_chunk<SINK, PLAIN>(p, m0 + c, n, v, sa + c, sw, bv, count);
         }
       } else {
         // Push the partial tile to its owners: 4-token group g belongs to CTA
@@ -571,7 +689,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
           const int m = m0 + 4 * g + q;
           if (m < p.M) {
             const float sa = SINK != static_cast<int>(GemmSink::kS32) ? sa_buf[m - m0] : 0.0f;
-            store_output<SINK, W8>(p, m, n, sv[q], sa, sw, bv);
+            store_output<SINK, PLAIN>(p, m, n, sv[q], sa, sw, bv);
           }
         }
       }
@@ -620,11 +738,11 @@ bool make_map_u8(CUtensorMap* map, const void* base, uint64_t rows, uint64_t col
   return r == CUDA_SUCCESS;
 }
 
-template <int SINK, bool W8>
-cudaError_t launch_sink(const CUtensorMap& tw, const CUtensorMap& tx, const PParams& prm, const GemmTiling& t,
-                        cudaStream_t stream) {
+template <int SINK, int WK>
+cudaError_t launch_sink(const CUtensorMap& tw, const CUtensorMap& tx, const CUtensorMap& ts, const PParams& prm,
+                        const GemmTiling& t, cudaStream_t stream) {
   static int cache[64] = {0};
-  const void* kfn = reinterpret_cast<const void*>(w4a4_tc_gemm_kernel<SINK, W8>);
+  const void* kfn = reinterpret_cast<const void*>(w4a4_tc_gemm_kernel<SINK, WK>);
   cudaError_t e = ensure_dynamic_smem(kfn, t.smem_bytes, cache);
   if (e != cudaSuccess) return note_cuda(e, "w4a4_gemm: dynamic shared memory attribute");
   cudaLaunchConfig_t cfg = {};
@@ -646,7 +764,7 @@ cudaError_t launch_sink(const CUtensorMap& tw, const CUtensorMap& tx, const PPar
   }
   cfg.attrs = attr;
   cfg.numAttrs = nattr;
-  return note_cuda(cudaLaunchKernelEx(&cfg, w4a4_tc_gemm_kernel<SINK, W8>, tw, tx, prm), "w4a4_gemm: launch");
+  return note_cuda(cudaLaunchKernelEx(&cfg, w4a4_tc_gemm_kernel<SINK, WK>, tw, tx, ts, prm), "w4a4_gemm: launch");
 }
 
 // Clusters of S CTAs (one CTA per SM) that can be resident at once on the
@@ -658,7 +776,7 @@ int max_active_clusters(int S, int num_sms) {
   if (cache[dev][S] > 0) return cache[dev][S];
   static int smem_cache[64] = {0};
   const int smem = 200 * 1024;
-  const void* kfn = reinterpret_cast<const void*>(w4a4_tc_gemm_kernel<0, false>);
+  const void* kfn = reinterpret_cast<const void*>(w4a4_tc_gemm_kernel<0, kW4>);
   int n = 0;
   if (ensure_dynamic_smem(kfn, smem, smem_cache) == cudaSuccess) {
     cudaLaunchConfig_t cfg = {};
@@ -672,7 +790,7 @@ int max_active_clusters(int S, int num_sms) {
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (cudaOccupancyMaxActiveClusters(&n, w4a4_tc_gemm_kernel<0, false>, &cfg) != cudaSuccess) n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, w4a4_tc_gemm_kernel<0, kW4>, &cfg) != cudaSuccess) n = 0;
   }
   cudaGetLastError();  // a failed query is not an error of the caller
   if (n <= 0) n = num_sms / (2 * S);
@@ -686,7 +804,8 @@ int max_active_clusters(int S, int num_sms) {
 // memory plus the unit's fixed costs, fitted to measured runs of this kernel
 // as about 700 + 3.2 * BT cycles (the BT-dependent part is the BT x 256
 // activation bytes); with int8 weights the weight tile is twice as large.
-long persistent_cost(int M, int N, int K, int BT, int num_sms, bool w8) {
+long persistent_cost(int M, int N, int K, int BT, int num_sms, int wk) {
+  const bool w8 = wk == kWInt8;
   const long tiles = static_cast<long>((M + BT - 1) / BT) * ((N + kRows - 1) / kRows);
   const long rounds = (tiles + num_sms - 1) / num_sms;
   const long mma = 4L * BT;
@@ -702,17 +821,23 @@ namespace {
 // groups x 128 rows x 16 bytes.
 int red_bytes(int BT, int S) { return S > 1 ? S * ((BT / 4 + S - 1) / S) * kRows * 16 : 0; }
 
+// Weight bytes of one unit's stage for a weight kind.
+int weight_stage_bytes(int wk) {
+  return wk == kWInt8 ? 2 * kWTileBytes : (wk == kWCodebook ? kWTileBytes + kSRelTileBytes : kWTileBytes);
+}
+
 // Stages of BT-token units that fit the shared memory of one CTA next to the
-// header (1 KB), the s_a staging (1.5 KB) and the split-K buffer, and the
-// dynamic shared memory for them (padded so that one CTA, which owns all of
-// tensor memory, occupies an SM).
-void set_stages(GemmTiling& t, bool w8) {
-  const int stage = (w8 ? 2 : 1) * kWTileBytes + t.BT * kKB;
+// header (1 KB), the s_a staging (1.5 KB), the split-K buffer and (codebook
+// weights) the 4 KB decode table, and the dynamic shared memory for them
+// (padded so that one CTA, which owns all of tensor memory, occupies an SM).
+void set_stages(GemmTiling& t, int wk) {
+  const int stage = weight_stage_bytes(wk) + t.BT * kKB;
   const int rb = red_bytes(t.BT, t.splits);
-  int ns = (220 * 1024 - 4096 - rb) / stage;
+  const int lut = wk == kWCodebook ? kLutBytes : 0;
+  int ns = (220 * 1024 - 4096 - rb - lut) / stage;
   if (ns > kMaxStages) ns = kMaxStages;
   t.nstages = ns;
-  t.smem_bytes = 1024 + ns * stage + 2560 + rb;
+  t.smem_bytes = 1024 + ns * stage + 2560 + rb + lut;
   if (t.smem_bytes < 120 * 1024) t.smem_bytes = 120 * 1024;
   // Tensor memory: two accumulators of BT (rounded up to 32) columns, then
   // 64-column A slots in the rest of the 512.
@@ -723,7 +848,7 @@ void set_stages(GemmTiling& t, bool w8) {
 
 }  // namespace
 
-GemmTiling choose_tiling(int M, int N, int K, int num_sms, bool w8) {
+GemmTiling choose_tiling(int M, int N, int K, int num_sms, int wk) {
   GemmTiling t{};
   const int kbn = K / kKB;
   const int G = num_sms < kMaxGemmGrid ? num_sms : kMaxGemmGrid;
@@ -738,7 +863,7 @@ GemmTiling choose_tiling(int M, int N, int K, int num_sms, bool w8) {
     for (int bt = 192; bt >= 64; bt -= 16) {
       const long tiles = static_cast<long>((M + bt - 1) / bt) * t.n_tiles;
       if (2 * tiles < G) continue;
-      const long c = persistent_cost(M, N, K, bt, G, w8);
+      const long c = persistent_cost(M, N, K, bt, G, wk);
       if (best < 0 || c < best) {
         best = c;
         best_bt = bt;
@@ -749,7 +874,7 @@ GemmTiling choose_tiling(int M, int N, int K, int num_sms, bool w8) {
       t.m_tiles = (M + best_bt - 1) / best_bt;
       const int tiles = t.m_tiles * t.n_tiles;
       t.grid = tiles < G ? tiles : G;
-      set_stages(t, w8);
+      set_stages(t, wk);
       return t;
     }
   }
@@ -777,15 +902,24 @@ GemmTiling choose_tiling(int M, int N, int K, int num_sms, bool w8) {
     }
   }
   t.grid = t.splits > 1 ? tiles * t.splits : (tiles < G ? tiles : G);
-  set_stages(t, w8);
+  set_stages(t, wk);
   return t;
 }
 
 cudaError_t launch_w4a4_gemm(const GemmArgs& a, GemmSink sink, const GemmTiling& t, cudaStream_t stream) {
-  CUtensorMap tw, tx;
-  if (!make_map_u8(&tw, a.Wq, static_cast<uint64_t>(a.N), static_cast<uint64_t>(a.w8 ? a.K : a.K / 2), kRows,
-                   a.w8 ? kXBox : kKB / 2, CU_TENSOR_MAP_SWIZZLE_128B))
+  CUtensorMap tw, tx, ts;
+  const bool w8 = a.wkind == kWInt8;
+  if (a.wkind < kW4 || a.wkind > kWCodebook || (a.wkind == kWCodebook && (!a.s_rel || !a.codebook)))
+    return note_cuda(cudaErrorInvalidValue, "w4a4_gemm: weight kind");
+  if (!make_map_u8(&tw, a.Wq, static_cast<uint64_t>(a.N), static_cast<uint64_t>(w8 ? a.K : a.K / 2), kRows,
+                   w8 ? kXBox : kKB / 2, CU_TENSOR_MAP_SWIZZLE_128B))
     return note_cuda(cudaErrorInvalidValue, "w4a4_gemm: weight tensor map");
+  // Group scales [N, K/16]: one 16-byte row piece per output channel and unit.
+  ts = tw;
+  if (a.wkind == kWCodebook &&
+      !make_map_u8(&ts, a.s_rel, static_cast<uint64_t>(a.N), static_cast<uint64_t>(a.K / 16), kRows, kKB / 16,
+                   CU_TENSOR_MAP_SWIZZLE_NONE))
+    return note_cuda(cudaErrorInvalidValue, "w4a4_gemm: group-scale tensor map");
   if (!make_map_u8(&tx, a.xs8, static_cast<uint64_t>(a.M), static_cast<uint64_t>(a.K),
                    static_cast<uint32_t>(t.BT), kXBox, CU_TENSOR_MAP_SWIZZLE_128B))
     return note_cuda(cudaErrorInvalidValue, "w4a4_gemm: activation tensor map");
@@ -808,21 +942,32 @@ cudaError_t launch_w4a4_gemm(const GemmArgs& a, GemmSink sink, const GemmTiling&
   pp.acc_stride = t.acc_stride;
   pp.a_slots = t.a_slots;
   pp.splits = t.splits;
-  pp.pair = (t.BT <= 128 && (a.w8 || t.a_slots >= 4) && t.nstages >= 4) ? 1 : 0;
+  pp.pair = (t.BT <= 128 && (w8 || t.a_slots >= 4) && t.nstages >= 4) ? 1 : 0;
   pp.sa_stride = a.sa_stride;
   pp.sw_stride = a.sw_stride;
+  pp.codebook = a.codebook;
+  pp.lut_off = 2560 + red_bytes(t.BT, t.splits);
+  if (a.wkind == kWCodebook && t.smem_bytes < 1024 + t.nstages * (weight_stage_bytes(kWCodebook) + t.BT * kKB) +
+                                                   pp.lut_off + kLutBytes)
+    return note_cuda(cudaErrorInvalidValue, "w4a4_gemm: tiling");
   cudaError_t e;
-  if (a.w8) {
+  if (w8) {
     switch (sink) {
-      case GemmSink::kBF16: e = launch_sink<0, true>(tw, tx, pp, t, stream); break;
-      case GemmSink::kF32: e = launch_sink<1, true>(tw, tx, pp, t, stream); break;
-      default: e = launch_sink<2, true>(tw, tx, pp, t, stream); break;
+      case GemmSink::kBF16: e = launch_sink<0, kWInt8>(tw, tx, ts, pp, t, stream); break;
+      case GemmSink::kF32: e = launch_sink<1, kWInt8>(tw, tx, ts, pp, t, stream); break;
+      default: e = launch_sink<2, kWInt8>(tw, tx, ts, pp, t, stream); break;
+    }
+  } else if (a.wkind == kWCodebook) {
+    switch (sink) {
+      case GemmSink::kBF16: e = launch_sink<0, kWCodebook>(tw, tx, ts, pp, t, stream); break;
+      case GemmSink::kF32: e = launch_sink<1, kWCodebook>(tw, tx, ts, pp, t, stream); break;
+      default: e = launch_sink<2, kWCodebook>(tw, tx, ts, pp, t, stream); break;
     }
   } else {
     switch (sink) {
-      case GemmSink::kBF16: e = launch_sink<0, false>(tw, tx, pp, t, stream); break;
-      case GemmSink::kF32: e = launch_sink<1, false>(tw, tx, pp, t, stream); break;
-      default: e = launch_sink<2, false>(tw, tx, pp, t, stream); break;
+      case GemmSink::kBF16: e = launch_sink<0, kW4>(tw, tx, ts, pp, t, stream); break;
+      case GemmSink::kF32: e = launch_sink<1, kW4>(tw, tx, ts, pp, t, stream); break;
+      default: e = launch_sink<2, kW4>(tw, tx, ts, pp, t, stream); break;
     }
   }
   count_dispatch(t.splits > 1 ? 3 : 2);

@@ -49,19 +49,24 @@ struct GemmTiling {
   int a_slots;      // 64-column tensor-memory slots for unpacked weights
 };
 
-// w8: the weights are int8 codes [N, K] (the W8A8 formats) instead of packed
-// 4-bit codes [N, K/2].
-GemmTiling choose_tiling(int M, int N, int K, int num_sms, bool w8 = false);
+// Weight kinds of the tensor-core GEMM.
+constexpr int kW4 = 0;         // packed two's-complement 4-bit codes [N, K/2]
+constexpr int kWInt8 = 1;      // int8 codes [N, K] (the W8A8 formats)
+constexpr int kWCodebook = 2;  // packed 4-bit codebook indices [N, K/2], e4m3 group scales [N, K/16], codebook [16]
+
+GemmTiling choose_tiling(int M, int N, int K, int num_sms, int wkind = kW4);
 
 struct GemmArgs {
-  const int8_t* xs8;      // [M, K] activation codes (operand layout; natural order with w8)
+  const int8_t* xs8;      // [M, K] activation codes (operand layout; natural order for 8-bit codes)
   const float* s_a;       // [M], or [1] with sa_stride 0 (ignored by the s32 sink)
-  const uint8_t* Wq;      // [N, K/2] packed weight codes, or [N, K] int8 codes with w8
+  const uint8_t* Wq;      // [N, K/2] packed weight codes or indices, or [N, K] int8 codes
   const float* s_w;       // [N], or [1] with sw_stride 0
   const uint16_t* bias;   // [N] or null
   void* out;              // [M, N] bf16 / f32 / s32
   int M, N, K;
-  int w8 = 0;             // 1: int8 weights (W8A8)
+  int wkind = kW4;        // kW4, kWInt8 or kWCodebook
+  const uint8_t* s_rel = nullptr;   // [N, K/16] e4m3 group scales (kWCodebook)
+  const float* codebook = nullptr;  // [16] levels (kWCodebook)
   int sa_stride = 1;      // 0: one activation scale for every row
   int sw_stride = 1;      // 0: one weight scale for every output channel
 };

@@ -158,7 +158,8 @@ class LinearShape:
     # of it serves all of them.
     input: str = ""
     # Weight/activation format: "w4a4" (ConvRot W4A4), "int8_tensorwise" or
-    # "convrot_int8" (the int8 W8A8 formats the pages mix with W4A4).
+    # "convrot_int8" (the int8 W8A8 formats the pages mix with W4A4), or
+    # "asym_w4a8" (4-bit codebook weights, ConvRot INT8 row-scaled activations).
     fmt: str = "w4a4"
 
     @property
@@ -174,9 +175,11 @@ _ACT = {
     "small_m": act_t4_outliers,
     "edit20b_int8": act_t4_outliers,
     "qwen3_4b_mixed": act_t4_outliers,
+    "qwen3_4b_w4a8": act_t4_outliers,
+    "small_m_w4a8": act_t4_outliers,
 }
 _BASE_SEED = {"small": 0, "qwen3_4b": 1, "dit6b": 2, "edit20b": 3, "small_m": 4, "edit20b_int8": 3,
-              "qwen3_4b_mixed": 1}
+              "qwen3_4b_mixed": 1, "qwen3_4b_w4a8": 1, "small_m_w4a8": 4}
 
 
 def workload_shapes(workload: str) -> list[LinearShape]:
@@ -212,6 +215,11 @@ def workload_shapes(workload: str) -> list[LinearShape]:
             fmt = "convrot_int8" if s.name.split("@")[0] in ("q_proj", "k_proj", "v_proj", "o_proj") else "w4a4"
             out.append(dataclasses.replace(s, fmt=fmt))
         return out
+    if workload == "qwen3_4b_w4a8":
+        # the Qwen3-VL-4B text encoder's decoder Linears in the asymmetric W4A8 format
+        return [dataclasses.replace(s, fmt="asym_w4a8") for s in workload_shapes("qwen3_4b")]
+    if workload == "small_m_w4a8":
+        return [dataclasses.replace(s, fmt="asym_w4a8") for s in workload_shapes("small_m")]
     if workload == "small_m":
         kn = [(2560, 9728), (9728, 2560), (3072, 12288), (12288, 3072)]
         return [LinearShape(f"k{K}_n{N}@{M}", M, K, N) for M in (1, 8, 16, 64, 128) for (K, N) in kn]
@@ -236,3 +244,18 @@ def weights(workload: str, N: int, K: int, seed_extra: int = 0):
     """(W bf16 bits [N, K], bias bf16 bits [N])."""
     base = _BASE_SEED[workload] ^ seed_extra
     return weight(derive_seed(base, "w", N, K), N, K), bias(derive_seed(base, "b", N, K), N)
+
+
+def asym_format(workload: str, N: int, K: int, seed_extra: int = 0):
+    """Random tensors in the asymmetric W4A8 storage layout, for timing and
+    for parity at sizes the offline converter is too slow for:
+    (idx uint8 [N, K/2] uniform bytes, s_rel uint8 [N, K/16] e4m3 bytes drawn
+    uniformly from 0x50..0x70 (the values 8 .. 128), codebook fp32 [16]:
+    16 sorted N(0, 0.4) draws clipped to [-1, 1], s_channel fp32 [N]:
+    (|N(0, 1)| + 0.5) * 1e-4).  Plain random draws; no quantizer runs here."""
+    base = derive_seed(_BASE_SEED[workload] ^ seed_extra, "asym", N, K)
+    idx = (splitmix64(base, N * K // 2) & np.uint64(0xFF)).astype(np.uint8).reshape(N, K // 2)
+    s_rel = (0x50 + (splitmix64(base ^ 0x5E1, N * K // 16) % np.uint64(0x21))).astype(np.uint8).reshape(N, K // 16)
+    codebook = np.sort(np.clip(0.4 * normal(base ^ 0xC0DE, 16), -1.0, 1.0)).astype(np.float32)
+    s_channel = ((np.abs(normal(base ^ 0x5C, N)) + 0.5) * 1e-4).astype(np.float32)
+    return idx, s_rel, codebook, s_channel
