@@ -129,3 +129,38 @@ def test_int8_and_group_arguments_rejected_before_any_device_call(lib):
     assert lib.w8a8_gemm_s32(bad, good, 4, 8, 256, good, null) == 3
     # a too small workspace for the fused int8 linear
     assert lib.w8a8_linear(good, good, good, null, 4, 8, 256, 0, good, good, 16, null) == 5
+
+
+def test_asym_workspace_sizes(lib):
+    # the asymmetric W4A8 activations are the ConvRot INT8 row-scaled codes and scales
+    assert lib.asym_w4a8_workspace_size(76, 1024, 2560) == _r256(76 * 2560) + _r256(76 * 4) + 256
+    assert lib.asym_w4a8_workspace_size(1, 8, 256) == _r256(256) + _r256(4) + 256
+    assert lib.asym_w4a8_workspace_size(76, 1024, 300) == 0   # K % 256
+    assert lib.asym_w4a8_workspace_size(76, 1020, 2560) == 0  # N % 8
+    assert lib.asym_w4a8_workspace_size(0, 8, 256) == 0       # M >= 1
+
+
+def test_asym_arguments_rejected_before_any_device_call(lib):
+    P = ctypes.c_void_p
+    buf = ctypes.create_string_buffer(1 << 16)
+    good = P(ctypes.addressof(buf) + (-ctypes.addressof(buf) % 16))
+    null = P(0)
+    # NULL operands: activations, indices, group scales, codebook; scales except for the s32 sink
+    assert lib.asym_w4a8_gemm(null, good, good, good, good, good, null, 4, 8, 256, good, null) == 1
+    assert lib.asym_w4a8_gemm(good, good, good, null, good, good, null, 4, 8, 256, good, null) == 1
+    assert lib.asym_w4a8_gemm(good, good, good, good, null, good, null, 4, 8, 256, good, null) == 1
+    assert lib.asym_w4a8_gemm_f32(good, null, good, good, good, good, null, 4, 8, 256, good, null) == 1
+    assert lib.asym_w4a8_gemm_f32(good, good, good, good, good, null, null, 4, 8, 256, good, null) == 1
+    assert lib.asym_w4a8_gemm_s32(good, good, good, null, 4, 8, 256, good, null) == 1
+    assert lib.asym_w4a8_linear(good, good, good, good, null, null, 4, 8, 256, good, good, 4096, null) == 1
+    # shapes: K % 256, N % 8, M >= 1
+    assert lib.asym_w4a8_gemm_s32(good, good, good, good, 4, 8, 128, good, null) == 2
+    assert lib.asym_w4a8_gemm_s32(good, good, good, good, 4, 12, 256, good, null) == 2
+    assert lib.asym_w4a8_gemm_s32(good, good, good, good, 0, 8, 256, good, null) == 2
+    assert lib.asym_w4a8_linear_f32(good, good, good, good, good, null, 4, 8, 300, good, good, 4096, null) == 2
+    # misaligned codebook / group scales
+    bad = P(good.value + 4)
+    assert lib.asym_w4a8_gemm_s32(good, good, good, bad, 4, 8, 256, good, null) == 3
+    assert lib.asym_w4a8_gemm_s32(good, good, bad, good, 4, 8, 256, good, null) == 3
+    # a too small workspace for the fused linear
+    assert lib.asym_w4a8_linear(good, good, good, good, good, null, 4, 8, 256, good, good, 16, null) == 5
