@@ -252,7 +252,21 @@ def cpu_baseline(shapes, workload, budget_s=15.0):
     return {"value": ops / dt / 1e12, "unit": UNIT, "cores": 1, "kind": "oracle",
             "sample": f"first {rows} rows (capped at M) of each of the {len(shapes)} linears of one step "
                       f"({ops / 1e9:.2f} GOP) in {dt:.1f} s; weight packing untimed",
-            "seconds": dt}
+            "seconds": dt, "host": host_cpu()}
+
+
+def host_cpu():
+    """The host the oracle ran on: logical CPUs and the CPU model name."""
+    model = ""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return {"logical_cpus": os.cpu_count(), "model": model}
 
 
 # ------------------------------------------------------------------ main
@@ -679,7 +693,8 @@ def reference_arm(args, shapes, config, world, rank):
             "warmup": max(args.warmup, 3), "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f32/int64", "data": "synthetic", "config": config,
             "impl": "reference",
-            "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample,
+                             "host": host_cpu()},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
