@@ -466,10 +466,13 @@ def main():
     t_grp = np.zeros(ngrp)
     t_quant = np.zeros(ngrp)
     t_gemm = np.zeros(nlin)
+    step_ms = np.zeros(args.steps)  # this rank's device time of each timed step
     for k in range(args.steps):
         for gi, (_src, idx) in enumerate(groups):
             ev = step_events[k][gi]
-            t_grp[gi] += ev[0].elapsed_time(ev[1 + len(idx)])
+            tg = ev[0].elapsed_time(ev[1 + len(idx)])
+            t_grp[gi] += tg
+            step_ms[k] += tg
             kv = kern_events[k][gi]
             t_quant[gi] += kv[0].elapsed_time(kv[1])
             for j, i in enumerate(idx):
@@ -542,7 +545,11 @@ def main():
 
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": max(world, 1), "steps": args.steps,
-        "warmup": max(args.warmup, 3), "ms_per_step": round(ms_per_step, 4), "higher_is_better": True,
+        "warmup": max(args.warmup, 3), "ms_per_step": round(ms_per_step, 4),
+        "step_ms_percentiles": {"p10": round(float(np.percentile(step_ms, 10)), 4),
+                                "median": round(float(np.median(step_ms)), 4),
+                                "p90": round(float(np.percentile(step_ms, 90)), 4), "rank": rank},
+        "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "s8", "data": "synthetic",
         "config": config, "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches,
         "clocks": clocks, "detail": detail,
