@@ -9,6 +9,7 @@
 #include <cstdint>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 
 #include "../../include/convrot.h"
 #include "kernels.cuh"
@@ -294,12 +295,17 @@ cudaError_t note_cuda(cudaError_t e, const char* where) {
   return e;
 }
 
-cudaError_t ensure_dynamic_smem(const void* kernel, int bytes, int* cache) {
+cudaError_t ensure_dynamic_smem(const void* kernel, int bytes, std::atomic<int>* cache) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-  if (bytes <= cache[dev]) return cudaSuccess;
+  if (bytes <= cache[dev].load(std::memory_order_acquire)) return cudaSuccess;
+  // Slow path, once per kernel and device: serialised, so that the limit a
+  // kernel is given only ever grows, whichever host thread gets here first.
+  static std::mutex mu;
+  std::lock_guard<std::mutex> lock(mu);
+  if (bytes <= cache[dev].load(std::memory_order_relaxed)) return cudaSuccess;
   int optin = 0;
   e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
   if (e != cudaSuccess) return e;
@@ -308,7 +314,7 @@ cudaError_t ensure_dynamic_smem(const void* kernel, int bytes, int* cache) {
   if (e != cudaSuccess) return e;
   if (bytes + static_cast<int>(fa.sharedSizeBytes) > optin) return cudaErrorInvalidValue;
   e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-  if (e == cudaSuccess) cache[dev] = bytes;
+  if (e == cudaSuccess) cache[dev].store(bytes, std::memory_order_release);
   return e;
 }
 

@@ -741,7 +741,7 @@ bool make_map_u8(CUtensorMap* map, const void* base, uint64_t rows, uint64_t col
 template <int SINK, int WK>
 cudaError_t launch_sink(const CUtensorMap& tw, const CUtensorMap& tx, const CUtensorMap& ts, const PParams& prm,
                         const GemmTiling& t, cudaStream_t stream) {
-  static int cache[64] = {0};
+  static std::atomic<int> cache[64];  // static storage: zero-initialised
   const void* kfn = reinterpret_cast<const void*>(w4a4_tc_gemm_kernel<SINK, WK>);
   cudaError_t e = ensure_dynamic_smem(kfn, t.smem_bytes, cache);
   if (e != cudaSuccess) return note_cuda(e, "w4a4_gemm: dynamic shared memory attribute");
@@ -770,11 +770,11 @@ cudaError_t launch_sink(const CUtensorMap& tw, const CUtensorMap& tx, const CUte
 // Clusters of S CTAs (one CTA per SM) that can be resident at once on the
 // current device; a conservative estimate when it cannot be queried.
 int max_active_clusters(int S, int num_sms) {
-  static int cache[64][9] = {};
+  static std::atomic<int> cache[64][9];  // clusters per device and size (0: not yet queried)
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64 || S < 1 || S > 8) return num_sms / (2 * S);
-  if (cache[dev][S] > 0) return cache[dev][S];
-  static int smem_cache[64] = {0};
+  if (cache[dev][S].load() > 0) return cache[dev][S].load();
+  static std::atomic<int> smem_cache[64];
   const int smem = 200 * 1024;
   const void* kfn = reinterpret_cast<const void*>(w4a4_tc_gemm_kernel<0, kW4>);
   int n = 0;
@@ -794,7 +794,7 @@ int max_active_clusters(int S, int num_sms) {
   }
   cudaGetLastError();  // a failed query is not an error of the caller
   if (n <= 0) n = num_sms / (2 * S);
-  cache[dev][S] = n;
+  cache[dev][S].store(n);
   return n;
 }
 

@@ -4,6 +4,7 @@
 
 #include <cuda.h>
 #include <cuda_runtime.h>
+#include <atomic>
 #include <cstdint>
 
 namespace convrot {
@@ -82,6 +83,8 @@ cudaError_t note_cuda(cudaError_t e, const char* where);
 
 // Raise a kernel's dynamic shared-memory limit to `bytes` on the current
 // device if needed (checked against the opt-in maximum minus static usage).
-cudaError_t ensure_dynamic_smem(const void* kernel, int bytes, int* cache);
+// `cache` is per kernel: one entry per device (the limit already set).  Safe
+// to call from several host threads.
+cudaError_t ensure_dynamic_smem(const void* kernel, int bytes, std::atomic<int>* cache);
 
 }  // namespace convrot

@@ -99,7 +99,7 @@ extern "C" convrot_status_t convrot_measure_mma_i8(int N, int a_in_tmem, int ite
     return CONVROT_ERR_DEVICE;
   const int grid = sms < kPeakMaxGrid ? sms : kPeakMaxGrid;
   const int smem = 1024 + 16384 + 32768;
-  static int cache[64] = {0};
+  static std::atomic<int> cache[64];
   if (ensure_dynamic_smem(reinterpret_cast<const void*>(mma_i8_rate_kernel), smem, cache) != cudaSuccess)
     return CONVROT_ERR_CUDA;
   cudaEvent_t e0, e1;

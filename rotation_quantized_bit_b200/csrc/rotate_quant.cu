@@ -430,7 +430,7 @@ int num_sms_cached() {
 
 template <int MODE, int LOG4G>
 cudaError_t launch_rq(const RQParams& p, int threads, cudaStream_t stream) {
-  static int cache[64] = {0};
+  static std::atomic<int> cache[64];
   const int smem = rq_smem_bytes(p.R, p.K, p.S, threads);
   const void* kfn = reinterpret_cast<const void*>(rotate_quant_kernel<MODE, LOG4G>);
   cudaError_t e = ensure_dynamic_smem(kfn, smem, cache);
