@@ -88,7 +88,7 @@ convrot_status_t convrot_rotate_quant(const uint16_t *x, int M, int K, uint8_t *
  * shape): the activation codes widened to bytes, M * K rounded up to 256. */
 size_t convrot_gemm_workspace_size(int M, int N, int K);
 
-/* Integer GEMM with the rank-one epilogue (the "rank-one s4 MMA", same card,
+/* Integer GEMM with the rank-one epilogue (the card's rank-one s4 MMA, same card,
  * speed table) on codes that are already quantized.
  *   xq   [M, K/2] uint8, s_a [M] float     (from convrot_rotate_quant)
  *   Wq   [N, K/2] uint8, s_w [N] float     (from convrot_pack_weight)
