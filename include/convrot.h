@@ -3,13 +3,14 @@
  *
  * The method (sources by page title and section):
  *   "Qwen-Image-Edit-2511 -- INT4 tensorwise W4A4 (+ConvRot, mixed int8
- *   fallback)", intro paragraph: weights are packed signed INT4, two codes per
- *   byte, after a group-256 regular-Hadamard ConvRot rotation; activations are
- *   rotated online and quantized dynamically to INT4 inside the kernel;
- *   calibration-free.  Same card, speed table: a fused ConvRot + rank-one s4
- *   MMA kernel (integer product rescaled by s_a[m] * s_w[n]).
- *   "rockerBOO/qwen3-4b-nvfp4-convrot", file table: group-wise Hadamard
- *   rotation, group size 256.
+ *   fallback)", intro paragraph: the weights are rotated by the ConvRot
+ *   transform (a regular Hadamard over groups of 256) and stored as signed
+ *   INT4, two codes to a byte; the activations get the same rotation at run
+ *   time and are quantized to INT4 on the fly; no calibration data is used.
+ *   Same card, speed table: one kernel does the rotation and an s4 MMA whose
+ *   integer product is rescaled by s_a[m] * s_w[n] (rank one).
+ *   "rockerBOO/qwen3-4b-nvfp4-convrot", file table: the Hadamard rotation is
+ *   applied per group of 256 channels.
  *   "Nicolaslas/Rebels_w4a8s", "What I do differently": the ConvRot group is
  *   exactly 256, so K must be divisible by 256.
  *
@@ -179,8 +180,8 @@ convrot_status_t convrot_w4a4_gemm_quantized(const uint8_t *Wq, const float *s_w
 
 /* ---- rotation group-size variants ---------------------------------------------
  * "JoaoZaokk/Z-Image-Turbo-W4A4-ConvRot", "Where Z-Image sits": the
- * convrot_groupsize ablation runs groups of 256, 64 and 16 (a rotation of size
- * N spreads each outlier over N channels).  These entry points are the ones
+ * convrot_groupsize ablation runs groups of 256, 64 and 16 (an outlier is
+ * shared out over the N channels of its rotation group).  These entry points are the ones
  * above with the group as a parameter: each group of `group` (256, 64 or 16)
  * channels is multiplied by H4 Kronecker'd log4(group) times, evaluated as
  * the first log4(group) butterfly stages of R (strides 1, 4, 16), then by

@@ -9,11 +9,12 @@
  *
  * What it computes (sources, by page title and section):
  *  - "Qwen-Image-Edit-2511 -- INT4 tensorwise W4A4 (+ConvRot, mixed int8
- *    fallback)" (HF card, intro paragraph): weights are packed signed INT4,
- *    two codes per byte, rotated with a group-256 regular-Hadamard ConvRot
- *    rotation; activations are rotated online and quantized dynamically to
- *    INT4; calibration-free.  Speed table: a "rank-one" s4 MMA kernel, i.e.
- *    the integer product is rescaled by s_a[m] * s_w[n].
+ *    fallback)" (HF card, intro paragraph): the weights go through the
+ *    ConvRot rotation (a regular Hadamard over groups of 256) and are stored
+ *    as signed INT4, two codes to a byte; the activations get the same
+ *    rotation at run time and are quantized to INT4 on the fly; no
+ *    calibration data.  Speed table: the integer product of an s4 MMA is
+ *    rescaled by s_a[m] * s_w[n] (rank one).
  *  - "rockerBOO/qwen3-4b-nvfp4-convrot" (file table): group-wise Hadamard
  *    rotation, group size 256.
  *  - "Nicolaslas/Rebels_w4a8s" ("What I do differently"): the ConvRot group is
@@ -43,8 +44,9 @@
  * The int8 formats the pages use next to W4A4 (a W8A8 path: int8 weights,
  * int8 activations, int32 accumulation, the same rank-one rescale):
  *  - "Qwen-Image-Edit-2511 -- INT4 tensorwise W4A4 (+ConvRot, mixed int8
- *    fallback)", intro: the sensitive layers (attention value/output
- *    projections) are stock "int8_tensorwise" -- read as one scale for the
+ *    fallback)", intro: the card keeps the layers that are sensitive to
+ *    quantization (among them the attention value and output projections)
+ *    in the stock "int8_tensorwise" format -- read as one scale for the
  *    whole weight tensor and one dynamic scale for the whole activation
  *    tensor, no rotation.
  *  - "rockerBOO/qwen3-4b-nvfp4-convrot", file table and notes: "ConvRot INT8

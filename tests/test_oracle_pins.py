@@ -6,7 +6,7 @@ The pins come from what the pages and the mathematics fix:
     Kronecker product built here with numpy, orthogonality H H^T = 256 I,
     symmetry, row sums of 16, exact inverse, norm preservation, and the
     outlier-spreading property ("JoaoZaokk/Z-Image-Turbo-W4A4-ConvRot", "Where
-    Z-Image sits": a rotation of size N spreads each outlier over N channels);
+    Z-Image sits": one outlier ends up shared over all N channels of its group);
   * the quantizer (amax/7, round half to even, clamp, two codes per byte):
     hand-derived ties in ``golden/quant_ties.txt``, an independent numpy
     re-derivation, power-of-two invariance;
@@ -361,8 +361,8 @@ def test_linear_error_band_and_rotation_helps_on_outliers():
 
 
 def test_larger_rotation_group_gives_lower_error():
-    # "JoaoZaokk/Z-Image-Turbo-W4A4-ConvRot", "Where Z-Image sits": a larger
-    # group mixes more and flattens outliers harder (cg 256 < 64 < 16 in error).
+    # "JoaoZaokk/Z-Image-Turbo-W4A4-ConvRot", "Where Z-Image sits": the error
+    # falls as the rotation group grows (cg 256 < 64 < 16 in error).
     x = synthetic.activations("qwen3_4b", 64, 2560)
     xf = synthetic.bf16_bits_to_f32(x).astype(np.float64)
     errs = []
