@@ -86,7 +86,10 @@ convrot_status_t convrot_rotate_quant(const uint16_t *x, int M, int K, uint8_t *
                                       void *stream);
 
 /* Bytes of workspace w4a4_gemm* needs for (M, N, K) (0 for an invalid
- * shape): the activation codes widened to bytes, M * K rounded up to 256. */
+ * shape).  M > 16: the activation codes widened to bytes, M * K rounded up
+ * to 256.  M <= 16 (the small-M kernel, which reads the packed codes as they
+ * are): 1 KB of arrival counters and the partial tiles of output tiles whose
+ * K range is split between CTAs, 2 * 160 * 128 * (M <= 8 ? 8 : 16) int32. */
 size_t convrot_gemm_workspace_size(int M, int N, int K);
 
 /* Integer GEMM with the rank-one epilogue (the card's rank-one s4 MMA, same card,
@@ -117,8 +120,9 @@ convrot_status_t w4a4_gemm_f32(const uint8_t *xq, const float *s_a, const uint8_
                                void *stream);
 
 /* Bytes of workspace convrot_w4a4_linear* needs for (M, N, K) (0 for an
- * invalid shape): the workspace of w4a4_gemm plus the M per-token scales,
- * each part rounded up to 256 bytes. */
+ * invalid shape): M * K bytes of activation codes and the M per-token
+ * scales, each part rounded up to 256 bytes; for M <= 16 followed by the
+ * small-M GEMM's counters and partial tiles (see convrot_gemm_workspace_size). */
 size_t convrot_w4a4_workspace_size(int M, int N, int K);
 
 /* The fused ConvRot W4A4 Linear: y = W4A4(x) with x rotated and quantized
@@ -128,7 +132,19 @@ size_t convrot_w4a4_workspace_size(int M, int N, int K);
  *   bias [N] bf16 bits or NULL
  *   y    [M, N] bf16 bits  (output)
  *   workspace: >= convrot_w4a4_workspace_size bytes of device scratch (holds
- *   the activation codes and scales between the two kernels). */
+ *   the activation codes and scales between the two kernels).
+ * Kernels.  M > 16: the rotate/quant prologue, then the tcgen05 tensor-core
+ * GEMM (kind::i8, accumulators in tensor memory).  M <= 16: a prologue with
+ * one CTA per token, then the bandwidth-bound small-M GEMM, which streams the
+ * packed weights with TMA into a ring of shared-memory stages and multiplies
+ * with mma.sync s8 (both operands widened from nibbles in registers).  Both
+ * give the same bits.
+ * Ordering.  Every GEMM here is launched with programmatic dependent launch:
+ * it starts streaming Wq while the preceding kernel on the stream finishes,
+ * and waits for that kernel before it reads anything else.  Wq must therefore
+ * be complete before the preceding kernel starts; convrot_pack_weight and any
+ * kernel that does not trigger its dependents early (griddepcontrol) meet
+ * this, as does a synchronisation. */
 convrot_status_t convrot_w4a4_linear(const uint16_t *x, const uint8_t *Wq, const float *s_w,
                                      const uint16_t *bias, int M, int N, int K, uint16_t *y,
                                      void *workspace, size_t workspace_bytes, void *stream);
@@ -165,17 +181,20 @@ convrot_status_t convrot_w4a4_linear_noalloc(const uint16_t *x, const uint8_t *W
  * convrot_w4a4_quantize followed by convrot_w4a4_gemm_quantized on the same
  * workspace and stream.
  *   convrot_w4a4_quantize: x [M, K] bf16 -> the workspace (activation codes
- *     in the GEMM's operand layout + per-token scales).  workspace_bytes >=
- *     convrot_w4a4_workspace_size(M, N, K) for every N it will be used with.
+ *     in the GEMM's operand layout, packed for M <= 16, + per-token scales).
+ *     workspace_bytes >= convrot_w4a4_workspace_size(M, N, K) for every N it
+ *     will be used with.
  *   convrot_w4a4_gemm_quantized: workspace (from convrot_w4a4_quantize with
- *     the same M, K) x Wq -> y [M, N] bf16.  It only reads the workspace, so
- *     one quantization may serve several GEMMs (e.g. projections that share
- *     their input). */
+ *     the same M, K) x Wq -> y [M, N] bf16.  It does not change the codes or
+ *     scales, so one quantization may serve several GEMMs (e.g. projections
+ *     that share their input), one after another on one stream: for M <= 16
+ *     the GEMM keeps its counters and partial tiles in the workspace's
+ *     scratch part (and leaves the counters at zero). */
 convrot_status_t convrot_w4a4_quantize(const uint16_t *x, int M, int K, void *workspace,
                                        size_t workspace_bytes, void *stream);
 convrot_status_t convrot_w4a4_gemm_quantized(const uint8_t *Wq, const float *s_w,
                                              const uint16_t *bias, int M, int N, int K,
-                                             uint16_t *y, const void *workspace,
+                                             uint16_t *y, void *workspace,
                                              size_t workspace_bytes, void *stream);
 
 /* ---- rotation group-size variants ---------------------------------------------
@@ -346,9 +365,10 @@ convrot_status_t convrot_selftest_timeout(unsigned int limit_us, void *stream);
 /* Host-side count of how many times each kernel path was enqueued by this
  * process: counts[0] = rotate/quant prologue, [1] = packed-code unpack pass,
  * [2] = tensor-core GEMM over whole output tiles, [3] = the same GEMM with
- * each tile's K split over a thread-block cluster (few tiles, small M; the
- * partial tiles are summed exactly in shared memory).  `n` is the array
- * length; at most 4 are written. */
+ * each tile's K split over a thread-block cluster (few tiles; the partial
+ * tiles are summed exactly in shared memory), [4] = the small-M prologue
+ * (one CTA per token), [5] = the small-M GEMM (M <= 16).  `n` is the array
+ * length; at most 6 are written. */
 void convrot_dispatch_counts(uint64_t *counts, int n);
 
 /* Description of the last CUDA call of this library that failed on the

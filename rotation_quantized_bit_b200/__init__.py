@@ -327,9 +327,10 @@ def convrot_selftest_timeout(limit_us: int = 20000, stream=None):
 
 def convrot_dispatch_counts():
     lib = load_library()
-    arr = (ctypes.c_uint64 * 4)()
-    lib.convrot_dispatch_counts(arr, 4)
-    return {"rotate_quant": arr[0], "unpack_codes": arr[1], "tc_gemm": arr[2], "tc_gemm_splitk": arr[3]}
+    arr = (ctypes.c_uint64 * 6)()
+    lib.convrot_dispatch_counts(arr, 6)
+    return {"rotate_quant": arr[0], "unpack_codes": arr[1], "tc_gemm": arr[2], "tc_gemm_splitk": arr[3],
+            "small_rotate_quant": arr[4], "small_gemm": arr[5]}
 
 
 def convrot_measure_mma_i8(N: int = 256, a_in_tmem: bool = False, iters: int = 4096):

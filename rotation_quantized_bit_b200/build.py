@@ -14,7 +14,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libconvrot_b200.so")
-SOURCES = ["api.cu", "rotate_quant.cu", "gemm.cu", "int8.cu", "noalloc.cu", "peak.cu"]
+SOURCES = ["api.cu", "rotate_quant.cu", "gemm.cu", "small_m.cu", "int8.cu", "noalloc.cu", "peak.cu"]
 HEADERS = ["ptx.cuh", "kernels.cuh"]
 
 

@@ -21,7 +21,7 @@ __device__ uint32_t g_device_error = 0;
 
 namespace {
 
-std::atomic<uint64_t> g_counts[4];
+std::atomic<uint64_t> g_counts[kDispatchKinds];
 
 constexpr int kMaxK = 32768;
 
@@ -78,6 +78,13 @@ size_t sa_offset(int M, int K) { return codes_bytes(M, K); }
 size_t workspace_bytes_for(int M, int K) {
   return sa_offset(M, K) + round_up(static_cast<size_t>(M) * sizeof(float), 256);
 }
+// M <= kSmallMaxM takes the small-M kernels: the codes region holds packed
+// codes (M*K/2 of its M*K bytes), and the GEMM's scratch (counters and
+// partial slabs where it splits K) follows the scales.
+bool small_m(int M) { return M <= kSmallMaxM; }
+size_t fused_ws_bytes(int M, int N, int K) {
+  return workspace_bytes_for(M, K) + (small_m(M) ? small_gemm_scratch_bytes(M, N, K) : 0);
+}
 
 convrot_status_t gemm_common(const uint8_t* xq, const float* s_a, const uint8_t* Wq, const float* s_w,
                              const uint16_t* bias, int M, int N, int K, void* out, GemmSink sink, void* ws,
@@ -89,12 +96,15 @@ convrot_status_t gemm_common(const uint8_t* xq, const float* s_a, const uint8_t*
   if (!aligned16(xq) || !aligned16(Wq) || !aligned16(out) || (s_a && !aligned16(s_a)) ||
       (s_w && !aligned16(s_w)) || (bias && !aligned16(bias)))
     return CONVROT_ERR_ALIGN;
-  if (!ws || ws_bytes < codes_bytes(M, K)) return CONVROT_ERR_WORKSPACE;
+  if (!ws || ws_bytes < (small_m(M) ? small_gemm_scratch_bytes(M, N, K) : codes_bytes(M, K)))
+    return CONVROT_ERR_WORKSPACE;
   if (!aligned16(ws)) return CONVROT_ERR_ALIGN;
   int sms = 0;
   st = check_device(&sms);
   if (st != CONVROT_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (small_m(M))  // the small-M GEMM reads the packed codes as they are
+    return from_cuda(launch_small_gemm(xq, s_a, Wq, s_w, bias, M, N, K, out, sink, ws, ws_bytes, s));
   int8_t* xs8 = static_cast<int8_t*>(ws);
   if (cudaError_t e = launch_unpack_codes(xq, M, K, xs8, s); e != cudaSuccess) return CONVROT_ERR_CUDA;
   GemmArgs a{xs8, s_a, Wq, s_w, bias, out, M, N, K};
@@ -114,24 +124,31 @@ convrot_status_t quantize_common(const uint16_t* x, int M, int K, void* ws, size
   st = check_device(nullptr);
   if (st != CONVROT_OK) return st;
   uint8_t* base = static_cast<uint8_t*>(ws);
+  if (small_m(M))
+    return from_cuda(launch_small_rotate_quant(x, M, K, group, base, reinterpret_cast<float*>(base + sa_offset(M, K)),
+                                               static_cast<cudaStream_t>(stream)));
   RotateQuantOut o{nullptr, reinterpret_cast<int8_t*>(base), reinterpret_cast<float*>(base + sa_offset(M, K))};
   o.group = group;
   return from_cuda(launch_rotate_quant(x, M, K, o, static_cast<cudaStream_t>(stream)));
 }
 
 convrot_status_t gemm_quantized_common(const uint8_t* Wq, const float* s_w, const uint16_t* bias, int M, int N,
-                                       int K, void* out, GemmSink sink, const void* ws, size_t ws_bytes,
+                                       int K, void* out, GemmSink sink, void* ws, size_t ws_bytes,
                                        void* stream) {
   if (!Wq || !s_w || !out) return CONVROT_ERR_NULL;
   convrot_status_t st = check_mnk(M, N, K);
   if (st != CONVROT_OK) return st;
   if (!aligned16(Wq) || !aligned16(s_w) || !aligned16(out) || (bias && !aligned16(bias))) return CONVROT_ERR_ALIGN;
-  if (!ws || ws_bytes < workspace_bytes_for(M, K)) return CONVROT_ERR_WORKSPACE;
+  if (!ws || ws_bytes < fused_ws_bytes(M, N, K)) return CONVROT_ERR_WORKSPACE;
   if (!aligned16(ws)) return CONVROT_ERR_ALIGN;
   int sms = 0;
   st = check_device(&sms);
   if (st != CONVROT_OK) return st;
-  const uint8_t* base = static_cast<const uint8_t*>(ws);
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  if (small_m(M))
+    return from_cuda(launch_small_gemm(base, reinterpret_cast<const float*>(base + sa_offset(M, K)), Wq, s_w, bias, M,
+                                       N, K, out, sink, base + workspace_bytes_for(M, K),
+                                       ws_bytes - workspace_bytes_for(M, K), static_cast<cudaStream_t>(stream)));
   GemmArgs a{reinterpret_cast<const int8_t*>(base), reinterpret_cast<const float*>(base + sa_offset(M, K)), Wq, s_w,
              bias, out, M, N, K};
   return from_cuda(launch_w4a4_gemm(a, sink, choose_tiling(M, N, K, sms), static_cast<cudaStream_t>(stream)));
@@ -145,7 +162,7 @@ convrot_status_t linear_common(const uint16_t* x, const uint8_t* Wq, const float
   if (st != CONVROT_OK) return st;
   if (!aligned16(x) || !aligned16(Wq) || !aligned16(s_w) || !aligned16(out) || (bias && !aligned16(bias)))
     return CONVROT_ERR_ALIGN;
-  if (!ws || ws_bytes < workspace_bytes_for(M, K)) return CONVROT_ERR_WORKSPACE;
+  if (!ws || ws_bytes < fused_ws_bytes(M, N, K)) return CONVROT_ERR_WORKSPACE;
   if (!aligned16(ws)) return CONVROT_ERR_ALIGN;
   if (!valid_group(group)) return CONVROT_ERR_SHAPE;
   st = quantize_common(x, M, K, ws, ws_bytes, stream, group);
@@ -165,7 +182,7 @@ size_t w8_workspace_bytes(int M, int K) { return w8_scratch_offset(M, K) + 256; 
 
 // Quantize rows of a bf16 [rows, K] matrix into int8 codes and scales.
 convrot_status_t quant8_common(const uint16_t* x, int rows, int K, int format, int8_t* codes, float* scales,
-                               void* ws, size_t ws_bytes, void* stream) {
+                               void* ws, size_t ws_bytes, void* stream, bool weights = false) {
   if (!x || !codes || !scales) return CONVROT_ERR_NULL;
   if (!valid_format(format)) return CONVROT_ERR_SHAPE;
   convrot_status_t st = check_mk(rows, K);
@@ -177,12 +194,13 @@ convrot_status_t quant8_common(const uint16_t* x, int rows, int K, int format, i
   if (format == W8A8_CONVROT_INT8_ROW) {
     RotateQuantOut o{nullptr, codes, scales};
     o.int8 = true;
+    o.early_trigger = !weights;
     return from_cuda(launch_rotate_quant(x, rows, K, o, s));
   }
   if (!ws || ws_bytes < 4) return CONVROT_ERR_WORKSPACE;
   if (!aligned16(ws)) return CONVROT_ERR_ALIGN;
   return from_cuda(launch_quant8_tensorwise(x, static_cast<size_t>(rows) * static_cast<size_t>(K), codes, scales,
-                                            static_cast<uint32_t*>(ws), s));
+                                            static_cast<uint32_t*>(ws), s, !weights));
 }
 
 convrot_status_t gemm8_common(const int8_t* x8, const float* s_x, const int8_t* Wq8, const float* s_w,
@@ -265,7 +283,7 @@ convrot_status_t linear_cb_common(const uint16_t* x, const uint8_t* idx, const u
 }  // namespace
 
 void count_dispatch(int which) {
-  if (which >= 0 && which < 4) g_counts[which].fetch_add(1, std::memory_order_relaxed);
+  if (which >= 0 && which < kDispatchKinds) g_counts[which].fetch_add(1, std::memory_order_relaxed);
 }
 
 namespace {
@@ -354,17 +372,17 @@ convrot_status_t convrot_rotate_quant(const uint16_t* x, int M, int K, uint8_t* 
 }
 
 convrot_status_t convrot_pack_weight(const uint16_t* W, int N, int K, uint8_t* Wq, float* s_w, void* stream) {
-  return convrot_rotate_quant(W, N, K, Wq, s_w, stream);
+  return convrot_pack_weight_g(W, N, K, 256, Wq, s_w, stream);
 }
 
 size_t convrot_gemm_workspace_size(int M, int N, int K) {
   if (check_mnk(M, N, K) != CONVROT_OK) return 0;
-  return codes_bytes(M, K);
+  return small_m(M) ? small_gemm_scratch_bytes(M, N, K) : codes_bytes(M, K);
 }
 
 size_t convrot_w4a4_workspace_size(int M, int N, int K) {
   if (check_mnk(M, N, K) != CONVROT_OK) return 0;
-  return workspace_bytes_for(M, K);
+  return fused_ws_bytes(M, N, K);
 }
 
 convrot_status_t w4a4_gemm(const uint8_t* xq, const float* s_a, const uint8_t* Wq, const float* s_w,
@@ -403,7 +421,7 @@ convrot_status_t convrot_w4a4_quantize(const uint16_t* x, int M, int K, void* wo
 }
 
 convrot_status_t convrot_w4a4_gemm_quantized(const uint8_t* Wq, const float* s_w, const uint16_t* bias, int M, int N,
-                                             int K, uint16_t* y, const void* workspace, size_t workspace_bytes,
+                                             int K, uint16_t* y, void* workspace, size_t workspace_bytes,
                                              void* stream) {
   return gemm_quantized_common(Wq, s_w, bias, M, N, K, y, GemmSink::kBF16, workspace, workspace_bytes, stream);
 }
@@ -429,7 +447,7 @@ convrot_status_t convrot_device_error(void* stream, uint32_t* code) {
 
 void convrot_dispatch_counts(uint64_t* counts, int n) {
   if (!counts) return;
-  for (int i = 0; i < n && i < 4; ++i) counts[i] = g_counts[i].load(std::memory_order_relaxed);
+  for (int i = 0; i < n && i < kDispatchKinds; ++i) counts[i] = g_counts[i].load(std::memory_order_relaxed);
 }
 
 }  // extern "C"
@@ -456,7 +474,17 @@ convrot_status_t w8a8_quantize(const uint16_t* x, int M, int K, int format, int8
 
 convrot_status_t w8a8_pack_weight(const uint16_t* W, int N, int K, int format, int8_t* Wq8, float* s_w,
                                   void* workspace, size_t workspace_bytes, void* stream) {
-  return w8a8_quantize(W, N, K, format, Wq8, s_w, workspace, workspace_bytes, stream);
+  // w8a8_quantize on W, except that no successor may start before the
+  // weights are complete (the GEMMs stream weights before they wait).
+  uint8_t* scratch = nullptr;
+  size_t scratch_bytes = 0;
+  if (workspace && check_mk(N, K) == CONVROT_OK && workspace_bytes >= w8_workspace_bytes(N, K)) {
+    scratch = static_cast<uint8_t*>(workspace) + w8_scratch_offset(N, K);
+    scratch_bytes = 256;
+  }
+  if (format == W8A8_INT8_TENSORWISE && !scratch && check_mk(N, K) == CONVROT_OK && W && Wq8 && s_w)
+    return CONVROT_ERR_WORKSPACE;
+  return quant8_common(W, N, K, format, Wq8, s_w, scratch, scratch_bytes, stream, /*weights=*/true);
 }
 
 convrot_status_t w8a8_gemm(const int8_t* x8, const float* s_x, const int8_t* Wq8, const float* s_w,
@@ -508,7 +536,19 @@ convrot_status_t convrot_rotate_quant_g(const uint16_t* x, int M, int K, int gro
 
 convrot_status_t convrot_pack_weight_g(const uint16_t* W, int N, int K, int group, uint8_t* Wq, float* s_w,
                                        void* stream) {
-  return convrot_rotate_quant_g(W, N, K, group, Wq, s_w, stream);
+  // convrot_rotate_quant_g on W, except that no successor may start before
+  // the weights are complete (the GEMMs stream weights before they wait).
+  if (!W || !Wq || !s_w) return CONVROT_ERR_NULL;
+  if (!valid_group(group)) return CONVROT_ERR_SHAPE;
+  convrot_status_t st = check_mk(N, K);
+  if (st != CONVROT_OK) return st;
+  if (!aligned16(W) || !aligned16(Wq) || !aligned16(s_w)) return CONVROT_ERR_ALIGN;
+  st = check_device(nullptr);
+  if (st != CONVROT_OK) return st;
+  RotateQuantOut o{Wq, nullptr, s_w};
+  o.group = group;
+  o.early_trigger = false;
+  return from_cuda(launch_rotate_quant(W, N, K, o, static_cast<cudaStream_t>(stream)));
 }
 
 convrot_status_t convrot_w4a4_quantize_g(const uint16_t* x, int M, int K, int group, void* workspace,

@@ -55,9 +55,12 @@ __global__ void __launch_bounds__(256) absmax_bf16_kernel(const uint4* __restric
 
 __global__ void __launch_bounds__(256) quant8_tensor_kernel(const uint4* __restrict__ x, size_t n16,
                                                             const uint32_t* __restrict__ amax_bits,
-                                                            uint2* __restrict__ codes, float* __restrict__ scale_out) {
-  // Let a dependent GEMM launch now: it streams its weights meanwhile.
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+                                                            uint2* __restrict__ codes, float* __restrict__ scale_out,
+                                                            int early_trigger) {
+  // Let a dependent GEMM launch now: it streams its weights meanwhile.  Not
+  // when this grid writes weights (the GEMMs read weights before they wait
+  // for their predecessor).
+  if (early_trigger) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const float s = __fdiv_rn(__uint_as_float(*amax_bits), 127.0f);
   if (blockIdx.x == 0 && threadIdx.x == 0) *scale_out = s;
   const float rcp = s >= kMinScale8 ? __frcp_rn(s) : 0.0f, ns = -s;
@@ -102,7 +105,7 @@ int sm_count() {
 }  // namespace
 
 cudaError_t launch_quant8_tensorwise(const uint16_t* x, size_t n, int8_t* codes, float* scale, uint32_t* scratch,
-                                     cudaStream_t stream) {
+                                     cudaStream_t stream, bool early_trigger) {
   const size_t n16 = n / 8;  // n is a multiple of 256
   cudaError_t e = cudaMemsetAsync(scratch, 0, sizeof(uint32_t), stream);
   if (e != cudaSuccess) return note_cuda(e, "int8_tensorwise: clear amax");
@@ -113,7 +116,7 @@ cudaError_t launch_quant8_tensorwise(const uint16_t* x, size_t n, int8_t* codes,
   e = cudaGetLastError();
   if (e != cudaSuccess) return note_cuda(e, "int8_tensorwise: amax launch");
   quant8_tensor_kernel<<<grid, 256, 0, stream>>>(reinterpret_cast<const uint4*>(x), n16, scratch,
-                                                  reinterpret_cast<uint2*>(codes), scale);
+                                                  reinterpret_cast<uint2*>(codes), scale, early_trigger ? 1 : 0);
   return note_cuda(cudaGetLastError(), "int8_tensorwise: quantize launch");
 }
 

@@ -21,13 +21,18 @@ struct RotateQuantOut {
   float* scale;     // [M]
   bool int8 = false;  // s8 holds 8-bit codes (amax / 127) in natural order instead
   int group = 256;    // rotation group: 256, 64 or 16 (int8: 256 only)
+  // Let the next kernel launch while this one runs (programmatic dependent
+  // launch).  Off for weight preparation: the GEMMs read weights before they
+  // wait for their predecessor, so the kernel that writes weights must not
+  // let any successor start before it has completed.
+  bool early_trigger = true;
 };
 
 // The int8_tensorwise quantizer: one scale s = amax|x| / 127 for the whole
 // [rows, K] tensor, codes clamp(rint(x / s), -127, 127), no rotation.
 // scratch: 4 bytes of device memory (the amax while it is reduced).
 cudaError_t launch_quant8_tensorwise(const uint16_t* x, size_t n, int8_t* codes, float* scale, uint32_t* scratch,
-                                     cudaStream_t stream);
+                                     cudaStream_t stream, bool early_trigger = true);
 
 cudaError_t launch_rotate_quant(const uint16_t* x, int M, int K, RotateQuantOut out, cudaStream_t stream);
 
@@ -75,7 +80,25 @@ struct GemmArgs {
 // Builds the tensor maps and launches the tensor-core GEMM.
 cudaError_t launch_w4a4_gemm(const GemmArgs& a, GemmSink sink, const GemmTiling& t, cudaStream_t stream);
 
-// Host-side dispatch counters (see convrot_dispatch_counts).
+// The small-M path (small_m.cu): M <= kSmallMaxM tokens.  A one-CTA-per-row
+// prologue writes packed codes (the convrot_rotate_quant layout) and scales;
+// the GEMM reads the packed codes as they are, streams each 16-channel slab
+// of packed weights with bulk copies and widens both operands in registers
+// for mma.sync s8.  Where it splits K over several CTAs it sums the partial
+// slabs through `scratch` (arrival counters, then partial slabs), whose size
+// small_gemm_scratch_bytes gives; it clears the counters itself.
+constexpr int kSmallMaxM = 16;
+size_t small_gemm_scratch_bytes(int M, int N, int K);
+cudaError_t launch_small_rotate_quant(const uint16_t* x, int M, int K, int group, uint8_t* xq, float* s_a,
+                                      cudaStream_t stream);
+cudaError_t launch_small_gemm(const uint8_t* xq, const float* s_a, const uint8_t* Wq, const float* s_w,
+                              const uint16_t* bias, int M, int N, int K, void* out, GemmSink sink, void* scratch,
+                              size_t scratch_bytes, cudaStream_t stream);
+
+// Host-side dispatch counters (see convrot_dispatch_counts): 0 rotate_quant,
+// 1 unpack_codes, 2 tensor-core GEMM, 3 split-K cluster GEMM, 4 small-M
+// prologue, 5 small-M GEMM.
+constexpr int kDispatchKinds = 6;
 void count_dispatch(int which);
 
 // Remember the last failing CUDA call (see convrot_last_error).

@@ -174,9 +174,11 @@ __global__ void __launch_bounds__(kMaxThreads) rotate_quant_kernel(const __grid_
   __shared__ uint32_t row_amax[3][kMaxRows];
   // Let the dependent GEMM launch now: it streams its weights meanwhile and
   // waits (griddepcontrol.wait) for this grid before reading codes or scales.
-  // This grid itself may have been launched before the preceding kernel
-  // finished: wait for it before reading x or writing any output.
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  // Not when this grid writes weights: then its successors start only once it
+  // has completed.  This grid itself may have been launched before the
+  // preceding kernel finished: wait for it before reading x or writing any
+  // output.
+  if (p.out.early_trigger) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   asm volatile("griddepcontrol.wait;" ::: "memory");
   // Parameters in registers (the inline-asm memory clobbers below would
   // otherwise reload them).

@@ -58,11 +58,30 @@ def _r256(v):
     return (v + 255) // 256 * 256
 
 
+def _small_scratch(M, N, K):
+    # The small-M GEMM takes one CTA per 16-channel slab; it splits K into
+    # parts only where a slab's K range would not fit its shared memory (96
+    # blocks of 128) or there are fewer slabs than SMs (148), at least 4
+    # blocks per part, at most 64 parts.  Split slabs need one counter per
+    # slab and one int32 partial slab (8 or 16 tokens x 16 channels) per part.
+    tiles, nb = (N + 15) // 16, K // 128
+    parts = max((nb + 95) // 96, (148 + tiles - 1) // tiles)
+    parts = max(1, min(parts, max(nb // 4, 1), 64))
+    if parts == 1:
+        return 256
+    return _r256(4 * tiles) + _r256(tiles * parts * (8 if M <= 8 else 16) * 16 * 4)
+
+
 def test_workspace_layout(lib):
-    # Codes (one byte each) then the per-token scales, each rounded to 256.
-    for M, N, K in ((4224, 3840, 3840), (1, 9728, 2560), (76, 2560, 9728), (77, 264, 768)):
+    # Codes (one byte each) then the per-token scales, each rounded to 256;
+    # for M <= 16 the small-M GEMM's scratch follows.
+    for M, N, K in ((4224, 3840, 3840), (76, 2560, 9728), (77, 264, 768), (17, 256, 512)):
         assert lib.convrot_gemm_workspace_size(M, N, K) == _r256(M * K)
         assert lib.convrot_w4a4_workspace_size(M, N, K) == _r256(M * K) + _r256(4 * M)
+    for M, N, K in ((1, 9728, 2560), (8, 256, 512), (9, 2560, 9728), (16, 12288, 3072), (16, 2560, 32768),
+                    (3, 1024, 2560)):
+        assert lib.convrot_gemm_workspace_size(M, N, K) == _small_scratch(M, N, K)
+        assert lib.convrot_w4a4_workspace_size(M, N, K) == _r256(M * K) + _r256(4 * M) + _small_scratch(M, N, K)
 
 
 FAKE = ctypes.c_void_p(0x10000)      # never dereferenced: validation fails first
@@ -90,10 +109,11 @@ def test_null_alignment_and_workspace_errors(lib):
 
 def test_dispatch_counters_without_a_gpu(lib):
     import torch
-    arr = (ctypes.c_uint64 * 4)()
-    lib.convrot_dispatch_counts(arr, 4)
+    arr = (ctypes.c_uint64 * 8)(*([7] * 8))
+    lib.convrot_dispatch_counts(arr, 8)
+    assert list(arr[6:]) == [7, 7]  # six kinds are counted; the rest of the array is left alone
     if not torch.cuda.is_available():
-        assert list(arr) == [0, 0, 0, 0]  # argument errors never reach a launch
+        assert list(arr[:6]) == [0] * 6  # argument errors never reach a launch
 
 
 def test_version(lib):
