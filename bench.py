@@ -6,18 +6,24 @@ input: for every linear of the workload, the fused ConvRot W4A4 Linear
 (online rotation + per-token INT4 quantization, then the tensor-core W4A4
 GEMM with the rank-one scale + bias epilogue, bf16 out).
 
-Default workload (``qwen3_4b``): the seven linears of one Qwen3-4B
-text-encoder decoder layer (q/k/v/o, gate/up/down; hidden 2560) at two prompt
-lengths, M = 76 and M = 1220 tokens -> 14 linear calls per step.  Other
-workloads: ``dit6b`` (M = 4224, hidden 3840), ``edit20b`` (M = 8704, hidden
-3072), ``small_m`` (M in 1..128), ``small``.
+Default workload (``edit20b``, the largest single-GPU configuration): the
+linears of one block of the 20B-class image-edit DiT, 8192 image + 512 text
+tokens (M = 8704), hidden 3072: to_q/k/v/out (3072 -> 3072), MLP up (3072 ->
+12288) and down (12288 -> 3072).  Other workloads: ``qwen3_4b`` (the Qwen3-4B
+text-encoder layer at M = 76 and 1220), ``dit6b`` (M = 4224, hidden 3840),
+``small_m`` (M in 1..128), ``small``, and the int8 / asymmetric W4A8 ones.
 
 Metric: effective TOPS = sum over the step's linears of 2*M*N*K / step time.
+The line also carries ``small_m``: HBM GB/s of the fused Linear and of the
+GEMM at M in {1, 8, 16} (the bandwidth-bound regime), each a steady-state
+per-call time over back-to-back calls on distinct weight copies.
 
 Usage:  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
         [--workload NAME] [--no-e2e]
-Multi-GPU: launched by torchrun; every rank runs the same workload (replicas,
-weak scaling, no data-path collective); the time is the max over ranks.
+Multi-GPU: every rank (one per GPU) runs the same workload (replicas, weak
+scaling, no data-path collective); the time is the max over ranks.  Under
+torchrun the ranks come from the environment; ``--gpus N`` without torchrun
+starts the N ranks itself.
 """
 from __future__ import annotations
 
@@ -67,7 +73,8 @@ def parse():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="qwen3_4b", choices=sorted(WORKLOAD_DESC))
+    ap.add_argument("--workload", default="edit20b", choices=sorted(WORKLOAD_DESC))
+    ap.add_argument("--no-small-m", action="store_true", help="leave out the M <= 16 HBM record")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--only", default=None, help="restrict the workload to the linear with this name")
@@ -231,28 +238,50 @@ def oracle_linear(oracle, s, x, wq, s_w, b):
     return oracle.linear8(x, wq, s_w, b, *ORACLE_FORMAT[s.fmt])
 
 
+def _oracle_rows(oracle, inputs, rows, threads):
+    """The oracle on the first ``rows`` rows of every linear, split into
+    ``threads`` row ranges run at once (the oracle's C calls release the GIL,
+    so each runs on its own core); returns (ops, seconds)."""
+    from concurrent.futures import ThreadPoolExecutor
+    jobs = []
+    for s, x, wq, s_w, b in inputs:
+        r = min(rows, s.M)
+        cuts = sorted({(r * i) // threads for i in range(threads + 1)})
+        jobs += [(s, x[a:c], wq, s_w, b) for a, c in zip(cuts[:-1], cuts[1:]) if c > a]
+    ops = sum(2.0 * j[1].shape[0] * j[0].N * j[0].K for j in jobs)
+    t0 = time.perf_counter()
+    if threads == 1:
+        for j in jobs:
+            oracle_linear(oracle, *j)
+    else:
+        with ThreadPoolExecutor(max_workers=threads) as ex:
+            list(ex.map(lambda j: oracle_linear(oracle, *j), jobs))
+    return ops, time.perf_counter() - t0
+
+
 def cpu_baseline(shapes, workload, budget_s=15.0):
-    """Time the CPU oracle (single thread, as it stands) on a bounded sample:
-    the first ``r`` rows of each linear of the step, r grown until the run
-    takes about ``budget_s``; throughput in the metric's unit (TOPS)."""
+    """Time the CPU oracle (as it stands) on a bounded sample: the first ``r``
+    rows of each linear of the step, r grown until one thread takes about
+    ``budget_s``; throughput in the metric's unit (TOPS).  The same sample is
+    then run again split over every core of the host (``all_cores``)."""
     import oracle
     inputs = [oracle_inputs(oracle, workload, s) for s in shapes]
     rows = 1
     while True:
-        t0 = time.perf_counter()
-        ops = 0.0
-        for s, x, wq, s_w, b in inputs:
-            r = min(rows, s.M)
-            oracle_linear(oracle, s, x[:r], wq, s_w, b)
-            ops += 2.0 * r * s.N * s.K
-        dt = time.perf_counter() - t0
+        ops, dt = _oracle_rows(oracle, inputs, rows, 1)
         if dt >= budget_s / 3 or rows >= max(s.M for s in shapes):
             break
         rows = min(max(s.M for s in shapes), rows * max(2, int(budget_s / 3 / max(dt, 1e-3))))
+    ncpu = os.cpu_count() or 1
+    ops_all, dt_all = _oracle_rows(oracle, inputs, rows, ncpu)
+    sample = (f"first {rows} rows (capped at M) of each of the {len(shapes)} linears of one step "
+              f"({ops / 1e9:.2f} GOP); weight packing untimed")
     return {"value": ops / dt / 1e12, "unit": UNIT, "cores": 1, "kind": "oracle",
-            "sample": f"first {rows} rows (capped at M) of each of the {len(shapes)} linears of one step "
-                      f"({ops / 1e9:.2f} GOP) in {dt:.1f} s; weight packing untimed",
-            "seconds": dt, "host": host_cpu()}
+            "sample": sample + f"; {dt:.1f} s on one thread",
+            "seconds": dt, "host": host_cpu(),
+            "all_cores": {"value": ops_all / dt_all / 1e12, "unit": UNIT, "cores": ncpu, "kind": "oracle",
+                          "sample": sample + f", split into {ncpu} row ranges run at once: {dt_all:.2f} s",
+                          "seconds": dt_all}}
 
 
 def host_cpu():
@@ -288,7 +317,7 @@ def main():
                     else "flushed between timed steps, outside the events: 256 MiB write",
               "launch": ("each step replayed from a CUDA graph" if not args.no_graph else "eager launches")
                         + ": per input tensor one rotate+quantize launch, then one GEMM launch per linear reading it",
-              "parallelism": f"replicas x{max(world, args.gpus)}" if max(world, args.gpus) > 1 else "single GPU",
+              "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
               "codes": "s4 packed weights, s4 activations widened to s8 for tcgen05 kind::i8, int32 accumulate, "
                        "fp32 epilogue, bf16 out"}
 
@@ -534,10 +563,16 @@ def main():
         roof["int8_mma_measured_tops"] = round(mma_i8_tops, 1)
         roof["frac_of_int8_mma_measured"] = roof["achieved"] / mma_i8_tops
     roof["traffic"] = committed_traffic(kname, s)
+    roof["timing"] = ("average launch duration from a second graph of the same step with an event between every "
+                      "two launches (this serialises the programmatic-launch overlap of the timed step)")
 
     e2e = None
     if not args.no_e2e:
         e2e = end_to_end(args, rq, torch, dev, stream, shapes, xs, layers, groups, ws, flush, world, dist)
+
+    small = None
+    if rank == 0 and not args.no_small_m:
+        small = small_m_record(rq, torch, dev, flush, peaks)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -552,7 +587,7 @@ def main():
         "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "s8", "data": "synthetic",
         "config": config, "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches,
-        "clocks": clocks, "detail": detail,
+        "clocks": clocks, "small_m": small, "detail": detail,
     }
     if rank == 0:
         print(json.dumps(line), flush=True)
@@ -585,6 +620,90 @@ def source_sha(kernel):
     fname = {"w4a4_tc_gemm_kernel": "gemm.cu", "rotate_quant_kernel": "rotate_quant.cu"}[kernel]
     with open(os.path.join(ROOT, "rotation_quantized_bit_b200", "csrc", fname), "rb") as f:
         return hashlib.sha256(f.read()).hexdigest()
+
+
+SMALL_M_SHAPES = [(2560, 9728), (9728, 2560), (3072, 12288), (12288, 3072)]  # (K, N) of the small-M sweep
+SMALL_M_TOKENS = [1, 8, 16]
+
+
+def small_m_record(rq, torch, dev, flush, peaks, reps=5):
+    """HBM GB/s of the fused Linear (rotate+quantize, then the GEMM) and of the
+    GEMM alone at M in {1, 8, 16} over the small-M sweep's (K, N) shapes.
+
+    Each figure is a steady-state per-call time: R back-to-back calls in one
+    CUDA graph, each on its own copy of the packed weights (R copies hold more
+    than three times the L2), L2 flushed before every replay, the median of
+    ``reps`` replays divided by R.  Bytes are the algorithmic ones: for the
+    Linear x (2MK) + weights (NK/2) + s_w, bias (6N) + y (2MN); for the GEMM
+    the packed codes and scales (MK/2 + 4M) instead of x.  The GEMM calls
+    share one quantization, as projections that read one tensor do."""
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    out = []
+    for K, N in SMALL_M_SHAPES:
+        w, b = synthetic.weights("small_m", N, K)
+        wd = torch.from_numpy(w.view(np.int16)).view(torch.bfloat16).to(dev)
+        wq0, s_w = rq.convrot_pack_weight(wd)
+        del wd
+        bias = torch.from_numpy(b.view(np.int16)).view(torch.bfloat16).to(dev)
+        R = max(8, int(np.ceil(3.0 * l2 / wq0.numel())))
+        wqs = [wq0] + [wq0.clone() for _ in range(R - 1)]
+        for M in SMALL_M_TOKENS:
+            x = torch.from_numpy(synthetic.activations("small_m", M, K).view(np.int16)).view(torch.bfloat16).to(dev)
+            ys = [torch.empty((M, N), dtype=torch.bfloat16, device=dev) for _ in range(R)]
+            ws = torch.empty(rq.convrot_w4a4_workspace_size(M, N, K), dtype=torch.uint8, device=dev)
+            rq.convrot_w4a4_quantize(x, ws)
+
+            def ring_gemm():
+                for r in range(R):
+                    rq.convrot_w4a4_gemm_quantized(ws, M, wqs[r], s_w, bias, out=ys[r])
+
+            def ring_linear():
+                for r in range(R):
+                    rq.convrot_w4a4_linear(x, wqs[r], s_w, bias, out=ys[r], workspace=ws)
+
+            rec = {"M": M, "K": K, "N": N, "calls_per_replay": R}
+            for name, fn, nbytes in (
+                    ("gemm", ring_gemm, N * K / 2 + 6 * N + M * K / 2 + 4 * M + 2 * M * N),
+                    ("linear", ring_linear, 2 * M * K + N * K / 2 + 6 * N + 2 * M * N)):
+                side = torch.cuda.Stream()
+                side.wait_stream(torch.cuda.current_stream())
+                with torch.cuda.stream(side):
+                    fn()  # warm-up outside the capture
+                torch.cuda.synchronize()
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g):
+                    fn()
+                times = []
+                for _ in range(reps):
+                    flush()
+                    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                    e0.record()
+                    g.replay()
+                    e1.record()
+                    e1.synchronize()
+                    times.append(e0.elapsed_time(e1))
+                us = statistics.median(times) * 1e3 / R
+                gbs = nbytes / (us * 1e-6) / 1e9
+                rec[f"{name}_us"] = round(us, 2)
+                rec[f"{name}_gbs"] = round(gbs, 1)
+                rec[f"{name}_frac_hbm"] = round(gbs / peaks["hbm_gbs"], 3)
+                del g
+            out.append(rec)
+            del ys, ws, x
+        del wqs, wq0
+        torch.cuda.empty_cache()
+    if rq.convrot_device_error():
+        raise RuntimeError("device error word set during the small-M record")
+    fr_l = [r["linear_frac_hbm"] for r in out]
+    fr_g = [r["gemm_frac_hbm"] for r in out]
+    return {"peak_gbs": peaks["hbm_gbs"], "peak_source": f"{peaks['source']} HBM copy",
+            "linear_frac_hbm": {"min": min(fr_l), "median": statistics.median(fr_l), "max": max(fr_l)},
+            "gemm_frac_hbm": {"min": min(fr_g), "median": statistics.median(fr_g), "max": max(fr_g)},
+            "method": "back-to-back calls in one CUDA graph over distinct weight copies (> 3x L2), L2 flushed "
+                      "before each replay; per-call time = median replay time / calls",
+            "kernels": "M <= 16: one-CTA-per-token prologue (rq_rows_kernel) + bandwidth-bound slab GEMM "
+                       "(w4a4_gemv_kernel: bulk-copied weight rows, mma.sync s8)",
+            "shapes": out}
 
 
 def end_to_end(args, rq, torch, dev, stream, shapes, xs, layers, groups, ws, flush, world, dist):
@@ -706,5 +825,26 @@ def reference_arm(args, shapes, config, world, rank):
     print(json.dumps(line), flush=True)
 
 
-if __name__ == "__main__":
+def _rank_entry(rank, world, port):
+    os.environ.update(RANK=str(rank), LOCAL_RANK=str(rank), WORLD_SIZE=str(world), MASTER_ADDR="127.0.0.1",
+                      MASTER_PORT=str(port))
     main()
+
+
+def self_launch(n):
+    """``--gpus N`` without torchrun: start the N ranks here (one process per
+    GPU, spawned), each running main() with the environment torchrun sets."""
+    import socket
+    import torch.multiprocessing as mp
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    mp.start_processes(_rank_entry, args=(n, port), nprocs=n, start_method="spawn", join=True)
+
+
+if __name__ == "__main__":
+    _args = parse()
+    if _args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        self_launch(_args.gpus)
+    else:
+        main()

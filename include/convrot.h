@@ -169,7 +169,11 @@ convrot_status_t convrot_w4a4_linear_f32(const uint16_t *x, const uint8_t *Wq, c
  *   no cudaFree.
  *   The first call on each device looks up the array's device address
  *   (cudaGetSymbolAddress) with that device current; make that first call
- *   before any stream capture.
+ *   before any stream capture.  The address is kept per device and looked up
+ *   again when the device's current CUDA context changes (for example after
+ *   cudaDeviceReset); the lookup is guarded, so several host threads may make
+ *   their first calls at once.  A device other than sm_100 gives
+ *   CONVROT_ERR_DEVICE before any lookup.
  *   Every call shares the one array and it keeps the last call's contents, so
  *   calls that overlap on the GPU (e.g. on two streams at once) race. */
 convrot_status_t convrot_w4a4_linear_noalloc(const uint16_t *x, const uint8_t *Wq,

@@ -12,12 +12,20 @@
 // GPU that loads the library holds until the process exits.
 //
 // Host code may not take the array's name as a device pointer (on the host it
-// is only a stand-in symbol), so the first call on each device looks its
-// device address up with cudaGetSymbolAddress and caches it.
+// is only a stand-in symbol), so the array's device address is looked up with
+// cudaGetSymbolAddress, with the device current, the first time a device (in
+// a given CUDA context) calls in, and kept for later calls.  The lookup is
+// repeated when the current context changes (after cudaDeviceReset, or with
+// another driver context current on the same device), since the array then
+// lives at another address.  A mutex guards the cache, so concurrent first
+// calls from several host threads are safe; the kernels of calls that
+// overlap on the GPU still share, and race on, the one array.
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <cstdint>
 #include <cstdio>
+#include <mutex>
 
 #include "../../include/convrot.h"
 #include "kernels.cuh"
@@ -30,8 +38,58 @@ constexpr int kMaxDevices = 64;
 
 static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
 
-// Device address of g_noalloc_scratch per device, looked up on first use.
-void* g_scratch_ptr[kMaxDevices] = {nullptr};
+struct ScratchSlot {
+  CUcontext ctx = nullptr;  // the context the address was looked up in
+  void* ptr = nullptr;
+};
+ScratchSlot g_scratch[kMaxDevices];
+std::mutex g_scratch_mu;
+
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+
+CtxGetCurrentFn ctx_get_current() {
+  static CtxGetCurrentFn fn = [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return static_cast<CtxGetCurrentFn>(nullptr);
+    return reinterpret_cast<CtxGetCurrentFn>(p);
+  }();
+  return fn;
+}
+
+// The scratch array's device address on the current device (and context), or
+// null with *st set.
+void* scratch_address(convrot_status_t* st) {
+  int dev = 0, major = 0, minor = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices ||
+      cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess || major != 10 ||
+      minor != 0) {
+    *st = CONVROT_ERR_DEVICE;  // checked before the library's image is touched on this device
+    return nullptr;
+  }
+  CUcontext ctx = nullptr;
+  CtxGetCurrentFn get = ctx_get_current();
+  if (get) (void)get(&ctx);
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  ScratchSlot& slot = g_scratch[dev];
+  if (slot.ptr == nullptr || slot.ctx != ctx) {
+    // Set-up, once per device and context, with that device current.
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess || p == nullptr) {
+      note_cuda(e != cudaSuccess ? e : cudaErrorInvalidSymbol, "convrot_w4a4_linear_noalloc: cudaGetSymbolAddress");
+      *st = CONVROT_ERR_CUDA;
+      return nullptr;
+    }
+    if (get) (void)get(&ctx);  // the runtime's primary context, now that it is surely initialised
+    slot.ctx = ctx;
+    slot.ptr = p;
+  }
+  return slot.ptr;
+}
 
 }  // namespace
 }  // namespace convrot
@@ -53,19 +111,11 @@ extern "C" convrot_status_t convrot_w4a4_linear_noalloc(const uint16_t* x, const
     note_cuda(cudaErrorInvalidValue, msg);
     return CONVROT_ERR_WORKSPACE;
   }
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return CONVROT_ERR_DEVICE;
-  if (g_scratch_ptr[dev] == nullptr) {
-    // Set-up, once per device, with that device current.
-    void* p = nullptr;
-    cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-    if (e != cudaSuccess || p == nullptr) {
-      note_cuda(e != cudaSuccess ? e : cudaErrorInvalidSymbol, "convrot_w4a4_linear_noalloc: cudaGetSymbolAddress");
-      return CONVROT_ERR_CUDA;
-    }
-    g_scratch_ptr[dev] = p;
-  }
+  convrot_status_t st = CONVROT_OK;
+  void* scratch = scratch_address(&st);
+  if (!scratch) return st;
   // Nothing in the scratch needs to start at zero: the first kernel writes
-  // every code and scale that the second one reads.
-  return convrot_w4a4_linear(x, Wq, s_w, bias, M, N, K, y, g_scratch_ptr[dev], kNoAllocScratchBytes, stream);
+  // every code and scale that the second one reads, and the small-M GEMM
+  // clears the counters it uses itself.
+  return convrot_w4a4_linear(x, Wq, s_w, bias, M, N, K, y, scratch, kNoAllocScratchBytes, stream);
 }

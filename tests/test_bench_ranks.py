@@ -69,3 +69,19 @@ def test_reference_arm_prints_on_rank_zero_only():
     assert r0.returncode == 0
     line = json.loads(r0.stdout.strip().splitlines()[-1])
     assert line["impl"] == "reference" and line["value"] > 0 and line["cpu_baseline"]["kind"] == "oracle"
+
+
+def test_gpus_flag_starts_its_own_ranks():
+    # `bench.py --gpus 2` without torchrun: the bench starts both ranks itself
+    # (spawned processes with the environment torchrun would set); the
+    # reference arm prints one line, from rank 0, with n_gpus = 2.
+    env = {k: v for k, v in os.environ.items() if k not in ("RANK", "WORLD_SIZE", "LOCAL_RANK")}
+    cmd = [sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--workload", "small",
+           "--gpus", "2", "--steps", "1", "--warmup", "0"]
+    r = subprocess.run(cmd, env=env, capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.strip().splitlines() if ln.startswith("{")]
+    assert len(lines) == 1
+    line = json.loads(lines[0])
+    assert line["impl"] == "reference" and line["n_gpus"] == 2
+    assert line["config"]["parallelism"] == "replicas x2"

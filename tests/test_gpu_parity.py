@@ -11,6 +11,8 @@ Small cases span several tiles and ragged tails; the full workload shapes
 configuration) are checked on sampled rows that include the first tile, a
 middle tile and the M tail.
 """
+import functools
+
 import numpy as np
 import pytest
 import torch
@@ -273,24 +275,36 @@ def sample_rows(M, BT_guess=192):
 FULL = [s for wl in ("qwen3_4b", "dit6b", "edit20b", "small_m") for s in synthetic.workload_shapes(wl)]
 
 
+@functools.lru_cache(maxsize=2)
+def _full_x(wl, M, K):
+    return synthetic.activations(wl, M, K)
+
+
+@functools.lru_cache(maxsize=2)
+def _full_w(wl, N, K):
+    """The weights and bias of a full-size linear, and the oracle's packing of
+    the whole weight matrix (its codes and scales are the reference)."""
+    w, b = synthetic.weights(wl, N, K)
+    wq_ref, sw_ref = oracle.pack_weight(w)
+    return w, b, wq_ref, sw_ref
+
+
 @pytest.mark.parametrize("shape", FULL, ids=lambda s: f"{s.name}-M{s.M}-K{s.K}-N{s.N}")
 def test_full_size_linear_sampled_rows(rq, shape):
     wl = next(w for w in ("qwen3_4b", "dit6b", "edit20b", "small_m")
               if shape in synthetic.workload_shapes(w))
     M, K, N = shape.M, shape.K, shape.N
-    x = synthetic.activations(wl, M, K)
-    w, b = synthetic.weights(wl, N, K)
+    x = _full_x(wl, M, K)
+    w, b, wq_ref, sw_ref = _full_w(wl, N, K)
+    # The weights prepared on the GPU are the oracle's, every code and scale.
     dwq, dsw = rq.convrot_pack_weight(dev_bf16(w))
-    wq = host(dwq)
+    assert np.array_equal(host(dwq), wq_ref)
+    assert np.array_equal(f32_bits(host(dsw)), f32_bits(sw_ref))
     y32 = host(rq.convrot_w4a4_linear_f32(dev_bf16(x), dwq, dsw, dev_bf16(b)))
     y16 = host_bits(rq.convrot_w4a4_linear(dev_bf16(x), dwq, dsw, dev_bf16(b)))
-    rows = sample_rows(M)
-    # the weights prepared on the GPU are the oracle's, checked on sampled rows
-    wrows = sorted(set(range(min(N, 4))) | set(range(max(0, N - 4), N)))
-    wq_ref, sw_ref = oracle.pack_weight(w[wrows])
-    assert np.array_equal(wq[wrows], wq_ref) and np.array_equal(f32_bits(host(dsw)[wrows]), f32_bits(sw_ref))
-    for r0, r1 in _runs(rows):
-        ref32, ref16 = oracle.linear(x, wq, host(dsw), b, K, rows=(r0, r1))
+    # The reference Linear uses the oracle's own codes and scales only.
+    for r0, r1 in _runs(sample_rows(M)):
+        ref32, ref16 = oracle.linear(x, wq_ref, sw_ref, b, K, rows=(r0, r1))
         check_f32(y32[r0:r1], ref32)
         assert np.array_equal(f32_bits(y32[r0:r1]), f32_bits(ref32))
         assert bf16_ulp_diff(y16[r0:r1], ref16).max() <= 1
