@@ -53,6 +53,7 @@ struct GemmTiling {
   int smem_bytes;   // dynamic shared memory per CTA
   int acc_stride;   // tensor-memory columns per accumulator
   int a_slots;      // 64-column tensor-memory slots for unpacked weights
+  int n_fast;       // whole-tile order: channel tile fastest (1) or token tile fastest (0)
 };
 
 // Weight kinds of the tensor-core GEMM.

@@ -20,13 +20,13 @@
 //
 // w4a4_gemv_kernel (K6)  one CTA (four warps) per slab of 16 output channels
 //   (and, only where K is very long or N small, per part of K).  The slab's
-//   packed weights are contiguous rows; each lane of a warp issues one bulk
-//   copy (cp.async.bulk) of its row's share of the warp's K range into shared
-//   memory at launch, before the grid waits for the prologue, so the whole
-//   matrix is requested from HBM at once and no tensor-map descriptor has to
-//   be fetched first.  Rows are padded to 64 bytes modulo 128 so that the
-//   16-byte fragment loads are free of bank conflicts.  Warp w multiplies the
-//   rows of its K quarter with mma.sync m16n8k32 s8: the weights are the A
+//   packed weights are contiguous rows; one bulk copy (cp.async.bulk) per row
+//   of the CTA's K range brings them into shared memory at launch, before
+//   the grid waits for the prologue, so the whole matrix is requested from
+//   HBM at once and no tensor-map descriptor has to be fetched first.  Rows
+//   are padded to 64 bytes modulo 128 so that the 16-byte fragment loads are
+//   free of bank conflicts.  Warp w multiplies the rows of its share of the
+//   K range with mma.sync m16n8k32 s8: the weights are the A
 //   operand (MMA rows = channels), the tokens the columns.  Both operands
 //   arrive as packed nibbles and are widened in registers: for a 32-bit word
 //   w of codes k .. k+7 (even code in the low nibble), (w << 4) & 0xF0F0F0F0
@@ -141,7 +141,9 @@ __global__ void __launch_bounds__(32 * W, W == 4 ? 6 : 2) w4a4_gemv_kernel(const
   constexpr int D = NT == 1 ? 8 : 4;  // blocks of activation words in flight per warp, in registers
   extern __shared__ __align__(128) uint8_t smem_raw[];
   uint8_t* slab = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
-  __shared__ __align__(8) uint64_t bar[W];
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ __align__(16) float s_sw[kSlabRows];        // the slab's weight scales
+  __shared__ __align__(16) uint16_t s_bias[kSlabRows];   // and bias
   __shared__ __align__(16) int32_t red[W][MT][kSlabRows];
   __shared__ uint32_t s_last;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -152,33 +154,39 @@ __global__ void __launch_bounds__(32 * W, W == 4 ? 6 : 2) w4a4_gemv_kernel(const
   const int wb0 = b0 + (warp * (b1 - b0)) / W, wb1 = b0 + ((warp + 1) * (b1 - b0)) / W;
   const size_t wrow = static_cast<size_t>(p.K) / 2;  // bytes per weight / activation row
 
-  if (threadIdx.x < W) mbar_init(&bar[threadIdx.x], 1);
-  fence_mbarrier_init();
-  __syncthreads();
+  // ---- weights: thread r < rows copies row r's share of the CTA's K range
+  // (one bulk copy per row: few, large copies keep the copy engine's per-copy
+  // cost out of the way); threads 16 and 17 copy the slab's weight scales and
+  // bias, which the epilogue reads from shared memory.  None of them depends
+  // on the preceding kernel: all are requested before waiting for it, and no
+  // register waits on them before the weights have landed.
+  const bool scaled = SINK != static_cast<int>(GemmSink::kS32);
+  const uint32_t rbytes = static_cast<uint32_t>((b1 - b0) * kBlockBytes);
+  const uint32_t swbytes = scaled ? static_cast<uint32_t>(rows) * 4u : 0u;
+  const uint32_t bbytes = p.bias ? static_cast<uint32_t>(rows) * 2u : 0u;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_mbarrier_init();
+    mbar_arrive_expect_tx(&bar, rbytes * static_cast<uint32_t>(rows) + swbytes + bbytes);
+  }
+  __syncwarp();
+  if (static_cast<int>(threadIdx.x) < rows)
+    bulk_load(slab + threadIdx.x * p.row_stride,
+              p.Wq + static_cast<size_t>(n0 + threadIdx.x) * wrow + static_cast<size_t>(b0) * kBlockBytes, rbytes,
+              &bar);
+  if (threadIdx.x == 16 && swbytes) bulk_load(s_sw, p.s_w + n0, swbytes, &bar);
+  if (threadIdx.x == 17 && bbytes) bulk_load(s_bias, p.bias + n0, bbytes, &bar);
+  __syncthreads();  // the barrier is initialised before any thread waits on it
   // The next kernel on the stream may launch now; it waits for this grid
   // before it touches anything this grid reads or writes.
   pdl_launch_dependents();
-  // ---- weights: lane r < rows copies row r's share of this warp's K range.
-  // They do not depend on the preceding kernel: requested before waiting.
   const uint32_t wbytes = static_cast<uint32_t>((wb1 - wb0) * kBlockBytes);
-  if (wbytes > 0) {
-    if (lane == 0) mbar_arrive_expect_tx(&bar[warp], wbytes * static_cast<uint32_t>(rows));
-    __syncwarp();
-    if (lane < rows)
-      bulk_load(slab + lane * p.row_stride + (wb0 - b0) * kBlockBytes,
-                p.Wq + static_cast<size_t>(n0 + lane) * wrow + static_cast<size_t>(wb0) * kBlockBytes, wbytes,
-                &bar[warp]);
-  }
-  // The epilogue's weight scale and bias (thread i stores channel n0 + i %
-  // 16): weight-side data, fetched before the wait like the weights.
+  // Thread i stores channel n0 + i % 16 in the epilogue.
   constexpr int kOut = MT * kSlabRows;
   constexpr int kPerThread = (kOut + 32 * W - 1) / (32 * W);  // 1 or 2
   const int r = threadIdx.x & 15;
   const bool mine_out = static_cast<int>(threadIdx.x) < kOut;  // (kOut is a multiple of 32 W or smaller)
-  const bool scaled = SINK != static_cast<int>(GemmSink::kS32);
   const bool chan = r < rows && mine_out;
-  const float sw = (scaled && chan) ? __ldg(p.s_w + n0 + r) : 0.0f;
-  const float bv = (p.bias && chan) ? __uint_as_float(static_cast<uint32_t>(__ldg(p.bias + n0 + r)) << 16) : 0.0f;
   pdl_wait();  // activations, scales, partial slabs and counters belong to the preceding kernels until now
 
   // ---- this warp's K range: 4 MMA k-steps per block, two accumulator sets
@@ -222,10 +230,12 @@ __global__ void __launch_bounds__(32 * W, W == 4 ? 6 : 2) w4a4_gemv_kernel(const
   };
 #pragma unroll
   for (int d = 0; d < D; ++d) load_x(wb0 + d, xbuf[d]);
-  const bool landed = wbytes == 0 || mbar_wait(&bar[warp], 0);
+  const bool landed = mbar_wait(&bar, 0);
   // After a wait that gave up, the copies still in flight must land (bounded)
   // before the block may exit.
-  if (!landed) (void)mbar_drain(&bar[warp], 0, 100000000ull);
+  if (!landed) (void)mbar_drain(&bar, 0, 100000000ull);
+  const float sw = (scaled && chan && landed) ? s_sw[r] : 0.0f;
+  const float bv = (bbytes && chan && landed) ? __uint_as_float(static_cast<uint32_t>(s_bias[r]) << 16) : 0.0f;
   if (landed && wbytes > 0) {
     const uint8_t* wr0 = slab + g * p.row_stride + 16 * t - b0 * kBlockBytes;
     const uint8_t* wr1 = wr0 + 8 * p.row_stride;
