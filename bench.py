@@ -605,13 +605,14 @@ def committed_traffic(kernel, s):
     try:
         with open(path) as f:
             rec = json.load(f)
-        ent = rec.get(kernel)
-        if not ent or ent.get("source_sha256") != source_sha(kernel):
-            return None
-        scale = 1.0
-        if ent.get("shape") != [s.M, s.K, s.N]:
-            return None
-        return ent["dram_bytes_per_launch"] * scale
+        ents = rec.get(kernel) or []
+        if isinstance(ents, dict):
+            ents = [ents]
+        sha = source_sha(kernel)
+        for ent in ents:
+            if ent.get("source_sha256") == sha and ent.get("shape") == [s.M, s.K, s.N]:
+                return ent["dram_bytes_per_launch"]
+        return None
     except (OSError, ValueError, KeyError):
         return None
 
