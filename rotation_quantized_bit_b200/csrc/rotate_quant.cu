@@ -40,20 +40,34 @@
 // run ahead of the arithmetic without holding registers.  A stage is
 // refilled right after the block barrier that ends its readers' use of it.
 //
-// Quantization.  The code is rint(q) with q the correctly rounded quotient
-// x' / s.  q is formed without a division by Markstein's correction (P.
-// Markstein, "Computation of elementary functions on the IBM RISC System/6000
-// processor", IBM J. Res. Develop. 34(1), 1990; restated as Markstein's
-// theorem in Muller et al., "Handbook of Floating-Point Arithmetic", ch. on
-// division with an FMA): with y = RN(1/s), q0 = RN(x' y) is within two ulps of
-// x'/s; one step q1 = RN(q0 + RN(x' - s q0) y) makes it faithful, and a second
-// step from a faithful q1, whose remainder x' - s q1 is exact, returns
-// RN(x'/s) itself.  Both remainders are fused multiply-adds.  The theorem needs
-// the remainders and products clear of underflow, which holds for every scale
-// s >= 2^-100 wherever the code can be nonzero; rows with a smaller scale (zero
-// included) take the IEEE division.  rint is the addition of 1.5 * 2^23, whose
-// low byte is then the two's-complement code (|x'/s| <= 7 up to rounding, so
-// no clamp is needed on this path).
+// Scales.  The butterflies leave v = 2^LOG4G x'; the amax is taken over |v|
+// and scaled once per row (RN is monotone, so RN(max|v| 2^-LOG4G) is the
+// amax of x' itself).  Every lane forms its two rows' scales
+// s = RN(amax / qmax) with two Markstein corrections of RN(amax fl(1/qmax))
+// (P. Markstein, "Computation of elementary functions on the IBM RISC
+// System/6000 processor", IBM J. Res. Develop. 34(1), 1990; restated as
+// Markstein's theorem in Muller et al., "Handbook of Floating-Point
+// Arithmetic", ch. on division with an FMA), which equals the IEEE quotient
+// for every amax in [2^-120, 2^120] and qmax 7 or 127 (checked against
+// division for each float of that range); other amax values take the IEEE
+// division.
+//
+// Quantization.  The code is c = rint(RN(x'/s)) (ties to even).  Fast path,
+// for 2^-100 <= s <= 2^100: k = rint(v y) with y ~ 1/(2^LOG4G s) from the
+// approximate reciprocal (one fused multiply-add with 1.5 * 2^23, whose low
+// byte is then k in two's complement), and the exact remainder
+// d = RN(v - 2^LOG4G s k) from a second one.  If |d| <= 2^LOG4G s (1/2 - m),
+// the quotient x'/s lies strictly inside (k - 1/2 + m', k + 1/2 - m') with m'
+// above half an ulp of any quotient of magnitude <= qmax (m = 2^-18 for the
+// 4-bit codes, 2^-14 for the 8-bit ones), so RN(x'/s) rounds to k as well, and
+// c = k; the reciprocal's error only decides how often the check fails.  A
+// lane whose check fails anywhere (a quotient within m of a half-integer:
+// about one element in 10^5 on random data, every one of an exact tie)
+// recomputes its codes by the exact quotient: y = RN(1/s), q0 = RN(x' y)
+// within two ulps of x'/s, one correction q1 = RN(q0 + RN(x' - s q0) y) makes
+// it faithful, and a second step from a faithful q1, whose remainder is exact,
+// returns RN(x'/s) itself (Markstein's theorem again; it needs s >= 2^-100).
+// Scales outside [2^-100, 2^100] (zero included) take the IEEE division.
 #include <cuda_runtime.h>
 
 #include <cstdint>
@@ -66,7 +80,8 @@ namespace convrot {
 namespace {
 
 constexpr float kMagic = 12582912.0f;           // 1.5 * 2^23: x + kMagic rounds x to an integer, ties to even
-constexpr float kMinScale = 7.88860905e-31f;    // 2^-100: below it, codes by division
+constexpr float kMinScale = 0x1p-100f;          // fast and exact-quotient paths: 2^-100 <= s <= 2^100
+constexpr float kMaxScale = 0x1p100f;
 constexpr int kTileRow = 144;                   // bytes per transpose-tile row: 16 fp32 pairs + 16 of padding
 constexpr int kTileBytes = 16 * kTileRow;       // per-half-warp transpose tile
 constexpr int kMaxRows = 64;                    // rows per row block (K = 256 -> 64 tasks)
@@ -109,6 +124,29 @@ __device__ __forceinline__ float max3(float a, float b, float c) {
   float d;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
   return d;
+}
+
+// Approximate reciprocal (the hardware's, about one ulp).
+__device__ __forceinline__ float rcp_approx(float a) {
+  float r;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(a));
+  return r;
+}
+
+// RN(a / QMAX) for QMAX = 7 or 127: two Markstein corrections of RN(a y),
+// y = RN(1 / QMAX), for a in [2^-120, 2^120] (equal to the IEEE quotient for
+// every float of that range), the IEEE division elsewhere.
+template <int QMAX>
+__device__ __forceinline__ float div_by_qmax(float a) {
+  constexpr float kQ = static_cast<float>(QMAX);
+  constexpr float kY = 1.0f / kQ;
+  if (a >= 0x1p-120f && a <= 0x1p120f) {
+    float q = __fmul_rn(a, kY);
+    q = __fmaf_rn(__fmaf_rn(-kQ, q, a), kY, q);
+    q = __fmaf_rn(__fmaf_rn(-kQ, q, a), kY, q);
+    return q;
+  }
+  return __fdiv_rn(a, kQ);
 }
 
 // One radix-4 butterfly on pairs: (a,b,c,d) -> (p+t, p-t, q+r, r-q).
@@ -168,7 +206,6 @@ __host__ __device__ constexpr int rq_smem_bytes(int R, int K, int S, int threads
 template <int MODE, int LOG4G>
 __global__ void __launch_bounds__(kMaxThreads) rotate_quant_kernel(const __grid_constant__ RQParams p) {
   constexpr bool PACKED = MODE == kPacked4;
-  constexpr float kQMax = MODE == kInt8 ? 127.0f : 7.0f;
   constexpr int kQLo = MODE == kInt8 ? -127 : -8, kQHi = MODE == kInt8 ? 127 : 7;
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ uint32_t row_amax[3][kMaxRows];
@@ -282,21 +319,15 @@ __global__ void __launch_bounds__(kMaxThreads) rotate_quant_kernel(const __grid_
 #pragma unroll
       for (int i = 0; i < 4; ++i) bfly4(P[i], P[i + 4], P[i + 8], P[i + 12]);
     }
-    // x' = v * 2^-LOG4G (1/16 for groups of 256), and the two tasks' amax
+    // the two tasks' max |v| (v = 2^LOG4G x'; the scaling waits for the row's amax)
     float m0 = 0.0f, m1 = 0.0f;
-    {
-      constexpr float kInvSqrtG = LOG4G == 4 ? 0.0625f : (LOG4G == 3 ? 0.125f : 0.25f);
-      const u64 sixteenth = f2(kInvSqrtG, kInvSqrtG);
 #pragma unroll
-      for (int i = 0; i < 16; i += 2) {
-        P[i] = f2_mul(P[i], sixteenth);
-        P[i + 1] = f2_mul(P[i + 1], sixteenth);
-        float x0, x1, y0, y1;
-        f2_split(P[i], x0, x1);
-        f2_split(P[i + 1], y0, y1);
-        m0 = max3(m0, fabsf(x0), fabsf(y0));
-        m1 = max3(m1, fabsf(x1), fabsf(y1));
-      }
+    for (int i = 0; i < 16; i += 2) {
+      float x0, x1, y0, y1;
+      f2_split(P[i], x0, x1);
+      f2_split(P[i + 1], y0, y1);
+      m0 = max3(m0, fabsf(x0), fabsf(y0));
+      m1 = max3(m1, fabsf(x1), fabsf(y1));
     }
     // ---- per-row amax: within each task (16 lanes), then across the row's tasks
 #pragma unroll
@@ -317,53 +348,73 @@ __global__ void __launch_bounds__(kMaxThreads) rotate_quant_kernel(const __grid_
     // in iteration it + 2, after one more barrier.
     if (threadIdx.x < kMaxRows) row_amax[slot == 0 ? 2 : slot - 1][threadIdx.x] = 0u;
 
-    // ---- quantize: lane 0 of the task forms the scale (one IEEE division)
-    // and its reciprocal; the half-warp shares them.
-    float scale0 = 0.0f, scale1 = 0.0f, rcp0 = 0.0f, rcp1 = 0.0f;
-    if (l == 0) {
-      scale0 = __fdiv_rn(__uint_as_float(row_amax[slot][rloc0]), kQMax);
-      scale1 = __fdiv_rn(__uint_as_float(row_amax[slot][rloc1]), kQMax);
-      rcp0 = __frcp_rn(scale0);
-      rcp1 = __frcp_rn(scale1);
-    }
-    const int src = threadIdx.x & 16;  // lane 0 of this half-warp
-    scale0 = __shfl_sync(0xffffffffu, scale0, src);
-    scale1 = __shfl_sync(0xffffffffu, scale1, src);
-    rcp0 = __shfl_sync(0xffffffffu, rcp0, src);
-    rcp1 = __shfl_sync(0xffffffffu, rcp1, src);
-    uint32_t c0[16], c1[16];  // code bytes (low byte) of channel 16 i + l
-    if (scale0 >= kMinScale && scale1 >= kMinScale) {
-      const u64 rr = f2(rcp0, rcp1), ns = f2(-scale0, -scale1);
+    // ---- quantize: every lane forms its two rows' scales from their amax
+    constexpr float kInvG = LOG4G == 4 ? 0.0625f : (LOG4G == 3 ? 0.125f : 0.25f);  // 2^-LOG4G
+    constexpr float kG = 1.0f / kInvG;
+    constexpr float kThr = kG * (0.5f - (MODE == kInt8 ? 0x1p-14f : 0x1p-18f));      // 2^LOG4G (1/2 - m)
+    const float scale0 = div_by_qmax<kQHi>(__uint_as_float(row_amax[slot][rloc0]) * kInvG);
+    const float scale1 = div_by_qmax<kQHi>(__uint_as_float(row_amax[slot][rloc1]) * kInvG);
+    const bool in_range = scale0 >= kMinScale && scale0 <= kMaxScale && scale1 >= kMinScale && scale1 <= kMaxScale;
+    // The code bytes of channel 16 i + l go to their row-order positions in
+    // the byte tiles as they are formed (a lane that falls back to the exact
+    // quotient writes its bytes again).
+    bool done = false;
+    if (in_range) {
+      // k = rint(v y) and the remainder v - 2^LOG4G s k; kept where no
+      // remainder reaches 2^LOG4G s (1/2 - m)
+      const u64 y = f2(rcp_approx(scale0) * kInvG, rcp_approx(scale1) * kInvG);
+      const u64 nd = f2(-(scale0 * kG), -(scale1 * kG));
       const u64 mg = f2(kMagic, kMagic);
+      float e0 = 0.0f, e1 = 0.0f;
 #pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        const u64 xv = P[i];
-        u64 q = f2_mul(xv, rr);
-        q = f2_fma(f2_fma(ns, q, xv), rr, q);  // faithful
-        q = f2_fma(f2_fma(ns, q, xv), rr, q);  // RN(x / s)
-        float t0, t1;
-        f2_split(f2_add(q, mg), t0, t1);       // low byte = rint(q)
-        c0[i] = __float_as_uint(t0);
-        c1[i] = __float_as_uint(t1);
+      for (int i = 0; i < 16; i += 2) {
+        const u64 ca = f2_fma(P[i], y, mg), cb = f2_fma(P[i + 1], y, mg);
+        const u64 da = f2_fma(nd, f2_sub(ca, mg), P[i]), db = f2_fma(nd, f2_sub(cb, mg), P[i + 1]);
+        float t0, t1, u0, u1;
+        f2_split(ca, t0, t1);
+        f2_split(cb, u0, u1);
+        bw0[16 * i] = static_cast<uint8_t>(__float_as_uint(t0));
+        bw1[16 * i] = static_cast<uint8_t>(__float_as_uint(t1));
+        bw0[16 * i + 16] = static_cast<uint8_t>(__float_as_uint(u0));
+        bw1[16 * i + 16] = static_cast<uint8_t>(__float_as_uint(u1));
+        f2_split(da, t0, t1);
+        f2_split(db, u0, u1);
+        e0 = max3(e0, fabsf(t0), fabsf(u0));
+        e1 = max3(e1, fabsf(t1), fabsf(u1));
       }
-    } else {
-      // A zero or tiny scale (a whole row takes this branch): IEEE division.
+      done = e0 <= scale0 * kThr && e1 <= scale1 * kThr;
+    }
+    if (!done) {
+      const u64 inv2 = f2(kInvG, kInvG);
+      if (in_range) {
+        // A quotient next to a half-integer: the exact quotient RN(x'/s).
+        const u64 rr = f2(__frcp_rn(scale0), __frcp_rn(scale1)), ns = f2(-scale0, -scale1);
+        const u64 mg = f2(kMagic, kMagic);
 #pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        float x0, x1;
-        f2_split(P[i], x0, x1);
-        const int q0 = scale0 != 0.0f ? __float2int_rn(__fdiv_rn(x0, scale0)) : 0;
-        const int q1 = scale1 != 0.0f ? __float2int_rn(__fdiv_rn(x1, scale1)) : 0;
-        c0[i] = static_cast<uint32_t>(min(kQHi, max(kQLo, q0)));
-        c1[i] = static_cast<uint32_t>(min(kQHi, max(kQLo, q1)));
+        for (int i = 0; i < 16; ++i) {
+          const u64 xv = f2_mul(P[i], inv2);
+          u64 q = f2_mul(xv, rr);
+          q = f2_fma(f2_fma(ns, q, xv), rr, q);  // faithful
+          q = f2_fma(f2_fma(ns, q, xv), rr, q);  // RN(x / s)
+          float t0, t1;
+          f2_split(f2_add(q, mg), t0, t1);       // low byte = rint(q)
+          bw0[16 * i] = static_cast<uint8_t>(__float_as_uint(t0));
+          bw1[16 * i] = static_cast<uint8_t>(__float_as_uint(t1));
+        }
+      } else {
+        // A zero, tiny or huge scale (a whole row takes this branch): IEEE division.
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          float x0, x1;
+          f2_split(f2_mul(P[i], inv2), x0, x1);
+          const int q0 = scale0 != 0.0f ? __float2int_rn(__fdiv_rn(x0, scale0)) : 0;
+          const int q1 = scale1 != 0.0f ? __float2int_rn(__fdiv_rn(x1, scale1)) : 0;
+          bw0[16 * i] = static_cast<uint8_t>(min(kQHi, max(kQLo, q0)));
+          bw1[16 * i] = static_cast<uint8_t>(min(kQHi, max(kQLo, q1)));
+        }
       }
     }
-    // ---- back to row order through the byte tiles, store
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      bw0[16 * i] = static_cast<uint8_t>(c0[i]);
-      bw1[16 * i] = static_cast<uint8_t>(c1[i]);
-    }
+    // ---- back to row order: read the byte tiles, store
     __syncwarp();
     const uint4 o0 = *reinterpret_cast<const uint4*>(btile0 + 16 * l);  // channels 16 l .. 16 l + 15
     const uint4 o1 = *reinterpret_cast<const uint4*>(btile1 + 16 * l);
