@@ -313,10 +313,12 @@ struct PHeader {
 // round to round, so activations larger than L2 are read from DRAM once
 // instead of once per round.
 __device__ __forceinline__ int tile_mi(const PParams& p, int tile) {
-  return p.n_fast ? tile / p.n_tiles : tile % p.m_tiles;
+  const int d = p.n_fast ? p.n_tiles : p.m_tiles, q = tile / d, r = tile - q * d;
+  return p.n_fast ? q : r;
 }
 __device__ __forceinline__ int tile_ni(const PParams& p, int tile) {
-  return p.n_fast ? tile % p.n_tiles : tile / p.m_tiles;
+  const int d = p.n_fast ? p.n_tiles : p.m_tiles, q = tile / d, r = tile - q * d;
+  return p.n_fast ? r : q;
 }
 
 // This CTA's first unit (tile, K block) and number of units.
@@ -405,38 +407,49 @@ __global__ void __launch_bounds__(kPThreads, 1)
     // ready[s] (the producer's arrival, together with the unpack warps').
     if (lane == 0) {
       const uint32_t xbytes = static_cast<uint32_t>(BT * kKB);
-      auto load_w = [&](int s, int tile, int kb) {
+      // The producer walks its units with a cursor that carries the tile's
+      // first weight and token rows; they change (two integer divisions)
+      // only when the cursor moves to the next tile, and the move is made
+      // before the producer waits for the stage it refills, so the waits
+      // are followed by the copies at once.
+      struct Cursor {
+        int tile, kb, wr, xr;
+      };
+      auto at = [&](int tile, int kb) { return Cursor{tile, kb, w_row(tile), x_row(tile)}; };
+      auto next = [&](Cursor& c) {
+        if (++c.kb == p.kbn) c = at(c.tile + static_cast<int>(gridDim.x), 0);
+      };
+      auto load_w = [&](int s, const Cursor& c) {
         if (W8) {
           mbar_arrive_expect_tx(&hdr->ready[s], static_cast<uint32_t>(kWBytes));
-          tma_load_2d(smem + s * stage_bytes, &tm_w, &hdr->ready[s], kb * kKB, w_row(tile));
-          tma_load_2d(smem + s * stage_bytes + kWTileBytes, &tm_w, &hdr->ready[s], kb * kKB + kXBox, w_row(tile));
+          tma_load_2d(smem + s * stage_bytes, &tm_w, &hdr->ready[s], c.kb * kKB, c.wr);
+          tma_load_2d(smem + s * stage_bytes + kWTileBytes, &tm_w, &hdr->ready[s], c.kb * kKB + kXBox, c.wr);
         } else {
           mbar_arrive_expect_tx(&hdr->wfull[s], static_cast<uint32_t>(kWBytes));
-          tma_load_2d(smem + s * stage_bytes, &tm_w, &hdr->wfull[s], kb * (kKB / 2), w_row(tile));
-          if (CB) tma_load_2d(smem + s * stage_bytes + kWTileBytes, &tm_s, &hdr->wfull[s], kb * (kKB / 16), w_row(tile));
+          tma_load_2d(smem + s * stage_bytes, &tm_w, &hdr->wfull[s], c.kb * (kKB / 2), c.wr);
+          if (CB) tma_load_2d(smem + s * stage_bytes + kWTileBytes, &tm_s, &hdr->wfull[s], c.kb * (kKB / 16), c.wr);
         }
       };
-      auto load_x = [&](int s, int tile, int kb) {
+      auto load_x = [&](int s, const Cursor& c) {
         uint8_t* xs = smem + s * stage_bytes + kWBytes;
         mbar_arrive_expect_tx(&hdr->ready[s], xbytes);
-        tma_load_2d(xs, &tm_x, &hdr->ready[s], kb * kKB, x_row(tile));
-        tma_load_2d(xs + BT * kXBox, &tm_x, &hdr->ready[s], kb * kKB + kXBox, x_row(tile));
+        tma_load_2d(xs, &tm_x, &hdr->ready[s], c.kb * kKB, c.xr);
+        tma_load_2d(xs + BT * kXBox, &tm_x, &hdr->ready[s], c.kb * kKB + kXBox, c.xr);
       };
       // Weight tiles of the first stages do not depend on the preceding
       // prologue kernel: request them before waiting for it.
       const int prime = total < ns ? total : ns;
-      int tile = tile0, kb = kb0;
-      for (int i = 0; i < prime; ++i, unit_next(p, tile, kb)) load_w(i, tile, kb);
+      Cursor c = at(tile0, kb0);
+      for (int i = 0; i < prime; ++i, next(c)) load_w(i, c);
       pdl_wait();
-      tile = tile0;
-      kb = kb0;
-      for (int i = 0; i < prime; ++i, unit_next(p, tile, kb)) load_x(i, tile, kb);
+      c = at(tile0, kb0);
+      for (int i = 0; i < prime; ++i, next(c)) load_x(i, c);
       int it = prime, s = prime % ns;  // stage of unit `it`
-      for (; it < total; ++it, unit_next(p, tile, kb)) {
+      for (; it < total; ++it, next(c)) {
         const int w = it - ns;  // the unit that last used stage s
         if (!mbar_wait(&hdr->done[w % kDoneRing], (w / kDoneRing) & 1)) break;
-        load_w(s, tile, kb);
-        load_x(s, tile, kb);
+        load_w(s, c);
+        load_x(s, c);
         if (++s == ns) s = 0;
       }
       // Drain: every issued load has landed before the block may exit.  In
