@@ -22,6 +22,7 @@ in (``out=``) or are allocated with torch; the workspace likewise.
 from __future__ import annotations
 
 import ctypes
+import functools
 import os
 
 import torch
@@ -166,6 +167,34 @@ def _need(t, name, dtype, shape=None):
         raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
 
 
+def _one_device(fn):
+    """Run a call with the device of its tensor arguments current.  Every
+    tensor argument must be a CUDA tensor and all must be on one device
+    (ValueError otherwise), and so must an explicit ``stream``; the default
+    stream is then that device's current stream, and the library's device
+    checks and launches refer to the same device."""
+    @functools.wraps(fn)
+    def wrapped(*args, **kwargs):
+        dev = None
+        for a in (*args, *kwargs.values()):
+            if not isinstance(a, torch.Tensor):
+                continue
+            if not a.is_cuda:
+                raise ValueError(f"{fn.__name__}: every tensor must be a CUDA tensor, got one on {a.device}")
+            if dev is None:
+                dev = a.device
+            elif a.device != dev:
+                raise ValueError(f"{fn.__name__}: tensors on {dev} and {a.device}; all must be on one device")
+        if dev is None:
+            return fn(*args, **kwargs)
+        stream = kwargs.get("stream")
+        if stream is not None and getattr(stream, "device", dev) != dev:
+            raise ValueError(f"{fn.__name__}: stream on {stream.device}, tensors on {dev}")
+        with torch.cuda.device(dev):
+            return fn(*args, **kwargs)
+    return wrapped
+
+
 def convrot_gemm_workspace_size(M: int, N: int, K: int) -> int:
     return int(load_library().convrot_gemm_workspace_size(M, N, K))
 
@@ -181,6 +210,7 @@ def _workspace(ws, nbytes, device):
     return ws
 
 
+@_one_device
 def convrot_rotate_quant(x, xq=None, s_a=None, stream=None):
     lib = load_library()
     M, K = x.shape
@@ -193,6 +223,7 @@ def convrot_rotate_quant(x, xq=None, s_a=None, stream=None):
     return xq, s_a
 
 
+@_one_device
 def convrot_pack_weight(W, Wq=None, s_w=None, stream=None):
     lib = load_library()
     N, K = W.shape
@@ -227,14 +258,17 @@ def _gemm(fn_name, out_dtype, xq, s_a, Wq, s_w, bias, out, workspace, stream):
     return out
 
 
+@_one_device
 def w4a4_gemm(xq, s_a, Wq, s_w, bias=None, out=None, workspace=None, stream=None):
     return _gemm("w4a4_gemm", torch.bfloat16, xq, s_a, Wq, s_w, bias, out, workspace, stream)
 
 
+@_one_device
 def w4a4_gemm_f32(xq, s_a, Wq, s_w, bias=None, out=None, workspace=None, stream=None):
     return _gemm("w4a4_gemm_f32", torch.float32, xq, s_a, Wq, s_w, bias, out, workspace, stream)
 
 
+@_one_device
 def w4a4_gemm_s32(xq, Wq, out=None, workspace=None, stream=None):
     return _gemm("w4a4_gemm_s32", torch.int32, xq, None, Wq, None, None, out, workspace, stream)
 
@@ -256,14 +290,17 @@ def _linear(fn_name, out_dtype, x, Wq, s_w, bias, out, workspace, stream):
     return out
 
 
+@_one_device
 def convrot_w4a4_linear(x, Wq, s_w, bias=None, out=None, workspace=None, stream=None):
     return _linear("convrot_w4a4_linear", torch.bfloat16, x, Wq, s_w, bias, out, workspace, stream)
 
 
+@_one_device
 def convrot_w4a4_linear_f32(x, Wq, s_w, bias=None, out=None, workspace=None, stream=None):
     return _linear("convrot_w4a4_linear_f32", torch.float32, x, Wq, s_w, bias, out, workspace, stream)
 
 
+@_one_device
 def convrot_w4a4_linear_noalloc(x, Wq, s_w, bias=None, out=None, stream=None):
     """The fused Linear using the library's own static scratch instead of a
     workspace (for callers that cannot allocate device memory; see
@@ -286,6 +323,7 @@ def convrot_w4a4_linear_noalloc(x, Wq, s_w, bias=None, out=None, stream=None):
     return out
 
 
+@_one_device
 def convrot_w4a4_quantize(x, workspace, stream=None):
     """First launch of the fused Linear: x -> activation codes + scales in ``workspace``."""
     M, K = x.shape
@@ -296,6 +334,7 @@ def convrot_w4a4_quantize(x, workspace, stream=None):
     return workspace
 
 
+@_one_device
 def convrot_w4a4_gemm_quantized(workspace, M, Wq, s_w, bias=None, out=None, stream=None):
     """Second launch of the fused Linear: ``workspace`` (from convrot_w4a4_quantize) x Wq -> y."""
     N, K = Wq.shape[0], Wq.shape[1] * 2
@@ -344,6 +383,7 @@ def convrot_measure_mma_i8(N: int = 256, a_in_tmem: bool = False, iters: int = 4
 
 # ---- rotation group-size variants (256, 64, 16)
 
+@_one_device
 def convrot_rotate_quant_g(x, group, xq=None, s_a=None, stream=None):
     """convrot_rotate_quant with rotation group ``group`` (256, 64 or 16)."""
     M, K = x.shape
@@ -357,6 +397,7 @@ def convrot_rotate_quant_g(x, group, xq=None, s_a=None, stream=None):
     return xq, s_a
 
 
+@_one_device
 def convrot_pack_weight_g(W, group, Wq=None, s_w=None, stream=None):
     """convrot_pack_weight with rotation group ``group`` (256, 64 or 16)."""
     N, K = W.shape
@@ -370,6 +411,7 @@ def convrot_pack_weight_g(W, group, Wq=None, s_w=None, stream=None):
     return Wq, s_w
 
 
+@_one_device
 def convrot_w4a4_quantize_g(x, workspace, group, stream=None):
     """convrot_w4a4_quantize with rotation group ``group`` (256, 64 or 16)."""
     M, K = x.shape
@@ -395,10 +437,12 @@ def _linear_g(fn_name, out_dtype, x, Wq, s_w, bias, group, out, workspace, strea
     return out
 
 
+@_one_device
 def convrot_w4a4_linear_g(x, Wq, s_w, bias=None, group=256, out=None, workspace=None, stream=None):
     return _linear_g("convrot_w4a4_linear_g", torch.bfloat16, x, Wq, s_w, bias, group, out, workspace, stream)
 
 
+@_one_device
 def convrot_w4a4_linear_g_f32(x, Wq, s_w, bias=None, group=256, out=None, workspace=None, stream=None):
     return _linear_g("convrot_w4a4_linear_g_f32", torch.float32, x, Wq, s_w, bias, group, out, workspace, stream)
 
@@ -413,6 +457,7 @@ def _n_scales(rows, fmt):
     return rows if fmt == W8A8_CONVROT_INT8_ROW else 1
 
 
+@_one_device
 def w8a8_quantize(x, fmt, x8=None, s_x=None, workspace=None, stream=None):
     """x [M, K] bf16 -> (int8 codes [M, K], scales fp32 [M] row-scaled / [1] tensorwise)."""
     M, K = x.shape
@@ -427,6 +472,7 @@ def w8a8_quantize(x, fmt, x8=None, s_x=None, workspace=None, stream=None):
     return x8, s_x
 
 
+@_one_device
 def w8a8_pack_weight(W, fmt, Wq8=None, s_w=None, workspace=None, stream=None):
     """W [N, K] bf16 -> (int8 codes [N, K], scales fp32 [N] row-scaled / [1] tensorwise)."""
     N, K = W.shape
@@ -456,14 +502,17 @@ def _gemm8(fn_name, out_dtype, x8, s_x, Wq8, s_w, bias, fmt, out, stream):
     return out
 
 
+@_one_device
 def w8a8_gemm(x8, s_x, Wq8, s_w, bias=None, fmt=W8A8_INT8_TENSORWISE, out=None, stream=None):
     return _gemm8("w8a8_gemm", torch.bfloat16, x8, s_x, Wq8, s_w, bias, fmt, out, stream)
 
 
+@_one_device
 def w8a8_gemm_f32(x8, s_x, Wq8, s_w, bias=None, fmt=W8A8_INT8_TENSORWISE, out=None, stream=None):
     return _gemm8("w8a8_gemm_f32", torch.float32, x8, s_x, Wq8, s_w, bias, fmt, out, stream)
 
 
+@_one_device
 def w8a8_gemm_s32(x8, Wq8, out=None, stream=None):
     M, K = x8.shape
     N = Wq8.shape[0]
@@ -490,10 +539,12 @@ def _linear8(fn_name, out_dtype, x, Wq8, s_w, bias, fmt, out, workspace, stream)
     return out
 
 
+@_one_device
 def w8a8_linear(x, Wq8, s_w, bias=None, fmt=W8A8_INT8_TENSORWISE, out=None, workspace=None, stream=None):
     return _linear8("w8a8_linear", torch.bfloat16, x, Wq8, s_w, bias, fmt, out, workspace, stream)
 
 
+@_one_device
 def w8a8_linear_f32(x, Wq8, s_w, bias=None, fmt=W8A8_INT8_TENSORWISE, out=None, workspace=None, stream=None):
     return _linear8("w8a8_linear_f32", torch.float32, x, Wq8, s_w, bias, fmt, out, workspace, stream)
 
@@ -529,15 +580,18 @@ def _gemm_asym(fn_name, out_dtype, x8, s_a, idx, s_rel, codebook, s_channel, bia
     return out
 
 
+@_one_device
 def asym_w4a8_gemm(x8, s_a, idx, s_rel, codebook, s_channel, bias=None, out=None, stream=None):
     return _gemm_asym("asym_w4a8_gemm", torch.bfloat16, x8, s_a, idx, s_rel, codebook, s_channel, bias, out, stream)
 
 
+@_one_device
 def asym_w4a8_gemm_f32(x8, s_a, idx, s_rel, codebook, s_channel, bias=None, out=None, stream=None):
     return _gemm_asym("asym_w4a8_gemm_f32", torch.float32, x8, s_a, idx, s_rel, codebook, s_channel, bias, out,
                       stream)
 
 
+@_one_device
 def asym_w4a8_gemm_s32(x8, idx, s_rel, codebook, out=None, stream=None):
     M, K = x8.shape
     _need(x8, "x8", torch.int8)
@@ -566,11 +620,13 @@ def _linear_asym(fn_name, out_dtype, x, idx, s_rel, codebook, s_channel, bias, o
     return out
 
 
+@_one_device
 def asym_w4a8_linear(x, idx, s_rel, codebook, s_channel, bias=None, out=None, workspace=None, stream=None):
     return _linear_asym("asym_w4a8_linear", torch.bfloat16, x, idx, s_rel, codebook, s_channel, bias, out, workspace,
                         stream)
 
 
+@_one_device
 def asym_w4a8_linear_f32(x, idx, s_rel, codebook, s_channel, bias=None, out=None, workspace=None, stream=None):
     return _linear_asym("asym_w4a8_linear_f32", torch.float32, x, idx, s_rel, codebook, s_channel, bias, out,
                         workspace, stream)

@@ -184,3 +184,22 @@ def test_asym_arguments_rejected_before_any_device_call(lib):
     assert lib.asym_w4a8_gemm_s32(good, good, bad, good, 4, 8, 256, good, null) == 3
     # a too small workspace for the fused linear
     assert lib.asym_w4a8_linear(good, good, good, good, good, null, 4, 8, 256, good, good, 16, null) == 5
+
+
+def test_binding_takes_cuda_tensors_on_one_device():
+    # Host tensors are refused by the binding itself, before any library call
+    # (no CPU path); tensors on several devices are refused the same way.
+    import torch
+    import rotation_quantized_bit_b200 as rq
+    x = torch.zeros(4, 256, dtype=torch.bfloat16)
+    wq = torch.zeros(8, 128, dtype=torch.uint8)
+    s = torch.zeros(8)
+    for call in (lambda: rq.convrot_w4a4_linear(x, wq, s), lambda: rq.convrot_rotate_quant(x),
+                 lambda: rq.convrot_pack_weight(x), lambda: rq.w4a4_gemm_s32(wq, wq),
+                 lambda: rq.convrot_w4a4_linear_noalloc(x, wq, s), lambda: rq.w8a8_quantize(x, rq.W8A8_INT8_TENSORWISE),
+                 lambda: rq.convrot_w4a4_linear_g(x, wq, s, group=64)):
+        with pytest.raises(ValueError, match="CUDA tensor"):
+            call()
+    meta = torch.zeros(8, 128, dtype=torch.uint8, device="meta")
+    with pytest.raises(ValueError):
+        rq.w4a4_gemm_s32(meta, meta)
