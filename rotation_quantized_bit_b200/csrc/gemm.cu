@@ -445,17 +445,29 @@ __global__ void __launch_bounds__(kPThreads, 1)
       c = at(tile0, kb0);
       for (int i = 0; i < prime; ++i, next(c)) load_x(i, c);
       int it = prime, s = prime % ns;  // stage of unit `it`
+      bool w_only = false;              // unit `it` has its weight copy issued but not its activations
       for (; it < total; ++it, next(c)) {
         const int w = it - ns;  // the unit that last used stage s
+        // The stage's weight region is free once unit w's weights are in
+        // tensor memory (its ready phase: the unpack warps arrive after their
+        // reads), an MMA's duration before the stage's activations are; int8
+        // weights are the MMA's own operand and wait for its completion.
+        if (!W8) {
+          if (!mbar_wait(&hdr->ready[s], (w / ns) & 1)) break;
+          load_w(s, c);
+          w_only = true;
+        }
         if (!mbar_wait(&hdr->done[w % kDoneRing], (w / kDoneRing) & 1)) break;
-        load_w(s, c);
+        w_only = false;
+        if (W8) load_w(s, c);
         load_x(s, c);
         if (++s == ns) s = 0;
       }
       // Drain: every issued load has landed before the block may exit.  In
       // the normal case the last stages' barriers have completed; after a
       // failed wait (anywhere in the grid) the weight tiles are awaited with a
-      // time limit that ignores the error word, and the activation tiles,
+      // time limit that ignores the error word (that of unit `it` too, when
+      // the loop stopped between its two copies), and the activation tiles,
       // whose barrier also needs the unpack warps, are given a fixed 100 us.
       bool clean = true;
       for (int i = (it > ns ? it - ns : 0); i < it; ++i) {
@@ -463,6 +475,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
           clean = (W8 || mbar_wait(&hdr->wfull[i % ns], (i / ns) & 1)) && mbar_wait(&hdr->ready[i % ns], (i / ns) & 1);
         if (!clean && !W8) (void)mbar_drain(&hdr->wfull[i % ns], (i / ns) & 1, 100000000ull);
       }
+      if (w_only) (void)mbar_drain(&hdr->wfull[it % ns], (it / ns) & 1, 100000000ull);
       if (!clean || it < total) {
         const unsigned long long t0 = globaltimer_ns();
         while (globaltimer_ns() - t0 < 100000ull) {
