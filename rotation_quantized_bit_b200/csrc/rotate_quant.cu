@@ -11,10 +11,12 @@
 //
 // Bit-exact contract.  The butterflies use the fixed stage order (stride 1,
 // 4, 16, 64) and association (p=a+b, q=a-b, r=c+d, t=c-d -> p+t, p-t, q+r,
-// r-q), every add is a correctly rounded fp32 add (no contraction), the 1/16
-// is one multiply, the scale is an IEEE division, and each code equals
-// rint(fl(x' / s)) with ties to even, so codes and scales are identical bit
-// for bit to any plain fp32 evaluation of that definition.
+// r-q) with correctly rounded fp32 adds (no contraction).  The results equal
+// those of the plain fp32 evaluation x' = fl(v / 16), s = fl(amax / 7) and
+// code = rint(fl(x' / s)) with ties to even, so codes and scales are
+// identical bit for bit to any such evaluation of the definition; the
+// Scales and Quantization paragraphs below say how they are reached without
+// a division per element.
 //
 // Layout.  A 256-channel group is one task of 16 lanes (half a warp); each
 // lane holds 16 channels of each of two tasks (two groups, from the same row
