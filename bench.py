@@ -155,18 +155,87 @@ def make_flusher(torch, dev, mode):
 # ------------------------------------------------------------------ clocks
 
 class ClockSampler:
-    """nvidia-smi clocks / throttle reasons sampled every 200 ms while running."""
+    """SM clock and throttle reasons while the timed steps run, from two
+    readers: `nvidia-smi` every 200 ms (the fields of the usual clocks line)
+    and, where the NVML library answers, a thread that reads the same
+    values every 2 ms, so that a timed region of a few ms still gets samples
+    from inside it.  Both only read; NVML failures leave the nvidia-smi
+    record alone."""
 
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
 
-    def __init__(self, gpu_index: int):
-        self.gpu = gpu_index
+    def __init__(self, torch_device: int):
+        self.torch_device = torch_device
+        self.gpu = torch_device  # NVML / nvidia-smi index; resolved by PCI location where NVML answers
         self.proc = None
         self.path = None
+        self.nvml_thread = None
+        self.nvml_stop = None
+        self.nvml_samples = []   # (sm MHz, max MHz, reason names)
+
+    def _nvml_loop(self, nvml, handle, bits):
+        try:
+            smax = float(nvml.nvmlDeviceGetMaxClockInfo(handle, nvml.NVML_CLOCK_SM))
+            while not self.nvml_stop.is_set():
+                sm = float(nvml.nvmlDeviceGetClockInfo(handle, nvml.NVML_CLOCK_SM))
+                active = nvml.nvmlDeviceGetCurrentClocksEventReasons(handle)
+                self.nvml_samples.append((sm, smax, [n for n, b in bits if active & b]))
+                self.nvml_stop.wait(0.002)
+        except Exception:  # noqa: BLE001 -- best effort: the nvidia-smi record stands
+            pass
+
+    def _resolve_index(self, nvml):
+        """The NVML index of the torch device (its PCI domain, bus and device),
+        which differs from the CUDA ordinal when CUDA_VISIBLE_DEVICES is set."""
+        import torch
+        props = torch.cuda.get_device_properties(self.torch_device)
+        want = (props.pci_domain_id, props.pci_bus_id, props.pci_device_id)
+        for i in range(nvml.nvmlDeviceGetCount()):
+            pi = nvml.nvmlDeviceGetPciInfo(nvml.nvmlDeviceGetHandleByIndex(i))
+            if (pi.domain, pi.bus, pi.device) == want:
+                return i
+        return None
+
+    def _start_nvml(self):
+        try:
+            import threading
+            import pynvml as nvml
+            handle = nvml.nvmlDeviceGetHandleByIndex(self.gpu)
+            bits = [("hw_slowdown", nvml.nvmlClocksEventReasonHwSlowdown),
+                    ("hw_thermal_slowdown", nvml.nvmlClocksEventReasonHwThermalSlowdown),
+                    ("sw_thermal_slowdown", nvml.nvmlClocksEventReasonSwThermalSlowdown),
+                    ("sw_power_cap", nvml.nvmlClocksEventReasonSwPowerCap)]
+            self.nvml_stop = threading.Event()
+            self.nvml_thread = threading.Thread(target=self._nvml_loop, args=(nvml, handle, bits), daemon=True)
+            self.nvml_thread.start()
+        except Exception:  # noqa: BLE001 -- no NVML here: nvidia-smi only
+            self.nvml_thread = None
+
+    def _stop_nvml(self):
+        if self.nvml_thread is not None:
+            self.nvml_stop.set()
+            self.nvml_thread.join(timeout=2.0)
+        if not getattr(self, "nvml_ok", False):
+            return
+        try:
+            import pynvml as nvml
+            nvml.nvmlShutdown()
+        except Exception:  # noqa: BLE001
+            pass
 
     def start(self):
+        try:
+            import pynvml as nvml
+            nvml.nvmlInit()
+            self.nvml_ok = True
+            idx = self._resolve_index(nvml)
+            if idx is not None:
+                self.gpu = idx
+        except Exception:  # noqa: BLE001 -- no NVML: the CUDA ordinal, nvidia-smi only
+            self.nvml_ok = False
         try:
             import tempfile
             fd, self.path = tempfile.mkstemp(prefix="clocks_", suffix=".csv")
@@ -177,37 +246,56 @@ class ClockSampler:
                  "-i", str(self.gpu)], stdout=self.fh, stderr=subprocess.DEVNULL)
         except (OSError, FileNotFoundError):
             self.proc = None
+        if self.nvml_ok:
+            self._start_nvml()
 
     def stop(self):
-        if self.proc is None:
-            return None
-        time.sleep(0.25)
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
-        self.fh.close()
+        self._stop_nvml()
         sm, smax, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        with open(self.path) as f:
-            for line in f:
-                parts = [p.strip() for p in line.split(",")]
-                if len(parts) < 9:
-                    continue
-                try:
-                    sm.append(float(parts[1]))
-                    smax = float(parts[2])
-                except ValueError:
-                    continue
-                for n, v in zip(names, parts[5:9]):
-                    if v.lower().startswith("active"):
-                        reasons.add(n)
-        os.unlink(self.path)
-        if not sm:
-            return None
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": smax, "reasons": sorted(reasons),
-                "samples": len(sm)}
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.fh.close()
+            with open(self.path) as f:
+                for line in f:
+                    parts = [p.strip() for p in line.split(",")]
+                    if len(parts) < 9:
+                        continue
+                    try:
+                        sm.append(float(parts[1]))
+                        smax = float(parts[2])
+                    except ValueError:
+                        continue
+                    for n, v in zip(self.REASONS, parts[5:9]):
+                        if v.lower().startswith("active"):
+                            reasons.add(n)
+            os.unlink(self.path)
+        out = None
+        if sm:
+            out = {"sm_mhz": statistics.median(sm), "sm_max_mhz": smax, "reasons": sorted(reasons),
+                   "samples": len(sm), "source": "nvidia-smi every 200 ms"}
+        if self.nvml_samples:
+            nsm = [x[0] for x in self.nvml_samples]
+            nreasons = set(r for x in self.nvml_samples for r in x[2])
+            nv = {"sm_mhz": statistics.median(nsm), "sm_min_mhz": min(nsm), "sm_max_mhz": self.nvml_samples[0][1],
+                  "reasons": sorted(nreasons), "samples": len(nsm),
+                  "source": "NVML every 2 ms during the timed steps (the thread runs while the host is free)",
+                  "nvml_index": self.gpu}
+            if out is None or len(nsm) >= 3:
+                # the headline: the samples taken inside the timed steps, with
+                # the reasons either reader saw
+                smi = out
+                out = dict(nv, reasons=sorted(nreasons | set(smi["reasons"] if smi else [])))
+                if smi is not None:
+                    out["nvidia_smi"] = smi
+            else:
+                out["reasons"] = sorted(set(out["reasons"]) | nreasons)
+                out["nvml"] = nv
+        return out
 
 
 # ------------------------------------------------------------------ the oracle leg
