@@ -187,9 +187,9 @@ def _one_device(fn):
                 raise ValueError(f"{fn.__name__}: tensors on {dev} and {a.device}; all must be on one device")
         if dev is None:
             return fn(*args, **kwargs)
-        stream = kwargs.get("stream")
-        if stream is not None and getattr(stream, "device", dev) != dev:
-            raise ValueError(f"{fn.__name__}: stream on {stream.device}, tensors on {dev}")
+        for a in (*args, *kwargs.values()):
+            if isinstance(a, torch.cuda.Stream) and a.device != dev:
+                raise ValueError(f"{fn.__name__}: stream on {a.device}, tensors on {dev}")
         with torch.cuda.device(dev):
             return fn(*args, **kwargs)
     return wrapped
