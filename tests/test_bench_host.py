@@ -44,3 +44,37 @@ def test_workload_formats(workload, fmt, count):
         assert {s.fmt for s in shapes} == {"convrot_int8", "w4a4"}
     assert all(s.K % 256 == 0 and s.N % 8 == 0 for s in shapes)
     assert workload in bench.WORKLOAD_DESC
+
+
+class _DoneProc:
+    def terminate(self):
+        pass
+
+    def wait(self, timeout=None):
+        return 0
+
+
+def _sampler_with(tmp_path, smi_lines, nvml):
+    c = bench.ClockSampler(0)
+    c.nvml_ok = False
+    if smi_lines is not None:
+        path = tmp_path / "clocks.csv"
+        path.write_text("".join(l + "\n" for l in smi_lines))
+        c.path, c.fh, c.proc = str(path), open(os.devnull, "w"), _DoneProc()
+    c.nvml_samples = nvml
+    return c
+
+
+def test_clock_record_merges_both_readers(tmp_path):
+    smi = ["0, 1965, 1965, 700.5, 0x0, Not Active, Not Active, Not Active, Not Active",
+           "0, 1950, 1965, 800.0, 0x4, Not Active, Not Active, Not Active, Active"]
+    # few NVML samples: the nvidia-smi record leads, NVML beside it, reasons united
+    r = _sampler_with(tmp_path, smi, [(1965.0, 1965.0, ["hw_slowdown"])]).stop()
+    assert r["source"].startswith("nvidia-smi") and r["samples"] == 2 and r["sm_mhz"] == 1957.5
+    assert r["reasons"] == ["hw_slowdown", "sw_power_cap"] and r["nvml"]["samples"] == 1
+    # enough NVML samples from inside the timed steps: they lead
+    r = _sampler_with(tmp_path, smi, [(1965.0, 1965.0, [])] * 3 + [(1900.0, 1965.0, [])]).stop()
+    assert r["source"].startswith("NVML") and r["samples"] == 4 and r["sm_min_mhz"] == 1900.0
+    assert r["reasons"] == ["sw_power_cap"] and r["nvidia_smi"]["samples"] == 2
+    # no reader at all (a host without a GPU): no record
+    assert _sampler_with(tmp_path, None, []).stop() is None
